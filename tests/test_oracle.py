@@ -1,0 +1,285 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself -- closed
+forms, brute force on tiny inputs, special cases that reduce to textbook formulas evaluated
+with torch float64 library matmuls, and a hand-worked example.  Definitions pinned:
+G(x) = Softmax(TopK(x . W_g)) and y = sum_i G(x)_i SwiGLU_i(x) ("Mixtral of Experts",
+arXiv 2401.04088, method section), and the statement that experts with zero gate need not
+be computed (Indonesian news summary, section on how the MoE layer is computed)."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _sig(z):
+    return 1.0 / (1.0 + math.exp(-z))
+
+
+def _silu(z):
+    return z * _sig(z)
+
+
+def _rand(shape, std, seed, dtype=torch.float32):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g, dtype=torch.float32) * std).to(dtype)
+
+
+def _layer(T, d, F, n, seed=0, dtype=torch.float32):
+    x = _rand((T, d), 1.0, seed, dtype)
+    Wg = _rand((d, n), d ** -0.5, seed + 1)
+    W1 = _rand((n, F, d), d ** -0.5, seed + 2, dtype)
+    W3 = _rand((n, F, d), d ** -0.5, seed + 3, dtype)
+    W2 = _rand((n, d, F), F ** -0.5, seed + 4, dtype)
+    return x, Wg, W1, W3, W2
+
+
+def _swiglu64(xt, W1e, W3e, W2e):
+    """SwiGLU expert with torch float64 library matmuls (independent of the oracle's loops)."""
+    a = W1e.double() @ xt.double()
+    b = W3e.double() @ xt.double()
+    return W2e.double() @ (torch.nn.functional.silu(a) * b)
+
+
+# ------------------------------------------------------------------ rounding helpers
+
+def test_round_bf16_matches_torch_rne(oracle_lib):
+    # Every fp32 value is exact in double, so torch's fp32 -> bf16 (round to nearest even)
+    # is the reference; include ties, subnormals and large values.
+    vals = torch.cat([
+        _rand((4000,), 1.0, 7), _rand((1000,), 1e-39, 8), _rand((1000,), 1e30, 9),
+        torch.tensor([1.00390625, 1.01171875, -1.00390625, 2.0 ** -130, 3.0e38, 0.0]),
+    ]).float()
+    ref = vals.to(torch.bfloat16).double()
+    got = torch.tensor([oracle_lib.round_bf16(float(v)) for v in vals], dtype=torch.float64)
+    assert torch.equal(got, ref)
+
+
+def test_round_bf16_ties_to_even(oracle_lib):
+    assert oracle_lib.round_bf16(1.0 + 2.0 ** -8) == 1.0          # tie -> even (1.0)
+    assert oracle_lib.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert oracle_lib.round_bf16(1.0 + 2.0 ** -8 + 2.0 ** -30) == 1.0 + 2.0 ** -7
+
+
+def test_silu_closed_forms(oracle_lib):
+    assert oracle_lib.silu(0.0) == 0.0
+    assert oracle_lib.silu(1.0) == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)
+    for z in (-5.0, -0.3, 0.7, 4.0):
+        # silu(z) - silu(-z) = z  (since sig(z) + sig(-z) = 1)
+        assert oracle_lib.silu(z) - oracle_lib.silu(-z) == pytest.approx(z, rel=1e-14)
+    assert oracle_lib.silu(40.0) == pytest.approx(40.0, rel=1e-15)
+    z = torch.linspace(-8, 8, 101, dtype=torch.float64)
+    ref = torch.nn.functional.silu(z)
+    got = torch.tensor([oracle_lib.silu(float(v)) for v in z], dtype=torch.float64)
+    assert torch.allclose(got, ref, rtol=1e-14, atol=1e-300)
+
+
+# ------------------------------------------------------------------ router: logits, TopK, G
+
+@pytest.mark.parametrize("n,K", [(8, 2), (8, 1), (6, 3), (5, 5), (16, 2)])
+def test_router_brute_force(oracle_lib, n, K):
+    T, d = 64, 24
+    x = _rand((T, d), 1.0, 11 + n)
+    Wg = _rand((d, n), d ** -0.5, 12 + K)
+    logits, idx, gate = oracle_lib.route(x, Wg, n, K)
+    ref_logits = (x.double() @ Wg.double()).numpy()
+    assert np.allclose(logits, ref_logits, rtol=1e-13, atol=1e-13)
+    for t in range(T):
+        l = logits[t]
+        # brute force: the chosen subset maximises the sum of kept logits (equivalently every
+        # kept logit >= every dropped one); ties resolved towards lower indices.
+        best = max(itertools.combinations(range(n), K),
+                   key=lambda s: (sorted((l[i] for i in s), reverse=True),
+                                  [-i for i in sorted(s)]))
+        assert sorted(idx[t].tolist()) == sorted(best)
+        assert len(set(idx[t].tolist())) == K
+        # slot order: descending logit
+        assert all(l[idx[t, k]] >= l[idx[t, k + 1]] for k in range(K - 1))
+        # G = softmax of the kept logits
+        kept = np.array([l[i] for i in idx[t]])
+        ref = np.exp(kept - kept.max()) / np.exp(kept - kept.max()).sum()
+        assert np.allclose(gate[t], ref, rtol=1e-14, atol=0)
+        assert gate[t].sum() == pytest.approx(1.0, abs=1e-15)
+        assert np.all(np.diff(gate[t]) <= 0) and gate[t][0] >= 1.0 / K - 1e-15
+
+
+def test_gate_closed_form_k2(oracle_lib):
+    T, d, n = 128, 32, 8
+    x = _rand((T, d), 1.0, 21)
+    Wg = _rand((d, n), d ** -0.5, 22)
+    logits, idx, gate = oracle_lib.route(x, Wg, n, 2)
+    for t in range(T):
+        l1, l2 = logits[t, idx[t, 0]], logits[t, idx[t, 1]]
+        assert gate[t, 0] == pytest.approx(_sig(l1 - l2), rel=1e-14)
+        assert gate[t, 1] == pytest.approx(_sig(l2 - l1), rel=1e-13)
+        assert gate[t, 0] >= 0.5
+
+
+def test_router_exact_ties_lowest_index(oracle_lib):
+    d, n = 4, 8
+    x = torch.tensor([[1.0, 2.0, -1.0, 0.5]])
+    Wg = torch.ones((d, n)) * 0.25                     # all logits equal
+    _, idx, gate = oracle_lib.route(x, Wg, n, 2)
+    assert idx[0].tolist() == [0, 1] and gate[0].tolist() == [0.5, 0.5]
+    Wg2 = Wg.clone()
+    Wg2[:, 5] = 0.5                                     # expert 5 strictly largest
+    Wg2[:, 3] = 0.4                                     # 3 and 6 tie for second
+    Wg2[:, 6] = 0.4
+    _, idx, _ = oracle_lib.route(x, Wg2, n, 2)
+    assert idx[0].tolist() == [5, 3]
+    _, idx, _ = oracle_lib.route(x, Wg2, n, 3)
+    assert idx[0].tolist() == [5, 3, 6]
+
+
+def test_tie_band_helper(oracle_lib):
+    ex, sets = oracle_lib.tie_band(np.array([3.0, 1.0, 2.0, 2.0 + 1e-6]), 2)
+    assert ex and sorted(sets) == [(0, 2), (0, 3)]
+    ex, sets = oracle_lib.tie_band(np.array([3.0, 1.0, 2.0, 2.5]), 2)
+    assert not ex and sets == [(0, 3)]
+
+
+# ------------------------------------------------------------------ experts and the block
+
+def test_hand_worked_token(oracle_lib):
+    with open(os.path.join(HERE, "golden", "hand_worked_token.json")) as f:
+        g = json.load(f)
+    x = torch.tensor(g["x"], dtype=torch.float32)
+    Wg = torch.tensor(g["W_g_rows_d_by_n"], dtype=torch.float32)
+    W1 = torch.tensor(g["W1_n_F_d"], dtype=torch.float32)
+    W3 = torch.tensor(g["W3_n_F_d"], dtype=torch.float32)
+    W2 = torch.tensor(g["W2_n_d_F"], dtype=torch.float32)
+    n, K = g["dims"]["n"], g["dims"]["K"]
+    env = {"sig": _sig, "silu": _silu}
+    logits, idx, gate = oracle_lib.route(x, Wg, n, K)
+    assert logits.tolist() == g["expected_logits"]
+    assert idx.tolist() == g["expected_idx"]
+    assert gate[0] == pytest.approx([eval(e, env) for e in g["expected_gate_expr"]], rel=1e-15)
+    y, idx2, _ = oracle_lib.moe_forward(x, Wg, W1, W3, W2, n, K, round_h=False)
+    assert idx2.tolist() == g["expected_idx"]
+    assert y[0] == pytest.approx([eval(e, env) for e in g["expected_y_expr"]], rel=1e-14)
+    yd = oracle_lib.moe_dense(x, Wg, W1, W3, W2, n, K, round_h=False)
+    assert yd[0] == pytest.approx(y[0], rel=1e-15)
+
+
+def test_identity_experts_reduce_to_silu_times_x(oracle_lib):
+    # F = d and W1 = W3 = W2 = I: every expert gives silu(x) * x, and the gates sum to 1.
+    T, d, n = 16, 32, 8
+    x = _rand((T, d), 2.0, 31)
+    Wg = _rand((d, n), d ** -0.5, 32)
+    eye = torch.eye(d).expand(n, d, d).contiguous()
+    y, _, _ = oracle_lib.moe_forward(x, Wg, eye, eye, eye, n, 2, round_h=False)
+    ref = (torch.nn.functional.silu(x.double()) * x.double()).numpy()
+    assert np.allclose(y, ref, rtol=1e-13, atol=1e-15)
+
+
+def test_single_expert_is_plain_ffn(oracle_lib):
+    # n = 1, K = 1: the block is one SwiGLU FFN (gate 1).  d != F catches transposed W.
+    T, d, F = 8, 24, 40
+    x, Wg, W1, W3, W2 = _layer(T, d, F, 1, seed=41)
+    y, idx, gate = oracle_lib.moe_forward(x, Wg, W1, W3, W2, 1, 1, round_h=False)
+    assert np.all(idx == 0) and np.all(gate == 1.0)
+    for t in range(T):
+        ref = _swiglu64(x[t], W1[0], W3[0], W2[0]).numpy()
+        assert np.allclose(y[t], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_k_equals_n_is_dense_softmax_moe(oracle_lib):
+    # K = n: G is the full softmax of the logits -- the textbook dense mixture.
+    T, d, F, n = 6, 16, 20, 4
+    x, Wg, W1, W3, W2 = _layer(T, d, F, n, seed=51)
+    y, _, _ = oracle_lib.moe_forward(x, Wg, W1, W3, W2, n, n, round_h=False)
+    G = torch.softmax(x.double() @ Wg.double(), dim=1)
+    for t in range(T):
+        ref = sum(G[t, e] * _swiglu64(x[t], W1[e], W3[e], W2[e]) for e in range(n)).numpy()
+        assert np.allclose(y[t], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_top2_matches_library_reference(oracle_lib):
+    # K = 2 of 8 against torch float64: topk (lowest index on ties is irrelevant for random
+    # data), softmax over the two kept logits, explicit weighted sum of two experts.
+    T, d, F, n = 12, 32, 48, 8
+    x, Wg, W1, W3, W2 = _layer(T, d, F, n, seed=61)
+    y, idx, gate = oracle_lib.moe_forward(x, Wg, W1, W3, W2, n, 2, round_h=False)
+    l = x.double() @ Wg.double()
+    top = torch.topk(l, 2, dim=1)
+    assert torch.equal(torch.from_numpy(idx).long(), top.indices)
+    G = torch.softmax(top.values, dim=1)
+    for t in range(T):
+        ref = sum(G[t, k] * _swiglu64(x[t], W1[top.indices[t, k]], W3[top.indices[t, k]],
+                                      W2[top.indices[t, k]]) for k in range(2)).numpy()
+        assert np.allclose(y[t], ref, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_sparse_equals_dense_masked(oracle_lib, dtype):
+    T, d, F, n = 10, 32, 64, 8
+    x, Wg, W1, W3, W2 = _layer(T, d, F, n, seed=71, dtype=dtype)
+    for round_h in (False, True):
+        ys, _, _ = oracle_lib.moe_forward(x, Wg, W1, W3, W2, n, 2, round_h=round_h)
+        yd = oracle_lib.moe_dense(x, Wg, W1, W3, W2, n, 2, round_h=round_h)
+        assert np.allclose(ys, yd, rtol=1e-12, atol=1e-15)
+
+
+def test_bf16_inputs_decoded_exactly(oracle_lib):
+    # bf16 tensors and fp32 tensors holding the same values must give identical results.
+    T, d, F, n = 8, 32, 40, 8
+    x, Wg, W1, W3, W2 = _layer(T, d, F, n, seed=81, dtype=torch.bfloat16)
+    yb, ib, gb = oracle_lib.moe_forward(x, Wg, W1, W3, W2, n, 2, round_h=False)
+    yf, i_f, gf = oracle_lib.moe_forward(x.float(), Wg, W1.float(), W3.float(), W2.float(),
+                                         n, 2, round_h=False)
+    assert np.array_equal(ib, i_f) and np.array_equal(gb, gf) and np.array_equal(yb, yf)
+
+
+def test_h_rounding_is_bf16(oracle_lib):
+    # With n = 1, K = 1 and W2 = I, y = h exactly, so round_h must give bf16-representable
+    # values equal to the library's fp64 -> fp32 -> bf16 rounding of silu(a)*b where that
+    # double rounding cannot differ (checked on fp32-exact intermediate values).
+    T, d = 6, 16
+    x = _rand((T, d), 1.0, 91, torch.bfloat16)
+    Wg = _rand((d, 1), 0.25, 92)
+    W1 = _rand((1, d, d), d ** -0.5, 93, torch.bfloat16)
+    W3 = _rand((1, d, d), d ** -0.5, 94, torch.bfloat16)
+    W2 = torch.eye(d, dtype=torch.bfloat16).unsqueeze(0).contiguous()
+    y, _, _ = oracle_lib.moe_forward(x, Wg, W1, W3, W2, 1, 1, round_h=True)
+    yu, _, _ = oracle_lib.moe_forward(x, Wg, W1, W3, W2, 1, 1, round_h=False)
+    yb = torch.from_numpy(y)
+    assert torch.equal(yb.float().to(torch.bfloat16).double(), yb)          # representable
+    assert np.all(np.abs(y - yu) <= np.abs(yu) * 2.0 ** -8 + 1e-30)          # half-ulp
+
+
+def test_token_with_experts_matches_forward(oracle_lib):
+    T, d, F, n = 5, 16, 24, 8
+    x, Wg, W1, W3, W2 = _layer(T, d, F, n, seed=101)
+    y, idx, _ = oracle_lib.moe_forward(x, Wg, W1, W3, W2, n, 2)
+    for t in range(T):
+        yt = oracle_lib.moe_token_with_experts(x, Wg, W1, W3, W2, n, t, idx[t])
+        assert np.allclose(yt, y[t], rtol=1e-15, atol=0)
+        yr = oracle_lib.moe_token_with_experts(x, Wg, W1, W3, W2, n, t, idx[t][::-1].copy())
+        assert np.allclose(yr, y[t], rtol=1e-14, atol=1e-16)
+
+
+# ------------------------------------------------------------------ stacked blocks
+
+def test_rmsnorm_closed_form(oracle_lib):
+    x = _rand((4, 64), 3.0, 111).double().numpy()
+    got = oracle_lib.rmsnorm(x, 1e-5, oracle_lib.F32)
+    ref = x / np.sqrt((x ** 2).mean(axis=1, keepdims=True) + 1e-5)
+    assert np.allclose(got, ref.astype(np.float32).astype(np.float64), rtol=0, atol=0)
+    c = np.full((1, 16), 3.0)
+    assert np.allclose(oracle_lib.rmsnorm(c, 0.0, oracle_lib.F32), 1.0)
+
+
+def test_block_forward_is_residual_plus_moe_of_norm(oracle_lib):
+    T, d, F, n, eps = 6, 32, 48, 8, 1e-5
+    x, Wg, W1, W3, W2 = _layer(T, d, F, n, seed=121)
+    x64 = x.double().numpy()
+    xn = oracle_lib.rmsnorm(x64, eps, oracle_lib.F32)
+    y, idx_ref, _ = oracle_lib.moe_forward(torch.from_numpy(xn).float(), Wg, W1, W3, W2, n, 2)
+    ref = (x64 + y).astype(np.float32).astype(np.float64)
+    got, idx, _ = oracle_lib.block_forward(x64, Wg, W1, W3, W2, n, 2, eps)
+    assert np.array_equal(idx, idx_ref)
+    assert np.allclose(got, ref, rtol=0, atol=0)
