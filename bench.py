@@ -1,0 +1,362 @@
+"""Benchmark of the Mixtral sparse-MoE block forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole block (router + TopK + softmax, permute, both expert GEMMs,
+gated combine) over one batch of seeded synthetic input of the workload's shapes.  Default
+workload: Mixtral-shaped decode batch (T=16, d=4096, F=14336, n=8, K=2, bf16).
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a device
+synchronisation, timed with CUDA events on the launching stream, max over ranks.  The expert
+weights (2.8 GB per layer) exceed the 126 MB L2, so no flush is needed between steps.
+  value   tokens/s of all ranks with inputs resident in HBM (moe_forward);
+  e2e     the same through moe_forward_host_io with pinned host x / out, host<->device
+          copies and a per-step synchronisation inside the timed region;
+  roofline  the dominant kernel (the gate/up expert GEMM), its duration from events the
+          library records on its own stream around each stage.
+With N > 1 (torchrun) every rank runs an independent replica on its own batch (the block
+has no exchange step on one node's data-parallel path): weak scaling.
+
+--impl reference times the CPU oracle (plain C, fp64, OpenMP) on the host cores on the same
+workload's metric, each step a bounded sample of tokens (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import moe_inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and TFLOP/s (bf16, top-2 of 8) as % of B200 roofline"
+DEFAULT_WORKLOAD = "decode_t16"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"],
+                "bf16_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return False
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.strip().splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) >= 9:
+                self.rows.append(f)
+        return False
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if r[5 + i].lower() == "active"})
+        loaded = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def _flops_per_token(w):
+    # routed work: 2 FLOPs per multiply-add; K experts x 3 d-by-F matrices + router d*n
+    return w.K * 3 * 2 * w.d * w.F + 2 * w.d * w.n
+
+
+def run_gpu(args, w):
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_18_b200 as moe
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=300))
+    peaks = _peaks()
+    # per-rank replica: its own batch (seed offset by rank), its own copy of the weights
+    wr = w.replace(seed=w.seed + 7919 * rank)
+    x = moe_inputs.make_x(wr, device=dev)
+    layer = moe_inputs.make_layer(wr, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    ws = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K, torch.bfloat16),
+                             dev, stream)
+    out = torch.empty_like(x)
+    L = moe.lib()
+    import ctypes
+    info = [ctypes.c_int(0) for _ in range(4)]
+    L.moe_plan_info(w.T, w.d, w.F, w.n, w.K, 1, *[ctypes.byref(v) for v in info])
+    small_batch, s13, s2, launches = (v.value for v in info)
+
+    def step():
+        moe.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.K, out=out,
+                        workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    _, idx, _, counts, _, _ = moe.moe_forward_debug(x, layer["Wg"], layer["W1"], layer["W3"],
+                                                    layer["W2"], w.K, workspace=ws,
+                                                    stream=stream)
+    torch.cuda.synchronize(dev)
+    counts = counts.cpu().tolist()
+    n_active = sum(1 for c in counts if c > 0)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        # ---- value: device-resident inputs
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+        ms = ev0.elapsed_time(ev1)
+        # ---- per-stage durations from events recorded by the library on its stream
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)]
+               for _ in range(args.steps)]
+        arr_t = ctypes.c_void_p * 6
+        for i in range(args.steps):
+            for e in evs[i]:
+                e.record(stream)  # creates the cudaEvent_t; the library re-records it
+            handles = arr_t(*[ctypes.c_void_p(e.cuda_event) for e in evs[i]])
+            rc = L.moe_forward_profiled(
+                ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(layer["Wg"].data_ptr()),
+                ctypes.c_void_p(layer["W1"].data_ptr()), ctypes.c_void_p(layer["W3"].data_ptr()),
+                ctypes.c_void_p(layer["W2"].data_ptr()), w.T, w.d, w.F, w.n, w.K, 1,
+                ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                ctypes.c_void_p(stream.cuda_stream), handles, 6)
+            if rc != 0:
+                raise RuntimeError(f"moe_forward_profiled failed: {rc}")
+        barrier()
+        stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
+                    for i in range(args.steps)]
+        # ---- e2e: pinned host x in, host out back, every step
+        xh = x.cpu().pin_memory()
+        oh = torch.empty_like(xh).pin_memory()
+        xd, od = torch.empty_like(x), torch.empty_like(x)
+        for _ in range(max(1, args.warmup)):
+            moe.moe_forward_host_io(xh, xd, layer["Wg"], layer["W1"], layer["W3"], layer["W2"],
+                                    w.K, od, oh, ws, stream=stream)
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            moe.moe_forward_host_io(xh, xd, layer["Wg"], layer["W1"], layer["W3"], layer["W2"],
+                                    w.K, od, oh, ws, stream=stream)
+            stream.synchronize()
+        ev1.record(stream)
+        barrier()
+        e2e_ms = ev0.elapsed_time(ev1)
+    code, raw = moe.moe_workspace_status(ws, stream)
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({raw:#x})")
+
+    # max over ranks
+    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, e2e_ms = t.tolist()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    ms_step = ms / args.steps
+    tok_s = world * w.T * args.steps / (ms / 1e3)
+    tflops = tok_s * _flops_per_token(w) / 1e12
+    g13 = statistics.mean(s[1] for s in stage_ms)          # gate/up GEMM (dominant kernel)
+    stage_avg = [statistics.mean(s[j] for s in stage_ms) for j in range(5)]
+    es = 2
+    weight_bytes_13 = n_active * 2 * w.F * w.d * es
+    weight_bytes_all = n_active * 3 * w.F * w.d * es
+    timed_s = ms / 1e3
+    bf16_peak = peaks["bf16_sustained"] if timed_s > 1.0 else peaks["bf16"]
+    if small_batch:
+        bound, unit = "hbm", "GB/s"
+        traffic_alg = weight_bytes_13 + w.T * w.K * w.d * es
+        achieved = traffic_alg / (g13 / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        step_alg = weight_bytes_all + w.d * w.n * 4 + 2 * w.T * w.d * es
+        step_frac = step_alg / (ms_step / 1e3) / 1e9 / peak
+    else:
+        bound, unit = "tensor", "TFLOP/s"
+        achieved = 4 * w.d * w.F * w.T * w.K / (g13 / 1e3) / 1e12
+        peak = bf16_peak
+        step_frac = tflops / peak
+    line = {
+        "metric": METRIC, "value": round(tok_s, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, RMS-normalised; N(0,1/fan_in) weights)",
+        "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K} bf16",
+                   "tokens_per_rank": w.T, "l2": "inputs larger than L2 "
+                   f"({3 * w.n * w.F * w.d * es / 1e9:.2f} GB of expert weights)",
+                   "parallelism": f"replicas x{world}", "tiling": "small-batch swap-AB "
+                   f"split-K {s13}/{s2}" if small_batch else "prefill 128-row tiles",
+                   "active_experts": n_active, "expert_counts": counts},
+        "tflops": round(tflops, 3),
+        "pct_roofline": {"bound": "hbm" if small_batch else "tensor",
+                         "frac": round(step_frac, 4),
+                         "basis": "unique expert-weight bytes of selected experts per step / "
+                                  "measured HBM copy GB/s" if small_batch else
+                                  "routed FLOPs per step / measured bf16 GEMM TFLOP/s"},
+        "roofline": {"bound": bound, "kernel": "tc_grouped_gemm G13 (gate/up + SwiGLU)",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": peaks["source"], "launch_ms": round(g13, 5)},
+        "stage_ms": {"route": round(stage_avg[0], 5), "gemm13": round(stage_avg[1], 5),
+                     "splitk_reduce": round(stage_avg[2], 5), "gemm2": round(stage_avg[3], 5),
+                     "combine": round(stage_avg[4], 5)},
+        "e2e": {"value": round(world * w.T * args.steps / (e2e_ms / 1e3), 2),
+                "unit": "tokens/s", "h2d_bytes_per_step": w.T * w.d * es,
+                "d2h_bytes_per_step": w.T * w.d * es},
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, x.cpu(), {k: v.cpu() for k, v in layer.items()},
+                                            args.cpu_tokens)
+    print(json.dumps(line), flush=True)
+    return line
+
+
+def cpu_baseline(w, x, layer, ntok):
+    """The oracle as it stands on the host cores, on a bounded sample of tokens."""
+    import oracle
+    oracle.build()
+    ntok = min(ntok, w.T)
+    toks = list(range(ntok))
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
+                       tokens=toks)
+    dt = time.perf_counter() - t0
+    return {"value": round(ntok / dt, 4), "unit": "tokens/s", "cores": _omp_threads(),
+            "kind": "oracle", "sample": f"{ntok} of {w.T} tokens of {w.name}, "
+                                        f"{dt:.1f} s (fp64 C, OpenMP over tokens)"}
+
+
+def _omp_threads():
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v and v.isdigit() else (len(os.sched_getaffinity(0))
+                                             if hasattr(os, "sched_getaffinity")
+                                             else os.cpu_count())
+
+
+def run_reference(args, w):
+    """Reference arm: the CPU oracle timed on the host cores (rank 0 only)."""
+    world, rank, _ = _dist()
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    x = moe_inputs.make_x(w)
+    layer = moe_inputs.make_layer(w)
+    per_step = min(w.T, args.cpu_tokens)
+    for i in range(args.warmup):
+        oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
+                           tokens=[i % w.T])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        toks = [(i * per_step + j) % w.T for j in range(per_step)]
+        oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
+                           tokens=toks)
+    dt = time.perf_counter() - t0
+    v = per_step * args.steps / dt
+    sample = (f"{per_step} of {w.T} tokens of {w.name} per step "
+              "(fp64 C oracle, OpenMP over tokens)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K}"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": _omp_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return line
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(moe_inputs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=4,
+                    help="tokens per oracle sample (CPU baseline / reference arm)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = moe_inputs.WORKLOADS[args.workload]
+    if w.layers > 1 or w.dtype != "bf16":
+        ap.error("the bench measures single bf16 blocks")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,157 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts block library (libmoe.so).
+ *
+ * What is computed, per token x (a row of the activation matrix), as defined in
+ * "Mixtral of Experts" (arXiv 2401.04088), method section, equations G(x) and y:
+ *
+ *   l    = x . W_g                         router logits over n experts, fp32, no bias
+ *   G(x) = Softmax(TopK(l))                TopK keeps the K largest logits (others -inf);
+ *                                          Mixtral uses K = 2 of n = 8
+ *   y    = sum_i G(x)_i * SwiGLU_i(x),     SwiGLU_i(x) = W2_i . (silu(W1_i . x) * (W3_i . x))
+ *
+ * Experts whose gate is zero are not evaluated (the Indonesian news summary, section on how
+ * the MoE layer is computed, notes this is exact); tokens are grouped per expert instead
+ * (the same page's implementation notes: variable token counts per expert).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument not marked "host" is a DEVICE pointer on the current CUDA device.
+ *  - Layouts are row-major:  x, out [T][d];  W_g [d][n] (always fp32);
+ *    W1, W3 [n][F][d];  W2 [n][d][F].  x, W1, W3, W2 and out share the dtype `dt`.
+ *  - Ties in TopK go to the lower expert index; slot 0 holds the larger logit.
+ *  - bf16 path: fp32 accumulation on the tensor cores; h = silu(a) * b is rounded to bf16
+ *    before the down-projection; each token's gated sum is accumulated in fp32 and rounded
+ *    once to bf16.  fp32 path: fp32 everywhere (no TF32).
+ *  - The caller owns all memory, including a workspace of at least moe_workspace_bytes()
+ *    bytes (256-byte aligned) that must be initialised once with moe_workspace_init().
+ *    The library never allocates or frees memory and never synchronises the stream on the
+ *    forward path; all work is enqueued on `stream` (a cudaStream_t; NULL = legacy stream).
+ *  - Argument errors are detected on the host before anything is enqueued and returned
+ *    synchronously.  Launch errors return MOE_ERR_CUDA.  Faults detected inside kernels
+ *    (a bounded wait that ran out, an index out of range) set bits in a status word in the
+ *    workspace; moe_workspace_status() synchronises the stream, reads and clears it.
+ *  - T = 0 is a valid no-op.  Requirements: 1 <= n <= 64, 1 <= K <= n, d and F multiples
+ *    of 64 on the bf16 path and of 8 on the fp32 path; otherwise MOE_ERR_UNSUPPORTED.
+ *  - out must not alias x.  Calls sharing one workspace must not overlap on the GPU.
+ *  - Thread safety: no mutable global state; concurrent calls need separate workspaces.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2, /* shape outside the supported set (see above) */
+  MOE_ERR_WORKSPACE = 3,   /* workspace smaller than moe_workspace_bytes() */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  MOE_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out (reported by status calls) */
+  MOE_ERR_DEVICE = 6       /* a kernel detected an out-of-range index (status calls) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Bytes of device workspace moe_forward / moe_forward_debug need for this shape
+ * (0 if the shape is unsupported).  moe_stack_forward needs moe_stack_workspace_bytes(). */
+MOE_API size_t moe_workspace_bytes(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt);
+
+/* Zero the workspace's status word and counters; call once after allocating it. */
+MOE_API moe_status moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, then read and clear the workspace status word written by kernels.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded wait ran out), MOE_ERR_DEVICE (an index out
+ * of range) or MOE_ERR_CUDA (the stream reported an error).  *raw (may be NULL) receives
+ * the raw bit mask. */
+MOE_API moe_status moe_workspace_status(void* workspace, void* stream, uint32_t* raw);
+
+/* One MoE block forward:  out[t] = sum_k G(x_t)_k * SwiGLU_{e_k}(x_t).
+ *   x    [T][d]   dt           token activations
+ *   W_g  [d][n]   fp32         router weight
+ *   W1   [n][F][d] dt          gate projection of each expert
+ *   W3   [n][F][d] dt          up projection of each expert
+ *   W2   [n][d][F] dt          down projection of each expert
+ *   out  [T][d]   dt           result (written, never read)
+ * Device pointers; x/W1/W3/W2/out 16-byte aligned, workspace 256-byte aligned. */
+MOE_API moe_status moe_forward(const void* x, const float* W_g, const void* W1, const void* W3,
+                       const void* W2, int64_t T, int64_t d, int64_t F, int n, int K,
+                       moe_dtype dt, void* out, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* moe_forward, then copies of the routing state into caller buffers (each may be NULL):
+ *   topk_idx [T][K] int32      selected experts, slot 0 = larger logit
+ *   topk_gate [T][K] fp32      G(x) over the kept experts (rows sum to 1)
+ *   expert_counts [n] int32    tokens routed to each expert
+ *   expert_offsets [n+1] int32 first row of each expert's group in the permuted layout
+ *   token_rows [T][K] int32    permuted row of each (token, slot)
+ * Enqueued on `stream` like moe_forward (no synchronisation). */
+MOE_API moe_status moe_forward_debug(const void* x, const float* W_g, const void* W1, const void* W3,
+                             const void* W2, int64_t T, int64_t d, int64_t F, int n, int K,
+                             moe_dtype dt, void* out, void* workspace, size_t workspace_bytes,
+                             void* stream, int32_t* topk_idx, float* topk_gate,
+                             int32_t* expert_counts, int32_t* expert_offsets,
+                             int32_t* token_rows);
+
+/* moe_forward with HOST input and output: copies x_host (pinned recommended) to x_dev,
+ * runs the block into out_dev and copies it back to out_host, all on `stream`; returns
+ * after enqueueing (synchronise the stream before reading out_host).  x_dev and out_dev
+ * are caller-owned device buffers of T*d elements. */
+MOE_API moe_status moe_forward_host_io(const void* x_host, void* x_dev, const float* W_g,
+                               const void* W1, const void* W3, const void* W2, int64_t T,
+                               int64_t d, int64_t F, int n, int K, moe_dtype dt,
+                               void* out_dev, void* out_host, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* moe_forward that also records caller-created CUDA events (cudaEvent_t, passed as void*)
+ * on `stream` at the stage boundaries, for timing each kernel live:
+ *   events[0] before routing            events[1] after router, scan and permute
+ *   events[2] after the gate/up GEMM    events[3] after the split-K reduction (== [2] when
+ *                                                  the small-batch tiling is not used)
+ *   events[4] after the down GEMM       events[5] after the combine
+ * n_events must be 6.  Otherwise identical to moe_forward. */
+MOE_API moe_status moe_forward_profiled(const void* x, const float* W_g, const void* W1,
+                                        const void* W3, const void* W2, int64_t T, int64_t d,
+                                        int64_t F, int n, int K, moe_dtype dt, void* out,
+                                        void* workspace, size_t workspace_bytes, void* stream,
+                                        void* const* events, int n_events);
+
+/* Work plan chosen for a shape (for reports): *small_batch = 1 if the weights are the MMA's
+ * 128-row operand (small token counts), 0 otherwise; *split13 / *split2 = K-splits of the
+ * two expert GEMMs on that path (1 otherwise); *launches = kernels one forward launches. */
+MOE_API moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt,
+                                 int* small_batch, int* split13, int* split2, int* launches);
+
+/* Stack of L blocks on a residual stream (attention omitted), in place on x [T][d]:
+ *   for l in 0..L-1:  x <- round(x + MoE_l(RMSNorm(x)))
+ * RMSNorm has unit gain: x / sqrt(mean(x^2) + eps), rounded to dt; the residual sum is
+ * taken in fp32 and rounded once.  W_g, W1, W3, W2 are HOST arrays of L device pointers
+ * (per-layer weights, layouts as above).  Only the bf16 path is supported. */
+MOE_API size_t moe_stack_workspace_bytes(int64_t T, int64_t d, int64_t F, int n, int K,
+                                 moe_dtype dt);
+MOE_API moe_status moe_stack_forward(void* x, const float* const* W_g, const void* const* W1,
+                             const void* const* W3, const void* const* W2, int L, int64_t T,
+                             int64_t d, int64_t F, int n, int K, moe_dtype dt, float eps,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Short description of a status code (static string). */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Library ABI version (increases when an entry point changes). */
+MOE_API int moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

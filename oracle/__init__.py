@@ -42,6 +42,8 @@ def lib():
         P, I64, I32, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
         L.oracle_round_bf16.restype = D
         L.oracle_round_bf16.argtypes = [D]
+        L.oracle_round_array.restype = None
+        L.oracle_round_array.argtypes = [P, I64, I32]
         L.oracle_silu.restype = D
         L.oracle_silu.argtypes = [D]
         L.oracle_route.restype = I32
@@ -100,6 +102,13 @@ def _wg(Wg):
 
 def round_bf16(v: float) -> float:
     return lib().oracle_round_bf16(float(v))
+
+
+def round_array(v: np.ndarray, dtype: int) -> np.ndarray:
+    """Copy of v (float64) rounded element-wise to bf16 (dtype=BF16) or fp32 (dtype=F32)."""
+    out = np.ascontiguousarray(v, np.float64).copy()
+    lib().oracle_round_array(_ptr(out), out.size, int(dtype))
+    return out
 
 
 def silu(z: float) -> float:

@@ -73,6 +73,12 @@ double oracle_round_bf16(double v) {
 
 double oracle_round_f32(double v) { return (double)(float)v; }
 
+/* In-place rounding of an array to dtype (the contract's single output rounding). */
+void oracle_round_array(double* v, int64_t count, int dtype) {
+  for (int64_t i = 0; i < count; ++i)
+    v[i] = dtype == ORACLE_BF16 ? oracle_round_bf16(v[i]) : oracle_round_f32(v[i]);
+}
+
 static double round_to(double v, int dtype) {
   return dtype == ORACLE_BF16 ? oracle_round_bf16(v) : oracle_round_f32(v);
 }

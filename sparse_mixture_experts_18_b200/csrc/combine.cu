@@ -1,0 +1,152 @@
+// combine.cu -- gate-weighted combine back to token order and the RMSNorm of the stacked
+// blocks.
+//
+//  combine:  out[t] = sum_k G(x_t)_k * y_{e_k}(x_t)  ("Mixtral of Experts", method section,
+//            equation y; expert outputs return to their token's original position, as the
+//            Indonesian news summary's expert-parallelism notes put it).  fp32 sum over the
+//            K slots in slot order (and over split slabs in split order), rounded once;
+//            16-byte vectorised loads and stores.  With a residual input, out = resid + sum,
+//            also in fp32 before the single rounding (the stacked-block workload).
+//  rmsnorm:  xn = x / sqrt(mean(x^2) + eps) with unit gain, fp32 math, bf16 result.
+#include "internal.h"
+
+namespace moe {
+
+template <typename Tout>
+struct Out8;
+
+template <>
+struct Out8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 r = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = bf16_lo(w[i]);
+      v[2 * i + 1] = bf16_hi(w[i]);
+    }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+};
+
+template <>
+struct Out8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    const float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[8]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+  }
+};
+
+template <typename Tout, bool RESID>
+__global__ void __launch_bounds__(256)
+    combine_kernel(const float* __restrict__ Y, int S, int64_t split_stride, int64_t T, int d,
+                   int K, const int32_t* __restrict__ inv, const float* __restrict__ gate,
+                   Tout* out, const Tout* resid) {
+  const int vpr = d / 8;
+  const int64_t total = T * vpr;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
+       v += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = v / vpr;
+    const int c = (int)(v % vpr) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < K; ++k) {
+      const int row = inv[t * K + k];
+      if (row < 0) continue;
+      const float g = gate[t * K + k];
+      float yk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < S; ++s) {
+        const float* src = Y + s * split_stride + (int64_t)row * d + c;
+        const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+        yk[0] += a.x; yk[1] += a.y; yk[2] += a.z; yk[3] += a.w;
+        yk[4] += b.x; yk[5] += b.y; yk[6] += b.z; yk[7] += b.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, yk[i], acc[i]);
+    }
+    if (RESID) {
+      float r[8];
+      Out8<Tout>::load(resid + t * d + c, r);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = r[i] + acc[i];
+    }
+    Out8<Tout>::store(out + t * d + c, acc);
+  }
+}
+
+cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
+                           cudaStream_t s) {
+  const int S = p.swap ? p.s2 : 1;
+  const int64_t split_stride = p.rows_max * p.d;
+  const int64_t total = p.T * (p.d / 8);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
+  if (blocks < 1) blocks = 1;
+  if (p.dt == 1) {
+    auto* o = static_cast<__nv_bfloat16*>(out);
+    if (resid)
+      combine_kernel<__nv_bfloat16, true><<<(unsigned)blocks, 256, 0, s>>>(
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
+          static_cast<const __nv_bfloat16*>(resid));
+    else
+      combine_kernel<__nv_bfloat16, false><<<(unsigned)blocks, 256, 0, s>>>(
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
+  } else {
+    auto* o = static_cast<float*>(out);
+    if (resid)
+      combine_kernel<float, true><<<(unsigned)blocks, 256, 0, s>>>(
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
+          static_cast<const float*>(resid));
+    else
+      combine_kernel<float, false><<<(unsigned)blocks, 256, 0, s>>>(
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
+  }
+  return cudaGetLastError();
+}
+
+// One warp per row: sum of squares in fp32 (lane-strided 8-element chunks, then a shuffle
+// tree), then x / sqrt(mean + eps) rounded to bf16.
+__global__ void __launch_bounds__(256)
+    rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ xn,
+                   int64_t T, int d, float eps) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= T) return;
+  const __nv_bfloat16* xr = x + row * d;
+  float ss = 0.f;
+  for (int c = lane * 8; c < d; c += 256) {
+    float v[8];
+    Out8<__nv_bfloat16>::load(xr + c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(v[i], v[i], ss);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  for (int c = lane * 8; c < d; c += 256) {
+    float v[8];
+    Out8<__nv_bfloat16>::load(xr + c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= inv;
+    Out8<__nv_bfloat16>::store(xn + row * d + c, v);
+  }
+}
+
+cudaError_t launch_rmsnorm(const void* x, void* xn, int64_t T, int64_t d, float eps,
+                           cudaStream_t s) {
+  const unsigned blocks = (unsigned)((T + 7) / 8);
+  rmsnorm_kernel<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
+                                        static_cast<__nv_bfloat16*>(xn), T, (int)d, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,535 @@
+// gemm_tc.cu -- grouped expert GEMMs on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Each expert is a SwiGLU FFN of intermediate width F ("Mixtral of Experts", method
+// section: n = 8 experts of width 14336 on hidden size 4096; glossary: Swish combined with
+// an element-wise product):
+//   G13:  h = silu(X_e . W1_e^T) * (X_e . W3_e^T)      rounded to bf16
+//   G2:   Y = h_e . W2_e^T                              kept in fp32
+// where X_e are the rows routed to expert e (grouped by the permute kernel).
+//
+// One persistent kernel per GEMM, one CTA per SM, 6 warps:
+//   warp 0      TMA producer (one thread) filling a ring of shared-memory stages,
+//   warp 1      owns the TMEM allocation; one thread issues tcgen05.mma,
+//   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulator, SwiGLU / store.
+// Accumulators are double-buffered in TMEM so the epilogue of one tile overlaps the MMAs
+// of the next.  All waits are bounded (see common.cuh).
+//
+// Two tilings:
+//   prefill (!SWAP): tile = 128 permuted rows x (G13: 128 columns of W1 and the same 128 of
+//     W3, stacked into one N = 256 MMA operand | G2: 256 columns of W2), full K per tile.
+//   small batch (SWAP): the weights are the 128-row MMA operand and the expert's tokens the
+//     N dimension (16..256), K split into `splits` ranges so that every SM streams weights;
+//     fp32 partial sums go to per-split slabs reduced in a fixed order afterwards.
+#include <stdio.h>
+
+#include "internal.h"
+
+namespace moe {
+
+enum { KIND_G13 = 0, KIND_G2 = 1 };
+constexpr int MAX_STAGES = 16;
+constexpr int GEMM_THREADS = 192;
+constexpr uint32_t TILE_BYTES = 128 * 128;  // 128 rows x 64 bf16 (one 128-byte row each)
+
+struct TcArgs {
+  const int32_t* offsets;  // [n+1] first permuted row of each expert
+  int n;
+  int num_kb;              // 64-wide K blocks per work unit
+  int nw;                  // weight rows (output features) per expert: F (G13) or d (G2)
+  int n_tiles;             // prefill: column tiles per 128-row tile
+  int wb;                  // small batch: 128-row weight blocks per expert
+  int splits;              // small batch: K ranges
+  int tok_tile;            // small batch: MMA N
+  int stages;
+  uint32_t stage_bytes;    // shared-memory bytes per stage (1024-aligned)
+  uint32_t tx_bytes;       // bytes the TMA loads of one stage deliver
+  uint32_t x_off;          // offset of the activation tile inside a stage
+  uint32_t acc_cols, nacc, tmem_cols;
+  void* out;
+  int64_t out_ld;          // elements per output row
+  int64_t split_stride;    // elements between split slabs
+  uint32_t* status;
+};
+
+struct Ctrl {
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t mma_done;
+  uint32_t issued[MAX_STAGES];
+  uint32_t tmem_slot;
+  int abort;
+  int nact;
+  int off[MAX_EXPERTS + 1];
+  int act[MAX_EXPERTS];
+};
+
+struct Work {
+  int e, mt, nt, wblk, s, row0, count;
+};
+
+template <bool SWAP>
+__device__ __forceinline__ int total_work(const TcArgs& a, const Ctrl* c) {
+  if (SWAP) return c->nact * a.wb * a.splits;
+  return (c->off[a.n] / TILE_M) * a.n_tiles;
+}
+
+// Prefill order: expert-major, then column tile, then row tile (consecutive CTAs share the
+// weight tile through L2).  Small-batch order: active expert, weight block, split.
+template <bool SWAP>
+__device__ __forceinline__ Work decode_work(const TcArgs& a, const Ctrl* c, int id) {
+  Work w{};
+  if (SWAP) {
+    const int per = a.wb * a.splits;
+    const int ai = id / per, rem = id % per;
+    w.e = c->act[ai];
+    w.wblk = rem / a.splits;
+    w.s = rem % a.splits;
+    w.row0 = c->off[w.e];
+    w.count = c->off[w.e + 1] - c->off[w.e];
+  } else {
+    int e = 0;
+    while (e + 1 < a.n && id >= (c->off[e + 1] / TILE_M) * a.n_tiles) ++e;
+    const int mt0 = c->off[e] / TILE_M;
+    const int mcnt = c->off[e + 1] / TILE_M - mt0;
+    const int local = id - mt0 * a.n_tiles;
+    w.e = e;
+    w.nt = local / mcnt;
+    w.mt = mt0 + local % mcnt;
+    w.row0 = w.mt * TILE_M;
+  }
+  return w;
+}
+
+__device__ __forceinline__ bool wait_short(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > (WAIT_LIMIT_CYCLES >> 4)) return false;
+  return true;
+}
+
+template <int KIND, bool SWAP>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
+                           const __grid_constant__ CUtensorMap tmW0,
+                           const __grid_constant__ CUtensorMap tmW1, const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  Ctrl* c = reinterpret_cast<Ctrl*>(smem + (size_t)a.stages * a.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&c->full[s], 1);
+      mbar_init(&c->empty[s], 1);
+      c->issued[s] = 0;
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&c->tfull[i], 1);
+      mbar_init(&c->tempty[i], 128);
+    }
+    mbar_init(&c->mma_done, 1);
+    c->abort = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW0);
+    if (KIND == KIND_G13) tma_prefetch_desc(&tmW1);
+  }
+  if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(&c->tmem_slot, a.tmem_cols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int na = 0;
+    for (int e = 0; e < a.n; ++e)
+      if (c->off[e + 1] > c->off[e]) c->act[na++] = e;
+    c->nact = na;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = c->tmem_slot;
+  const int total = total_work<SWAP>(a, c);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = SWAP ? policy_evict_first() : policy_evict_normal();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int id = blockIdx.x; id < total; id += gridDim.x) {
+        const Work w = decode_work<SWAP>(a, c, id);
+        bool ok = true;
+        for (int kb = 0; kb < a.num_kb; ++kb) {
+          if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort)) { ok = false; break; }
+          uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+          uint64_t* fb = &c->full[stage];
+          mbar_arrive_expect_tx(fb, a.tx_bytes);
+          const int k = (SWAP ? w.s * a.num_kb + kb : kb) * 64;
+          if (!SWAP) {
+            tma_load_2d(st, &tmX, fb, k, w.mt * TILE_M, pol_x);
+            if (KIND == KIND_G13) {
+              const int wr = w.e * a.nw + w.nt * 128;
+              tma_load_2d(st + TILE_BYTES, &tmW0, fb, k, wr, pol_w);
+              tma_load_2d(st + 2 * TILE_BYTES, &tmW1, fb, k, wr, pol_w);
+            } else {
+              tma_load_2d(st + TILE_BYTES, &tmW0, fb, k, w.e * a.nw + w.nt * 256, pol_w);
+            }
+          } else {
+            const int wr = w.e * a.nw + w.wblk * 128;
+            tma_load_2d(st, &tmW0, fb, k, wr, pol_w);
+            if (KIND == KIND_G13) tma_load_2d(st + TILE_BYTES, &tmW1, fb, k, wr, pol_w);
+            tma_load_2d(st + a.x_off, &tmX, fb, k, w.row0, pol_x);
+          }
+          c->issued[stage] += 1;
+          if (++stage == a.stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      if (c->abort) {  // let every issued copy land before the CTA's shared memory goes away
+        for (int s = 0; s < a.stages; ++s)
+          if (c->issued[s]) wait_short(&c->full[s], (c->issued[s] - 1u) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(128, SWAP ? a.tok_tile : 256);
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++it) {
+        const uint32_t acc = (uint32_t)it % a.nacc;
+        const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
+        if (!mbar_wait(&c->tempty[acc], aph ^ 1u, a.status, &c->abort)) break;
+        tc_fence_after();
+        const uint32_t dtm = tmem_base + acc * a.acc_cols;
+        for (int kb = 0; kb < a.num_kb; ++kb) {
+          if (!mbar_wait(&c->full[stage], phase, a.status, &c->abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(smem + (size_t)stage * a.stage_bytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t kofs = kk * 32;  // 16 bf16 along K inside the 128-byte row
+            const uint32_t accum = (kb | kk) != 0;
+            if (!SWAP) {
+              umma_bf16(dtm, umma_desc_k128(sb + kofs), umma_desc_k128(sb + TILE_BYTES + kofs),
+                        idesc, accum);
+            } else {
+              const uint64_t bd = umma_desc_k128(sb + a.x_off + kofs);
+              umma_bf16(dtm, umma_desc_k128(sb + kofs), bd, idesc, accum);
+              if (KIND == KIND_G13)
+                umma_bf16(dtm + a.tok_tile, umma_desc_k128(sb + TILE_BYTES + kofs), bd, idesc,
+                          accum);
+            }
+          }
+          umma_commit(&c->empty[stage]);  // frees the stage once these MMAs have read it
+          if (++stage == a.stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&c->tfull[acc]);  // accumulator complete
+      }
+      if (c->abort) {
+        umma_commit(&c->mma_done);
+        wait_short(&c->mma_done, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;
+    int it = 0;
+    for (int id = blockIdx.x; id < total; id += gridDim.x, ++it) {
+      const Work w = decode_work<SWAP>(a, c, id);
+      const uint32_t acc = (uint32_t)it % a.nacc;
+      const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
+      const bool ok = mbar_wait(&c->tfull[acc], aph, a.status, &c->abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * a.acc_cols;
+      if (!SWAP && KIND == KIND_G13) {
+        __nv_bfloat16* h = static_cast<__nv_bfloat16*>(a.out) + (int64_t)(w.row0 + r) * a.out_ld;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tb + cc * 32, va);
+          tmem_ld32(tb + 128 + cc * 32, vb);
+          tmem_ld_wait();
+          const int col = w.nt * 128 + cc * 32;
+          if (col < a.nw) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu(__uint_as_float(va[2 * i])) * __uint_as_float(vb[2 * i]);
+              const float h1 =
+                  silu(__uint_as_float(va[2 * i + 1])) * __uint_as_float(vb[2 * i + 1]);
+              pk[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(h + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else if (!SWAP && KIND == KIND_G2) {
+        float* y = static_cast<float*>(a.out) + (int64_t)(w.row0 + r) * a.out_ld;
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tb + cc * 32, v);
+          tmem_ld_wait();
+          const int col = w.nt * 256 + cc * 32;
+          if (col < a.nw) {
+            float4* dst = reinterpret_cast<float4*>(y + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+        }
+      } else {
+        // small batch: accumulator row = weight row, column = token of this expert
+        float* p = static_cast<float*>(a.out) + (int64_t)w.s * a.split_stride;
+        const int f = w.wblk * 128 + r;
+        const bool frow = f < a.nw;
+#pragma unroll 1
+        for (int cc = 0; cc < a.tok_tile / 16; ++cc) {
+          uint32_t v1[16], v3[16];
+          tmem_ld16(tb + cc * 16, v1);
+          if (KIND == KIND_G13) tmem_ld16(tb + a.tok_tile + cc * 16, v3);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = cc * 16 + jj;
+            if (frow && j < w.count) {
+              float* rowp = p + (int64_t)(w.row0 + j) * a.out_ld;
+              rowp[f] = __uint_as_float(v1[jj]);
+              if (KIND == KIND_G13) rowp[a.nw + f] = __uint_as_float(v3[jj]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&c->tempty[acc]);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, a.tmem_cols);
+}
+
+// Small batch: h = bf16(silu(sum_s A_s) * sum_s B_s), splits summed in order 0..S-1.
+__global__ void __launch_bounds__(256)
+    swiglu_reduce_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
+                         int64_t rows, int F, __nv_bfloat16* __restrict__ h) {
+  const int vpr = F / 4;
+  const int64_t total = rows * vpr;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
+       v += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = v / vpr;
+    const int c = (int)(v % vpr) * 4;
+    const float* pa = p13 + r * 2 * F + c;
+    float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
+    for (int s = 0; s < S; ++s) {
+      const float4 ta = *reinterpret_cast<const float4*>(pa + s * split_stride);
+      const float4 tb = *reinterpret_cast<const float4*>(pa + s * split_stride + F);
+      sa.x += ta.x; sa.y += ta.y; sa.z += ta.z; sa.w += ta.w;
+      sb.x += tb.x; sb.y += tb.y; sb.z += tb.z; sb.w += tb.w;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(silu(sa.x) * sb.x, silu(sa.y) * sb.y);
+    o.y = pack_bf16x2(silu(sa.z) * sb.z, silu(sa.w) * sb.w);
+    *reinterpret_cast<uint2*>(h + r * F + c) = o;
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [outer][inner] (row-major), box = box_rows x 64 elements, 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                     uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr uint32_t SMEM_STAGE_BUDGET = 200 * 1024;
+
+template <int KIND, bool SWAP>
+static cudaError_t launch_one(const CUtensorMap& mx, const CUtensorMap& mw0,
+                              const CUtensorMap& mw1, TcArgs a, int max_work, cudaStream_t s) {
+  const size_t smem = (size_t)a.stages * a.stage_bytes + sizeof(Ctrl) + 1024;
+  auto kern = tc_grouped_gemm_kernel<KIND, SWAP>;
+  static int configured = 0;
+  if (configured < (int)smem) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = (int)smem;
+  }
+  const int grid = max_work < num_sms() ? (max_work > 0 ? max_work : 1) : num_sms();
+  kern<<<grid, GEMM_THREADS, smem, s>>>(mx, mw0, mw1, a);
+  return cudaGetLastError();
+}
+
+static int stages_for(uint32_t stage_bytes) {
+  int st = (int)(SMEM_STAGE_BUDGET / stage_bytes);
+  return st > MAX_STAGES ? MAX_STAGES : st;
+}
+
+static uint32_t pow2_cols(uint32_t c) {
+  uint32_t p = 32;
+  while (p < c) p <<= 1;
+  return p;
+}
+
+static cudaError_t record(cudaEvent_t const* ev, int i, cudaStream_t s) {
+  return ev ? cudaEventRecord(ev[i], s) : cudaSuccess;
+}
+
+cudaError_t launch_expert_gemms_tc(const Plan& p, const void* W1, const void* W3,
+                                   const void* W2, const Workspace& w, cudaStream_t s,
+                                   cudaEvent_t const* ev) {
+  CUtensorMap mX, mW1, mW3, mH, mW2;
+  const int d = (int)p.d, F = (int)p.F, n = p.n;
+  cudaError_t err;
+  if (!p.swap) {
+    if (!make_map(&mX, w.xperm, d, p.rows_max, 128) ||
+        !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||
+        !make_map(&mW3, W3, d, (uint64_t)n * F, 128) ||
+        !make_map(&mH, w.h, F, p.rows_max, 128) ||
+        !make_map(&mW2, W2, F, (uint64_t)n * d, 256))
+      return cudaErrorInvalidValue;
+    const int m_tiles_max = (int)(p.rows_max / TILE_M);
+    TcArgs a{};
+    a.offsets = w.offsets;
+    a.n = n;
+    a.stage_bytes = 3 * TILE_BYTES;
+    a.tx_bytes = 3 * TILE_BYTES;
+    a.stages = stages_for(a.stage_bytes);
+    a.acc_cols = 256;
+    a.nacc = 2;
+    a.tmem_cols = 512;
+    a.status = w.status;
+    // G13
+    a.num_kb = d / 64;
+    a.nw = F;
+    a.n_tiles = (F + 127) / 128;
+    a.out = w.h;
+    a.out_ld = F;
+    if ((err = launch_one<KIND_G13, false>(mX, mW1, mW3, a, m_tiles_max * a.n_tiles, s)) !=
+        cudaSuccess)
+      return err;
+    if ((err = record(ev, 0, s)) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
+      return err;
+    // G2
+    a.num_kb = F / 64;
+    a.nw = d;
+    a.n_tiles = (d + 255) / 256;
+    a.out = w.y;
+    a.out_ld = d;
+    if ((err = launch_one<KIND_G2, false>(mH, mW2, mW2, a, m_tiles_max * a.n_tiles, s)) !=
+        cudaSuccess)
+      return err;
+    return record(ev, 2, s);
+  }
+  // small batch
+  const int tok = p.tok_tile;
+  const uint32_t xbytes = (uint32_t)tok * 128;
+  const uint32_t xslot = (xbytes + 1023u) & ~1023u;
+  if (!make_map(&mX, w.xperm, d, p.rows_max, tok) ||
+      !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||
+      !make_map(&mW3, W3, d, (uint64_t)n * F, 128) || !make_map(&mH, w.h, F, p.rows_max, tok) ||
+      !make_map(&mW2, W2, F, (uint64_t)n * d, 128))
+    return cudaErrorInvalidValue;
+  TcArgs a{};
+  a.offsets = w.offsets;
+  a.n = n;
+  a.tok_tile = tok;
+  a.status = w.status;
+  // G13: partial sums of x.W1 and x.W3 per split
+  a.splits = p.s13;
+  a.num_kb = d / 64 / p.s13;
+  a.nw = F;
+  a.wb = (F + 127) / 128;
+  a.x_off = 2 * TILE_BYTES;
+  a.stage_bytes = 2 * TILE_BYTES + xslot;
+  a.tx_bytes = 2 * TILE_BYTES + xbytes;
+  a.stages = stages_for(a.stage_bytes);
+  a.acc_cols = 2 * tok;
+  a.nacc = 2 * a.acc_cols <= 512 ? 2 : 1;
+  a.tmem_cols = pow2_cols(a.nacc * a.acc_cols);
+  a.out = w.p13;
+  a.out_ld = 2 * (int64_t)F;
+  a.split_stride = p.rows_max * 2 * (int64_t)F;
+  if ((err = launch_one<KIND_G13, true>(mX, mW1, mW3, a, n * a.wb * a.splits, s)) !=
+      cudaSuccess)
+    return err;
+  if ((err = record(ev, 0, s)) != cudaSuccess) return err;
+  const int64_t rows = p.T * p.K;
+  const int64_t vec = rows * F / 4;
+  const int rgrid = (int)((vec + 255) / 256 < 4 * num_sms() ? (vec + 255) / 256 : 4 * num_sms());
+  swiglu_reduce_kernel<<<rgrid > 0 ? rgrid : 1, 256, 0, s>>>(
+      w.p13, p.s13, a.split_stride, rows, F, static_cast<__nv_bfloat16*>(w.h));
+  if ((err = cudaGetLastError()) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
+    return err;
+  // G2: per-split partial sums of h.W2
+  a.splits = p.s2;
+  a.num_kb = F / 64 / p.s2;
+  a.nw = d;
+  a.wb = (d + 127) / 128;
+  a.x_off = TILE_BYTES;
+  a.stage_bytes = TILE_BYTES + xslot;
+  a.tx_bytes = TILE_BYTES + xbytes;
+  a.stages = stages_for(a.stage_bytes);
+  a.acc_cols = tok;
+  a.nacc = 2 * a.acc_cols <= 512 ? 2 : 1;
+  a.tmem_cols = pow2_cols(a.nacc * a.acc_cols);
+  a.out = w.y;
+  a.out_ld = d;
+  a.split_stride = p.rows_max * (int64_t)d;
+  if ((err = launch_one<KIND_G2, true>(mH, mW2, mW2, a, n * a.wb * a.splits, s)) !=
+      cudaSuccess)
+    return err;
+  return record(ev, 2, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,66 @@
+// internal.h -- host-side plan, workspace carving and kernel launchers shared by the
+// library's translation units.  Not part of the public ABI (see include/moe.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int TILE_M = 128;       // rows of one tensor-core accumulator tile
+constexpr int SIMT_TILE = 64;     // rows of one fp32 SIMT tile
+constexpr int MAX_EXPERTS = 64;
+
+// Everything about a forward call that depends only on its shape.
+struct Plan {
+  int64_t T = 0, d = 0, F = 0;
+  int n = 0, K = 0;
+  int dt = 1;              // 0 = fp32 (SIMT path), 1 = bf16 (tensor-core path)
+  bool swap = false;       // small-batch path: weights are the MMA's 128-row operand
+  int row_align = 1;       // each expert's group is padded to a multiple of this
+  int64_t rows_max = 0;    // upper bound of permuted rows (T*K plus padding)
+  int64_t nblk = 0;        // router / permute blocks
+  int tok_tile = 0;        // swap: MMA N (tokens per expert tile), multiple of 16
+  int s13 = 1, s2 = 1;     // swap: split-K factors of the two expert GEMMs
+  bool stack = false;      // workspace also holds the normalised activations
+  // workspace byte offsets
+  size_t o_status, o_idx, o_gate, o_blk_counts, o_blk_base, o_counts, o_offsets, o_inv,
+      o_xperm, o_h, o_y, o_p13, o_xn, total;
+};
+
+// Device pointers into the workspace.
+struct Workspace {
+  uint32_t* status;
+  int32_t *idx, *blk_counts, *blk_base, *counts, *offsets, *inv;
+  float* gate;
+  void* xperm;  // [rows_max][d] activations in permuted order
+  void* h;      // [rows_max][F] silu(a) * b (bf16 on the tensor-core path, fp32 on SIMT)
+  float* y;     // [s2][rows_max][d] expert outputs (per split on the swap path)
+  float* p13;   // swap: [s13][rows_max][2F] split-K partial sums of x.W1 | x.W3
+  void* xn;     // stack: normalised activations [T][d]
+};
+
+bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p);
+Workspace carve(const Plan& p, void* base);
+
+int route_tokens_per_block(int n);
+cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Workspace& w,
+                         cudaStream_t s);
+// ev (may be null): events recorded after G13, after the split-K reduction, after G2.
+cudaError_t launch_expert_gemms_tc(const Plan& p, const void* W1, const void* W3,
+                                   const void* W2, const Workspace& w, cudaStream_t s,
+                                   cudaEvent_t const* ev = nullptr);
+cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float* W3,
+                                     const float* W2, const Workspace& w, cudaStream_t s,
+                                     cudaEvent_t const* ev = nullptr);
+cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
+                           cudaStream_t s);
+cudaError_t launch_rmsnorm(const void* x, void* xn, int64_t T, int64_t d, float eps,
+                           cudaStream_t s);
+int num_sms();
+
+}  // namespace moe

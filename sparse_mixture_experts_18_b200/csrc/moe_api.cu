@@ -1,0 +1,324 @@
+// moe_api.cu -- the C ABI of libmoe.so (declared in include/moe.h): argument validation,
+// the per-shape plan, workspace carving, and the kernel sequence of one MoE block forward:
+//   router + TopK + softmax  ->  histogram scan  ->  permute / gather
+//   ->  expert GEMMs (tensor cores for bf16, CUDA cores for fp32)  ->  gated combine.
+#include <string.h>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+namespace moe {
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cached[dev] = v;
+  }
+  return cached[dev];
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Smallest split of `num_kb` K-blocks (a divisor, at least 4 blocks per split, at most 16
+// splits) for which `units_per_split` * splits work units fill whole waves of the SMs to
+// within 5%; otherwise the best fill found.
+static int choose_split(int num_kb, int units_per_split, int sms) {
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 16; ++s) {
+    if (num_kb % s || num_kb / s < 4) continue;
+    const double u = (double)units_per_split * s;
+    const double waves = u / sms;
+    const double eff = waves / (double)((int64_t)((u + sms - 1) / sms));
+    if (eff >= 0.95) return s;
+    if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+  }
+  return best;
+}
+
+bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p) {
+  if (T < 0 || d <= 0 || F <= 0 || n < 1 || n > MAX_EXPERTS || K < 1 || K > n) return false;
+  if (dt == 1) {
+    if (d % 64 || F % 64) return false;
+  } else if (dt == 0) {
+    if (d % 8 || F % 8) return false;
+  } else {
+    return false;
+  }
+  if (d > (1 << 20) || F > (1 << 20) || T > (int64_t)1 << 26) return false;
+  Plan q;
+  q.T = T; q.d = d; q.F = F; q.n = n; q.K = K; q.dt = dt; q.stack = stack;
+  q.swap = dt == 1 && T <= 256 && T * K < 64 * (int64_t)n;
+  q.row_align = dt == 0 ? SIMT_TILE : (q.swap ? 1 : TILE_M);
+  const int64_t P = T * K;
+  q.rows_max = (P + (int64_t)n * (q.row_align - 1) + q.row_align - 1) / q.row_align * q.row_align;
+  if (q.swap) q.rows_max = (P + 15) / 16 * 16;  // >= tok_tile rows for the token TMA box
+  if (q.rows_max >= ((int64_t)1 << 31) / 2) return false;
+  const int tokb = route_tokens_per_block(n);
+  q.nblk = (T + tokb - 1) / tokb;
+  if (q.swap) {
+    q.tok_tile = (int)((T + 15) / 16 * 16);
+    const int sms = num_sms();
+    q.s13 = choose_split((int)(d / 64), n * (int)((F + 127) / 128), sms);
+    q.s2 = choose_split((int)(F / 64), n * (int)((d + 127) / 128), sms);
+  }
+  const size_t es = dt == 1 ? 2 : 4;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = align256(o + bytes); return at; };
+  q.o_status = take(256);
+  q.o_idx = take((size_t)P * 4);
+  q.o_gate = take((size_t)P * 4);
+  q.o_blk_counts = take((size_t)q.nblk * n * 4);
+  q.o_blk_base = take((size_t)q.nblk * n * 4);
+  q.o_counts = take((size_t)n * 4);
+  q.o_offsets = take((size_t)(n + 1) * 4);
+  q.o_inv = take((size_t)P * 4);
+  q.o_xperm = take((size_t)q.rows_max * d * es);
+  q.o_h = take((size_t)q.rows_max * F * es);
+  q.o_y = take((size_t)(q.swap ? q.s2 : 1) * q.rows_max * d * 4);
+  q.o_p13 = take(q.swap ? (size_t)q.s13 * q.rows_max * 2 * F * 4 : 0);
+  q.o_xn = take(stack ? (size_t)T * d * es : 0);
+  q.total = o;
+  *p = q;
+  return true;
+}
+
+Workspace carve(const Plan& p, void* base) {
+  uint8_t* b = static_cast<uint8_t*>(base);
+  Workspace w;
+  w.status = reinterpret_cast<uint32_t*>(b + p.o_status);
+  w.idx = reinterpret_cast<int32_t*>(b + p.o_idx);
+  w.gate = reinterpret_cast<float*>(b + p.o_gate);
+  w.blk_counts = reinterpret_cast<int32_t*>(b + p.o_blk_counts);
+  w.blk_base = reinterpret_cast<int32_t*>(b + p.o_blk_base);
+  w.counts = reinterpret_cast<int32_t*>(b + p.o_counts);
+  w.offsets = reinterpret_cast<int32_t*>(b + p.o_offsets);
+  w.inv = reinterpret_cast<int32_t*>(b + p.o_inv);
+  w.xperm = b + p.o_xperm;
+  w.h = b + p.o_h;
+  w.y = reinterpret_cast<float*>(b + p.o_y);
+  w.p13 = reinterpret_cast<float*>(b + p.o_p13);
+  w.xn = b + p.o_xn;
+  return w;
+}
+
+static bool aligned(const void* ptr, size_t a) {
+  return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0;
+}
+
+static moe_status check_common(const void* x, const float* W_g, const void* W1, const void* W3,
+                               const void* W2, const void* out, const void* ws) {
+  if (!x || !W_g || !W1 || !W3 || !W2 || !out || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(W_g, 16) || !aligned(W1, 16) || !aligned(W3, 16) ||
+      !aligned(W2, 16) || !aligned(out, 16) || !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+static moe_status shape_status(int64_t T, int64_t d, int64_t F, int n, int K, int dt) {
+  if (T < 0 || d <= 0 || F <= 0 || n < 1 || K < 1 || K > n) return MOE_ERR_INVALID_ARG;
+  if (dt != 0 && dt != 1) return MOE_ERR_INVALID_ARG;
+  return MOE_ERR_UNSUPPORTED;
+}
+
+// The kernel sequence of one block on already-validated arguments.
+// ev (may be null): six events recorded at the stage boundaries (see moe_forward_profiled).
+static moe_status forward_impl(const Plan& p, const void* x, const float* W_g, const void* W1,
+                               const void* W3, const void* W2, void* out, const void* resid,
+                               const Workspace& w, cudaStream_t s,
+                               cudaEvent_t const* ev = nullptr) {
+  if (ev && cudaEventRecord(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_route(p, x, W_g, w, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (ev && cudaEventRecord(ev[1], s) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t err =
+      p.dt == 1 ? launch_expert_gemms_tc(p, W1, W3, W2, w, s, ev ? ev + 2 : nullptr)
+                : launch_expert_gemms_simt(p, static_cast<const float*>(W1),
+                                           static_cast<const float*>(W3),
+                                           static_cast<const float*>(W2), w, s,
+                                           ev ? ev + 2 : nullptr);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_combine(p, w, out, resid, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (ev && cudaEventRecord(ev[5], s) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_abi_version(void) { return 1; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument (null, misaligned or bad size)";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+    case MOE_ERR_DEVICE: return "a kernel detected an out-of-range index";
+  }
+  return "unknown status";
+}
+
+size_t moe_workspace_bytes(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt) {
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, false, &p)) return 0;
+  return p.total;
+}
+
+size_t moe_stack_workspace_bytes(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt) {
+  Plan p;
+  if (dt != MOE_BF16 || !make_plan(T, d, F, n, K, (int)dt, true, &p)) return 0;
+  return p.total;
+}
+
+moe_status moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < 256 || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_status(void* workspace, void* stream, uint32_t* raw) {
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t bits = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&bits, workspace, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemset(workspace, 0, sizeof bits) != cudaSuccess) return MOE_ERR_CUDA;
+  if (raw) *raw = bits;
+  if (bits & DEV_ERR_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (bits) return MOE_ERR_DEVICE;
+  return MOE_OK;
+}
+
+moe_status moe_forward(const void* x, const float* W_g, const void* W1, const void* W3,
+                       const void* W2, int64_t T, int64_t d, int64_t F, int n, int K,
+                       moe_dtype dt, void* out, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, false, &p)) return shape_status(T, d, F, n, K, dt);
+  if (T == 0) return MOE_OK;
+  moe_status st = check_common(x, W_g, W1, W3, W2, out, workspace);
+  if (st != MOE_OK) return st;
+  if (out == x) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  const Workspace w = carve(p, workspace);
+  return forward_impl(p, x, W_g, W1, W3, W2, out, nullptr, w, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_profiled(const void* x, const float* W_g, const void* W1,
+                                const void* W3, const void* W2, int64_t T, int64_t d, int64_t F,
+                                int n, int K, moe_dtype dt, void* out, void* workspace,
+                                size_t workspace_bytes, void* stream, void* const* events,
+                                int n_events) {
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, false, &p)) return shape_status(T, d, F, n, K, dt);
+  if (!events || n_events != 6) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  moe_status st = check_common(x, W_g, W1, W3, W2, out, workspace);
+  if (st != MOE_OK) return st;
+  if (out == x) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  const Workspace w = carve(p, workspace);
+  cudaEvent_t ev[6];
+  for (int i = 0; i < 6; ++i) ev[i] = static_cast<cudaEvent_t>(events[i]);
+  return forward_impl(p, x, W_g, W1, W3, W2, out, nullptr, w, static_cast<cudaStream_t>(stream),
+                      ev);
+}
+
+moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt,
+                         int* small_batch, int* split13, int* split2, int* launches) {
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, false, &p)) return shape_status(T, d, F, n, K, dt);
+  if (small_batch) *small_batch = p.swap ? 1 : 0;
+  if (split13) *split13 = p.swap ? p.s13 : 1;
+  if (split2) *split2 = p.swap ? p.s2 : 1;
+  if (launches) *launches = T == 0 ? 0 : 3 + (p.swap ? 3 : 2) + 1;
+  return MOE_OK;
+}
+
+moe_status moe_forward_debug(const void* x, const float* W_g, const void* W1, const void* W3,
+                             const void* W2, int64_t T, int64_t d, int64_t F, int n, int K,
+                             moe_dtype dt, void* out, void* workspace, size_t workspace_bytes,
+                             void* stream, int32_t* topk_idx, float* topk_gate,
+                             int32_t* expert_counts, int32_t* expert_offsets,
+                             int32_t* token_rows) {
+  moe_status st = moe_forward(x, W_g, W1, W3, W2, T, d, F, n, K, dt, out, workspace,
+                              workspace_bytes, stream);
+  if (st != MOE_OK || T == 0) return st;
+  Plan p;
+  make_plan(T, d, F, n, K, (int)dt, false, &p);
+  const Workspace w = carve(p, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t tk = (size_t)T * K * 4;
+  struct { void* dst; const void* src; size_t bytes; } cp[5] = {
+      {topk_idx, w.idx, tk}, {topk_gate, w.gate, tk}, {expert_counts, w.counts, (size_t)n * 4},
+      {expert_offsets, w.offsets, (size_t)(n + 1) * 4}, {token_rows, w.inv, tk}};
+  for (auto& c : cp)
+    if (c.dst && cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_forward_host_io(const void* x_host, void* x_dev, const float* W_g,
+                               const void* W1, const void* W3, const void* W2, int64_t T,
+                               int64_t d, int64_t F, int n, int K, moe_dtype dt,
+                               void* out_dev, void* out_host, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, false, &p)) return shape_status(T, d, F, n, K, dt);
+  if (T == 0) return MOE_OK;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_common(x_dev, W_g, W1, W3, W2, out_dev, workspace);
+  if (st != MOE_OK) return st;
+  if (out_dev == x_dev) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)T * d * (dt == MOE_BF16 ? 2 : 4);
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const Workspace w = carve(p, workspace);
+  st = forward_impl(p, x_dev, W_g, W1, W3, W2, out_dev, nullptr, w, s);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_stack_forward(void* x, const float* const* W_g, const void* const* W1,
+                             const void* const* W3, const void* const* W2, int L, int64_t T,
+                             int64_t d, int64_t F, int n, int K, moe_dtype dt, float eps,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, true, &p)) return shape_status(T, d, F, n, K, dt);
+  if (L < 0 || !W_g || !W1 || !W3 || !W2 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (T == 0 || L == 0) return MOE_OK;
+  for (int l = 0; l < L; ++l) {
+    moe_status st = check_common(x, W_g[l], W1[l], W3[l], W2[l], x, workspace);
+    if (st != MOE_OK) return st;
+  }
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Workspace w = carve(p, workspace);
+  for (int l = 0; l < L; ++l) {
+    if (launch_rmsnorm(x, w.xn, T, d, eps, s) != cudaSuccess) return MOE_ERR_CUDA;
+    moe_status st = forward_impl(p, w.xn, W_g[l], W1[l], W3[l], W2[l], x, x, w, s);
+    if (st != MOE_OK) return st;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

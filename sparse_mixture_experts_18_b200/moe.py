@@ -1,0 +1,185 @@
+"""Thin ctypes binding of libmoe.so (declared in include/moe.h).
+
+Argument marshalling only: every step of the MoE block runs in the library's CUDA kernels.
+torch supplies device memory and streams.  There is no fallback: if the library is missing
+or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+          3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_DEVICE"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn}: {STATUS.get(code, code)} ({msg})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (built in-tree by sparse_mixture_experts_18_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m sparse_mixture_experts_18_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.moe_workspace_bytes.restype = SZ
+        L.moe_workspace_bytes.argtypes = [I64, I64, I64, I32, I32, I32]
+        L.moe_stack_workspace_bytes.restype = SZ
+        L.moe_stack_workspace_bytes.argtypes = [I64, I64, I64, I32, I32, I32]
+        L.moe_workspace_init.restype = I32
+        L.moe_workspace_init.argtypes = [P, SZ, P]
+        L.moe_workspace_status.restype = I32
+        L.moe_workspace_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+        L.moe_forward.restype = I32
+        L.moe_forward.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P, P, SZ, P]
+        L.moe_forward_debug.restype = I32
+        L.moe_forward_debug.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P, P, SZ, P,
+                                        P, P, P, P, P]
+        L.moe_forward_host_io.restype = I32
+        L.moe_forward_host_io.argtypes = [P, P, P, P, P, P, I64, I64, I64, I32, I32, I32, P, P, P,
+                                          SZ, P]
+        L.moe_stack_forward.restype = I32
+        L.moe_stack_forward.argtypes = [P, P, P, P, P, I32, I64, I64, I64, I32, I32, I32,
+                                        ctypes.c_float, P, SZ, P]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [I32]
+        L.moe_abi_version.restype = I32
+        L.moe_abi_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise MoeError(fn, code, lib().moe_status_string(code).decode())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def moe_workspace_bytes(T, d, F, n, K, dtype) -> int:
+    dt = MOE_BF16 if dtype in (torch.bfloat16, MOE_BF16) else MOE_F32
+    return int(lib().moe_workspace_bytes(T, d, F, n, K, dt))
+
+
+def moe_stack_workspace_bytes(T, d, F, n, K, dtype=torch.bfloat16) -> int:
+    dt = MOE_BF16 if dtype in (torch.bfloat16, MOE_BF16) else MOE_F32
+    return int(lib().moe_stack_workspace_bytes(T, d, F, n, K, dt))
+
+
+def alloc_workspace(nbytes: int, device=None, stream=None) -> torch.Tensor:
+    """Device buffer of nbytes (256-byte aligned by torch's allocator), initialised."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+    _check("moe_workspace_init", lib().moe_workspace_init(_ptr(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def moe_workspace_status(ws: torch.Tensor, stream=None) -> tuple[int, int]:
+    raw = ctypes.c_uint32(0)
+    code = lib().moe_workspace_status(_ptr(ws), _stream(stream), ctypes.byref(raw))
+    return code, raw.value
+
+
+def _dims(x, W1, W_g):
+    T, d = x.shape
+    n, F, d1 = W1.shape
+    if d1 != d or tuple(W_g.shape) != (d, n):
+        raise ValueError("shape mismatch between x, W_g and W1")
+    return T, d, F, n
+
+
+def moe_forward(x, W_g, W1, W3, W2, K: int, out=None, workspace=None, stream=None):
+    """out[t] = sum_k G(x_t)_k SwiGLU_{e_k}(x_t) on the GPU; returns out."""
+    T, d, F, n = _dims(x, W1, W_g)
+    dt = _dt(x)
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = alloc_workspace(moe_workspace_bytes(T, d, F, n, K, dt), x.device, stream)
+    _check("moe_forward", lib().moe_forward(
+        _ptr(x), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt, _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def moe_forward_debug(x, W_g, W1, W3, W2, K: int, out=None, workspace=None, stream=None):
+    """moe_forward plus the routing state: (out, topk_idx, topk_gate, expert_counts,
+    expert_offsets, token_rows)."""
+    T, d, F, n = _dims(x, W1, W_g)
+    dt = _dt(x)
+    dev = x.device
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = alloc_workspace(moe_workspace_bytes(T, d, F, n, K, dt), dev, stream)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    gate = torch.empty((T, K), dtype=torch.float32, device=dev)
+    counts = torch.empty((n,), dtype=torch.int32, device=dev)
+    offsets = torch.empty((n + 1,), dtype=torch.int32, device=dev)
+    rows = torch.empty((T, K), dtype=torch.int32, device=dev)
+    _check("moe_forward_debug", lib().moe_forward_debug(
+        _ptr(x), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt, _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream(stream), _ptr(idx), _ptr(gate),
+        _ptr(counts), _ptr(offsets), _ptr(rows)))
+    return out, idx, gate, counts, offsets, rows
+
+
+def moe_forward_host_io(x_host, x_dev, W_g, W1, W3, W2, K: int, out_dev, out_host, workspace,
+                        stream=None):
+    """Host x in, host out: H2D copy, forward, D2H copy, all enqueued on the stream."""
+    T, d, F, n = _dims(x_host, W1, W_g)
+    dt = _dt(x_host)
+    _check("moe_forward_host_io", lib().moe_forward_host_io(
+        _ptr(x_host), _ptr(x_dev), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt,
+        _ptr(out_dev), _ptr(out_host), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out_host
+
+
+def moe_stack_forward(x, layers, K: int, eps: float = 1e-5, workspace=None, stream=None):
+    """In place on x: for each layer dict (W_g, W1, W3, W2), x <- x + MoE(RMSNorm(x))."""
+    L = len(layers)
+    T, d = x.shape
+    n, F, _ = layers[0]["W1"].shape
+    dt = _dt(x)
+    if workspace is None:
+        workspace = alloc_workspace(moe_stack_workspace_bytes(T, d, F, n, K, dt), x.device,
+                                    stream)
+    arr = ctypes.c_void_p * max(L, 1)
+    pg = arr(*[l["Wg"].data_ptr() for l in layers])
+    p1 = arr(*[l["W1"].data_ptr() for l in layers])
+    p3 = arr(*[l["W3"].data_ptr() for l in layers])
+    p2 = arr(*[l["W2"].data_ptr() for l in layers])
+    _check("moe_stack_forward", lib().moe_stack_forward(
+        _ptr(x), pg, p1, p3, p2, L, T, d, F, n, K, dt, float(eps), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return x

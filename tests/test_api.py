@@ -1,0 +1,161 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point the header
+declares, sizes workspaces, and rejects bad arguments synchronously, before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_mixture_experts_18_b200 as moe
+from sparse_mixture_experts_18_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+BF16, F32 = 1, 0
+
+
+@pytest.fixture(scope="module")
+def L():
+    moe_build.build()
+    return moe.lib()
+
+
+def _declared():
+    with open(HEADER) as f:
+        src = f.read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for want in ("moe_forward", "moe_forward_debug", "moe_workspace_bytes", "moe_stack_forward",
+                 "moe_status_string", "moe_forward_host_io", "moe_workspace_init",
+                 "moe_workspace_status", "moe_forward_profiled", "moe_plan_info"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name   # dlsym through ctypes
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.moe_abi_version() >= 1
+    for code in range(7):
+        assert L.moe_status_string(code)
+    assert L.moe_status_string(99) == b"unknown status"
+
+
+def test_workspace_bytes(L):
+    ws = moe.moe_workspace_bytes
+    assert ws(16, 4096, 14336, 8, 2, BF16) > 0
+    assert ws(4096, 4096, 14336, 8, 2, BF16) > ws(16, 4096, 14336, 8, 2, BF16)
+    assert ws(0, 4096, 14336, 8, 2, BF16) > 0                   # T = 0 is valid
+    assert ws(16, 4000, 14336, 8, 2, BF16) == 0                 # d % 64 on the bf16 path
+    assert ws(16, 4096, 14300, 8, 2, BF16) == 0                 # F % 64
+    assert ws(16, 136, 200, 8, 2, F32) > 0                      # fp32 path: multiples of 8
+    assert ws(16, 4096, 14336, 65, 2, BF16) == 0                # n > 64
+    assert ws(16, 4096, 14336, 8, 9, BF16) == 0                 # K > n
+    assert ws(16, 4096, 14336, 8, 0, BF16) == 0                 # K < 1
+    # the prefill layout holds at least the routed rows of X, h and Y
+    T, d, F = 4096, 4096, 14336
+    assert ws(T, d, F, 8, 2, BF16) >= T * 2 * (d * 2 + F * 2 + d * 4)
+    assert moe.moe_stack_workspace_bytes(8192, 4096, 14336, 8, 2) > ws(8192, 4096, 14336, 8, 2,
+                                                                       BF16)
+    assert moe.moe_stack_workspace_bytes(64, 128, 256, 8, 2, F32) == 0
+
+
+def _plan(L, T, d, F, n, K, dt=BF16):
+    v = [ctypes.c_int(-1) for _ in range(4)]
+    rc = L.moe_plan_info(T, d, F, n, K, dt, *[ctypes.byref(i) for i in v])
+    return rc, [i.value for i in v]
+
+
+def test_plan_selection(L):
+    rc, (small, s13, s2, launches) = _plan(L, 16, 4096, 14336, 8, 2)
+    assert rc == OK and small == 1 and s13 >= 1 and s2 >= 1 and launches == 7
+    assert 4096 // 64 % s13 == 0 and 14336 // 64 % s2 == 0
+    rc, (small, s13, s2, launches) = _plan(L, 4096, 4096, 14336, 8, 2)
+    assert rc == OK and small == 0 and s13 == 1 and s2 == 1 and launches == 6
+    rc, (small, _, _, _) = _plan(L, 64, 128, 256, 8, 2, F32)
+    assert rc == OK and small == 0
+    assert _plan(L, 16, 100, 256, 8, 2)[0] == UNSUPPORTED
+    assert _plan(L, 16, 128, 256, 8, 9)[0] == INVALID
+
+
+P = ctypes.c_void_p
+
+
+def _fwd(L, x=0x1000, wg=0x2000, w1=0x3000, w3=0x4000, w2=0x5000, T=16, d=256, F=256, n=8,
+         K=2, dt=BF16, out=0x6000, ws=0x10000, ws_bytes=1 << 40):
+    return L.moe_forward(P(x), P(wg), P(w1), P(w3), P(w2), T, d, F, n, K, dt, P(out), P(ws),
+                         ws_bytes, None)
+
+
+def test_forward_rejects_bad_arguments_before_launch(L):
+    assert _fwd(L, x=0) == INVALID
+    assert _fwd(L, wg=0) == INVALID
+    assert _fwd(L, w1=0) == INVALID and _fwd(L, w3=0) == INVALID and _fwd(L, w2=0) == INVALID
+    assert _fwd(L, out=0) == INVALID
+    assert _fwd(L, ws=0) == INVALID
+    assert _fwd(L, x=0x1008) == INVALID            # x not 16-byte aligned
+    assert _fwd(L, ws=0x10080) == INVALID          # workspace not 256-byte aligned
+    assert _fwd(L, out=0x1000) == INVALID          # out aliases x
+    assert _fwd(L, K=0) == INVALID and _fwd(L, K=9) == INVALID and _fwd(L, n=0) == INVALID
+    assert _fwd(L, T=-1) == INVALID
+    assert _fwd(L, d=200) == UNSUPPORTED
+    assert _fwd(L, n=65, K=2) == UNSUPPORTED
+    assert _fwd(L, dt=7) == INVALID
+    assert _fwd(L, ws_bytes=1024) == WORKSPACE
+
+
+def test_zero_tokens_is_a_noop_without_touching_pointers(L):
+    assert _fwd(L, T=0, x=0, w1=0, out=0, ws=0) == OK
+
+
+def test_profiled_needs_six_events(L):
+    evs = (P * 6)(*([P(0x1)] * 6))
+    rc = L.moe_forward_profiled(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), 16, 256,
+                                256, 8, 2, BF16, P(0x6000), P(0x10000), 1 << 40, None, evs, 5)
+    assert rc == INVALID
+
+
+def test_stack_validation(L):
+    arr = (P * 2)(P(0x3000), P(0x3000))
+    assert L.moe_stack_forward(P(0x1000), arr, arr, arr, arr, 2, 16, 256, 256, 8, 2, F32,
+                               ctypes.c_float(1e-5), P(0x10000), 1 << 40, None) == UNSUPPORTED
+    assert L.moe_stack_forward(P(0x1000), None, arr, arr, arr, 2, 16, 256, 256, 8, 2, BF16,
+                               ctypes.c_float(1e-5), P(0x10000), 1 << 40, None) == INVALID
+    assert L.moe_stack_forward(P(0x1000), arr, arr, arr, arr, 2, 16, 256, 256, 8, 2, BF16,
+                               ctypes.c_float(1e-5), P(0x10000), 1024, None) == WORKSPACE
+
+
+def test_host_io_validation(L):
+    rc = L.moe_forward_host_io(None, P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), 16,
+                               256, 256, 8, 2, BF16, P(0x6000), P(0x7000), P(0x10000), 1 << 40,
+                               None)
+    assert rc == INVALID
+
+
+def test_product_path_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "sparse_mixture_experts_18_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    src = f.read()
+                assert not re.search(r"\boracle\b", src), fn
+    with open(os.path.join(ROOT, "include", "moe.h")) as f:
+        assert "oracle" not in f.read()
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import importlib
+    from sparse_mixture_experts_18_b200 import moe as binding
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(ImportError):
+        binding.lib()
+    importlib.reload(binding)

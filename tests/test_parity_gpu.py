@@ -1,0 +1,188 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle, element by
+element on the same seeded inputs.  Small cases span several tiles and ragged tails on both
+the prefill tiling and the small-batch (swap-AB, split-K) tiling; full-size workloads are
+checked on all tokens' routing and on sampled tokens' outputs."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+cuda = pytest.importorskip("torch").cuda
+if not cuda.is_available():  # pragma: no cover - the driver runs this file on a B200 only
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import sparse_mixture_experts_18_b200 as moe  # noqa: E402
+
+
+def _run(w: moe_inputs.Workload, gen_device="cpu", budget=None, layer_kw=None, x=None,
+         layer=None):
+    """Run one block on the GPU and compare with the oracle.  Returns a report dict."""
+    if x is None:
+        x = moe_inputs.make_x(w, device=gen_device)
+    if layer is None:
+        layer = moe_inputs.make_layer(w, device=gen_device, **(layer_kw or {}))
+    xd = x.cuda()
+    L = {k: v.cuda() for k, v in layer.items()}
+    out, idx, gate, counts, offsets, rows = moe.moe_forward_debug(
+        xd, L["Wg"], L["W1"], L["W3"], L["W2"], w.K)
+    ws_status = None
+    torch.cuda.synchronize()
+    xc = x.cpu()
+    lc = {k: v.cpu() for k, v in layer.items()}
+    del L, xd
+    idx_h, gate_h = idx.cpu().numpy(), gate.cpu().numpy()
+    logits, _, _ = parity.oracle.route(xc, lc["Wg"], w.n, w.K)
+    exempt, errors = parity.check_routing(logits, idx_h, gate_h, w.K)
+    assert not errors, errors[:5]
+    parity.check_permutation(idx_h, counts.cpu().numpy(), offsets.cpu().numpy(),
+                             rows.cpu().numpy(), w.n, w.K)
+    tokens = parity.sample_tokens(w.T, idx_h, exempt, w.n, budget or w.T)
+    ref = parity.oracle_outputs(xc, lc["Wg"], lc["W1"], lc["W3"], lc["W2"], w.n, w.K, tokens,
+                                idx_h, exempt)
+    got = out.float().cpu().numpy()[tokens]
+    rep = parity.compare_outputs(got, ref, x.dtype)
+    rep.update(exempt=len(exempt), tokens=len(tokens), counts=counts.cpu().tolist(),
+               status=ws_status)
+    assert rep["ok"], rep
+    return rep
+
+
+# ------------------------------------------------------------------ small, ragged cases
+
+def test_tiny_f32_full():
+    rep = _run(moe_inputs.WORKLOADS["tiny_f32"])
+    assert rep["tokens"] == 64
+
+
+@pytest.mark.parametrize("T,d,F", [(700, 320, 448), (1000, 256, 384), (600, 512, 1024)])
+def test_prefill_tiling_small(T, d, F):
+    # T*K >= 64*n: the 128-row tile path; d % 256 and F % 128 ragged in the first case
+    _run(moe_inputs.small(T=T, d=d, F=F))
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 37, 100, 255])
+def test_small_batch_tiling(T):
+    # T <= 256 and T*K < 64*n: weights as the 128-row MMA operand, split-K
+    _run(moe_inputs.small(T=T, d=512, F=768))
+
+
+@pytest.mark.parametrize("n,K", [(8, 1), (4, 4), (16, 2), (64, 2), (1, 1), (32, 3)])
+def test_expert_counts(n, K):
+    _run(moe_inputs.small(T=333, d=256, F=256, n=n, K=K))
+    _run(moe_inputs.small(T=24, d=256, F=256, n=n, K=K))
+
+
+@pytest.mark.parametrize("T", [7, 200])
+def test_f32_path_ragged(T):
+    _run(moe_inputs.small(T=T, d=136, F=200, dtype="f32", rms_x=False))
+
+
+def _biased_layer(w, bias):
+    layer = moe_inputs.make_layer(w)
+    layer["Wg"][0, :] = torch.tensor(bias, dtype=torch.float32)
+    return layer
+
+
+@pytest.mark.parametrize("T", [16, 900])
+def test_all_tokens_to_two_experts(T):
+    w = moe_inputs.small(T=T, d=256, F=384, zipf=0.0)
+    x = moe_inputs.make_x(w)
+    x[:, 0] = 1.0
+    layer = _biased_layer(w, [0, 0, 0, 40.0, 0, 30.0, 0, 0])
+    rep = _run(w, x=x, layer=layer)
+    assert rep["counts"] == [0, 0, 0, T, 0, T, 0, 0]
+
+
+def test_expert_with_no_tokens():
+    w = moe_inputs.small(T=640, d=256, F=256)
+    x = moe_inputs.make_x(w)
+    x[:, 0] = 1.0
+    layer = _biased_layer(w, [0, -50.0, 0, 0, 0, 0, -50.0, 0])
+    rep = _run(w, x=x, layer=layer)
+    assert rep["counts"][1] == 0 and rep["counts"][6] == 0
+
+
+def test_exact_ties_pick_lowest_index():
+    w = moe_inputs.small(T=40, d=128, F=128)
+    x = moe_inputs.make_x(w)
+    layer = moe_inputs.make_layer(w)
+    layer["Wg"][:] = layer["Wg"][:, :1]          # identical columns: every logit ties
+    xd = x.cuda()
+    L = {k: v.cuda() for k, v in layer.items()}
+    out, idx, gate, counts, _, _ = moe.moe_forward_debug(xd, L["Wg"], L["W1"], L["W3"], L["W2"],
+                                                         w.K)
+    assert torch.all(idx.cpu() == torch.tensor([0, 1], dtype=torch.int32))
+    assert torch.all(gate.cpu() == 0.5)
+    ref = parity.oracle_outputs(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n,
+                                w.K, np.arange(w.T), idx.cpu().numpy(), [])
+    assert parity.compare_outputs(out.float().cpu().numpy(), ref, x.dtype)["ok"]
+
+
+def test_zero_tokens_is_noop():
+    w = moe_inputs.small(T=8, d=128, F=128)
+    layer = {k: v.cuda() for k, v in moe_inputs.make_layer(w).items()}
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    out = moe.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], 2)
+    assert out.shape == (0, 128)
+
+
+def test_repeat_calls_same_workspace_bitwise():
+    w = moe_inputs.small(T=300, d=256, F=384)
+    x = moe_inputs.make_x(w).cuda()
+    L = {k: v.cuda() for k, v in moe_inputs.make_layer(w).items()}
+    ws = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K, torch.bfloat16))
+    a = moe.moe_forward(x, L["Wg"], L["W1"], L["W3"], L["W2"], w.K, workspace=ws)
+    b = moe.moe_forward(x, L["Wg"], L["W1"], L["W3"], L["W2"], w.K, workspace=ws)
+    assert torch.equal(a, b)
+    assert moe.moe_workspace_status(ws) == (0, 0)
+
+
+def test_host_io_matches_device_path():
+    w = moe_inputs.small(T=64, d=256, F=384)
+    x = moe_inputs.make_x(w)
+    L = {k: v.cuda() for k, v in moe_inputs.make_layer(w).items()}
+    ws = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K, torch.bfloat16))
+    ref = moe.moe_forward(x.cuda(), L["Wg"], L["W1"], L["W3"], L["W2"], w.K, workspace=ws)
+    xh = x.pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    xd, od = torch.empty_like(ref), torch.empty_like(ref)
+    moe.moe_forward_host_io(xh, xd, L["Wg"], L["W1"], L["W3"], L["W2"], w.K, od, oh, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, ref.cpu())
+
+
+def test_stack_small():
+    w = moe_inputs.small(T=300, d=256, F=512, layers=4)
+    x = moe_inputs.make_x(w)
+    layers = [moe_inputs.make_layer(w, layer=l) for l in range(w.layers)]
+    xd = x.cuda()
+    moe.moe_stack_forward(xd, [{k: v.cuda() for k, v in l.items()} for l in layers], w.K)
+    torch.cuda.synchronize()
+    ref = x.double().numpy()
+    for l in layers:
+        ref, _, _ = parity.oracle.block_forward(ref, l["Wg"], l["W1"], l["W3"], l["W2"], w.n,
+                                                w.K, 1e-5)
+    rep = parity.compare_outputs(xd.float().cpu().numpy(), ref, torch.bfloat16)
+    assert rep["ok"], rep
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def test_decode_t16_full():
+    rep = _run(moe_inputs.WORKLOADS["decode_t16"])
+    assert rep["tokens"] == 16
+
+
+def test_prefill_t4096_sampled():
+    _run(moe_inputs.WORKLOADS["prefill_t4096"], gen_device="cuda", budget=24)
+
+
+def test_skewed_t32768_sampled():
+    w = moe_inputs.WORKLOADS["skewed_t32768"]
+    rep = _run(w, gen_device="cuda", budget=16)
+    c = np.array(rep["counts"])
+    assert c[0] > 2.5 * c.mean(), c   # busiest expert about 3x the mean load
