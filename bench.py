@@ -137,11 +137,9 @@ def run_gpu(args, w):
     ws = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K, torch.bfloat16),
                              dev, stream)
     out = torch.empty_like(x)
-    L = moe.lib()
-    import ctypes
-    info = [ctypes.c_int(0) for _ in range(4)]
-    L.moe_plan_info(w.T, w.d, w.F, w.n, w.K, 1, *[ctypes.byref(v) for v in info])
-    small_batch, s13, s2, launches = (v.value for v in info)
+    plan = moe.moe_plan_info(w.T, w.d, w.F, w.n, w.K)
+    small_batch, s13, s2, launches = (plan["small_batch"], plan["split13"], plan["split2"],
+                                      plan["launches"])
 
     def step():
         moe.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.K, out=out,
@@ -175,19 +173,11 @@ def run_gpu(args, w):
         # ---- per-stage durations from events recorded by the library on its stream
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)]
                for _ in range(args.steps)]
-        arr_t = ctypes.c_void_p * 6
         for i in range(args.steps):
             for e in evs[i]:
                 e.record(stream)  # creates the cudaEvent_t; the library re-records it
-            handles = arr_t(*[ctypes.c_void_p(e.cuda_event) for e in evs[i]])
-            rc = L.moe_forward_profiled(
-                ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(layer["Wg"].data_ptr()),
-                ctypes.c_void_p(layer["W1"].data_ptr()), ctypes.c_void_p(layer["W3"].data_ptr()),
-                ctypes.c_void_p(layer["W2"].data_ptr()), w.T, w.d, w.F, w.n, w.K, 1,
-                ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
-                ctypes.c_void_p(stream.cuda_stream), handles, 6)
-            if rc != 0:
-                raise RuntimeError(f"moe_forward_profiled failed: {rc}")
+            moe.moe_forward_profiled(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.K,
+                                     evs[i], out=out, workspace=ws, stream=stream)
         barrier()
         stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
                     for i in range(args.steps)]

@@ -56,6 +56,12 @@ def lib() -> ctypes.CDLL:
         L.moe_stack_forward.restype = I32
         L.moe_stack_forward.argtypes = [P, P, P, P, P, I32, I64, I64, I64, I32, I32, I32,
                                         ctypes.c_float, P, SZ, P]
+        L.moe_forward_profiled.restype = I32
+        L.moe_forward_profiled.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P, P, SZ,
+                                           P, ctypes.POINTER(P), I32]
+        IP = ctypes.POINTER(ctypes.c_int)
+        L.moe_plan_info.restype = I32
+        L.moe_plan_info.argtypes = [I64, I64, I64, I32, I32, I32, IP, IP, IP, IP]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [I32]
         L.moe_abi_version.restype = I32
@@ -130,6 +136,32 @@ def moe_forward(x, W_g, W1, W3, W2, K: int, out=None, workspace=None, stream=Non
         _ptr(x), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt, _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
+
+
+def moe_forward_profiled(x, W_g, W1, W3, W2, K: int, events, out=None, workspace=None,
+                         stream=None):
+    """moe_forward that records six torch.cuda.Event objects at the stage boundaries (see
+    include/moe.h).  The events must have been recorded once (so they exist)."""
+    T, d, F, n = _dims(x, W1, W_g)
+    dt = _dt(x)
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = alloc_workspace(moe_workspace_bytes(T, d, F, n, K, dt), x.device, stream)
+    handles = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check("moe_forward_profiled", lib().moe_forward_profiled(
+        _ptr(x), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt, _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream(stream), handles, len(events)))
+    return out
+
+
+def moe_plan_info(T, d, F, n, K, dtype=torch.bfloat16) -> dict:
+    """The work plan the library picks for a shape."""
+    dt = MOE_BF16 if dtype in (torch.bfloat16, MOE_BF16) else MOE_F32
+    v = [ctypes.c_int(0) for _ in range(4)]
+    _check("moe_plan_info", lib().moe_plan_info(T, d, F, n, K, dt, *[ctypes.byref(i) for i in v]))
+    return {"small_batch": bool(v[0].value), "split13": v[1].value, "split2": v[2].value,
+            "launches": v[3].value}
 
 
 def moe_forward_debug(x, W_g, W1, W3, W2, K: int, out=None, workspace=None, stream=None):

@@ -20,6 +20,7 @@ import torch
 import oracle
 
 TIE_REL = 1e-4
+STACK_TIE_REL = 1e-2   # stacked blocks: residual streams differ by bf16 rounding after block 1
 BF16_MAX_ABS, BF16_REL_L2 = 2e-2, 5e-3
 F32_REL = 1e-5
 GATE_ABS = 1e-5
@@ -97,11 +98,17 @@ def oracle_outputs(x, Wg, W1, W3, W2, n, K, tokens, idx_gpu, exempt):
     return oracle.round_array(y, dt)
 
 
-def compare_outputs(out_gpu: np.ndarray, ref: np.ndarray, dtype) -> dict:
+def compare_outputs(out_gpu: np.ndarray, ref: np.ndarray, dtype, stacked: bool = False) -> dict:
+    """stacked=True: the residual stream of stacked blocks grows past the magnitudes the
+    absolute bar was set for, so each element may also differ by 2^-7 |ref| (two bf16 ulps)
+    on top of 2e-2; the relative L2 bar is unchanged."""
     err = out_gpu.astype(np.float64) - ref
     max_abs = float(np.max(np.abs(err))) if err.size else 0.0
     rel_l2 = float(np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300)) if err.size else 0.0
-    if dtype == torch.bfloat16:
+    if dtype == torch.bfloat16 and stacked:
+        ok = bool(np.all(np.abs(err) <= BF16_MAX_ABS + 2.0 ** -7 * np.abs(ref))) and \
+            rel_l2 <= BF16_REL_L2
+    elif dtype == torch.bfloat16:
         ok = max_abs <= BF16_MAX_ABS and rel_l2 <= BF16_REL_L2
     else:
         ok = rel_l2 <= F32_REL and max_abs <= F32_REL * max(float(np.max(np.abs(ref))), 1e-30)
