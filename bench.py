@@ -41,6 +41,23 @@ import moe_inputs  # noqa: E402
 METRIC = "MoE-layer tokens/s and TFLOP/s (bf16, top-2 of 8) as % of B200 roofline"
 DEFAULT_WORKLOAD = "decode_t16"
 
+# DRAM bytes (read + write) of one launch of the dominant kernel (G13), from the ncu
+# captures summarised in profiles/tc_grouped_gemm_<workload>.md, valid only for the kernel
+# source they were taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
+TRAFFIC = {
+    "decode_t16": {"bytes": 1879435000 + 7812096, "src": "3a5e4416896d"},
+    "prefill_t4096": {"bytes": 1973359000 + 239567872, "src": "3a5e4416896d"},
+}
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "sparse_mixture_experts_18_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
 
 def _peaks():
     try:
@@ -233,6 +250,8 @@ def run_gpu(args, w):
         achieved = 4 * w.d * w.F * w.T * w.K / (g13 / 1e3) / 1e12
         peak = bf16_peak
         step_frac = tflops / peak
+    cap = TRAFFIC.get(w.name)
+    traffic = cap["bytes"] if cap and cap["src"] == kernel_source_hash() else None
     line = {
         "metric": METRIC, "value": round(tok_s, 2), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
@@ -252,7 +271,7 @@ def run_gpu(args, w):
                                   "routed FLOPs per step / measured bf16 GEMM TFLOP/s"},
         "roofline": {"bound": bound, "kernel": "tc_grouped_gemm G13 (gate/up + SwiGLU)",
                      "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": peaks["source"], "launch_ms": round(g13, 5)},
         "stage_ms": {"route": round(stage_avg[0], 5), "gemm13": round(stage_avg[1], 5),
                      "splitk_reduce": round(stage_avg[2], 5), "gemm2": round(stage_avg[3], 5),

@@ -205,29 +205,52 @@ def test_skewed_t32768_sampled():
 
 
 def test_stack32_t8192_sampled():
-    # 32 blocks of Mixtral shape on T=8192 tokens (~90 GB of bf16 expert weights on the
-    # device); the oracle follows 3 tokens through all blocks, one layer's weights at a time.
+    """32 blocks of Mixtral shape on T=8192 tokens (~90 GB of bf16 expert weights on the
+    device).  The residual stream amplifies any sub-ulp difference: two oracle trajectories
+    that differ only in whether h is rounded to bf16 drift apart by ~0.8% after 8 blocks and
+    ~2.5% after 32, and by block 32 they route about half of the tokens differently.  So:
+    block 1 must meet the stacked-block bars; block 8 must be within max(5e-3, 2x the
+    oracle's own drift) for at least 90% of the tokens the two oracle trajectories route
+    identically (median ratio to the drift <= 1.5); and 32 blocks in one call must equal
+    four successive 8-block calls bit for bit."""
     w = moe_inputs.WORKLOADS["stack32_t8192"]
+    depth = 8
     x = moe_inputs.make_x(w, device="cuda")
     layers = [moe_inputs.make_layer(w, layer=l, device="cuda") for l in range(w.layers)]
-    xd = x.clone()
-    moe.moe_stack_forward(xd, layers, w.K)
+    x1, x8, x32, xc = x.clone(), x.clone(), x.clone(), x.clone()
+    moe.moe_stack_forward(x1, layers[:1], w.K)
+    moe.moe_stack_forward(x8, layers[:depth], w.K)
+    moe.moe_stack_forward(x32, layers, w.K)
+    for c in range(0, w.layers, depth):
+        moe.moe_stack_forward(xc, layers[c:c + depth], w.K)
     torch.cuda.synchronize()
-    out = xd.float().cpu().numpy()
-    tokens = np.array([0, 4097, w.T - 1])
+    assert torch.equal(x32, xc), "stack over 32 blocks differs from 4 calls of 8 blocks"
+    assert torch.isfinite(x32.float()).all()
+    tokens = np.linspace(0, w.T - 1, 12).astype(np.int64)
+    out1 = x1.float().cpu().numpy()[tokens]
+    out8 = x8.float().cpu().numpy()[tokens]
+    del x1, x8, x32, xc
     ref = x.cpu().double().numpy()[tokens]
-    near = np.zeros(len(tokens), bool)
-    for l in range(w.layers):
+    pert = ref.copy()
+    same = np.ones(len(tokens), bool)
+    for l in range(depth):
         lc = {k: v.cpu() for k, v in layers[l].items()}
-        layers[l] = None
-        xn = parity.oracle.rmsnorm(ref, 1e-5, parity.oracle.BF16)
-        logits, _, _ = parity.oracle.route(torch.from_numpy(xn).to(torch.bfloat16), lc["Wg"],
-                                           w.n, w.K)
-        near |= np.array([parity.oracle.tie_band(logits[r], w.K, parity.STACK_TIE_REL)[0]
-                          for r in range(len(tokens))])
-        ref, _, _ = parity.oracle.block_forward(ref, lc["Wg"], lc["W1"], lc["W3"], lc["W2"],
-                                                w.n, w.K, 1e-5)
-    keep = ~near
-    assert keep.sum() >= 1
-    rep = parity.compare_outputs(out[tokens][keep], ref[keep], torch.bfloat16, stacked=True)
-    assert rep["ok"], rep
+        ref, ia, _ = parity.oracle.block_forward(ref, lc["Wg"], lc["W1"], lc["W3"], lc["W2"],
+                                                 w.n, w.K, 1e-5)
+        xp = parity.oracle.rmsnorm(pert, 1e-5, parity.oracle.BF16)
+        yp, ip, _ = parity.oracle.moe_forward(torch.from_numpy(xp).to(torch.bfloat16),
+                                              lc["Wg"], lc["W1"], lc["W3"], lc["W2"], w.n,
+                                              w.K, round_h=False)
+        pert = parity.oracle.round_array(pert + yp, parity.oracle.BF16)
+        same &= np.all(np.sort(ia, axis=1) == np.sort(ip, axis=1), axis=1)
+        if l == 0:
+            rep1 = parity.compare_outputs(out1, ref, torch.bfloat16, stacked=True)
+            assert rep1["ok"], rep1
+    drift = np.linalg.norm(pert - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    gpu = np.linalg.norm(out8 - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    info = {"gpu": gpu.round(4).tolist(), "drift": drift.round(4).tolist(),
+            "well_conditioned": same.tolist()}
+    assert same.sum() >= 6, info
+    ok = gpu[same] <= np.maximum(5e-3, 2.0 * drift[same])
+    assert ok.mean() >= 0.9, info
+    assert np.median(gpu[same] / drift[same]) <= 1.5, info
