@@ -144,6 +144,26 @@ MOE_API moe_status moe_stack_forward(void* x, const float* const* W_g, const voi
                              int64_t d, int64_t F, int n, int K, moe_dtype dt, float eps,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_forward without a caller-supplied workspace, for callers that cannot allocate device
+ * memory (e.g. a plugin inside an application whose own pool owns every allocation, or a
+ * loop that must never call cudaMalloc because it can synchronise the device).  The paper
+ * has no counterpart to this entry point; it exists only for such callers.
+ *   - The workspace is a fixed device array of MOE_NOALLOC_WORKSPACE_BYTES inside the
+ *     library; every GPU that loads the library holds it until the process exits.  Shapes
+ *     whose moe_workspace_bytes() exceeds it return MOE_ERR_WORKSPACE (at Mixtral's sizes it
+ *     fits decode batches of up to 24 tokens).
+ *   - The first call on a device, with that device current, looks up the array's address
+ *     and zeroes its status word (synchronously); make that first call before any stream
+ *     capture.  Nothing is allocated, and nothing is freed.
+ *   - All calls share the one array and it keeps the last call's contents: calls that
+ *     overlap on the GPU (other streams, other threads) race on it.
+ * Arguments, layouts and errors otherwise as moe_forward. */
+#define MOE_NOALLOC_WORKSPACE_BYTES (32u << 20)
+MOE_API moe_status moe_forward_noalloc(const void* x, const float* W_g, const void* W1,
+                                       const void* W3, const void* W2, int64_t T, int64_t d,
+                                       int64_t F, int n, int K, moe_dtype dt, void* out,
+                                       void* stream);
+
 /* Short description of a status code (static string). */
 MOE_API const char* moe_status_string(moe_status s);
 

@@ -5,9 +5,10 @@ include/moe.h); this package is its build script and a ctypes binding.
 """
 from .moe import (MOE_BF16, MOE_F32, MoeError, alloc_workspace, lib, moe_forward,
                   moe_forward_debug, moe_forward_host_io,
-                  moe_forward_profiled, moe_plan_info, moe_stack_forward,
+                  moe_forward_noalloc, moe_forward_profiled, moe_plan_info, moe_stack_forward,
                   moe_stack_workspace_bytes, moe_workspace_bytes, moe_workspace_status)
 
 __all__ = ["MOE_BF16", "MOE_F32", "MoeError", "alloc_workspace", "lib", "moe_forward",
-           "moe_forward_debug", "moe_forward_host_io", "moe_forward_profiled", "moe_plan_info", "moe_stack_forward",
+           "moe_forward_debug", "moe_forward_host_io", "moe_forward_noalloc", "moe_forward_profiled",
+           "moe_plan_info", "moe_stack_forward",
            "moe_stack_workspace_bytes", "moe_workspace_bytes", "moe_workspace_status"]

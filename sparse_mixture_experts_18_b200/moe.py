@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         IP = ctypes.POINTER(ctypes.c_int)
         L.moe_plan_info.restype = I32
         L.moe_plan_info.argtypes = [I64, I64, I64, I32, I32, I32, IP, IP, IP, IP]
+        L.moe_forward_noalloc.restype = I32
+        L.moe_forward_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P, P]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [I32]
         L.moe_abi_version.restype = I32
@@ -135,6 +137,20 @@ def moe_forward(x, W_g, W1, W3, W2, K: int, out=None, workspace=None, stream=Non
     _check("moe_forward", lib().moe_forward(
         _ptr(x), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt, _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def moe_forward_noalloc(x, W_g, W1, W3, W2, K: int, out=None, stream=None):
+    """moe_forward for callers that cannot allocate device memory: the library's own
+    fixed-size device workspace is used (see include/moe.h for its size, its first-call
+    set-up and why overlapping calls race).  `out` may be preallocated by the caller."""
+    T, d, F, n = _dims(x, W1, W_g)
+    dt = _dt(x)
+    if out is None:
+        out = torch.empty_like(x)
+    _check("moe_forward_noalloc", lib().moe_forward_noalloc(
+        _ptr(x), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt, _ptr(out),
+        _stream(stream)))
     return out
 
 
