@@ -46,40 +46,73 @@ struct Out8<float> {
   }
 };
 
+// One thread per 4 output columns of a token.  All K x S loads of a thread are issued
+// before they are summed (splits unrolled up to MAX_S), then the fp32 sum over slots is
+// taken in slot order and rounded once.
+constexpr int COMBINE_MAX_S = 8;
+
+template <typename Tout>
+struct Out4;
+template <>
+struct Out4<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[4]) {
+    const uint2 r = *reinterpret_cast<const uint2*>(p);
+    v[0] = bf16_lo(r.x); v[1] = bf16_hi(r.x); v[2] = bf16_lo(r.y); v[3] = bf16_hi(r.y);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+  }
+};
+template <>
+struct Out4<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+
 template <typename Tout, bool RESID>
 __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ Y, int S, int64_t split_stride, int64_t T, int d,
                    int K, const int32_t* __restrict__ inv, const float* __restrict__ gate,
                    Tout* out, const Tout* resid) {
-  const int vpr = d / 8;
+  const int vpr = d / 4;
   const int64_t total = T * vpr;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
        v += (int64_t)gridDim.x * blockDim.x) {
     const int64_t t = v / vpr;
-    const int c = (int)(v % vpr) * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const int c = (int)(v % vpr) * 4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int k = 0; k < K; ++k) {
       const int row = inv[t * K + k];
       if (row < 0) continue;
       const float g = gate[t * K + k];
-      float yk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int s = 0; s < S; ++s) {
-        const float* src = Y + s * split_stride + (int64_t)row * d + c;
-        const float4 a = __ldg(reinterpret_cast<const float4*>(src));
-        const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
-        yk[0] += a.x; yk[1] += a.y; yk[2] += a.z; yk[3] += a.w;
-        yk[4] += b.x; yk[5] += b.y; yk[6] += b.z; yk[7] += b.w;
-      }
+      const float* src = Y + (int64_t)row * d + c;
+      float4 part[COMBINE_MAX_S];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, yk[i], acc[i]);
+      for (int s = 0; s < COMBINE_MAX_S; ++s)
+        if (s < S) part[s] = __ldg(reinterpret_cast<const float4*>(src + s * split_stride));
+      float4 yk = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s = 0; s < COMBINE_MAX_S; ++s)
+        if (s < S) {
+          yk.x += part[s].x; yk.y += part[s].y; yk.z += part[s].z; yk.w += part[s].w;
+        }
+      acc[0] = fmaf(g, yk.x, acc[0]);
+      acc[1] = fmaf(g, yk.y, acc[1]);
+      acc[2] = fmaf(g, yk.z, acc[2]);
+      acc[3] = fmaf(g, yk.w, acc[3]);
     }
     if (RESID) {
-      float r[8];
-      Out8<Tout>::load(resid + t * d + c, r);
+      float r[4];
+      Out4<Tout>::load(resid + t * d + c, r);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = r[i] + acc[i];
+      for (int i = 0; i < 4; ++i) acc[i] = r[i] + acc[i];
     }
-    Out8<Tout>::store(out + t * d + c, acc);
+    Out4<Tout>::store(out + t * d + c, acc);
   }
 }
 
@@ -87,7 +120,7 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
                            cudaStream_t s) {
   const int S = p.swap ? p.s2 : 1;
   const int64_t split_stride = p.rows_max * p.d;
-  const int64_t total = p.T * (p.d / 8);
+  const int64_t total = p.T * (p.d / 4);
   int64_t blocks = (total + 255) / 256;
   if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
   if (blocks < 1) blocks = 1;

@@ -329,7 +329,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, a.tmem_cols);
 }
 
-// Small batch: h = bf16(silu(sum_s A_s) * sum_s B_s), splits summed in order 0..S-1.
+// Small batch: h = bf16(silu(sum_s A_s) * sum_s B_s), splits summed in order 0..S-1.  All
+// 2*S loads of a thread are issued before the sums (splits unrolled up to 8).
+constexpr int REDUCE_MAX_S = 8;
+
 __global__ void __launch_bounds__(256)
     swiglu_reduce_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
                          int64_t rows, int F, __nv_bfloat16* __restrict__ h) {
@@ -340,13 +343,20 @@ __global__ void __launch_bounds__(256)
     const int64_t r = v / vpr;
     const int c = (int)(v % vpr) * 4;
     const float* pa = p13 + r * 2 * F + c;
+    float4 ta[REDUCE_MAX_S], tb[REDUCE_MAX_S];
+#pragma unroll
+    for (int s = 0; s < REDUCE_MAX_S; ++s)
+      if (s < S) {
+        ta[s] = __ldg(reinterpret_cast<const float4*>(pa + s * split_stride));
+        tb[s] = __ldg(reinterpret_cast<const float4*>(pa + s * split_stride + F));
+      }
     float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
-    for (int s = 0; s < S; ++s) {
-      const float4 ta = *reinterpret_cast<const float4*>(pa + s * split_stride);
-      const float4 tb = *reinterpret_cast<const float4*>(pa + s * split_stride + F);
-      sa.x += ta.x; sa.y += ta.y; sa.z += ta.z; sa.w += ta.w;
-      sb.x += tb.x; sb.y += tb.y; sb.z += tb.z; sb.w += tb.w;
-    }
+#pragma unroll
+    for (int s = 0; s < REDUCE_MAX_S; ++s)
+      if (s < S) {
+        sa.x += ta[s].x; sa.y += ta[s].y; sa.z += ta[s].z; sa.w += ta[s].w;
+        sb.x += tb[s].x; sb.y += tb[s].y; sb.z += tb[s].z; sb.w += tb[s].w;
+      }
     uint2 o;
     o.x = pack_bf16x2(silu(sa.x) * sb.x, silu(sa.y) * sb.y);
     o.y = pack_bf16x2(silu(sa.z) * sb.z, silu(sa.w) * sb.w);
@@ -425,9 +435,9 @@ static cudaError_t record(cudaEvent_t const* ev, int i, cudaStream_t s) {
   return ev ? cudaEventRecord(ev[i], s) : cudaSuccess;
 }
 
-cudaError_t launch_expert_gemms_tc(const Plan& p, const void* W1, const void* W3,
-                                   const void* W2, const Workspace& w, cudaStream_t s,
-                                   cudaEvent_t const* ev) {
+cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
+                                   const void* W3, const void* W2, const Workspace& w,
+                                   cudaStream_t s, cudaEvent_t const* ev) {
   CUtensorMap mX, mW1, mW3, mH, mW2;
   const int d = (int)p.d, F = (int)p.F, n = p.n;
   cudaError_t err;

@@ -24,10 +24,13 @@ struct Plan {
   int row_align = 1;       // each expert's group is padded to a multiple of this
   int64_t rows_max = 0;    // upper bound of permuted rows (T*K plus padding)
   int64_t nblk = 0;        // router / permute blocks
+  bool fused_route = false;  // small batch: routing in one launch (route_split_kernel)
   int tok_tile = 0;        // swap: MMA N (tokens per expert tile), multiple of 16
   int s13 = 1, s2 = 1;     // swap: split-K factors of the two expert GEMMs
   bool stack = false;      // workspace also holds the normalised activations
   // workspace byte offsets
+  size_t o_rpart;          // small batch: partial router logits [ceil(d/64)][T][n]
+  size_t o_rowtok;         // small batch: token of each permuted row [rows_max]
   size_t o_status, o_idx, o_gate, o_blk_counts, o_blk_base, o_counts, o_offsets, o_inv,
       o_xperm, o_h, o_y, o_p13, o_xn, total;
 };
@@ -35,6 +38,9 @@ struct Plan {
 // Device pointers into the workspace.
 struct Workspace {
   uint32_t* status;
+  unsigned int* ticket;  // small-batch routing: CTAs finished (in the status header, starts 0)
+  float* rpart;          // small-batch routing: partial logits
+  int32_t* row_tok;      // small batch: token of each permuted row
   int32_t *idx, *blk_counts, *blk_base, *counts, *offsets, *inv;
   float* gate;
   void* xperm;  // [rows_max][d] activations in permuted order
@@ -51,9 +57,9 @@ int route_tokens_per_block(int n);
 cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Workspace& w,
                          cudaStream_t s);
 // ev (may be null): events recorded after G13, after the split-K reduction, after G2.
-cudaError_t launch_expert_gemms_tc(const Plan& p, const void* W1, const void* W3,
-                                   const void* W2, const Workspace& w, cudaStream_t s,
-                                   cudaEvent_t const* ev = nullptr);
+cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
+                                   const void* W3, const void* W2, const Workspace& w,
+                                   cudaStream_t s, cudaEvent_t const* ev = nullptr);
 cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float* W3,
                                      const float* W2, const Workspace& w, cudaStream_t s,
                                      cudaEvent_t const* ev = nullptr);

@@ -31,7 +31,7 @@ static int choose_split(int num_kb, int units_per_split, int sms) {
   int best = 1;
   double best_eff = 0.0;
   for (int s = 1; s <= 16; ++s) {
-    if (num_kb % s || num_kb / s < 4) continue;
+    if (num_kb % s || num_kb / s < 4 || s > 8) continue;  // the combine unrolls <= 8 splits
     const double u = (double)units_per_split * s;
     const double waves = u / sms;
     const double eff = waves / (double)((int64_t)((u + sms - 1) / sms));
@@ -61,6 +61,7 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   if (q.rows_max >= ((int64_t)1 << 31) / 2) return false;
   const int tokb = route_tokens_per_block(n);
   q.nblk = (T + tokb - 1) / tokb;
+  q.fused_route = T <= 64 && T * K <= 1024;  // limits of route_split_kernel
   if (q.swap) {
     q.tok_tile = (int)((T + 15) / 16 * 16);
     const int sms = num_sms();
@@ -83,6 +84,8 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   q.o_y = take((size_t)(q.swap ? q.s2 : 1) * q.rows_max * d * 4);
   q.o_p13 = take(q.swap ? (size_t)q.s13 * q.rows_max * 2 * F * 4 : 0);
   q.o_xn = take(stack ? (size_t)T * d * es : 0);
+  q.o_rpart = take(q.fused_route ? (size_t)((d + 63) / 64) * T * n * 4 : 0);
+  q.o_rowtok = take(q.fused_route ? (size_t)q.rows_max * 4 : 0);
   q.total = o;
   *p = q;
   return true;
@@ -92,6 +95,9 @@ Workspace carve(const Plan& p, void* base) {
   uint8_t* b = static_cast<uint8_t*>(base);
   Workspace w;
   w.status = reinterpret_cast<uint32_t*>(b + p.o_status);
+  w.ticket = reinterpret_cast<unsigned int*>(b + p.o_status + 64);
+  w.rpart = reinterpret_cast<float*>(b + p.o_rpart);
+  w.row_tok = reinterpret_cast<int32_t*>(b + p.o_rowtok);
   w.idx = reinterpret_cast<int32_t*>(b + p.o_idx);
   w.gate = reinterpret_cast<float*>(b + p.o_gate);
   w.blk_counts = reinterpret_cast<int32_t*>(b + p.o_blk_counts);
@@ -136,7 +142,7 @@ static moe_status forward_impl(const Plan& p, const void* x, const float* W_g, c
   if (launch_route(p, x, W_g, w, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], s) != cudaSuccess) return MOE_ERR_CUDA;
   cudaError_t err =
-      p.dt == 1 ? launch_expert_gemms_tc(p, W1, W3, W2, w, s, ev ? ev + 2 : nullptr)
+      p.dt == 1 ? launch_expert_gemms_tc(p, x, W1, W3, W2, w, s, ev ? ev + 2 : nullptr)
                 : launch_expert_gemms_simt(p, static_cast<const float*>(W1),
                                            static_cast<const float*>(W3),
                                            static_cast<const float*>(W2), w, s,
@@ -245,7 +251,7 @@ moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtyp
   if (small_batch) *small_batch = p.swap ? 1 : 0;
   if (split13) *split13 = p.swap ? p.s13 : 1;
   if (split2) *split2 = p.swap ? p.s2 : 1;
-  if (launches) *launches = T == 0 ? 0 : 3 + (p.swap ? 3 : 2) + 1;
+  if (launches) *launches = T == 0 ? 0 : (p.fused_route ? 1 : 3) + (p.swap ? 3 : 2) + 1;
   return MOE_OK;
 }
 

@@ -46,24 +46,29 @@ struct Vec8<float> {
   }
 };
 
-// Block b handles tokens [b*TOKB, b*TOKB + TOKB).  Each thread accumulates the logits of all
-// TOKB tokens over its 8-element chunks of the hidden dimension (so a W_g row is loaded once
-// per TOKB tokens); lanes and then warps are summed in a fixed order.
-template <typename Tin, int NPAD, int TOKB>
-__global__ void __launch_bounds__(ROUTE_THREADS)
-    router_topk_kernel(const Tin* __restrict__ x, const float* __restrict__ Wg, int64_t T,
-                       int d, int n, int K, int32_t* __restrict__ idx,
-                       float* __restrict__ gate, int32_t* __restrict__ blk_counts) {
+// Synchronisation of the threads that route one token block: the whole CTA, or one
+// 256-thread group of a larger CTA (named barrier 1 + group).
+struct CtaSync {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+struct GroupSync {
+  int id;
+  __device__ __forceinline__ void operator()() const {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(ROUTE_THREADS) : "memory");
+  }
+};
+
+// Router, TopK and softmax of tokens [t0, t0 + ntok), ntok <= TOKB, by ROUTE_THREADS threads
+// (tid = 0..255).  Each thread accumulates the logits of all TOKB tokens over its 8-element
+// chunks of the hidden dimension (so a W_g row is loaded once per TOKB tokens); lanes and
+// then warps are summed in a fixed order.  hist (shared, may be null) counts selections.
+template <typename Tin, int NPAD, int TOKB, typename Sync>
+__device__ __forceinline__ void route_token_block(
+    const Tin* __restrict__ x, const float* __restrict__ Wg, int64_t t0, int ntok, int d, int n,
+    int K, int tid, float (*red)[64], float (*logits)[NPAD], int* hist,
+    int32_t* __restrict__ idx, float* __restrict__ gate, Sync sync) {
   static_assert(NPAD * TOKB == 64, "64 partial sums per lane");
-  __shared__ float red[ROUTE_THREADS / 32][64];
-  __shared__ float logits[TOKB][NPAD];
-  __shared__ int hist[64];
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t0 = (int64_t)blockIdx.x * TOKB;
-  const int ntok = (int)(T - t0 < TOKB ? T - t0 : TOKB);
-  if (threadIdx.x < 64) hist[threadIdx.x] = 0;
-
+  const int warp = tid >> 5, lane = tid & 31;
   float acc[TOKB][NPAD];
 #pragma unroll
   for (int a = 0; a < TOKB; ++a)
@@ -71,7 +76,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
     for (int e = 0; e < NPAD; ++e) acc[a][e] = 0.f;
 
   // 8-element chunks of the hidden dimension, thread-interleaved (coalesced 16-byte loads)
-  for (int ci = threadIdx.x; ci < d / 8; ci += ROUTE_THREADS) {
+  for (int ci = tid; ci < d / 8; ci += ROUTE_THREADS) {
     const int j0 = ci * 8;
     Vec8<Tin> xv[TOKB];
 #pragma unroll
@@ -122,19 +127,19 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
   }
   red[warp][base] = v[0];
   red[warp][base + 1] = v[1];
-  __syncthreads();
-  if (threadIdx.x < 64) {
+  sync();
+  if (tid < 64) {
     float s = 0.f;
 #pragma unroll
-    for (int w = 0; w < ROUTE_THREADS / 32; ++w) s += red[w][threadIdx.x];
-    logits[threadIdx.x / NPAD][threadIdx.x % NPAD] = s;
+    for (int w = 0; w < ROUTE_THREADS / 32; ++w) s += red[w][tid];
+    logits[tid / NPAD][tid % NPAD] = s;
   }
-  __syncthreads();
+  sync();
 
   // TopK by repeated arg-max (strict '>' keeps the lower index on ties), then Softmax over
   // the kept logits shifted by the largest.
-  if (threadIdx.x < ntok) {
-    const int a = threadIdx.x;
+  if (tid < ntok) {
+    const int a = tid;
     const int64_t t = t0 + a;
     uint64_t used = 0;
     float top = 0.f, z = 0.f;
@@ -153,15 +158,251 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
       val[k] = bv;
       if (k == 0) top = bv;
       z += expf(bv - top);
-      atomicAdd(&hist[best], 1);
+      if (hist) atomicAdd(&hist[best], 1);
     }
     for (int k = 0; k < K; ++k) {
       idx[t * K + k] = sel[k];
       gate[t * K + k] = expf(val[k] - top) / z;
     }
   }
+  sync();
+}
+
+// Block b routes tokens [b*TOKB, b*TOKB + TOKB) and writes its expert histogram.
+template <typename Tin, int NPAD, int TOKB>
+__global__ void __launch_bounds__(ROUTE_THREADS)
+    router_topk_kernel(const Tin* __restrict__ x, const float* __restrict__ Wg, int64_t T,
+                       int d, int n, int K, int32_t* __restrict__ idx,
+                       float* __restrict__ gate, int32_t* __restrict__ blk_counts) {
+  __shared__ float red[ROUTE_THREADS / 32][64];
+  __shared__ float logits[TOKB][NPAD];
+  __shared__ int hist[64];
+  const int64_t t0 = (int64_t)blockIdx.x * TOKB;
+  const int ntok = (int)(T - t0 < TOKB ? T - t0 : TOKB);
+  if (threadIdx.x < 64) hist[threadIdx.x] = 0;
   __syncthreads();
+  route_token_block<Tin, NPAD, TOKB>(x, Wg, t0, ntok, d, n, K, threadIdx.x, red, logits, hist,
+                                     idx, gate, CtaSync{});
   if (threadIdx.x < n) blk_counts[(int64_t)blockIdx.x * n + threadIdx.x] = hist[threadIdx.x];
+}
+
+// Copy the x rows of `E` entries (entry i = (token t0 + i / K, slot i % K)) to their
+// permuted rows (row[i] < 0: skip).  One warp per row, 16-byte vectors, U loads in flight per
+// lane before the stores; no per-vector index arithmetic beyond the lane stride.
+template <typename Tact>
+__device__ __forceinline__ void gather_rows(const Tact* __restrict__ x, int64_t t0, int d, int K,
+                                            int E, const int* row, Tact* __restrict__ xperm,
+                                            int tid, int nthreads) {
+  constexpr int U = 8;
+  const int lane = tid & 31, nwarps = nthreads >> 5;
+  const int vpr = d * (int)sizeof(Tact) / 16;
+  for (int i = tid >> 5; i < E; i += nwarps) {
+    const int r = row[i];
+    if (r < 0) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (t0 + i / K) * d);
+    uint4* dst = reinterpret_cast<uint4*>(xperm + (int64_t)r * d);
+    for (int c0 = lane; c0 < vpr; c0 += 32 * U) {
+      uint4 buf[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + 32 * u < vpr) buf[u] = __ldg(src + c0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + 32 * u < vpr) dst[c0 + 32 * u] = buf[u];
+    }
+  }
+}
+
+// Small batches (T <= 64, T*K <= 1024) in ONE launch of G = ceil(d / 64) CTAs of 1024 threads.
+// CTA c owns hidden elements [64c, 64c + 64): 8 lanes per token each take one 8-element chunk, sum
+// their products with W_g and reduce over the 8 lanes in a fixed butterfly order; the CTA
+// writes partial logits [c][t][e].  The last CTA to finish (ticket counter, wrapped by
+// atomicInc so it is back at 0 for the next call) sums the partials in CTA order, then does
+// TopK and softmax, the expert counts, group offsets (padded to row_align), the stable rank
+// of every (token, slot) (per-warp match + per-expert prefix over 32-entry chunks), the
+// inverse map token -> row, the map row -> token, and (if xperm is given) the gather of x
+// rows.
+constexpr int RS_THREADS = 1024;
+constexpr int RS_MAX_T = 64;
+constexpr int RS_MAX_ENTRIES = 1024;
+
+template <typename Tact>
+__global__ void __launch_bounds__(RS_THREADS)
+    route_split_kernel(const Tact* __restrict__ x, const float* __restrict__ Wg, int T, int d,
+                       int n, int K, int row_align, int64_t rows_max,
+                       float* __restrict__ part, unsigned int* ticket,
+                       int32_t* __restrict__ idx, float* __restrict__ gate,
+                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                       int32_t* __restrict__ inv, int32_t* __restrict__ row_tok,
+                       Tact* __restrict__ xperm, uint32_t* status) {
+  constexpr int PER = RS_MAX_ENTRIES / RS_THREADS;  // entries per thread in the rank phase
+  constexpr int CPL = 1;                            // 8-element chunks per lane
+  __shared__ float logit[RS_MAX_T * MAX_EXPERTS];
+  __shared__ int ccnt[RS_MAX_ENTRIES / 32][MAX_EXPERTS];  // per (32-entry chunk, expert)
+  __shared__ int s_off[MAX_EXPERTS + 1];
+  __shared__ int s_row[RS_MAX_ENTRIES];
+  __shared__ int s_idx[RS_MAX_ENTRIES];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x, c = blockIdx.x;
+
+  // ---- partial logits of this CTA's 64 hidden elements
+  const int sub = lane & 7;
+  for (int tb = warp * 4; tb < T; tb += (RS_THREADS / 32) * 4) {
+    const int t = tb + (lane >> 3);
+    Vec8<Tact> xv[CPL];
+    int j0[CPL];
+#pragma unroll
+    for (int q = 0; q < CPL; ++q) {
+      j0[q] = (c * 8 * CPL + q * 8 + sub) * 8;
+      if (t < T && j0[q] < d) xv[q].load(x + (int64_t)t * d + j0[q]);
+    }
+    for (int eg = 0; eg < n; eg += 8) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < CPL; ++q) {
+        if (t >= T || j0[q] >= d) continue;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float xi = xv[q].get(i);
+          const float* wr = Wg + (int64_t)(j0[q] + i) * n + eg;
+          if (n == 8) {
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr));
+            const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr) + 1);
+            acc[0] = fmaf(xi, w0.x, acc[0]); acc[1] = fmaf(xi, w0.y, acc[1]);
+            acc[2] = fmaf(xi, w0.z, acc[2]); acc[3] = fmaf(xi, w0.w, acc[3]);
+            acc[4] = fmaf(xi, w1.x, acc[4]); acc[5] = fmaf(xi, w1.y, acc[5]);
+            acc[6] = fmaf(xi, w1.z, acc[6]); acc[7] = fmaf(xi, w1.w, acc[7]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (eg + e < n) acc[e] = fmaf(xi, __ldg(wr + e), acc[e]);
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+      if (sub == 0 && t < T) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (eg + e < n) part[((int64_t)c * T + t) * n + eg + e] = acc[e];
+      }
+    }
+  }
+
+  // ---- the last CTA to finish does the rest
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicInc(ticket, (unsigned)G - 1u) == (unsigned)G - 1u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int i = tid; i < RS_MAX_ENTRIES / 32 * MAX_EXPERTS; i += RS_THREADS) (&ccnt[0][0])[i] = 0;
+  // logit (t, e) = sum over CTAs of the partials: 8 threads per logit each sum every 8th CTA
+  // in order, then a fixed xor-butterfly over the 8 (one round of loads, deterministic)
+  for (int v0 = 0; v0 < T * n; v0 += RS_THREADS / 8) {
+    const int v = v0 + (tid >> 3), sub8 = tid & 7;
+    float sum = 0.f;
+    if (v < T * n) {
+      float pv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int cc = sub8 + 8 * u;
+        pv[u] = cc < G ? __ldcg(part + (int64_t)cc * T * n + v) : 0.f;
+      }
+      for (int cc0 = 64; cc0 < G; cc0 += 8)  // G > 64 (d > 4096): remaining CTAs
+        if (cc0 + sub8 < G) pv[7] += __ldcg(part + (int64_t)(cc0 + sub8) * T * n + v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += pv[u];
+    }
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (v < T * n && sub8 == 0) logit[v] = sum;
+  }
+  __syncthreads();
+  if (tid < T) {  // TopK by repeated arg-max (ties -> lower index), softmax over the kept;
+                  // the selection is run twice (normaliser, then output) to stay in registers
+    const float* l = logit + tid * n;
+    float top = 0.f, z = 0.f;
+    for (int pass = 0; pass < 2; ++pass) {
+      uint64_t used = 0;
+      for (int k = 0; k < K; ++k) {
+        int best = -1;
+        float bv = 0.f;
+        for (int e = 0; e < n; ++e) {
+          if ((used >> e) & 1ull) continue;
+          if (best < 0 || l[e] > bv) { best = e; bv = l[e]; }
+        }
+        used |= 1ull << best;
+        if (pass == 0) {
+          if (k == 0) top = bv;
+          z += expf(bv - top);
+        } else {
+          idx[tid * K + k] = best;
+          s_idx[tid * K + k] = best;
+          gate[tid * K + k] = expf(bv - top) / z;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int E = T * K;
+  int e_i[PER], rank_c[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {  // entry i = j*256 + tid lies in chunk i/32 = j*8 + warp
+    const int i = j * RS_THREADS + tid;
+    e_i[j] = i < E ? s_idx[i] : -1;
+    const unsigned vmask = __ballot_sync(0xffffffffu, e_i[j] >= 0);
+    const unsigned peers = __match_any_sync(0xffffffffu, e_i[j]) & vmask;
+    rank_c[j] = __popc(peers & ((1u << lane) - 1u));
+    if (e_i[j] >= 0 && rank_c[j] == 0)
+      ccnt[j * (RS_THREADS / 32) + warp][e_i[j]] = __popc(peers);
+  }
+  __syncthreads();
+  for (int e = warp; e < n; e += RS_THREADS / 32) {  // expert e: prefix over the 32 chunks
+    const int v = ccnt[lane][e];
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    ccnt[lane][e] = incl - v;
+    if (lane == 31) s_off[e] = incl;  // total for now
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int64_t off = 0;
+    for (int e = 0; e < n; ++e) {
+      const int cnt = s_off[e];
+      counts[e] = cnt;
+      s_off[e] = (int)off;
+      offsets[e] = (int)off;
+      off += (int64_t)(cnt + row_align - 1) / row_align * row_align;
+    }
+    s_off[n] = (int)off;
+    offsets[n] = (int)off;
+    if (off > rows_max) set_status(status, DEV_ERR_ROW);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    const int i = j * RS_THREADS + tid;
+    if (i >= E) continue;
+    int row = s_off[e_i[j]] + ccnt[j * (RS_THREADS / 32) + warp][e_i[j]] + rank_c[j];
+    if (row >= rows_max) {
+      set_status(status, DEV_ERR_ROW);
+      row = -1;
+    }
+    s_row[i] = row;
+    inv[i] = row;
+    if (row >= 0) row_tok[row] = i / K;
+  }
+  if (xperm == nullptr) return;  // the GEMM loads token rows straight from x
+  __syncthreads();
+  gather_rows(x, 0, d, K, E, s_row, xperm, tid, RS_THREADS);
 }
 
 // One CTA: for every expert, exclusive prefix of the block histograms over blocks, the
@@ -255,16 +496,7 @@ __global__ void __launch_bounds__(256)
     inv[t0 * K + i] = row;
   }
   __syncthreads();
-  // gather: 16-byte vectors of each selected x row into its permuted row
-  const int vpr = d * (int)sizeof(Tact) / 16;
-  for (int v = threadIdx.x; v < E * vpr; v += blockDim.x) {
-    const int ei = v / vpr, c = v % vpr;
-    const int row = ent_row[ei];
-    if (row < 0) continue;
-    const int64_t t = t0 + ei / K;
-    const uint4 val = __ldg(reinterpret_cast<const uint4*>(x + t * d) + c);
-    reinterpret_cast<uint4*>(xperm + (int64_t)row * d)[c] = val;
-  }
+  gather_rows(x, t0, d, K, E, ent_row, xperm, threadIdx.x, blockDim.x);
 }
 
 // ---------------------------------------------------------------- host launchers
@@ -292,8 +524,22 @@ static cudaError_t launch_router_t(const Tin* x, const float* Wg, int64_t T, int
   return cudaGetLastError();
 }
 
+template <typename Tact>
+static cudaError_t launch_route_small_t(const Plan& p, const Tact* x, const float* Wg,
+                                        const Workspace& w, cudaStream_t s) {
+  const int G = (int)((p.d + 63) / 64);
+  route_split_kernel<Tact><<<G, RS_THREADS, 0, s>>>(
+      x, Wg, (int)p.T, (int)p.d, p.n, p.K, p.row_align, p.rows_max, w.rpart, w.ticket, w.idx,
+      w.gate, w.counts, w.offsets, w.inv, w.row_tok,
+      static_cast<Tact*>(w.xperm), w.status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Workspace& w,
                          cudaStream_t s) {
+  if (p.fused_route)
+    return p.dt == 1 ? launch_route_small_t(p, static_cast<const __nv_bfloat16*>(x), Wg, w, s)
+                     : launch_route_small_t(p, static_cast<const float*>(x), Wg, w, s);
   cudaError_t err;
   if (p.dt == 1)
     err = launch_router_t(static_cast<const __nv_bfloat16*>(x), Wg, p.T, (int)p.d, p.n, p.K,
