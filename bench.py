@@ -129,6 +129,20 @@ class ClockSampler:
                 "samples": len(self.rows)}
 
 
+def replica_workload(w, rank: int):
+    """Each rank's independent replica: its own seeded batch and weights."""
+    return w.replace(seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings (identity on one rank)."""
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def _flops_per_token(w):
     # routed work: 2 FLOPs per multiply-add; K experts x 3 d-by-F matrices + router d*n
     return w.K * 3 * 2 * w.d * w.F + 2 * w.d * w.n
@@ -147,9 +161,10 @@ def run_gpu(args, w):
                                 timeout=__import__("datetime").timedelta(seconds=300))
     peaks = _peaks()
     # per-rank replica: its own batch (seed offset by rank), its own copy of the weights
-    wr = w.replace(seed=w.seed + 7919 * rank)
+    wr = replica_workload(w, rank)
     x = moe_inputs.make_x(wr, device=dev)
-    layer = moe_inputs.make_layer(wr, device=dev)
+    layers = [moe_inputs.make_layer(wr, layer=l, device=dev) for l in range(w.layers)]
+    layer = layers[0]
     stream = torch.cuda.Stream(device=dev)
     ws = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K, torch.bfloat16),
                              dev, stream)
@@ -157,10 +172,21 @@ def run_gpu(args, w):
     plan = moe.moe_plan_info(w.T, w.d, w.F, w.n, w.K)
     small_batch, s13, s2, launches = (plan["small_batch"], plan["split13"], plan["split2"],
                                       plan["launches"])
+    stacked = w.layers > 1
+    if stacked:  # x is the residual stream: every step restarts from the same input
+        ws_stack = moe.alloc_workspace(
+            moe.moe_stack_workspace_bytes(w.T, w.d, w.F, w.n, w.K), dev, stream)
+        xs = torch.empty_like(x)
+        launches = w.layers * (1 + launches) + 1  # RMSNorm per block, the restart copy
 
     def step():
-        moe.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.K, out=out,
-                        workspace=ws, stream=stream)
+        if stacked:
+            with torch.cuda.stream(stream):
+                xs.copy_(x, non_blocking=True)
+            moe.moe_stack_forward(xs, layers, w.K, workspace=ws_stack, stream=stream)
+        else:
+            moe.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.K, out=out,
+                            workspace=ws, stream=stream)
 
     def barrier():
         if world > 1:
@@ -202,14 +228,24 @@ def run_gpu(args, w):
         xh = x.cpu().pin_memory()
         oh = torch.empty_like(xh).pin_memory()
         xd, od = torch.empty_like(x), torch.empty_like(x)
+
+        def e2e_step():
+            if stacked:  # host -> device, the 32-block stack in place, device -> host
+                with torch.cuda.stream(stream):
+                    xd.copy_(xh, non_blocking=True)
+                moe.moe_stack_forward(xd, layers, w.K, workspace=ws_stack, stream=stream)
+                with torch.cuda.stream(stream):
+                    oh.copy_(xd, non_blocking=True)
+            else:
+                moe.moe_forward_host_io(xh, xd, layer["Wg"], layer["W1"], layer["W3"],
+                                        layer["W2"], w.K, od, oh, ws, stream=stream)
+
         for _ in range(max(1, args.warmup)):
-            moe.moe_forward_host_io(xh, xd, layer["Wg"], layer["W1"], layer["W3"], layer["W2"],
-                                    w.K, od, oh, ws, stream=stream)
+            e2e_step()
         barrier()
         ev0.record(stream)
         for _ in range(args.steps):
-            moe.moe_forward_host_io(xh, xd, layer["Wg"], layer["W1"], layer["W3"], layer["W2"],
-                                    w.K, od, oh, ws, stream=stream)
+            e2e_step()
             stream.synchronize()
         ev1.record(stream)
         barrier()
@@ -218,11 +254,7 @@ def run_gpu(args, w):
     if code != 0:
         raise RuntimeError(f"device status {code} ({raw:#x})")
 
-    # max over ranks
-    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms = t.tolist()
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -230,7 +262,7 @@ def run_gpu(args, w):
 
     ms_step = ms / args.steps
     tok_s = world * w.T * args.steps / (ms / 1e3)
-    tflops = tok_s * _flops_per_token(w) / 1e12
+    tflops = tok_s * w.layers * _flops_per_token(w) / 1e12
     g13 = statistics.mean(s[1] for s in stage_ms)          # gate/up GEMM (dominant kernel)
     stage_avg = [statistics.mean(s[j] for s in stage_ms) for j in range(5)]
     es = 2
@@ -257,9 +289,11 @@ def run_gpu(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations, RMS-normalised; N(0,1/fan_in) weights)",
-        "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K} bf16",
+        "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K} bf16"
+                               + (f", {w.layers} x (RMSNorm -> MoE -> residual)" if stacked
+                                  else ""),
                    "tokens_per_rank": w.T, "l2": "inputs larger than L2 "
-                   f"({3 * w.n * w.F * w.d * es / 1e9:.2f} GB of expert weights)",
+                   f"({w.layers * 3 * w.n * w.F * w.d * es / 1e9:.2f} GB of expert weights)",
                    "parallelism": f"replicas x{world}", "tiling": "small-batch swap-AB "
                    f"split-K {s13}/{s2}" if small_batch else "prefill 128-row tiles",
                    "active_experts": n_active, "expert_counts": counts},
@@ -285,6 +319,7 @@ def run_gpu(args, w):
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, x.cpu(), {k: v.cpu() for k, v in layer.items()},
                                             args.cpu_tokens)
+    del layers
     print(json.dumps(line), flush=True)
     return line
 
@@ -299,9 +334,12 @@ def cpu_baseline(w, x, layer, ntok):
     oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
                        tokens=toks)
     dt = time.perf_counter() - t0
-    return {"value": round(ntok / dt, 4), "unit": "tokens/s", "cores": _omp_threads(),
-            "kind": "oracle", "sample": f"{ntok} of {w.T} tokens of {w.name}, "
-                                        f"{dt:.1f} s (fp64 C, OpenMP over tokens)"}
+    per_block = f", one of the {w.layers} blocks (rate divided by {w.layers})" \
+        if w.layers > 1 else ""
+    return {"value": round(ntok / dt / w.layers, 4), "unit": "tokens/s",
+            "cores": _omp_threads(), "kind": "oracle",
+            "sample": f"{ntok} of {w.T} tokens of {w.name}{per_block}, "
+                      f"{dt:.1f} s (fp64 C, OpenMP over tokens)"}
 
 
 def _omp_threads():
@@ -330,9 +368,10 @@ def run_reference(args, w):
         oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
                            tokens=toks)
     dt = time.perf_counter() - t0
-    v = per_step * args.steps / dt
+    v = per_step * args.steps / dt / w.layers
     sample = (f"{per_step} of {w.T} tokens of {w.name} per step "
-              "(fp64 C oracle, OpenMP over tokens)")
+              "(fp64 C oracle, OpenMP over tokens)"
+              + (f"; one block, rate divided by {w.layers} blocks" if w.layers > 1 else ""))
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
@@ -360,8 +399,8 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = moe_inputs.WORKLOADS[args.workload]
-    if w.layers > 1 or w.dtype != "bf16":
-        ap.error("the bench measures single bf16 blocks")
+    if w.dtype != "bf16":
+        ap.error("the bench measures the bf16 path")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)
