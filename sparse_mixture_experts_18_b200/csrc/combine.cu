@@ -121,8 +121,8 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
   const int S = p.swap ? p.s2 : 1;
   const int64_t split_stride = p.rows_max * p.d;
   const int64_t total = p.T * (p.d / 4);
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
+  int64_t blocks = (total + 255) / 256;  // one 4-column item per thread: all loads in flight
+  if (blocks > ((int64_t)1 << 30)) blocks = (int64_t)1 << 30;
   if (blocks < 1) blocks = 1;
   if (p.dt == 1) {
     auto* o = static_cast<__nv_bfloat16*>(out);

@@ -275,8 +275,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             }
             uint4* dst = reinterpret_cast<uint4*>(h + col);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < 4; ++i)  // streaming: keep L2 for the weight and X tiles
+              __stcs(dst + i, make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
           }
         }
       } else if (!SWAP && KIND == KIND_G2) {
@@ -291,8 +291,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             float4* dst = reinterpret_cast<float4*>(y + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+              __stcs(dst + i, make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                          __uint_as_float(v[4 * i + 2]),
+                                          __uint_as_float(v[4 * i + 3])));
           }
         }
       } else {
@@ -327,6 +328,236 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, a.tmem_cols);
+}
+
+// ---------------------------------------------------------------- CTA-pair prefill tiling
+// Tile = 256 permuted rows x 256 MMA columns computed by a cluster of two CTAs with
+// tcgen05.mma.cta_group::2 (M = 256).  CTA r holds its 128 rows of A and half of the N = 256
+// operand -- G13: W1 rows (r = 0) or the same W3 rows (r = 1); G2: W2 rows [128r, 128r + 128)
+// of the column tile -- so each CTA stages 32 KB per 64-wide K block instead of 48 KB, and
+// twice as many K blocks are in flight.  The even CTA (leader) issues every MMA; both CTAs'
+// TMA loads complete on the leader's full barrier; the leader's commits arrive on both CTAs'
+// empty and accumulator-full barriers; both epilogues release accumulators on the leader's
+// barrier.  Expert groups are padded to 256 rows on this path.
+constexpr int PAIR_ROWS = 256;
+
+struct PairCtrl {
+  uint64_t full[MAX_STAGES];   // leader: the stage's bytes of both CTAs have landed
+  uint64_t empty[MAX_STAGES];  // each CTA: its stage may be refilled
+  uint64_t tfull[2];           // each CTA: accumulator complete
+  uint64_t tempty[2];          // leader: both epilogues drained the accumulator (256 threads)
+  uint64_t peer_done;          // each CTA: the peer CTA is finished with TMEM
+  uint32_t tmem_slot;
+  int abort;
+  int off[MAX_EXPERTS + 1];
+};
+
+__device__ __forceinline__ Work decode_pair_work(const TcArgs& a, const int* off, int id) {
+  Work w{};
+  int e = 0;
+  while (e + 1 < a.n && id >= (off[e + 1] / PAIR_ROWS) * a.n_tiles) ++e;
+  const int mt0 = off[e] / PAIR_ROWS;
+  const int mcnt = off[e + 1] / PAIR_ROWS - mt0;
+  const int local = id - mt0 * a.n_tiles;
+  w.e = e;
+  w.nt = local / mcnt;
+  w.mt = mt0 + local % mcnt;  // 256-row tile index
+  return w;
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
+                        const __grid_constant__ CUtensorMap tmW0,
+                        const __grid_constant__ CUtensorMap tmW1, const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  PairCtrl* c = reinterpret_cast<PairCtrl*>(smem + (size_t)a.stages * a.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&c->full[s], 1);
+      mbar_init(&c->empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&c->tfull[i], 1);
+      mbar_init(&c->tempty[i], 256);
+    }
+    mbar_init(&c->peer_done, 1);
+    c->abort = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW0);
+    if (KIND == KIND_G13) tma_prefetch_desc(&tmW1);
+  }
+  if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc_pair(&c->tmem_slot, a.tmem_cols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barrier initialisation and the TMEM allocation, in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = c->tmem_slot;
+  const int total = (c->off[a.n] / PAIR_ROWS) * a.n_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_normal();
+      const uint64_t pol_x = policy_evict_last();
+      const uint32_t full0 = map_to_rank(&c->full[0], 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int id = pair; id < total && ok; id += npairs) {
+        const Work w = decode_pair_work(a, c->off, id);
+        const int row = w.mt * PAIR_ROWS + (int)rank * 128;
+        for (int kb = 0; kb < a.num_kb; ++kb) {
+          if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort)) { ok = false; break; }
+          uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+          if (leader) mbar_arrive_expect_tx(&c->full[stage], 2 * a.tx_bytes);
+          const uint32_t fb = full0 + (uint32_t)stage * 8u;
+          const int k = kb * 64;
+          tma_load_2d_pair(st, &tmX, fb, k, row, pol_x);
+          if (KIND == KIND_G13)
+            tma_load_2d_pair(st + TILE_BYTES, rank == 0 ? &tmW0 : &tmW1, fb, k,
+                             w.e * a.nw + w.nt * 128, pol_w);
+          else
+            tma_load_2d_pair(st + TILE_BYTES, &tmW0, fb, k,
+                             w.e * a.nw + w.nt * 256 + (int)rank * 128, pol_w);
+          if (++stage == a.stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // every MMA commit aimed at this CTA's empty barriers has landed before it may exit
+      for (int s = 0; ok && s < a.stages; ++s) {
+        if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort)) break;
+        if (++stage == a.stages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      const uint32_t idesc = umma_idesc_bf16(256, 256);
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int id = pair; id < total && ok; id += npairs, ++it) {
+        const uint32_t acc = (uint32_t)it % a.nacc;
+        const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
+        if (!mbar_wait(&c->tempty[acc], aph ^ 1u, a.status, &c->abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dtm = tmem_base + acc * a.acc_cols;
+        for (int kb = 0; kb < a.num_kb; ++kb) {
+          if (!mbar_wait(&c->full[stage], phase, a.status, &c->abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(smem + (size_t)stage * a.stage_bytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t kofs = kk * 32;
+            umma_bf16_pair(dtm, umma_desc_k128(sb + kofs), umma_desc_k128(sb + TILE_BYTES + kofs),
+                           idesc, (kb | kk) != 0);
+          }
+          umma_commit_pair(&c->empty[stage], 0x3);
+          if (++stage == a.stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&c->tfull[acc], 0x3);
+      }
+      // both epilogues have released every accumulator before TMEM is torn down
+      for (uint32_t j = 0; ok && j < a.nacc; ++j, ++it) {
+        const uint32_t acc = (uint32_t)it % a.nacc;
+        const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
+        if (!mbar_wait(&c->tempty[acc], aph ^ 1u, a.status, &c->abort)) break;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t tempty0 = map_to_rank(&c->tempty[0], 0);
+    int it = 0;
+    for (int id = pair; id < total; id += npairs, ++it) {
+      const Work w = decode_pair_work(a, c->off, id);
+      const uint32_t acc = (uint32_t)it % a.nacc;
+      const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
+      const bool ok = mbar_wait(&c->tfull[acc], aph, a.status, &c->abort);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * a.acc_cols;
+      const int64_t row = (int64_t)w.mt * PAIR_ROWS + rank * 128 + r;
+      if (KIND == KIND_G13) {
+        __nv_bfloat16* h = static_cast<__nv_bfloat16*>(a.out) + row * a.out_ld;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t va[32], vb[32];
+          tmem_ld32(tb + cc * 32, va);
+          tmem_ld32(tb + 128 + cc * 32, vb);
+          tmem_ld_wait();
+          const int col = w.nt * 128 + cc * 32;
+          if (col < a.nw) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu(__uint_as_float(va[2 * i])) * __uint_as_float(vb[2 * i]);
+              const float h1 =
+                  silu(__uint_as_float(va[2 * i + 1])) * __uint_as_float(vb[2 * i + 1]);
+              pk[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(h + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)  // streaming: keep L2 for the weight and X tiles
+              __stcs(dst + i, make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+          }
+        }
+      } else {
+        float* y = static_cast<float*>(a.out) + row * a.out_ld;
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tb + cc * 32, v);
+          tmem_ld_wait();
+          const int col = w.nt * 256 + cc * 32;
+          if (col < a.nw) {
+            float4* dst = reinterpret_cast<float4*>(y + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              __stcs(dst + i, make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                          __uint_as_float(v[4 * i + 2]),
+                                          __uint_as_float(v[4 * i + 3])));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(tempty0 + acc * 8u);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {  // both CTAs are done with TMEM before the pair deallocates it
+    if (lane == 0) {
+      mbar_arrive_cluster(map_to_rank(&c->peer_done, rank ^ 1u));
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&c->peer_done, 0))
+        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+          set_status(a.status, DEV_ERR_TIMEOUT);
+          break;
+        }
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, a.tmem_cols);
+  }
 }
 
 // Small batch: h = bf16(silu(sum_s A_s) * sum_s B_s), splits summed in order 0..S-1.  All
@@ -420,6 +651,44 @@ static cudaError_t launch_one(const CUtensorMap& mx, const CUtensorMap& mw0,
   return cudaGetLastError();
 }
 
+template <int KIND>
+static cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw0,
+                               const CUtensorMap& mw1, TcArgs a, int max_work, cudaStream_t s) {
+  const size_t smem = (size_t)a.stages * a.stage_bytes + sizeof(PairCtrl) + 1024;
+  auto kern = tc_pair_gemm_kernel<KIND>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int pairs_fit[64] = {0};  // co-resident clusters per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!pairs_fit[dev]) {
+    int nclusters = 0;
+    cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters < 1)
+      nclusters = num_sms() / 2;
+    pairs_fit[dev] = nclusters;
+  }
+  int pairs = max_work < pairs_fit[dev] ? max_work : pairs_fit[dev];
+  if (pairs < 1) pairs = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  e = cudaLaunchKernelEx(&cfg, kern, mx, mw0, mw1, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 static int stages_for(uint32_t stage_bytes) {
   int st = (int)(SMEM_STAGE_BUDGET / stage_bytes);
   return st > MAX_STAGES ? MAX_STAGES : st;
@@ -441,6 +710,44 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   CUtensorMap mX, mW1, mW3, mH, mW2;
   const int d = (int)p.d, F = (int)p.F, n = p.n;
   cudaError_t err;
+  if (p.pair) {  // 256-row tiles on CTA pairs
+    if (!make_map(&mX, w.xperm, d, p.rows_max, 128) ||
+        !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||
+        !make_map(&mW3, W3, d, (uint64_t)n * F, 128) ||
+        !make_map(&mH, w.h, F, p.rows_max, 128) ||
+        !make_map(&mW2, W2, F, (uint64_t)n * d, 128))
+      return cudaErrorInvalidValue;
+    const int pair_tiles_max = (int)(p.rows_max / 256);
+    TcArgs a{};
+    a.offsets = w.offsets;
+    a.n = n;
+    a.stage_bytes = 2 * TILE_BYTES;
+    a.tx_bytes = 2 * TILE_BYTES;  // per CTA; the leader expects both CTAs' bytes
+    a.stages = stages_for(a.stage_bytes);
+    a.acc_cols = 256;
+    a.nacc = 2;
+    a.tmem_cols = 512;
+    a.status = w.status;
+    a.num_kb = d / 64;
+    a.nw = F;
+    a.n_tiles = (F + 127) / 128;
+    a.out = w.h;
+    a.out_ld = F;
+    if ((err = launch_pair<KIND_G13>(mX, mW1, mW3, a, pair_tiles_max * a.n_tiles, s)) !=
+        cudaSuccess)
+      return err;
+    if ((err = record(ev, 0, s)) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
+      return err;
+    a.num_kb = F / 64;
+    a.nw = d;
+    a.n_tiles = (d + 255) / 256;
+    a.out = w.y;
+    a.out_ld = d;
+    if ((err = launch_pair<KIND_G2>(mH, mW2, mW2, a, pair_tiles_max * a.n_tiles, s)) !=
+        cudaSuccess)
+      return err;
+    return record(ev, 2, s);
+  }
   if (!p.swap) {
     if (!make_map(&mX, w.xperm, d, p.rows_max, 128) ||
         !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||

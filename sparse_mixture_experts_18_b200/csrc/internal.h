@@ -21,6 +21,7 @@ struct Plan {
   int n = 0, K = 0;
   int dt = 1;              // 0 = fp32 (SIMT path), 1 = bf16 (tensor-core path)
   bool swap = false;       // small-batch path: weights are the MMA's 128-row operand
+  bool pair = false;       // large batches: 256-row tiles on 2-CTA clusters (cta_group::2)
   int row_align = 1;       // each expert's group is padded to a multiple of this
   int64_t rows_max = 0;    // upper bound of permuted rows (T*K plus padding)
   int64_t nblk = 0;        // router / permute blocks

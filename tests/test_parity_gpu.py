@@ -64,6 +64,14 @@ def test_prefill_tiling_small(T, d, F):
     _run(moe_inputs.small(T=T, d=d, F=F))
 
 
+@pytest.mark.parametrize("T,d,F,n,K", [(3000, 256, 384, 8, 2), (2700, 320, 448, 8, 2),
+                                       (2600, 256, 256, 4, 1), (5200, 128, 256, 16, 2)])
+def test_pair_tiling_small(T, d, F, n, K):
+    # T*K >= 640*n: 256-row tiles on CTA pairs (cta_group::2); ragged d and F tails
+    assert moe.moe_plan_info(T, d, F, n, K)["small_batch"] is False
+    _run(moe_inputs.small(T=T, d=d, F=F, n=n, K=K))
+
+
 @pytest.mark.parametrize("T", [1, 5, 16, 37, 100, 255])
 def test_small_batch_tiling(T):
     # T <= 256 and T*K < 64*n: weights as the 128-row MMA operand, split-K
