@@ -73,7 +73,8 @@ MOE_API moe_status moe_workspace_init(void* workspace, size_t workspace_bytes, v
 /* Synchronise `stream`, then read and clear the workspace status word written by kernels.
  * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded wait ran out), MOE_ERR_DEVICE (an index out
  * of range) or MOE_ERR_CUDA (the stream reported an error).  *raw (may be NULL) receives
- * the raw bit mask. */
+ * the raw bit mask.  After any error, call moe_workspace_init() again before reusing the
+ * workspace (an interrupted call can leave its counters mid-count). */
 MOE_API moe_status moe_workspace_status(void* workspace, void* stream, uint32_t* raw);
 
 /* One MoE block forward:  out[t] = sum_k G(x_t)_k * SwiGLU_{e_k}(x_t).

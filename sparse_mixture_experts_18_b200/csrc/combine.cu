@@ -116,10 +116,97 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Large batches: one warp per token, each lane 8 groups of 4 columns (128 columns apart)
+// per pass, with all of a slot's loads in flight before they are summed.  Same arithmetic
+// (split order, then slot order, one rounding) as combine_kernel.
+constexpr int COMBINE_U = 8;
+
+template <typename Tout, bool RESID>
+__global__ void __launch_bounds__(256)
+    combine_rows_kernel(const float* __restrict__ Y, int S, int64_t split_stride, int64_t T,
+                        int d, int K, const int32_t* __restrict__ inv,
+                        const float* __restrict__ gate, Tout* out, const Tout* resid) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
+       t += nwarps) {
+    for (int c0 = lane * 4; c0 < d; c0 += 128 * COMBINE_U) {
+      float4 acc[COMBINE_U];
+#pragma unroll
+      for (int u = 0; u < COMBINE_U; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < K; ++k) {
+        const int row = inv[t * K + k];
+        if (row < 0) continue;
+        const float g = gate[t * K + k];
+        float4 yk[COMBINE_U];
+#pragma unroll
+        for (int u = 0; u < COMBINE_U; ++u) yk[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < S; ++s) {
+          const float* src = Y + s * split_stride + (int64_t)row * d + c0;
+          float4 v[COMBINE_U];
+#pragma unroll
+          for (int u = 0; u < COMBINE_U; ++u)
+            if (c0 + 128 * u < d) v[u] = __ldg(reinterpret_cast<const float4*>(src + 128 * u));
+#pragma unroll
+          for (int u = 0; u < COMBINE_U; ++u)
+            if (c0 + 128 * u < d) {
+              yk[u].x += v[u].x; yk[u].y += v[u].y; yk[u].z += v[u].z; yk[u].w += v[u].w;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < COMBINE_U; ++u) {
+          acc[u].x = fmaf(g, yk[u].x, acc[u].x);
+          acc[u].y = fmaf(g, yk[u].y, acc[u].y);
+          acc[u].z = fmaf(g, yk[u].z, acc[u].z);
+          acc[u].w = fmaf(g, yk[u].w, acc[u].w);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < COMBINE_U; ++u) {
+        const int c = c0 + 128 * u;
+        if (c >= d) continue;
+        float o[4] = {acc[u].x, acc[u].y, acc[u].z, acc[u].w};
+        if (RESID) {
+          float r[4];
+          Out4<Tout>::load(resid + t * d + c, r);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[i] = r[i] + o[i];
+        }
+        Out4<Tout>::store(out + t * d + c, o);
+      }
+    }
+  }
+}
+
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
                            cudaStream_t s) {
   const int S = p.swap ? p.s2 : 1;
   const int64_t split_stride = p.rows_max * p.d;
+  if (p.T >= 1024) {  // enough tokens for one warp each
+    const int64_t blocks = (p.T + 7) / 8;
+    const unsigned g = (unsigned)(blocks < ((int64_t)1 << 30) ? blocks : ((int64_t)1 << 30));
+    if (p.dt == 1) {
+      auto* o = static_cast<__nv_bfloat16*>(out);
+      if (resid)
+        combine_rows_kernel<__nv_bfloat16, true><<<g, 256, 0, s>>>(
+            w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
+            static_cast<const __nv_bfloat16*>(resid));
+      else
+        combine_rows_kernel<__nv_bfloat16, false><<<g, 256, 0, s>>>(
+            w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
+    } else {
+      auto* o = static_cast<float*>(out);
+      if (resid)
+        combine_rows_kernel<float, true><<<g, 256, 0, s>>>(w.y, S, split_stride, p.T, (int)p.d,
+                                                           p.K, w.inv, w.gate, o,
+                                                           static_cast<const float*>(resid));
+      else
+        combine_rows_kernel<float, false><<<g, 256, 0, s>>>(w.y, S, split_stride, p.T,
+                                                            (int)p.d, p.K, w.inv, w.gate, o,
+                                                            nullptr);
+    }
+    return cudaGetLastError();
+  }
   const int64_t total = p.T * (p.d / 4);
   int64_t blocks = (total + 255) / 256;  // one 4-column item per thread: all loads in flight
   if (blocks > ((int64_t)1 << 30)) blocks = (int64_t)1 << 30;

@@ -137,32 +137,32 @@ __device__ __forceinline__ void route_token_block(
   sync();
 
   // TopK by repeated arg-max (strict '>' keeps the lower index on ties), then Softmax over
-  // the kept logits shifted by the largest.
+  // the kept logits shifted by the largest; the selection runs twice (normaliser, then
+  // output) so that nothing is kept in per-thread arrays.
   if (tid < ntok) {
     const int a = tid;
     const int64_t t = t0 + a;
-    uint64_t used = 0;
     float top = 0.f, z = 0.f;
-    int sel[64];
-    float val[64];
-    for (int k = 0; k < K; ++k) {
-      int best = -1;
-      float bv = 0.f;
-      for (int e = 0; e < n; ++e) {
-        if ((used >> e) & 1ull) continue;
-        const float le = logits[a][e];
-        if (best < 0 || le > bv) { best = e; bv = le; }
+    for (int pass = 0; pass < 2; ++pass) {
+      uint64_t used = 0;
+      for (int k = 0; k < K; ++k) {
+        int best = -1;
+        float bv = 0.f;
+        for (int e = 0; e < n; ++e) {
+          if ((used >> e) & 1ull) continue;
+          const float le = logits[a][e];
+          if (best < 0 || le > bv) { best = e; bv = le; }
+        }
+        used |= 1ull << best;
+        if (pass == 0) {
+          if (k == 0) top = bv;
+          z += expf(bv - top);
+        } else {
+          idx[t * K + k] = best;
+          gate[t * K + k] = expf(bv - top) / z;
+          if (hist) atomicAdd(&hist[best], 1);
+        }
       }
-      used |= 1ull << best;
-      sel[k] = best;
-      val[k] = bv;
-      if (k == 0) top = bv;
-      z += expf(bv - top);
-      if (hist) atomicAdd(&hist[best], 1);
-    }
-    for (int k = 0; k < K; ++k) {
-      idx[t * K + k] = sel[k];
-      gate[t * K + k] = expf(val[k] - top) / z;
     }
   }
   sync();
@@ -406,53 +406,49 @@ __global__ void __launch_bounds__(RS_THREADS)
 }
 
 // One CTA: for every expert, exclusive prefix of the block histograms over blocks, the
-// expert's total, and the start row of its group (groups padded to row_align rows).
+// expert's total, and the start row of its group (groups padded to row_align rows).  The
+// experts are scanned side by side: G = 1024 / n' threads per expert (n' = n rounded up to a
+// power of two), each summing a contiguous range of blocks, then a shared-memory scan.
 __global__ void __launch_bounds__(1024)
     route_scan_kernel(const int32_t* __restrict__ blk_counts, int64_t nblk, int n,
                       int row_align, int64_t rows_max, int32_t* __restrict__ blk_base,
                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                       uint32_t* status) {
-  __shared__ int wsum[32];
-  __shared__ int total[64];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t chunk = (nblk + blockDim.x - 1) / blockDim.x;
-  const int64_t b0 = tid * chunk, b1 = b0 + chunk < nblk ? b0 + chunk : nblk;
-  for (int e = 0; e < n; ++e) {
-    int local = 0;
+  __shared__ int part[1024];
+  __shared__ int total[MAX_EXPERTS];
+  int np = 1;
+  while (np < n) np <<= 1;
+  const int G = 1024 / np;                      // threads per expert (>= 16)
+  const int e = threadIdx.x / G, i = threadIdx.x % G;
+  const int64_t chunk = (nblk + G - 1) / G;
+  const int64_t b0 = i * chunk, b1 = b0 + chunk < nblk ? b0 + chunk : nblk;
+  int local = 0;
+  if (e < n)
     for (int64_t b = b0; b < b1; ++b) local += blk_counts[b * n + e];
-    // inclusive warp scan, then across warps
-    int incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
+  part[threadIdx.x] = local;
+  __syncthreads();
+  // inclusive Hillis-Steele scan inside each expert's G-thread segment
+  for (int off = 1; off < G; off <<= 1) {
+    const int v = i >= off ? part[threadIdx.x - off] : 0;
     __syncthreads();
-    if (warp == 0) {
-      int s = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, s, off);
-        if (lane >= off) s += y;
-      }
-      wsum[lane] = s;  // inclusive over warps
-    }
+    part[threadIdx.x] += v;
     __syncthreads();
-    int run = incl - local + (warp > 0 ? wsum[warp - 1] : 0);
+  }
+  if (e < n) {
+    int run = part[threadIdx.x] - local;  // exclusive prefix of this thread's range
     for (int64_t b = b0; b < b1; ++b) {
       blk_base[b * n + e] = run;
       run += blk_counts[b * n + e];
     }
-    if (tid == 0) total[e] = wsum[(blockDim.x >> 5) - 1];
-    __syncthreads();
+    if (i == G - 1) total[e] = part[threadIdx.x];
   }
-  if (tid == 0) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
     int64_t off = 0;
-    for (int e = 0; e < n; ++e) {
-      counts[e] = total[e];
-      offsets[e] = (int32_t)off;
-      off += (int64_t)(total[e] + row_align - 1) / row_align * row_align;
+    for (int x = 0; x < n; ++x) {
+      counts[x] = total[x];
+      offsets[x] = (int32_t)off;
+      off += (int64_t)(total[x] + row_align - 1) / row_align * row_align;
     }
     offsets[n] = (int32_t)off;
     if (off > rows_max) set_status(status, DEV_ERR_ROW);

@@ -84,7 +84,7 @@ def test_expert_counts(n, K):
     _run(moe_inputs.small(T=24, d=256, F=256, n=n, K=K))
 
 
-@pytest.mark.parametrize("T", [7, 200])
+@pytest.mark.parametrize("T", [7, 200, 1100])
 def test_f32_path_ragged(T):
     _run(moe_inputs.small(T=T, d=136, F=200, dtype="f32", rms_x=False))
 
