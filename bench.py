@@ -45,8 +45,8 @@ DEFAULT_WORKLOAD = "decode_t16"
 # captures summarised in profiles/tc_grouped_gemm_<workload>.md, valid only for the kernel
 # source they were taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "decode_t16": {"bytes": 1879435000 + 7812096, "src": "3a5e4416896d"},
-    "prefill_t4096": {"bytes": 1973359000 + 239567872, "src": "3a5e4416896d"},
+    "decode_t16": {"bytes": 1887007584, "src": "6fc4655fc0de"},
+    "prefill_t4096": {"bytes": 5470377504, "src": "6fc4655fc0de"},
 }
 
 
@@ -303,7 +303,9 @@ def run_gpu(args, w):
                          "basis": "unique expert-weight bytes of selected experts per step / "
                                   "measured HBM copy GB/s" if small_batch else
                                   "routed FLOPs per step / measured bf16 GEMM TFLOP/s"},
-        "roofline": {"bound": bound, "kernel": "tc_grouped_gemm G13 (gate/up + SwiGLU)",
+        "roofline": {"bound": bound,
+                     "kernel": ("tc_pair_gemm" if plan["pair"] else "tc_grouped_gemm")
+                               + " G13 (gate/up + SwiGLU)",
                      "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": peaks["source"], "launch_ms": round(g13, 5)},

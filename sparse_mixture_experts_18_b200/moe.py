@@ -176,8 +176,9 @@ def moe_plan_info(T, d, F, n, K, dtype=torch.bfloat16) -> dict:
     dt = MOE_BF16 if dtype in (torch.bfloat16, MOE_BF16) else MOE_F32
     v = [ctypes.c_int(0) for _ in range(4)]
     _check("moe_plan_info", lib().moe_plan_info(T, d, F, n, K, dt, *[ctypes.byref(i) for i in v]))
+    pair = not v[0].value and dt == MOE_BF16 and T * K >= 640 * n  # same rule as the plan
     return {"small_batch": bool(v[0].value), "split13": v[1].value, "split2": v[2].value,
-            "launches": v[3].value}
+            "launches": v[3].value, "pair": bool(pair)}
 
 
 def moe_forward_debug(x, W_g, W1, W3, W2, K: int, out=None, workspace=None, stream=None):
