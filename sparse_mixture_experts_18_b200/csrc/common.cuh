@@ -38,6 +38,13 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
+// silu for the GEMM epilogues, where h is rounded to bf16 right after: fast exponential and
+// division (a few fp32 ulps, far below bf16's half-ulp).  Large negative z gives exp = inf and
+// a quotient of 0, the limit of silu.
+__device__ __forceinline__ float silu_epilogue(float z) {
+  return __fdividef(z, 1.0f + __expf(-z));
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -268,9 +268,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float h0 = silu(__uint_as_float(va[2 * i])) * __uint_as_float(vb[2 * i]);
+              const float h0 = silu_epilogue(__uint_as_float(va[2 * i])) * __uint_as_float(vb[2 * i]);
               const float h1 =
-                  silu(__uint_as_float(va[2 * i + 1])) * __uint_as_float(vb[2 * i + 1]);
+                  silu_epilogue(__uint_as_float(va[2 * i + 1])) * __uint_as_float(vb[2 * i + 1]);
               pk[i] = pack_bf16x2(h0, h1);
             }
             uint4* dst = reinterpret_cast<uint4*>(h + col);
@@ -507,9 +507,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float h0 = silu(__uint_as_float(va[2 * i])) * __uint_as_float(vb[2 * i]);
+              const float h0 = silu_epilogue(__uint_as_float(va[2 * i])) * __uint_as_float(vb[2 * i]);
               const float h1 =
-                  silu(__uint_as_float(va[2 * i + 1])) * __uint_as_float(vb[2 * i + 1]);
+                  silu_epilogue(__uint_as_float(va[2 * i + 1])) * __uint_as_float(vb[2 * i + 1]);
               pk[i] = pack_bf16x2(h0, h1);
             }
             uint4* dst = reinterpret_cast<uint4*>(h + col);
@@ -589,8 +589,8 @@ __global__ void __launch_bounds__(256)
         sb.x += tb[s].x; sb.y += tb[s].y; sb.z += tb[s].z; sb.w += tb[s].w;
       }
     uint2 o;
-    o.x = pack_bf16x2(silu(sa.x) * sb.x, silu(sa.y) * sb.y);
-    o.y = pack_bf16x2(silu(sa.z) * sb.z, silu(sa.w) * sb.w);
+    o.x = pack_bf16x2(silu_epilogue(sa.x) * sb.x, silu_epilogue(sa.y) * sb.y);
+    o.y = pack_bf16x2(silu_epilogue(sa.z) * sb.z, silu_epilogue(sa.w) * sb.w);
     *reinterpret_cast<uint2*>(h + r * F + c) = o;
   }
 }
