@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ Y, int S, int64_t split_stride, int64_t T, int d,
                    int K, const int32_t* __restrict__ inv, const float* __restrict__ gate,
                    Tout* out, const Tout* resid) {
+  pdl_wait();
+  pdl_trigger();
   const int vpr = d / 4;
   const int64_t total = T * vpr;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
@@ -126,6 +128,8 @@ __global__ void __launch_bounds__(256)
     combine_rows_kernel(const float* __restrict__ Y, int S, int64_t split_stride, int64_t T,
                         int d, int K, const int32_t* __restrict__ inv,
                         const float* __restrict__ gate, Tout* out, const Tout* resid) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
@@ -188,20 +192,20 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
     if (p.dt == 1) {
       auto* o = static_cast<__nv_bfloat16*>(out);
       if (resid)
-        combine_rows_kernel<__nv_bfloat16, true><<<g, 256, 0, s>>>(
+        pdl(combine_rows_kernel<__nv_bfloat16, true>, g, 256, 0, s)(
             w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
             static_cast<const __nv_bfloat16*>(resid));
       else
-        combine_rows_kernel<__nv_bfloat16, false><<<g, 256, 0, s>>>(
+        pdl(combine_rows_kernel<__nv_bfloat16, false>, g, 256, 0, s)(
             w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
     } else {
       auto* o = static_cast<float*>(out);
       if (resid)
-        combine_rows_kernel<float, true><<<g, 256, 0, s>>>(w.y, S, split_stride, p.T, (int)p.d,
+        pdl(combine_rows_kernel<float, true>, g, 256, 0, s)(w.y, S, split_stride, p.T, (int)p.d,
                                                            p.K, w.inv, w.gate, o,
                                                            static_cast<const float*>(resid));
       else
-        combine_rows_kernel<float, false><<<g, 256, 0, s>>>(w.y, S, split_stride, p.T,
+        pdl(combine_rows_kernel<float, false>, g, 256, 0, s)(w.y, S, split_stride, p.T,
                                                             (int)p.d, p.K, w.inv, w.gate, o,
                                                             nullptr);
     }
@@ -214,20 +218,20 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
   if (p.dt == 1) {
     auto* o = static_cast<__nv_bfloat16*>(out);
     if (resid)
-      combine_kernel<__nv_bfloat16, true><<<(unsigned)blocks, 256, 0, s>>>(
+      pdl(combine_kernel<__nv_bfloat16, true>, (unsigned)blocks, 256, 0, s)(
           w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
           static_cast<const __nv_bfloat16*>(resid));
     else
-      combine_kernel<__nv_bfloat16, false><<<(unsigned)blocks, 256, 0, s>>>(
+      pdl(combine_kernel<__nv_bfloat16, false>, (unsigned)blocks, 256, 0, s)(
           w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
   } else {
     auto* o = static_cast<float*>(out);
     if (resid)
-      combine_kernel<float, true><<<(unsigned)blocks, 256, 0, s>>>(
+      pdl(combine_kernel<float, true>, (unsigned)blocks, 256, 0, s)(
           w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
           static_cast<const float*>(resid));
     else
-      combine_kernel<float, false><<<(unsigned)blocks, 256, 0, s>>>(
+      pdl(combine_kernel<float, false>, (unsigned)blocks, 256, 0, s)(
           w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
   }
   return cudaGetLastError();
@@ -238,6 +242,8 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
 __global__ void __launch_bounds__(256)
     rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ xn,
                    int64_t T, int d, float eps) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= T) return;
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_rmsnorm(const void* x, void* xn, int64_t T, int64_t d, float eps,
                            cudaStream_t s) {
   const unsigned blocks = (unsigned)((T + 7) / 8);
-  rmsnorm_kernel<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
+  pdl(rmsnorm_kernel, blocks, 256, 0, s)(static_cast<const __nv_bfloat16*>(x),
                                         static_cast<__nv_bfloat16*>(xn), T, (int)d, eps);
   return cudaGetLastError();
 }

@@ -23,6 +23,16 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel is launched so that it may start while the previous kernel of the stream is
+// still finishing.  pdl_wait() blocks until that kernel has completed and its writes are
+// visible, so it comes before any access to data it produced (and before any write another
+// kernel of the previous call may still read); pdl_trigger() lets the next kernel launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- small helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

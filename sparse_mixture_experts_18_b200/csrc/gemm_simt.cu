@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(256)
                              const float* __restrict__ W0, const float* __restrict__ W1,
                              int nw, const int32_t* __restrict__ offsets, int n,
                              float* __restrict__ out, int64_t out_ld) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[SK][SIMT_TILE + 4];
   __shared__ float B0s[SK][SIMT_TILE + 4];
   __shared__ float B1s[SK][SIMT_TILE + 4];
@@ -87,7 +89,7 @@ cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float
   const int d = (int)p.d, F = (int)p.F;
   const unsigned mtiles = (unsigned)(p.rows_max / SIMT_TILE);
   dim3 g13((F + SIMT_TILE - 1) / SIMT_TILE, mtiles);
-  simt_grouped_gemm_kernel<true><<<g13, 256, 0, s>>>(static_cast<const float*>(w.xperm), d, d,
+  pdl(simt_grouped_gemm_kernel<true>, g13, 256, 0, s)(static_cast<const float*>(w.xperm), d, d,
                                                       W1, W3, F, w.offsets, p.n,
                                                       static_cast<float*>(w.h), F);
   cudaError_t err = cudaGetLastError();
@@ -96,7 +98,7 @@ cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float
              (err = cudaEventRecord(ev[1], s)) != cudaSuccess))
     return err;
   dim3 g2((d + SIMT_TILE - 1) / SIMT_TILE, mtiles);
-  simt_grouped_gemm_kernel<false><<<g2, 256, 0, s>>>(static_cast<const float*>(w.h), F, F, W2,
+  pdl(simt_grouped_gemm_kernel<false>, g2, 256, 0, s)(static_cast<const float*>(w.h), F, F, W2,
                                                       nullptr, d, w.offsets, p.n, w.y, d);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   return ev ? cudaEventRecord(ev[2], s) : cudaSuccess;

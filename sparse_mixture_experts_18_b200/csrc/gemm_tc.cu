@@ -138,11 +138,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tma_prefetch_desc(&tmW0);
     if (KIND == KIND_G13) tma_prefetch_desc(&tmW1);
   }
-  if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
   if (warp == 1) {
     tmem_alloc(&c->tmem_slot, a.tmem_cols);
     tmem_relinquish();
   }
+  pdl_wait();  // expert offsets and operands come from the previous kernels
+  pdl_trigger();
+  if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
   __syncthreads();
   if (threadIdx.x == 0) {
     int na = 0;
@@ -396,11 +398,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tma_prefetch_desc(&tmW0);
     if (KIND == KIND_G13) tma_prefetch_desc(&tmW1);
   }
-  if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
   if (warp == 1) {
     tmem_alloc_pair(&c->tmem_slot, a.tmem_cols);
     tmem_relinquish_pair();
   }
+  pdl_wait();  // expert offsets and operands come from the previous kernels
+  pdl_trigger();
+  if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
   tc_fence_before();
   cluster_sync_all();  // barrier initialisation and the TMEM allocation, in both CTAs
   tc_fence_after();
@@ -567,6 +571,8 @@ constexpr int REDUCE_MAX_S = 8;
 __global__ void __launch_bounds__(256)
     swiglu_reduce_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
                          int64_t rows, int F, __nv_bfloat16* __restrict__ h) {
+  pdl_wait();
+  pdl_trigger();
   const int vpr = F / 4;
   const int64_t total = rows * vpr;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
@@ -647,7 +653,7 @@ static cudaError_t launch_one(const CUtensorMap& mx, const CUtensorMap& mw0,
     configured = (int)smem;
   }
   const int grid = max_work < num_sms() ? (max_work > 0 ? max_work : 1) : num_sms();
-  kern<<<grid, GEMM_THREADS, smem, s>>>(mx, mw0, mw1, a);
+  pdl(kern, grid, GEMM_THREADS, smem, s)(mx, mw0, mw1, a);
   return cudaGetLastError();
 }
 
@@ -660,11 +666,13 @@ static cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw0,
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -684,6 +692,7 @@ static cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw0,
   int pairs = max_work < pairs_fit[dev] ? max_work : pairs_fit[dev];
   if (pairs < 1) pairs = 1;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, mx, mw0, mw1, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -824,7 +833,7 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   const int64_t rows = p.T * p.K;
   const int64_t vec = rows * F / 4;
   const int rgrid = (int)((vec + 255) / 256 < 4 * num_sms() ? (vec + 255) / 256 : 4 * num_sms());
-  swiglu_reduce_kernel<<<rgrid > 0 ? rgrid : 1, 256, 0, s>>>(
+  pdl(swiglu_reduce_kernel, rgrid > 0 ? rgrid : 1, 256, 0, s)(
       w.p13, p.s13, a.split_stride, rows, F, static_cast<__nv_bfloat16*>(w.h));
   if ((err = cudaGetLastError()) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
     return err;

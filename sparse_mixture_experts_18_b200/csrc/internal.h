@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace moe {
@@ -50,6 +52,35 @@ struct Workspace {
   float* p13;   // swap: [s13][rows_max][2F] split-K partial sums of x.W1 | x.W3
   void* xn;     // stack: normalised activations [T][d]
 };
+
+// Launch with programmatic stream serialization (the kernel may begin while its predecessor
+// in the stream finishes; see pdl_wait / pdl_trigger):  pdl(kernel, grid, block, smem, s)(args)
+template <typename... KArgs>
+struct PdlLaunch {
+  void (*kern)(KArgs...);
+  dim3 grid, block;
+  size_t smem;
+  cudaStream_t stream;
+  template <typename... Args>
+  cudaError_t operator()(Args&&... args) const {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  }
+};
+template <typename... KArgs>
+PdlLaunch<KArgs...> pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                        cudaStream_t s) {
+  return PdlLaunch<KArgs...>{kern, grid, block, smem, s};
+}
 
 bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p);
 Workspace carve(const Plan& p, void* base);

@@ -174,6 +174,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
     router_topk_kernel(const Tin* __restrict__ x, const float* __restrict__ Wg, int64_t T,
                        int d, int n, int K, int32_t* __restrict__ idx,
                        float* __restrict__ gate, int32_t* __restrict__ blk_counts) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[ROUTE_THREADS / 32][64];
   __shared__ float logits[TOKB][NPAD];
   __shared__ int hist[64];
@@ -235,6 +237,8 @@ __global__ void __launch_bounds__(RS_THREADS)
                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                        int32_t* __restrict__ inv, int32_t* __restrict__ row_tok,
                        Tact* __restrict__ xperm, uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int PER = RS_MAX_ENTRIES / RS_THREADS;  // entries per thread in the rank phase
   constexpr int CPL = 1;                            // 8-element chunks per lane
   __shared__ float logit[RS_MAX_T * MAX_EXPERTS];
@@ -414,6 +418,8 @@ __global__ void __launch_bounds__(1024)
                       int row_align, int64_t rows_max, int32_t* __restrict__ blk_base,
                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                       uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int part[1024];
   __shared__ int total[MAX_EXPERTS];
   int np = 1;
@@ -466,6 +472,8 @@ __global__ void __launch_bounds__(256)
                           const int32_t* __restrict__ offsets, int64_t rows_max,
                           int32_t* __restrict__ inv, Tact* __restrict__ xperm,
                           uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int ent_e[64];
   __shared__ int ent_row[64];
   const int64_t t0 = (int64_t)blockIdx.x * tokb;
@@ -506,16 +514,16 @@ static cudaError_t launch_router_t(const Tin* x, const float* Wg, int64_t T, int
   const int tokb = route_tokens_per_block(n);
   const unsigned grid = (unsigned)((T + tokb - 1) / tokb);
   if (n <= 8)
-    router_topk_kernel<Tin, 8, 8><<<grid, ROUTE_THREADS, 0, s>>>(x, Wg, T, d, n, K, idx, gate,
+    pdl(router_topk_kernel<Tin, 8, 8>, grid, ROUTE_THREADS, 0, s)(x, Wg, T, d, n, K, idx, gate,
                                                                  blk_counts);
   else if (n <= 16)
-    router_topk_kernel<Tin, 16, 4><<<grid, ROUTE_THREADS, 0, s>>>(x, Wg, T, d, n, K, idx,
+    pdl(router_topk_kernel<Tin, 16, 4>, grid, ROUTE_THREADS, 0, s)(x, Wg, T, d, n, K, idx,
                                                                   gate, blk_counts);
   else if (n <= 32)
-    router_topk_kernel<Tin, 32, 2><<<grid, ROUTE_THREADS, 0, s>>>(x, Wg, T, d, n, K, idx,
+    pdl(router_topk_kernel<Tin, 32, 2>, grid, ROUTE_THREADS, 0, s)(x, Wg, T, d, n, K, idx,
                                                                   gate, blk_counts);
   else
-    router_topk_kernel<Tin, 64, 1><<<grid, ROUTE_THREADS, 0, s>>>(x, Wg, T, d, n, K, idx,
+    pdl(router_topk_kernel<Tin, 64, 1>, grid, ROUTE_THREADS, 0, s)(x, Wg, T, d, n, K, idx,
                                                                   gate, blk_counts);
   return cudaGetLastError();
 }
@@ -524,7 +532,7 @@ template <typename Tact>
 static cudaError_t launch_route_small_t(const Plan& p, const Tact* x, const float* Wg,
                                         const Workspace& w, cudaStream_t s) {
   const int G = (int)((p.d + 63) / 64);
-  route_split_kernel<Tact><<<G, RS_THREADS, 0, s>>>(
+  pdl(route_split_kernel<Tact>, G, RS_THREADS, 0, s)(
       x, Wg, (int)p.T, (int)p.d, p.n, p.K, p.row_align, p.rows_max, w.rpart, w.ticket, w.idx,
       w.gate, w.counts, w.offsets, w.inv, w.row_tok,
       static_cast<Tact*>(w.xperm), w.status);
@@ -544,17 +552,17 @@ cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Wo
     err = launch_router_t(static_cast<const float*>(x), Wg, p.T, (int)p.d, p.n, p.K, w.idx,
                           w.gate, w.blk_counts, s);
   if (err != cudaSuccess) return err;
-  route_scan_kernel<<<1, 1024, 0, s>>>(w.blk_counts, p.nblk, p.n, p.row_align, p.rows_max,
+  pdl(route_scan_kernel, 1, 1024, 0, s)(w.blk_counts, p.nblk, p.n, p.row_align, p.rows_max,
                                        w.blk_base, w.counts, w.offsets, w.status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int tokb = route_tokens_per_block(p.n);
   if (p.dt == 1)
-    permute_gather_kernel<__nv_bfloat16><<<(unsigned)p.nblk, 256, 0, s>>>(
+    pdl(permute_gather_kernel<__nv_bfloat16>, (unsigned)p.nblk, 256, 0, s)(
         static_cast<const __nv_bfloat16*>(x), p.T, (int)p.d, p.n, p.K, tokb, w.idx,
         w.blk_base, w.offsets, p.rows_max, w.inv, static_cast<__nv_bfloat16*>(w.xperm),
         w.status);
   else
-    permute_gather_kernel<float><<<(unsigned)p.nblk, 256, 0, s>>>(
+    pdl(permute_gather_kernel<float>, (unsigned)p.nblk, 256, 0, s)(
         static_cast<const float*>(x), p.T, (int)p.d, p.n, p.K, tokb, w.idx, w.blk_base,
         w.offsets, p.rows_max, w.inv, static_cast<float*>(w.xperm), w.status);
   return cudaGetLastError();
