@@ -266,22 +266,26 @@ def run_gpu(args, w):
     g13 = statistics.mean(s[1] for s in stage_ms)          # gate/up GEMM (dominant kernel)
     stage_avg = [statistics.mean(s[j] for s in stage_ms) for j in range(5)]
     es = 2
-    weight_bytes_13 = n_active * 2 * w.F * w.d * es
-    weight_bytes_all = n_active * 3 * w.F * w.d * es
     timed_s = ms / 1e3
     bf16_peak = peaks["bf16_sustained"] if timed_s > 1.0 else peaks["bf16"]
-    if small_batch:
-        bound, unit = "hbm", "GB/s"
-        traffic_alg = weight_bytes_13 + w.T * w.K * w.d * es
-        achieved = traffic_alg / (g13 / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        step_alg = weight_bytes_all + w.d * w.n * 4 + 2 * w.T * w.d * es
-        step_frac = step_alg / (ms_step / 1e3) / 1e9 / peak
+    # The bound of each is the larger of its two floors: algorithmic bytes at the measured HBM
+    # copy rate, algorithmic FLOPs at the measured bf16 GEMM rate.
+    rows = w.T * w.K
+    bytes13 = n_active * 2 * w.F * w.d * es + rows * w.d * es + rows * w.F * es
+    flops13 = 4 * w.d * w.F * rows
+    if bytes13 / (peaks["hbm_gbs"] * 1e9) >= flops13 / (bf16_peak * 1e12):
+        bound, unit, peak = "hbm", "GB/s", peaks["hbm_gbs"]
+        achieved = bytes13 / (g13 / 1e3) / 1e9
     else:
-        bound, unit = "tensor", "TFLOP/s"
-        achieved = 4 * w.d * w.F * w.T * w.K / (g13 / 1e3) / 1e12
-        peak = bf16_peak
-        step_frac = tflops / peak
+        bound, unit, peak = "tensor", "TFLOP/s", bf16_peak
+        achieved = flops13 / (g13 / 1e3) / 1e12
+    step_bytes = (w.layers * (n_active * 3 * w.F * w.d * es + w.d * w.n * 4)
+                  + 2 * w.T * w.d * es)
+    step_hbm = step_bytes / (peaks["hbm_gbs"] * 1e9) >= tflops * ms_step / 1e3 / bf16_peak
+    step_frac = (step_bytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"] if step_hbm
+                 else tflops / bf16_peak)
+    tiling = (f"small-batch swap-AB split-K {s13}/{s2}" if small_batch else
+              "CTA-pair 256-row tiles" if plan["pair"] else "128-row tiles")
     cap = TRAFFIC.get(w.name)
     traffic = cap["bytes"] if cap and cap["src"] == kernel_source_hash() else None
     line = {
@@ -294,14 +298,13 @@ def run_gpu(args, w):
                                   else ""),
                    "tokens_per_rank": w.T, "l2": "inputs larger than L2 "
                    f"({w.layers * 3 * w.n * w.F * w.d * es / 1e9:.2f} GB of expert weights)",
-                   "parallelism": f"replicas x{world}", "tiling": "small-batch swap-AB "
-                   f"split-K {s13}/{s2}" if small_batch else "prefill 128-row tiles",
+                   "parallelism": f"replicas x{world}", "tiling": tiling,
                    "active_experts": n_active, "expert_counts": counts},
         "tflops": round(tflops, 3),
-        "pct_roofline": {"bound": "hbm" if small_batch else "tensor",
+        "pct_roofline": {"bound": "hbm" if step_hbm else "tensor",
                          "frac": round(step_frac, 4),
                          "basis": "unique expert-weight bytes of selected experts per step / "
-                                  "measured HBM copy GB/s" if small_batch else
+                                  "measured HBM copy GB/s" if step_hbm else
                                   "routed FLOPs per step / measured bf16 GEMM TFLOP/s"},
         "roofline": {"bound": bound,
                      "kernel": ("tc_pair_gemm" if plan["pair"] else "tc_grouped_gemm")

@@ -55,13 +55,23 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads of the benchmark and parity suite.
+# The five workloads of the benchmark and parity suite, then variants of the expert count n
+# and of K on the same hidden and expert widths (the paper's remark that n and K are free
+# parameters of the layer): they move the rows per expert M_e = T*K/n down to ~128, where
+# the expert GEMMs sit near the HBM/tensor ridge, and exercise grouping with many groups.
 WORKLOADS = {
     "tiny_f32": Workload("tiny_f32", T=64, d=128, F=256, dtype="f32", rms_x=False),
     "decode_t16": Workload("decode_t16", T=16, d=4096, F=14336),
     "prefill_t4096": Workload("prefill_t4096", T=4096, d=4096, F=14336),
     "skewed_t32768": Workload("skewed_t32768", T=32768, d=4096, F=14336, zipf=1.2),
     "stack32_t8192": Workload("stack32_t8192", T=8192, d=4096, F=14336, layers=32),
+    "experts16_top1_t4096": Workload("experts16_top1_t4096", T=4096, d=4096, F=14336, n=16,
+                                     K=1),
+    "experts16_top4_t4096": Workload("experts16_top4_t4096", T=4096, d=4096, F=14336, n=16,
+                                     K=4),
+    "experts64_top2_t4096": Workload("experts64_top2_t4096", T=4096, d=4096, F=14336, n=64,
+                                     K=2),
+    "experts64_top4_t16": Workload("experts64_top4_t16", T=16, d=4096, F=14336, n=64, K=4),
 }
 
 

@@ -212,6 +212,16 @@ def test_skewed_t32768_sampled():
     assert c[0] > 2.5 * c.mean(), c   # busiest expert about 3x the mean load
 
 
+@pytest.mark.parametrize("name", ["experts16_top1_t4096", "experts16_top4_t4096",
+                                  "experts64_top2_t4096", "experts64_top4_t16"])
+def test_expert_count_variants_full_size(name):
+    """n = 16 / 64 experts with K = 1 / 2 / 4 at Mixtral's hidden and expert widths: every
+    token's routing, the grouping, and sampled tokens' outputs."""
+    w = moe_inputs.WORKLOADS[name]
+    rep = _run(w, gen_device="cuda", budget=16)
+    assert sum(rep["counts"]) == w.T * w.K
+
+
 def test_stack32_t8192_sampled():
     """32 blocks of Mixtral shape on T=8192 tokens (~90 GB of bf16 expert weights on the
     device).  The residual stream amplifies any sub-ulp difference: two oracle trajectories
