@@ -45,8 +45,8 @@ DEFAULT_WORKLOAD = "decode_t16"
 # captures summarised in profiles/tc_grouped_gemm_<workload>.md, valid only for the kernel
 # source they were taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "decode_t16": {"bytes": 1887007584, "src": "6fc4655fc0de"},
-    "prefill_t4096": {"bytes": 5470377504, "src": "6fc4655fc0de"},
+    "decode_t16": {"bytes": 1887546456, "src": "3c55670d6d98"},
+    "prefill_t4096": {"bytes": 2670625064, "src": "3c55670d6d98"},
 }
 
 
