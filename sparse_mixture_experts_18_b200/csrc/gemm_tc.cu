@@ -36,7 +36,8 @@ struct TcArgs {
   int n;
   int num_kb;              // 64-wide K blocks per work unit
   int nw;                  // weight rows (output features) per expert: F (G13) or d (G2)
-  int n_tiles;             // prefill: column tiles per 128-row tile
+  int n_tiles;             // prefill: column tiles per row tile (pairs: column-block pairs)
+  int n_blocks;            // CTA pairs: column blocks per expert, two per tile
   int wb;                  // small batch: 128-row weight blocks per expert
   int splits;              // small batch: K ranges
   int tok_tile;            // small batch: MMA N
@@ -67,6 +68,8 @@ struct Ctrl {
 
 struct Work {
   int e, mt, nt, wblk, s, row0, count;
+  int m;  // CTA pairs: MMA M of the tile (256, or 128 for an expert's last 128 rows)
+          // (and s: the tile's first column block)
 };
 
 template <bool SWAP>
@@ -333,45 +336,86 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 }
 
 // ---------------------------------------------------------------- CTA-pair prefill tiling
-// Tile = 256 permuted rows x 256 MMA columns computed by a cluster of two CTAs with
-// tcgen05.mma.cta_group::2 (M = 256).  CTA r holds its 128 rows of A and half of the N = 256
-// operand -- G13: W1 rows (r = 0) or the same W3 rows (r = 1); G2: W2 rows [128r, 128r + 128)
-// of the column tile -- so each CTA stages 32 KB per 64-wide K block instead of 48 KB, and
-// twice as many K blocks are in flight.  The even CTA (leader) issues every MMA; both CTAs'
-// TMA loads complete on the leader's full barrier; the leader's commits arrive on both CTAs'
-// empty and accumulator-full barriers; both epilogues release accumulators on the leader's
-// barrier.  Expert groups are padded to 256 rows on this path.
+// Tile = 256 permuted rows x two 256-column blocks, computed by a cluster of two CTAs with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256 per block).  CTA r holds its 128 rows of A and
+// half of each block's N = 256 operand -- G13: W1 rows (r = 0) or the same W3 rows (r = 1),
+// so a block is 128 columns of h; G2: W2 rows [128r, 128r + 128) of the block's 256 output
+// columns.  Both blocks share the A rows, so a CTA stages 48 KB per 64-wide K block for two
+// blocks' MMAs: 48 bytes per MMA cycle, where one block per tile needs 64, which is about what
+// an SM can pull from L2.  The even CTA (leader) issues every MMA; both CTAs' TMA loads
+// complete on the leader's full barrier; the leader's commits arrive on both CTAs' empty and
+// accumulator-full barriers.  The two accumulators fill TMEM (2 x 256 columns), so there is
+// no second buffer: the eight epilogue warps drain accumulator 0, release it on the leader's
+// barrier, then drain accumulator 1, and the next tile's MMAs start on accumulator 0 in the
+// meantime.  A tile whose second block lies past the last column block computes one block.  Expert groups are padded to 256 rows on this path.
 constexpr int PAIR_ROWS = 256;
+constexpr int PAIR_THREADS = 320;
 
 struct PairCtrl {
   uint64_t full[MAX_STAGES];   // leader: the stage's bytes of both CTAs have landed
   uint64_t empty[MAX_STAGES];  // each CTA: its stage may be refilled
-  uint64_t tfull[2];           // each CTA: accumulator complete
-  uint64_t tempty[2];          // leader: both epilogues drained the accumulator (256 threads)
+  uint64_t tfull;              // each CTA: both accumulators complete
+  uint64_t tempty[2];          // leader: accumulator g drained by both CTAs' epilogues
   uint64_t peer_done;          // each CTA: the peer CTA is finished with TMEM
   uint32_t tmem_slot;
   int abort;
   int off[MAX_EXPERTS + 1];
+  int tbase[MAX_EXPERTS + 1];  // row tiles of experts before e
 };
 
-__device__ __forceinline__ Work decode_pair_work(const TcArgs& a, const int* off, int id) {
+// Tile order: expert, then column-block pair, then row tile (the row tiles of a column-block
+// pair run side by side and share its weight tiles through L2).  Tiles go round-robin to the
+// pairs; when the last round would keep at most half of the pairs busy, its `split` tiles are
+// cut into one-block tiles (ids from wide - split on: two per tile) so that it takes half
+// as long.  count = 0 marks the missing second half of a one-block tile.
+struct PairSchedule {
+  int wide;   // two-block tiles
+  int split;  // of which the last `split` are cut in two
+};
+
+__device__ __forceinline__ PairSchedule pair_schedule(const TcArgs& a, const PairCtrl* c,
+                                                      int npairs) {
+  PairSchedule ps;
+  ps.wide = c->tbase[a.n] * a.n_tiles;
+  const int r = ps.wide % npairs;
+  ps.split = a.n_blocks > 1 && r > 0 && 2 * r <= npairs ? r : 0;
+  return ps;
+}
+
+__device__ __forceinline__ Work decode_pair_work(const TcArgs& a, const PairCtrl* c,
+                                                 const PairSchedule& ps, int id) {
+  int wid = id, part = -1;
+  if (id >= ps.wide - ps.split) {
+    const int u = id - (ps.wide - ps.split);
+    wid = ps.wide - ps.split + (u >> 1);
+    part = u & 1;
+  }
   Work w{};
   int e = 0;
-  while (e + 1 < a.n && id >= (off[e + 1] / PAIR_ROWS) * a.n_tiles) ++e;
-  const int mt0 = off[e] / PAIR_ROWS;
-  const int mcnt = off[e + 1] / PAIR_ROWS - mt0;
-  const int local = id - mt0 * a.n_tiles;
+  while (e + 1 < a.n && wid >= c->tbase[e + 1] * a.n_tiles) ++e;
+  const int mcnt = c->tbase[e + 1] - c->tbase[e];
+  const int local = wid - c->tbase[e] * a.n_tiles;
+  const int mloc = local % mcnt;
   w.e = e;
-  w.nt = local / mcnt;
-  w.mt = mt0 + local % mcnt;  // 256-row tile index
+  w.nt = local / mcnt;  // column-block pair: blocks 2 nt and 2 nt + 1
+  w.row0 = c->off[e] + mloc * PAIR_ROWS;
+  w.m = c->off[e + 1] - w.row0 < PAIR_ROWS ? 128 : 256;
+  w.count = 2 * w.nt + 1 < a.n_blocks ? 2 : 1;  // blocks in this tile
+  w.s = 2 * w.nt;                               // first column block
+  if (part >= 0) {
+    w.s += part;
+    w.count = part < w.count ? 1 : 0;
+  }
   return w;
 }
 
 template <int KIND>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(PAIR_THREADS, 1)
     tc_pair_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmW0,
-                        const __grid_constant__ CUtensorMap tmW1, const TcArgs a) {
+                        const __grid_constant__ CUtensorMap tmW1,
+                        const __grid_constant__ CUtensorMap tmW0h,
+                        const __grid_constant__ CUtensorMap tmW1h, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   PairCtrl* c = reinterpret_cast<PairCtrl*>(smem + (size_t)a.stages * a.stage_bytes);
@@ -385,10 +429,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&c->full[s], 1);
       mbar_init(&c->empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&c->tfull[i], 1);
-      mbar_init(&c->tempty[i], 256);
-    }
+    mbar_init(&c->tfull, 1);
+    mbar_init(&c->tempty[0], 512);  // 256 epilogue threads in each of the two CTAs
+    mbar_init(&c->tempty[1], 512);
     mbar_init(&c->peer_done, 1);
     c->abort = 0;
     fence_mbar_init();
@@ -396,20 +439,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (threadIdx.x == 32) {
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW0);
-    if (KIND == KIND_G13) tma_prefetch_desc(&tmW1);
+    if (KIND == KIND_G13) {
+      tma_prefetch_desc(&tmW1);
+      tma_prefetch_desc(&tmW0h);
+      tma_prefetch_desc(&tmW1h);
+    }
   }
   if (warp == 1) {
-    tmem_alloc_pair(&c->tmem_slot, a.tmem_cols);
+    tmem_alloc_pair(&c->tmem_slot, 512);
     tmem_relinquish_pair();
   }
   pdl_wait();  // expert offsets and operands come from the previous kernels
   pdl_trigger();
   if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    c->tbase[0] = 0;
+    for (int e = 0; e < a.n; ++e)
+      c->tbase[e + 1] = c->tbase[e] + (c->off[e + 1] - c->off[e] + PAIR_ROWS - 1) / PAIR_ROWS;
+  }
   tc_fence_before();
   cluster_sync_all();  // barrier initialisation and the TMEM allocation, in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = c->tmem_slot;
-  const int total = (c->off[a.n] / PAIR_ROWS) * a.n_tiles;
+  const PairSchedule ps = pair_schedule(a, c, npairs);
+  const int total = ps.wide + ps.split;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -421,21 +475,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int id = pair; id < total && ok; id += npairs) {
-        const Work w = decode_pair_work(a, c->off, id);
-        const int row = w.mt * PAIR_ROWS + (int)rank * 128;
+        const Work w = decode_pair_work(a, c, ps, id);
+        if (w.count == 0) continue;
+        const int row = w.row0 + (int)rank * (w.m >> 1);
         for (int kb = 0; kb < a.num_kb; ++kb) {
           if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort)) { ok = false; break; }
           uint8_t* st = smem + (size_t)stage * a.stage_bytes;
-          if (leader) mbar_arrive_expect_tx(&c->full[stage], 2 * a.tx_bytes);
+          if (leader)
+            mbar_arrive_expect_tx(&c->full[stage], 2u * (uint32_t)(1 + w.count) * TILE_BYTES);
           const uint32_t fb = full0 + (uint32_t)stage * 8u;
           const int k = kb * 64;
           tma_load_2d_pair(st, &tmX, fb, k, row, pol_x);
-          if (KIND == KIND_G13)
-            tma_load_2d_pair(st + TILE_BYTES, rank == 0 ? &tmW0 : &tmW1, fb, k,
-                             w.e * a.nw + w.nt * 128, pol_w);
-          else
-            tma_load_2d_pair(st + TILE_BYTES, &tmW0, fb, k,
-                             w.e * a.nw + w.nt * 256 + (int)rank * 128, pol_w);
+          for (int j = 0; j < w.count; ++j) {
+            const int cb = w.s + j;
+            uint8_t* bt = st + (1 + j) * TILE_BYTES;
+            if (KIND == KIND_G13 && w.m == 128) {  // 64 W1 rows, then the same 64 W3 rows
+              const int wr = w.e * a.nw + cb * 128 + (int)rank * 64;
+              tma_load_2d_pair(bt, &tmW0h, fb, k, wr, pol_w);
+              tma_load_2d_pair(bt + TILE_BYTES / 2, &tmW1h, fb, k, wr, pol_w);
+            } else if (KIND == KIND_G13)
+              tma_load_2d_pair(bt, rank == 0 ? &tmW0 : &tmW1, fb, k,
+                               w.e * a.nw + cb * 128, pol_w);
+            else
+              tma_load_2d_pair(bt, &tmW0, fb, k, w.e * a.nw + cb * 256 + (int)rank * 128, pol_w);
+          }
           if (++stage == a.stages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -448,100 +511,171 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
+    // The epilogue drains accumulator 0 before accumulator 1, so a tile starts with the first
+    // `lead` K blocks of accumulator 0 (their stages are held) while accumulator 1 is still
+    // being drained; accumulator 1 then catches up on the held stages, releasing them.
     if (lane == 0 && leader) {
-      const uint32_t idesc = umma_idesc_bf16(256, 256);
-      int stage = 0, it = 0;
-      uint32_t phase = 0;
+      const int lead = a.stages < a.num_kb ? a.stages : a.num_kb;
+      int stage = 0;
+      uint32_t it = 0, phase = 0;
       bool ok = true;
-      for (int id = pair; id < total && ok; id += npairs, ++it) {
-        const uint32_t acc = (uint32_t)it % a.nacc;
-        const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
-        if (!mbar_wait(&c->tempty[acc], aph ^ 1u, a.status, &c->abort)) { ok = false; break; }
+      for (int id = pair; id < total && ok; id += npairs) {
+        const Work w = decode_pair_work(a, c, ps, id);
+        if (w.count == 0) continue;
+        const uint32_t idesc = umma_idesc_bf16(w.m, 256);
+        const uint32_t tpar = (it & 1u) ^ 1u;  // tile it - 1 drained
+        if (!mbar_wait(&c->tempty[0], tpar, a.status, &c->abort)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t dtm = tmem_base + acc * a.acc_cols;
-        for (int kb = 0; kb < a.num_kb; ++kb) {
+        const int stage0 = stage;
+        const uint32_t phase0 = phase;
+        for (int kb = 0; kb < lead; ++kb) {
           if (!mbar_wait(&c->full[stage], phase, a.status, &c->abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sb = smem_u32(smem + (size_t)stage * a.stage_bytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t kofs = kk * 32;
-            umma_bf16_pair(dtm, umma_desc_k128(sb + kofs), umma_desc_k128(sb + TILE_BYTES + kofs),
-                           idesc, (kb | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_pair(tmem_base, umma_desc_k128(sb + kk * 32),
+                           umma_desc_k128(sb + TILE_BYTES + kk * 32), idesc, (kb | kk) != 0);
+          if (++stage == a.stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (w.count == 2) {
+          if (!mbar_wait(&c->tempty[1], tpar, a.status, &c->abort)) { ok = false; break; }
+          tc_fence_after();
+        }
+        stage = stage0;
+        phase = phase0;
+        for (int kb = 0; kb < lead; ++kb) {
+          if (w.count == 2) {
+            const uint32_t sb = smem_u32(smem + (size_t)stage * a.stage_bytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_pair(tmem_base + 256u, umma_desc_k128(sb + kk * 32),
+                             umma_desc_k128(sb + 2 * TILE_BYTES + kk * 32), idesc,
+                             (kb | kk) != 0);
+          }
+          umma_commit_pair(&c->empty[stage], 0x3);
+          if (++stage == a.stages) { stage = 0; phase ^= 1u; }
+        }
+        for (int kb = lead; kb < a.num_kb; ++kb) {
+          if (!mbar_wait(&c->full[stage], phase, a.status, &c->abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(smem + (size_t)stage * a.stage_bytes);
+          for (int j = 0; j < w.count; ++j) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_pair(tmem_base + (uint32_t)j * 256u, umma_desc_k128(sb + kk * 32),
+                             umma_desc_k128(sb + (uint32_t)(1 + j) * TILE_BYTES + kk * 32),
+                             idesc, 1u);
           }
           umma_commit_pair(&c->empty[stage], 0x3);
           if (++stage == a.stages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit_pair(&c->tfull[acc], 0x3);
+        umma_commit_pair(&c->tfull, 0x3);
+        ++it;
       }
-      // both epilogues have released every accumulator before TMEM is torn down
-      for (uint32_t j = 0; ok && j < a.nacc; ++j, ++it) {
-        const uint32_t acc = (uint32_t)it % a.nacc;
-        const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
-        if (!mbar_wait(&c->tempty[acc], aph ^ 1u, a.status, &c->abort)) break;
-      }
+      // both accumulators released before TMEM is torn down
+      if (ok && mbar_wait(&c->tempty[0], (it & 1u) ^ 1u, a.status, &c->abort))
+        mbar_wait(&c->tempty[1], (it & 1u) ^ 1u, a.status, &c->abort);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Two warps per TMEM lane quarter (warps q + 2 and q + 6, q = warp & 3 being the quarter
+    // a warp may access) split the columns; accumulator 0 is drained and released first.
+    const int half = (warp - 2) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t tempty0 = map_to_rank(&c->tempty[0], 0);
-    int it = 0;
+    uint32_t it = 0;
     for (int id = pair; id < total; id += npairs, ++it) {
-      const Work w = decode_pair_work(a, c->off, id);
-      const uint32_t acc = (uint32_t)it % a.nacc;
-      const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
-      const bool ok = mbar_wait(&c->tfull[acc], aph, a.status, &c->abort);
+      const Work w = decode_pair_work(a, c, ps, id);
+      if (w.count == 0) { --it; continue; }
+      const bool ok = mbar_wait(&c->tfull, it & 1u, a.status, &c->abort);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * a.acc_cols;
-      const int64_t row = (int64_t)w.mt * PAIR_ROWS + rank * 128 + r;
-      if (KIND == KIND_G13) {
-        __nv_bfloat16* h = static_cast<__nv_bfloat16*>(a.out) + row * a.out_ld;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t va[32], vb[32];
-          tmem_ld32(tb + cc * 32, va);
-          tmem_ld32(tb + 128 + cc * 32, vb);
-          tmem_ld_wait();
-          const int col = w.nt * 128 + cc * 32;
-          if (col < a.nw) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_epilogue(__uint_as_float(va[2 * i])) * __uint_as_float(vb[2 * i]);
-              const float h1 =
-                  silu_epilogue(__uint_as_float(va[2 * i + 1])) * __uint_as_float(vb[2 * i + 1]);
-              pk[i] = pack_bf16x2(h0, h1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(h + col);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)  // streaming: keep L2 for the weight and X tiles
-              __stcs(dst + i, make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+      // M = 256: lane r is row r of this CTA's 128, all 256 columns of the block.
+      // M = 128: lane r is row r % 64 of this CTA's 64; lanes >= 64 hold the second half of N.
+      const bool full = w.m == 256;
+      const int sub = full ? 0 : r >> 6;
+      const int64_t row = w.row0 + (full ? (int)rank * 128 + r : (int)rank * 64 + (r & 63));
+      for (int g = 0; g < 2; ++g) {
+        if (g >= w.count) {
+          tc_fence_before();
+          mbar_arrive_cluster(tempty0 + (uint32_t)g * 8u);
+          continue;
+        }
+        const int cb = w.s + g;
+        const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)g * 256u;
+        // This warp's share of the accumulator goes to registers first; the accumulator is
+        // released to the next tile's MMAs before the SwiGLU and the stores.
+        uint32_t v[4][32];
+        if (KIND == KIND_G13) {
+          if (full) {  // a in columns [0,128), b in [128,256); this warp: 64*half + [0,64)
+            const uint32_t c0 = 64u * half;
+            tmem_ld32(tb + c0, v[0]);
+            tmem_ld32(tb + c0 + 32, v[1]);
+            tmem_ld32(tb + 128 + c0, v[2]);
+            tmem_ld32(tb + 128 + c0 + 32, v[3]);
+          } else {     // a in [0,64), b in [64,128); this warp: 32*half + [0,32)
+            const uint32_t c0 = 32u * half;
+            tmem_ld32(tb + c0, v[0]);
+            tmem_ld32(tb + 64 + c0, v[2]);
+          }
+        } else {       // this warp: 128*half + [0,128) (full) or 64*half + [0,64) (half)
+          const uint32_t c0 = full ? 128u * half : 64u * half;
+          tmem_ld32(tb + c0, v[0]);
+          tmem_ld32(tb + c0 + 32, v[1]);
+          if (full) {
+            tmem_ld32(tb + c0 + 64, v[2]);
+            tmem_ld32(tb + c0 + 96, v[3]);
           }
         }
-      } else {
-        float* y = static_cast<float*>(a.out) + row * a.out_ld;
-#pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tb + cc * 32, v);
-          tmem_ld_wait();
-          const int col = w.nt * 256 + cc * 32;
-          if (col < a.nw) {
-            float4* dst = reinterpret_cast<float4*>(y + col);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive_cluster(tempty0 + (uint32_t)g * 8u);
+        if (KIND == KIND_G13) {
+          __nv_bfloat16* h = static_cast<__nv_bfloat16*>(a.out) + row * a.out_ld;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              __stcs(dst + i, make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                          __uint_as_float(v[4 * i + 2]),
-                                          __uint_as_float(v[4 * i + 3])));
+          for (int j = 0; j < 2; ++j) {
+            if (j == 1 && !full) break;
+            const int col = cb * 128 + sub * 64 + (full ? 64 * half + 32 * j : 32 * half);
+            if (col < a.nw) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float h0 = silu_epilogue(__uint_as_float(v[j][2 * i])) *
+                                 __uint_as_float(v[2 + j][2 * i]);
+                const float h1 = silu_epilogue(__uint_as_float(v[j][2 * i + 1])) *
+                                 __uint_as_float(v[2 + j][2 * i + 1]);
+                pk[i] = pack_bf16x2(h0, h1);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(h + col);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)  // streaming: keep L2 for the weight and X tiles
+                __stcs(dst + i,
+                       make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]));
+            }
+          }
+        } else {
+          float* y = static_cast<float*>(a.out) + row * a.out_ld;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j >= 2 && !full) break;
+            const int col = cb * 256 + sub * 128 + (full ? 128 * half : 64 * half) + 32 * j;
+            if (col < a.nw) {
+              float4* dst = reinterpret_cast<float4*>(y + col);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                __stcs(dst + i, make_float4(__uint_as_float(v[j][4 * i]),
+                                            __uint_as_float(v[j][4 * i + 1]),
+                                            __uint_as_float(v[j][4 * i + 2]),
+                                            __uint_as_float(v[j][4 * i + 3])));
+            }
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive_cluster(tempty0 + acc * 8u);
     }
     __syncwarp();
   }
@@ -560,7 +694,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, a.tmem_cols);
+    tmem_dealloc_pair(tmem_base, 512);
   }
 }
 
@@ -659,7 +793,8 @@ static cudaError_t launch_one(const CUtensorMap& mx, const CUtensorMap& mw0,
 
 template <int KIND>
 static cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw0,
-                               const CUtensorMap& mw1, TcArgs a, int max_work, cudaStream_t s) {
+                               const CUtensorMap& mw1, const CUtensorMap& mw0h,
+                               const CUtensorMap& mw1h, TcArgs a, int max_work, cudaStream_t s) {
   const size_t smem = (size_t)a.stages * a.stage_bytes + sizeof(PairCtrl) + 1024;
   auto kern = tc_pair_gemm_kernel<KIND>;
   cudaError_t e =
@@ -673,7 +808,7 @@ static cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw0,
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.blockDim = dim3(PAIR_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
@@ -693,7 +828,7 @@ static cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw0,
   if (pairs < 1) pairs = 1;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, kern, mx, mw0, mw1, a);
+  e = cudaLaunchKernelEx(&cfg, kern, mx, mw0, mw1, mw0h, mw1h, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -720,39 +855,41 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   const int d = (int)p.d, F = (int)p.F, n = p.n;
   cudaError_t err;
   if (p.pair) {  // 256-row tiles on CTA pairs
+    CUtensorMap mW1h, mW3h;  // 64-row boxes for the M = 128 tiles of G13
     if (!make_map(&mX, w.xperm, d, p.rows_max, 128) ||
         !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||
         !make_map(&mW3, W3, d, (uint64_t)n * F, 128) ||
+        !make_map(&mW1h, W1, d, (uint64_t)n * F, 64) ||
+        !make_map(&mW3h, W3, d, (uint64_t)n * F, 64) ||
         !make_map(&mH, w.h, F, p.rows_max, 128) ||
         !make_map(&mW2, W2, F, (uint64_t)n * d, 128))
       return cudaErrorInvalidValue;
-    const int pair_tiles_max = (int)(p.rows_max / 256);
+    const int pair_tiles_max = (int)(p.rows_max / 128);  // bound on row tiles (grid size)
     TcArgs a{};
     a.offsets = w.offsets;
     a.n = n;
-    a.stage_bytes = 2 * TILE_BYTES;
-    a.tx_bytes = 2 * TILE_BYTES;  // per CTA; the leader expects both CTAs' bytes
+    a.stage_bytes = 3 * TILE_BYTES;  // A rows + two column blocks' halves
     a.stages = stages_for(a.stage_bytes);
-    a.acc_cols = 256;
-    a.nacc = 2;
-    a.tmem_cols = 512;
     a.status = w.status;
     a.num_kb = d / 64;
     a.nw = F;
-    a.n_tiles = (F + 127) / 128;
+    a.n_blocks = (F + 127) / 128;
+    a.n_tiles = (a.n_blocks + 1) / 2;
     a.out = w.h;
     a.out_ld = F;
-    if ((err = launch_pair<KIND_G13>(mX, mW1, mW3, a, pair_tiles_max * a.n_tiles, s)) !=
+    if ((err = launch_pair<KIND_G13>(mX, mW1, mW3, mW1h, mW3h, a, pair_tiles_max * a.n_tiles,
+                                     s)) !=
         cudaSuccess)
       return err;
     if ((err = record(ev, 0, s)) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
       return err;
     a.num_kb = F / 64;
     a.nw = d;
-    a.n_tiles = (d + 255) / 256;
+    a.n_blocks = (d + 255) / 256;
+    a.n_tiles = (a.n_blocks + 1) / 2;
     a.out = w.y;
     a.out_ld = d;
-    if ((err = launch_pair<KIND_G2>(mH, mW2, mW2, a, pair_tiles_max * a.n_tiles, s)) !=
+    if ((err = launch_pair<KIND_G2>(mH, mW2, mW2, mW2, mW2, a, pair_tiles_max * a.n_tiles, s)) !=
         cudaSuccess)
       return err;
     return record(ev, 2, s);

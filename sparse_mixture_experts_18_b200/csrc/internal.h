@@ -85,7 +85,7 @@ PdlLaunch<KArgs...> pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
 bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p);
 Workspace carve(const Plan& p, void* base);
 
-int route_tokens_per_block(int n);
+int route_tokens_per_block(int K);
 cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Workspace& w,
                          cudaStream_t s);
 // ev (may be null): events recorded after G13, after the split-K reduction, after G2.

@@ -54,15 +54,14 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   Plan q;
   q.T = T; q.d = d; q.F = F; q.n = n; q.K = K; q.dt = dt; q.stack = stack;
   q.swap = dt == 1 && T <= 256 && T * K < 64 * (int64_t)n;
-  // CTA pairs once the extra padding (~64 rows per expert more than 128-row tiles) costs
-  // less than the pair tiles' higher tensor-pipe utilisation gains.
+  // CTA pairs (256-row tiles, 128-row tails) from about 80 rows per expert on.
   q.pair = dt == 1 && !q.swap && T * K >= 640 * (int64_t)n;
-  q.row_align = dt == 0 ? SIMT_TILE : (q.swap ? 1 : (q.pair ? 2 * TILE_M : TILE_M));
+  q.row_align = dt == 0 ? SIMT_TILE : (q.swap ? 1 : TILE_M);
   const int64_t P = T * K;
   q.rows_max = (P + (int64_t)n * (q.row_align - 1) + q.row_align - 1) / q.row_align * q.row_align;
   if (q.swap) q.rows_max = (P + 15) / 16 * 16;  // >= tok_tile rows for the token TMA box
   if (q.rows_max >= ((int64_t)1 << 31) / 2) return false;
-  const int tokb = route_tokens_per_block(n);
+  const int tokb = route_tokens_per_block(K);
   q.nblk = (T + tokb - 1) / tokb;
   q.fused_route = T <= 64 && T * K <= 1024;  // limits of route_split_kernel
   if (q.swap) {

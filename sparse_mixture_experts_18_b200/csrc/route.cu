@@ -58,83 +58,87 @@ struct GroupSync {
   }
 };
 
-// Router, TopK and softmax of tokens [t0, t0 + ntok), ntok <= TOKB, by ROUTE_THREADS threads
-// (tid = 0..255).  Each thread accumulates the logits of all TOKB tokens over its 8-element
-// chunks of the hidden dimension (so a W_g row is loaded once per TOKB tokens); lanes and
-// then warps are summed in a fixed order.  hist (shared, may be null) counts selections.
-template <typename Tin, int NPAD, int TOKB, typename Sync>
-__device__ __forceinline__ void route_token_block(
-    const Tin* __restrict__ x, const float* __restrict__ Wg, int64_t t0, int ntok, int d, int n,
-    int K, int tid, float (*red)[64], float (*logits)[NPAD], int* hist,
-    int32_t* __restrict__ idx, float* __restrict__ gate, Sync sync) {
-  static_assert(NPAD * TOKB == 64, "64 partial sums per lane");
-  const int warp = tid >> 5, lane = tid & 31;
-  float acc[TOKB][NPAD];
-#pragma unroll
-  for (int a = 0; a < TOKB; ++a)
-#pragma unroll
-    for (int e = 0; e < NPAD; ++e) acc[a][e] = 0.f;
+// Router, TopK and softmax of tokens [t0, t0 + ntok), ntok <= RT_TOK, by ROUTE_THREADS
+// threads (tid = 0..255).  Experts are taken eight at a time: each thread accumulates the
+// logits of the block's tokens for eight experts over its 8-element chunks of the hidden
+// dimension (so each W_g row segment is loaded once per RT_TOK tokens); lanes and then warps
+// are summed in a fixed order.  hist (shared, may be null) counts selections.
+constexpr int RT_TOK = 8;
 
-  // 8-element chunks of the hidden dimension, thread-interleaved (coalesced 16-byte loads)
-  for (int ci = tid; ci < d / 8; ci += ROUTE_THREADS) {
-    const int j0 = ci * 8;
-    Vec8<Tin> xv[TOKB];
+template <typename Tin, typename Sync>
+__device__ __forceinline__ void route_token_block(
+    const Tin* __restrict__ x, const float* __restrict__ Wg, bool w_vec, int64_t t0, int ntok,
+    int d, int n, int K, int tid, float (*red)[64], float (*logits)[MAX_EXPERTS], int* hist,
+    int32_t* __restrict__ idx, float* __restrict__ gate, Sync sync) {
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int eg = 0; eg < n; eg += 8) {
+    float acc[RT_TOK][8];
 #pragma unroll
-    for (int a = 0; a < TOKB; ++a)
-      if (a < ntok) xv[a].load(x + (t0 + a) * (int64_t)d + j0);
+    for (int a = 0; a < RT_TOK; ++a)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float w[NPAD];
-      const float* wr = Wg + (int64_t)(j0 + i) * n;
-      if (NPAD == 8 && n == 8) {  // one 32-byte row: two aligned float4 loads
-        const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr));
-        const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr) + 1);
-        w[0] = w0.x; w[1] = w0.y; w[2] = w0.z; w[3] = w0.w;
-        w[4] = w1.x; w[5] = w1.y; w[6] = w1.z; w[7] = w1.w;
-      } else {
+      for (int e = 0; e < 8; ++e) acc[a][e] = 0.f;
+
+    // 8-element chunks of the hidden dimension, thread-interleaved (coalesced 16-byte loads)
+    for (int ci = tid; ci < d / 8; ci += ROUTE_THREADS) {
+      const int j0 = ci * 8;
+      Vec8<Tin> xv[RT_TOK];
 #pragma unroll
-        for (int e = 0; e < NPAD; ++e) w[e] = e < n ? __ldg(wr + e) : 0.f;
-      }
+      for (int a = 0; a < RT_TOK; ++a)
+        if (a < ntok) xv[a].load(x + (t0 + a) * (int64_t)d + j0);
 #pragma unroll
-      for (int a = 0; a < TOKB; ++a) {
-        if (a < ntok) {
-          const float xa = xv[a].get(i);
+      for (int i = 0; i < 8; ++i) {
+        float w[8];
+        const float* wr = Wg + (int64_t)(j0 + i) * n + eg;
+        if (w_vec) {  // eight experts of one row: two aligned float4 loads
+          const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr));
+          const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr) + 1);
+          w[0] = w0.x; w[1] = w0.y; w[2] = w0.z; w[3] = w0.w;
+          w[4] = w1.x; w[5] = w1.y; w[6] = w1.z; w[7] = w1.w;
+        } else {
 #pragma unroll
-          for (int e = 0; e < NPAD; ++e) acc[a][e] = fmaf(xa, w[e], acc[a][e]);
+          for (int e = 0; e < 8; ++e) w[e] = eg + e < n ? __ldg(wr + e) : 0.f;
+        }
+#pragma unroll
+        for (int a = 0; a < RT_TOK; ++a) {
+          if (a < ntok) {
+            const float xa = xv[a].get(i);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[a][e] = fmaf(xa, w[e], acc[a][e]);
+          }
         }
       }
     }
-  }
 
-  // Butterfly reduce-scatter of the 64 partial sums over the 32 lanes: after five steps
-  // each lane owns two complete warp sums.
-  float v[64];
+    // Butterfly reduce-scatter of the 64 partial sums over the 32 lanes: after five steps
+    // each lane owns two complete warp sums.
+    float v[64];
 #pragma unroll
-  for (int a = 0; a < TOKB; ++a)
+    for (int a = 0; a < RT_TOK; ++a)
 #pragma unroll
-    for (int e = 0; e < NPAD; ++e) v[a * NPAD + e] = acc[a][e];
-  int base = 0;
+      for (int e = 0; e < 8; ++e) v[a * 8 + e] = acc[a][e];
+    int base = 0;
 #pragma unroll
-  for (int half = 32, off = 16; off >= 1; half >>= 1, off >>= 1) {
-    const bool upper = (lane & off) != 0;
+    for (int half = 32, off = 16; off >= 1; half >>= 1, off >>= 1) {
+      const bool upper = (lane & off) != 0;
 #pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = upper ? v[i] : v[half + i];
-      const float keep = upper ? v[half + i] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      for (int i = 0; i < half; ++i) {
+        const float send = upper ? v[i] : v[half + i];
+        const float keep = upper ? v[half + i] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      }
+      if (upper) base += half;
     }
-    if (upper) base += half;
-  }
-  red[warp][base] = v[0];
-  red[warp][base + 1] = v[1];
-  sync();
-  if (tid < 64) {
-    float s = 0.f;
+    red[warp][base] = v[0];
+    red[warp][base + 1] = v[1];
+    sync();
+    if (tid < 64 && eg + (tid & 7) < n) {
+      float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < ROUTE_THREADS / 32; ++w) s += red[w][tid];
-    logits[tid / NPAD][tid % NPAD] = s;
+      for (int w = 0; w < ROUTE_THREADS / 32; ++w) sum += red[w][tid];
+      logits[tid >> 3][eg + (tid & 7)] = sum;
+    }
+    sync();
   }
-  sync();
 
   // TopK by repeated arg-max (strict '>' keeps the lower index on ties), then Softmax over
   // the kept logits shifted by the largest; the selection runs twice (normaliser, then
@@ -168,23 +172,24 @@ __device__ __forceinline__ void route_token_block(
   sync();
 }
 
-// Block b routes tokens [b*TOKB, b*TOKB + TOKB) and writes its expert histogram.
-template <typename Tin, int NPAD, int TOKB>
+// Block b routes tokens [b*tokb, b*tokb + tokb) (tokb <= RT_TOK) and writes its expert
+// histogram.
+template <typename Tin>
 __global__ void __launch_bounds__(ROUTE_THREADS)
-    router_topk_kernel(const Tin* __restrict__ x, const float* __restrict__ Wg, int64_t T,
-                       int d, int n, int K, int32_t* __restrict__ idx,
+    router_topk_kernel(const Tin* __restrict__ x, const float* __restrict__ Wg, bool w_vec,
+                       int64_t T, int d, int n, int K, int tokb, int32_t* __restrict__ idx,
                        float* __restrict__ gate, int32_t* __restrict__ blk_counts) {
   pdl_wait();
   pdl_trigger();
   __shared__ float red[ROUTE_THREADS / 32][64];
-  __shared__ float logits[TOKB][NPAD];
-  __shared__ int hist[64];
-  const int64_t t0 = (int64_t)blockIdx.x * TOKB;
-  const int ntok = (int)(T - t0 < TOKB ? T - t0 : TOKB);
-  if (threadIdx.x < 64) hist[threadIdx.x] = 0;
+  __shared__ float logits[RT_TOK][MAX_EXPERTS];
+  __shared__ int hist[MAX_EXPERTS];
+  const int64_t t0 = (int64_t)blockIdx.x * tokb;
+  const int ntok = (int)(T - t0 < tokb ? T - t0 : tokb);
+  if (threadIdx.x < MAX_EXPERTS) hist[threadIdx.x] = 0;
   __syncthreads();
-  route_token_block<Tin, NPAD, TOKB>(x, Wg, t0, ntok, d, n, K, threadIdx.x, red, logits, hist,
-                                     idx, gate, CtaSync{});
+  route_token_block<Tin>(x, Wg, w_vec, t0, ntok, d, n, K, threadIdx.x, red, logits, hist, idx,
+                         gate, CtaSync{});
   if (threadIdx.x < n) blk_counts[(int64_t)blockIdx.x * n + threadIdx.x] = hist[threadIdx.x];
 }
 
@@ -429,8 +434,10 @@ __global__ void __launch_bounds__(1024)
   const int64_t chunk = (nblk + G - 1) / G;
   const int64_t b0 = i * chunk, b1 = b0 + chunk < nblk ? b0 + chunk : nblk;
   int local = 0;
-  if (e < n)
+  if (e < n) {
+#pragma unroll 8
     for (int64_t b = b0; b < b1; ++b) local += blk_counts[b * n + e];
+  }
   part[threadIdx.x] = local;
   __syncthreads();
   // inclusive Hillis-Steele scan inside each expert's G-thread segment
@@ -442,6 +449,7 @@ __global__ void __launch_bounds__(1024)
   }
   if (e < n) {
     int run = part[threadIdx.x] - local;  // exclusive prefix of this thread's range
+#pragma unroll 8
     for (int64_t b = b0; b < b1; ++b) {
       blk_base[b * n + e] = run;
       run += blk_counts[b * n + e];
@@ -478,7 +486,7 @@ __global__ void __launch_bounds__(256)
   __shared__ int ent_row[64];
   const int64_t t0 = (int64_t)blockIdx.x * tokb;
   const int ntok = (int)(T - t0 < tokb ? T - t0 : tokb);
-  const int E = ntok * K;  // <= 64 by construction (tokb * K <= tokb * NPAD = 64)
+  const int E = ntok * K;  // <= 64: tokb = route_tokens_per_block(K)
   const int i = threadIdx.x;
   if (i < E) ent_e[i] = idx[t0 * K + i];
   __syncthreads();
@@ -505,26 +513,19 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------- host launchers
 
-int route_tokens_per_block(int n) { return n <= 8 ? 8 : n <= 16 ? 4 : n <= 32 ? 2 : 1; }
+// Tokens per router / permute block: eight, or fewer when K > 8 so that a block's
+// (token, slot) entries stay within 64.
+int route_tokens_per_block(int K) { return K <= 8 ? RT_TOK : (64 / K > 0 ? 64 / K : 1); }
 
 template <typename Tin>
 static cudaError_t launch_router_t(const Tin* x, const float* Wg, int64_t T, int d, int n,
                                    int K, int32_t* idx, float* gate, int32_t* blk_counts,
                                    cudaStream_t s) {
-  const int tokb = route_tokens_per_block(n);
+  const int tokb = route_tokens_per_block(K);
   const unsigned grid = (unsigned)((T + tokb - 1) / tokb);
-  if (n <= 8)
-    pdl(router_topk_kernel<Tin, 8, 8>, grid, ROUTE_THREADS, 0, s)(x, Wg, T, d, n, K, idx, gate,
-                                                                 blk_counts);
-  else if (n <= 16)
-    pdl(router_topk_kernel<Tin, 16, 4>, grid, ROUTE_THREADS, 0, s)(x, Wg, T, d, n, K, idx,
-                                                                  gate, blk_counts);
-  else if (n <= 32)
-    pdl(router_topk_kernel<Tin, 32, 2>, grid, ROUTE_THREADS, 0, s)(x, Wg, T, d, n, K, idx,
-                                                                  gate, blk_counts);
-  else
-    pdl(router_topk_kernel<Tin, 64, 1>, grid, ROUTE_THREADS, 0, s)(x, Wg, T, d, n, K, idx,
-                                                                  gate, blk_counts);
+  const bool w_vec = n % 8 == 0 && (reinterpret_cast<uintptr_t>(Wg) & 15u) == 0;
+  pdl(router_topk_kernel<Tin>, grid, ROUTE_THREADS, 0, s)(x, Wg, w_vec, T, d, n, K, tokb, idx,
+                                                          gate, blk_counts);
   return cudaGetLastError();
 }
 
@@ -555,7 +556,7 @@ cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Wo
   pdl(route_scan_kernel, 1, 1024, 0, s)(w.blk_counts, p.nblk, p.n, p.row_align, p.rows_max,
                                        w.blk_base, w.counts, w.offsets, w.status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const int tokb = route_tokens_per_block(p.n);
+  const int tokb = route_tokens_per_block(p.K);
   if (p.dt == 1)
     pdl(permute_gather_kernel<__nv_bfloat16>, (unsigned)p.nblk, 256, 0, s)(
         static_cast<const __nv_bfloat16*>(x), p.T, (int)p.d, p.n, p.K, tokb, w.idx,

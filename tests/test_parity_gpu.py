@@ -95,8 +95,10 @@ def _biased_layer(w, bias):
     return layer
 
 
-@pytest.mark.parametrize("T", [16, 900])
+@pytest.mark.parametrize("T", [16, 900, 2600])
 def test_all_tokens_to_two_experts(T):
+    # T = 2600 takes the CTA-pair tiling: 2600 rows per expert are ten 256-row tiles and one
+    # 128-row tile (M = 128), and six experts have no rows
     w = moe_inputs.small(T=T, d=256, F=384, zipf=0.0)
     x = moe_inputs.make_x(w)
     x[:, 0] = 1.0
