@@ -298,7 +298,9 @@ def run_gpu(args, w):
                                   else ""),
                    "tokens_per_rank": w.T, "l2": "inputs larger than L2 "
                    f"({w.layers * 3 * w.n * w.F * w.d * es / 1e9:.2f} GB of expert weights)",
-                   "parallelism": f"replicas x{world}", "tiling": tiling,
+                   "parallelism": f"replicas x{world}",
+                   "tiling": tiling + (", A rows gathered from x" if args.gather_x and plan["pair"]
+                                       else ""),
                    "active_experts": n_active, "expert_counts": counts},
         "tflops": round(tflops, 3),
         "pct_roofline": {"bound": "hbm" if step_hbm else "tensor",
@@ -400,7 +402,12 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=4,
                     help="tokens per oracle sample (CPU baseline / reference arm)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gather-x", action="store_true",
+                    help="CTA-pair path: gather G13's A rows from x (TMA gather4) instead of "
+                         "X_perm, gates applied in G2 (sets MOE_GATHER_X=1)")
     args = ap.parse_args(argv)
+    if args.gather_x:
+        os.environ["MOE_GATHER_X"] = "1"
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = moe_inputs.WORKLOADS[args.workload]

@@ -6,7 +6,9 @@
 //            Indonesian news summary's expert-parallelism notes put it).  fp32 sum over the
 //            K slots in slot order (and over split slabs in split order), rounded once;
 //            16-byte vectorised loads and stores.  With a residual input, out = resid + sum,
-//            also in fp32 before the single rounding (the stacked-block workload).
+//            also in fp32 before the single rounding (the stacked-block workload).  On the
+//            CTA-pair path the down-projection epilogue has already multiplied each row by
+//            its gate, and the combine only sums the K rows.
 //  rmsnorm:  xn = x / sqrt(mean(x^2) + eps) with unit gain, fp32 math, bf16 result.
 #include "internal.h"
 
@@ -91,7 +93,7 @@ __global__ void __launch_bounds__(256)
     for (int k = 0; k < K; ++k) {
       const int row = inv[t * K + k];
       if (row < 0) continue;
-      const float g = gate[t * K + k];
+      const float g = gate ? gate[t * K + k] : 1.f;  // null: rows already gated
       const float* src = Y + (int64_t)row * d + c;
       float4 part[COMBINE_MAX_S];
 #pragma unroll
@@ -141,7 +143,7 @@ __global__ void __launch_bounds__(256)
       for (int k = 0; k < K; ++k) {
         const int row = inv[t * K + k];
         if (row < 0) continue;
-        const float g = gate[t * K + k];
+        const float g = gate ? gate[t * K + k] : 1.f;  // null: rows already gated
         float4 yk[COMBINE_U];
 #pragma unroll
         for (int u = 0; u < COMBINE_U; ++u) yk[u] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -186,6 +188,7 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
                            cudaStream_t s) {
   const int S = p.swap ? p.s2 : 1;
   const int64_t split_stride = p.rows_max * p.d;
+  const float* gates = p.gather_x ? nullptr : w.gate;  // gather_x: G2 applied the gates
   if (p.T >= 1024) {  // enough tokens for one warp each
     const int64_t blocks = (p.T + 7) / 8;
     const unsigned g = (unsigned)(blocks < ((int64_t)1 << 30) ? blocks : ((int64_t)1 << 30));
@@ -193,20 +196,20 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
       auto* o = static_cast<__nv_bfloat16*>(out);
       if (resid)
         pdl(combine_rows_kernel<__nv_bfloat16, true>, g, 256, 0, s)(
-            w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
+            w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o,
             static_cast<const __nv_bfloat16*>(resid));
       else
         pdl(combine_rows_kernel<__nv_bfloat16, false>, g, 256, 0, s)(
-            w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
+            w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr);
     } else {
       auto* o = static_cast<float*>(out);
       if (resid)
         pdl(combine_rows_kernel<float, true>, g, 256, 0, s)(w.y, S, split_stride, p.T, (int)p.d,
-                                                           p.K, w.inv, w.gate, o,
+                                                           p.K, w.inv, gates, o,
                                                            static_cast<const float*>(resid));
       else
         pdl(combine_rows_kernel<float, false>, g, 256, 0, s)(w.y, S, split_stride, p.T,
-                                                            (int)p.d, p.K, w.inv, w.gate, o,
+                                                            (int)p.d, p.K, w.inv, gates, o,
                                                             nullptr);
     }
     return cudaGetLastError();
@@ -219,20 +222,20 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
     auto* o = static_cast<__nv_bfloat16*>(out);
     if (resid)
       pdl(combine_kernel<__nv_bfloat16, true>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o,
           static_cast<const __nv_bfloat16*>(resid));
     else
       pdl(combine_kernel<__nv_bfloat16, false>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr);
   } else {
     auto* o = static_cast<float*>(out);
     if (resid)
       pdl(combine_kernel<float, true>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o,
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o,
           static_cast<const float*>(resid));
     else
       pdl(combine_kernel<float, false>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate, o, nullptr);
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr);
   }
   return cudaGetLastError();
 }

@@ -269,6 +269,22 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// Four rows y0..y3 of a 2-D bf16 tensor whose map has a one-row box (64 elements, 128-byte
+// swizzle) into 512 consecutive bytes of shared memory, by either CTA of a pair; completion
+// is counted on the leader's barrier.  Rows outside the tensor (e.g. y = number of rows)
+// arrive as zeros.  No multicast.
+__device__ __forceinline__ void tma_gather4_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster_addr, int32_t x,
+                                                 int32_t y0, int32_t y1, int32_t y2, int32_t y3,
+                                                 uint64_t cache_hint) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr),
+      "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "l"(cache_hint)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst_smem)),

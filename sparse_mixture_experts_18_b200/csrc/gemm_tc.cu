@@ -50,6 +50,12 @@ struct TcArgs {
   int64_t out_ld;          // elements per output row
   int64_t split_stride;    // elements between split slabs
   uint32_t* status;
+  // CTA pairs reading x directly (G13: row_tok, counts, gather_T) and applying the gates
+  // (G2: row_gate); null otherwise
+  const int32_t* row_tok;  // token of each permuted row
+  const int32_t* counts;   // [n] rows routed to each expert
+  int gather_T;            // rows of x (a row index past the end reads zeros)
+  const float* row_gate;   // gate of each permuted row
 };
 
 struct Ctrl {
@@ -361,6 +367,7 @@ struct PairCtrl {
   int abort;
   int off[MAX_EXPERTS + 1];
   int tbase[MAX_EXPERTS + 1];  // row tiles of experts before e
+  int cnt[MAX_EXPERTS];        // gather: rows routed to each expert
 };
 
 // Tile order: expert, then column-block pair, then row tile (the row tiles of a column-block
@@ -452,6 +459,7 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
   pdl_wait();  // expert offsets and operands come from the previous kernels
   pdl_trigger();
   if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
+  if (a.counts != nullptr && threadIdx.x < a.n) c->cnt[threadIdx.x] = a.counts[threadIdx.x];
   __syncthreads();
   if (threadIdx.x == 0) {
     c->tbase[0] = 0;
@@ -467,25 +475,41 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_normal();
-      const uint64_t pol_x = policy_evict_last();
-      const uint32_t full0 = map_to_rank(&c->full[0], 0);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int id = pair; id < total && ok; id += npairs) {
-        const Work w = decode_pair_work(a, c, ps, id);
-        if (w.count == 0) continue;
-        const int row = w.row0 + (int)rank * (w.m >> 1);
-        for (int kb = 0; kb < a.num_kb; ++kb) {
-          if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort)) { ok = false; break; }
-          uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+    // Lane 0 waits for free stages and loads the weight halves (and X_perm rows).  When G13
+    // reads x directly, every lane gathers four of the CTA's 128 A rows per stage (one
+    // tile::gather4 of the x rows of their tokens; padding rows read zeros).
+    const bool gather = KIND == KIND_G13 && a.row_tok != nullptr;
+    const uint64_t pol_w = policy_evict_normal();
+    const uint64_t pol_x = policy_evict_last();
+    const uint32_t full0 = map_to_rank(&c->full[0], 0);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int id = pair; id < total && ok; id += npairs) {
+      const Work w = decode_pair_work(a, c, ps, id);
+      if (w.count == 0) continue;
+      const int rows_cta = w.m >> 1;
+      const int row = w.row0 + (int)rank * rows_cta;
+      int tok[4] = {0, 0, 0, 0};
+      if (gather) {
+        const int end = c->off[w.e] + c->cnt[w.e];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = 4 * lane + j;
+          tok[j] = i < rows_cta && row + i < end ? a.row_tok[row + i] : a.gather_T;
+        }
+      }
+      for (int kb = 0; kb < a.num_kb; ++kb) {
+        if (lane == 0) ok = mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        uint8_t* st = smem + (size_t)stage * a.stage_bytes;
+        const uint32_t fb = full0 + (uint32_t)stage * 8u;
+        const int k = kb * 64;
+        if (lane == 0) {
           if (leader)
             mbar_arrive_expect_tx(&c->full[stage], 2u * (uint32_t)(1 + w.count) * TILE_BYTES);
-          const uint32_t fb = full0 + (uint32_t)stage * 8u;
-          const int k = kb * 64;
-          tma_load_2d_pair(st, &tmX, fb, k, row, pol_x);
+          if (!gather) tma_load_2d_pair(st, &tmX, fb, k, row, pol_x);
           for (int j = 0; j < w.count; ++j) {
             const int cb = w.s + j;
             uint8_t* bt = st + (1 + j) * TILE_BYTES;
@@ -499,10 +523,14 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
             else
               tma_load_2d_pair(bt, &tmW0, fb, k, w.e * a.nw + cb * 256 + (int)rank * 128, pol_w);
           }
-          if (++stage == a.stages) { stage = 0; phase ^= 1u; }
         }
+        if (gather)
+          tma_gather4_pair(st + lane * 512, &tmX, fb, k, tok[0], tok[1], tok[2], tok[3], pol_x);
+        if (++stage == a.stages) { stage = 0; phase ^= 1u; }
       }
-      // every MMA commit aimed at this CTA's empty barriers has landed before it may exit
+    }
+    // every MMA commit aimed at this CTA's empty barriers has landed before it may exit
+    if (lane == 0) {
       for (int s = 0; ok && s < a.stages; ++s) {
         if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort)) break;
         if (++stage == a.stages) { stage = 0; phase ^= 1u; }
@@ -660,6 +688,8 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
           }
         } else {
           float* y = static_cast<float*>(a.out) + row * a.out_ld;
+          // the row's gate (the combine then only sums); padding rows are never read
+          const float g = a.row_gate != nullptr ? a.row_gate[row] : 1.f;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (j >= 2 && !full) break;
@@ -668,10 +698,10 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
               float4* dst = reinterpret_cast<float4*>(y + col);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
-                __stcs(dst + i, make_float4(__uint_as_float(v[j][4 * i]),
-                                            __uint_as_float(v[j][4 * i + 1]),
-                                            __uint_as_float(v[j][4 * i + 2]),
-                                            __uint_as_float(v[j][4 * i + 3])));
+                __stcs(dst + i, make_float4(g * __uint_as_float(v[j][4 * i]),
+                                            g * __uint_as_float(v[j][4 * i + 1]),
+                                            g * __uint_as_float(v[j][4 * i + 2]),
+                                            g * __uint_as_float(v[j][4 * i + 3])));
             }
           }
         }
@@ -856,7 +886,9 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   cudaError_t err;
   if (p.pair) {  // 256-row tiles on CTA pairs
     CUtensorMap mW1h, mW3h;  // 64-row boxes for the M = 128 tiles of G13
-    if (!make_map(&mX, w.xperm, d, p.rows_max, 128) ||
+    // gather_x: G13's A rows are gathered from x (one-row boxes), else loaded from X_perm
+    if (!(p.gather_x ? make_map(&mX, x, d, (uint64_t)p.T, 1)
+                     : make_map(&mX, w.xperm, d, p.rows_max, 128)) ||
         !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||
         !make_map(&mW3, W3, d, (uint64_t)n * F, 128) ||
         !make_map(&mW1h, W1, d, (uint64_t)n * F, 64) ||
@@ -877,6 +909,11 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
     a.n_tiles = (a.n_blocks + 1) / 2;
     a.out = w.h;
     a.out_ld = F;
+    if (p.gather_x) {
+      a.row_tok = w.row_tok;
+      a.counts = w.counts;
+      a.gather_T = (int)p.T;
+    }
     if ((err = launch_pair<KIND_G13>(mX, mW1, mW3, mW1h, mW3h, a, pair_tiles_max * a.n_tiles,
                                      s)) !=
         cudaSuccess)
@@ -889,6 +926,9 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
     a.n_tiles = (a.n_blocks + 1) / 2;
     a.out = w.y;
     a.out_ld = d;
+    a.row_tok = nullptr;
+    a.counts = nullptr;
+    if (p.gather_x) a.row_gate = w.row_gate;
     if ((err = launch_pair<KIND_G2>(mH, mW2, mW2, mW2, mW2, a, pair_tiles_max * a.n_tiles, s)) !=
         cudaSuccess)
       return err;

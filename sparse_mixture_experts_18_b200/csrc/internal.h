@@ -24,6 +24,8 @@ struct Plan {
   int dt = 1;              // 0 = fp32 (SIMT path), 1 = bf16 (tensor-core path)
   bool swap = false;       // small-batch path: weights are the MMA's 128-row operand
   bool pair = false;       // large batches: 256-row tiles on 2-CTA clusters (cta_group::2)
+  bool gather_x = false;   // pair path: G13 gathers its A rows from x by token (no X_perm),
+                           // G2 applies the gates in its epilogue
   int row_align = 1;       // each expert's group is padded to a multiple of this
   int64_t rows_max = 0;    // upper bound of permuted rows (T*K plus padding)
   int64_t nblk = 0;        // router / permute blocks
@@ -33,7 +35,8 @@ struct Plan {
   bool stack = false;      // workspace also holds the normalised activations
   // workspace byte offsets
   size_t o_rpart;          // small batch: partial router logits [ceil(d/64)][T][n]
-  size_t o_rowtok;         // small batch: token of each permuted row [rows_max]
+  size_t o_rowtok;         // token of each permuted row [rows_max] (small batch, gather_x)
+  size_t o_rowgate;        // gather_x: gate of each permuted row [rows_max]
   size_t o_status, o_idx, o_gate, o_blk_counts, o_blk_base, o_counts, o_offsets, o_inv,
       o_xperm, o_h, o_y, o_p13, o_xn, total;
 };
@@ -43,7 +46,8 @@ struct Workspace {
   uint32_t* status;
   unsigned int* ticket;  // small-batch routing: CTAs finished (in the status header, starts 0)
   float* rpart;          // small-batch routing: partial logits
-  int32_t* row_tok;      // small batch: token of each permuted row
+  int32_t* row_tok;      // token of each permuted row (small batch, gather_x)
+  float* row_gate;       // gather_x: gate of each permuted row
   int32_t *idx, *blk_counts, *blk_base, *counts, *offsets, *inv;
   float* gate;
   void* xperm;  // [rows_max][d] activations in permuted order

@@ -2,6 +2,7 @@
 // the per-shape plan, workspace carving, and the kernel sequence of one MoE block forward:
 //   router + TopK + softmax  ->  histogram scan  ->  permute / gather
 //   ->  expert GEMMs (tensor cores for bf16, CUDA cores for fp32)  ->  gated combine.
+#include <stdlib.h>
 #include <string.h>
 
 #include "../../include/moe.h"
@@ -41,6 +42,16 @@ static int choose_split(int num_kb, int units_per_split, int sms) {
   return best;
 }
 
+// The CTA-pair path's alternative data path (MOE_GATHER_X=1 in the environment, read at
+// every call): G13 gathers its A rows from x by token with TMA tile::gather4 instead of
+// reading X_perm, and G2 applies the gates in its epilogue.  Off by default: on B200 the
+// 512-byte gathers starve the tensor cores (G13 2.3x slower at T = 4096), which costs far
+// more than the X_perm pass it saves.
+static bool gather_x_requested() {
+  const char* v = getenv("MOE_GATHER_X");
+  return v != nullptr && v[0] == '1';
+}
+
 bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p) {
   if (T < 0 || d <= 0 || F <= 0 || n < 1 || n > MAX_EXPERTS || K < 1 || K > n) return false;
   if (dt == 1) {
@@ -57,6 +68,7 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   // CTA pairs (256-row tiles, 128-row tails) from about 80 rows per expert on.
   q.pair = dt == 1 && !q.swap && T * K >= 640 * (int64_t)n;
   q.row_align = dt == 0 ? SIMT_TILE : (q.swap ? 1 : TILE_M);
+  q.gather_x = q.pair && gather_x_requested();
   const int64_t P = T * K;
   q.rows_max = (P + (int64_t)n * (q.row_align - 1) + q.row_align - 1) / q.row_align * q.row_align;
   if (q.swap) q.rows_max = (P + 15) / 16 * 16;  // >= tok_tile rows for the token TMA box
@@ -87,7 +99,9 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   q.o_p13 = take(q.swap ? (size_t)q.s13 * q.rows_max * 2 * F * 4 : 0);
   q.o_xn = take(stack ? (size_t)T * d * es : 0);
   q.o_rpart = take(q.fused_route ? (size_t)((d + 63) / 64) * T * n * 4 : 0);
-  q.o_rowtok = take(q.fused_route ? (size_t)q.rows_max * 4 : 0);
+  // (the layout does not depend on gather_x, so a workspace sized earlier stays valid)
+  q.o_rowtok = take(q.fused_route || q.pair ? (size_t)q.rows_max * 4 : 0);
+  q.o_rowgate = take(q.pair ? (size_t)q.rows_max * 4 : 0);
   q.total = o;
   *p = q;
   return true;
@@ -100,6 +114,7 @@ Workspace carve(const Plan& p, void* base) {
   w.ticket = reinterpret_cast<unsigned int*>(b + p.o_status + 64);
   w.rpart = reinterpret_cast<float*>(b + p.o_rpart);
   w.row_tok = reinterpret_cast<int32_t*>(b + p.o_rowtok);
+  w.row_gate = reinterpret_cast<float*>(b + p.o_rowgate);
   w.idx = reinterpret_cast<int32_t*>(b + p.o_idx);
   w.gate = reinterpret_cast<float*>(b + p.o_gate);
   w.blk_counts = reinterpret_cast<int32_t*>(b + p.o_blk_counts);

@@ -471,14 +471,18 @@ __global__ void __launch_bounds__(1024)
 
 // Block b takes the same tokens as router block b.  Entry i = (token, slot) in token-major
 // order gets rank = number of earlier entries of this block routed to the same expert, so
-// the placement is stable (rows of an expert ordered by token, then slot).
+// the placement is stable (rows of an expert ordered by token, then slot).  Writes the
+// inverse map and either gathers the x rows into X_perm or (xperm == null) records the token
+// and the gate of each row for the GEMMs that read x directly.
 template <typename Tact>
 __global__ void __launch_bounds__(256)
     permute_gather_kernel(const Tact* __restrict__ x, int64_t T, int d, int n, int K,
                           int tokb, const int32_t* __restrict__ idx,
+                          const float* __restrict__ gate,
                           const int32_t* __restrict__ blk_base,
                           const int32_t* __restrict__ offsets, int64_t rows_max,
                           int32_t* __restrict__ inv, Tact* __restrict__ xperm,
+                          int32_t* __restrict__ row_tok, float* __restrict__ row_gate,
                           uint32_t* status) {
   pdl_wait();
   pdl_trigger();
@@ -506,7 +510,12 @@ __global__ void __launch_bounds__(256)
     }
     ent_row[i] = row;
     inv[t0 * K + i] = row;
+    if (xperm == nullptr && row >= 0) {
+      row_tok[row] = (int32_t)(t0 + i / K);
+      row_gate[row] = gate[t0 * K + i];
+    }
   }
+  if (xperm == nullptr) return;
   __syncthreads();
   gather_rows(x, t0, d, K, E, ent_row, xperm, threadIdx.x, blockDim.x);
 }
@@ -559,13 +568,15 @@ cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Wo
   const int tokb = route_tokens_per_block(p.K);
   if (p.dt == 1)
     pdl(permute_gather_kernel<__nv_bfloat16>, (unsigned)p.nblk, 256, 0, s)(
-        static_cast<const __nv_bfloat16*>(x), p.T, (int)p.d, p.n, p.K, tokb, w.idx,
-        w.blk_base, w.offsets, p.rows_max, w.inv, static_cast<__nv_bfloat16*>(w.xperm),
+        static_cast<const __nv_bfloat16*>(x), p.T, (int)p.d, p.n, p.K, tokb, w.idx, w.gate,
+        w.blk_base, w.offsets, p.rows_max, w.inv,
+        p.gather_x ? nullptr : static_cast<__nv_bfloat16*>(w.xperm), w.row_tok, w.row_gate,
         w.status);
   else
     pdl(permute_gather_kernel<float>, (unsigned)p.nblk, 256, 0, s)(
-        static_cast<const float*>(x), p.T, (int)p.d, p.n, p.K, tokb, w.idx, w.blk_base,
-        w.offsets, p.rows_max, w.inv, static_cast<float*>(w.xperm), w.status);
+        static_cast<const float*>(x), p.T, (int)p.d, p.n, p.K, tokb, w.idx, w.gate, w.blk_base,
+        w.offsets, p.rows_max, w.inv, static_cast<float*>(w.xperm), w.row_tok, w.row_gate,
+        w.status);
   return cudaGetLastError();
 }
 

@@ -59,9 +59,10 @@ def test_workspace_bytes(L):
     assert ws(16, 4096, 14336, 65, 2, BF16) == 0                # n > 64
     assert ws(16, 4096, 14336, 8, 9, BF16) == 0                 # K > n
     assert ws(16, 4096, 14336, 8, 0, BF16) == 0                 # K < 1
-    # the prefill layout holds at least the routed rows of X, h and Y
-    T, d, F = 4096, 4096, 14336
-    assert ws(T, d, F, 8, 2, BF16) >= T * 2 * (d * 2 + F * 2 + d * 4)
+    # the prefill layouts hold at least the routed rows of X, h and Y (128-row tiles at
+    # T = 1024, CTA pairs at T = 4096)
+    for T, d, F in ((1024, 4096, 14336), (4096, 4096, 14336)):
+        assert ws(T, d, F, 8, 2, BF16) >= T * 2 * (d * 2 + F * 2 + d * 4)
     assert moe.moe_stack_workspace_bytes(8192, 4096, 14336, 8, 2) > ws(8192, 4096, 14336, 8, 2,
                                                                        BF16)
     assert moe.moe_stack_workspace_bytes(64, 128, 256, 8, 2, F32) == 0

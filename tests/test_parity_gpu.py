@@ -72,6 +72,20 @@ def test_pair_tiling_small(T, d, F, n, K):
     _run(moe_inputs.small(T=T, d=d, F=F, n=n, K=K))
 
 
+@pytest.mark.parametrize("T,d,F,n,K", [(3000, 256, 384, 8, 2), (2700, 320, 448, 8, 2)])
+def test_pair_tiling_gather_x(monkeypatch, T, d, F, n, K):
+    # the alternative CTA-pair data path: A rows gathered from x by token (TMA gather4), gates
+    # applied in the down-projection epilogue
+    monkeypatch.setenv("MOE_GATHER_X", "1")
+    _run(moe_inputs.small(T=T, d=d, F=F, n=n, K=K))
+
+
+@pytest.mark.parametrize("T", [2600])
+def test_all_tokens_to_two_experts_gather_x(monkeypatch, T):
+    monkeypatch.setenv("MOE_GATHER_X", "1")
+    test_all_tokens_to_two_experts(T)
+
+
 @pytest.mark.parametrize("T", [1, 5, 16, 37, 100, 255])
 def test_small_batch_tiling(T):
     # T <= 256 and T*K < 64*n: weights as the 128-row MMA operand, split-K
