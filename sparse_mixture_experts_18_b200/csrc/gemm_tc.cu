@@ -475,9 +475,10 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    // Lane 0 waits for free stages and loads the weight halves (and X_perm rows).  When G13
-    // reads x directly, every lane gathers four of the CTA's 128 A rows per stage (one
-    // tile::gather4 of the x rows of their tokens; padding rows read zeros).
+    // Lane 0 waits for free stages and loads the weight halves and the X_perm rows.  When G13
+    // reads x directly, the whole warp runs the loop and every lane gathers four of the CTA's
+    // 128 A rows per stage (one tile::gather4 of the x rows of their tokens; padding rows read
+    // zeros).
     const bool gather = KIND == KIND_G13 && a.row_tok != nullptr;
     const uint64_t pol_w = policy_evict_normal();
     const uint64_t pol_x = policy_evict_last();
@@ -485,7 +486,7 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int id = pair; id < total && ok; id += npairs) {
+    for (int id = pair; id < total && ok && (gather || lane == 0); id += npairs) {
       const Work w = decode_pair_work(a, c, ps, id);
       if (w.count == 0) continue;
       const int rows_cta = w.m >> 1;
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
       }
       for (int kb = 0; kb < a.num_kb; ++kb) {
         if (lane == 0) ok = mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (gather) ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         uint8_t* st = smem + (size_t)stage * a.stage_bytes;
         const uint32_t fb = full0 + (uint32_t)stage * 8u;

@@ -45,6 +45,7 @@ struct Plan {
 struct Workspace {
   uint32_t* status;
   unsigned int* ticket;  // small-batch routing: CTAs finished (in the status header, starts 0)
+  unsigned int* scan_ticket;  // routing scan: expert CTAs finished (status header, starts 0)
   float* rpart;          // small-batch routing: partial logits
   int32_t* row_tok;      // token of each permuted row (small batch, gather_x)
   float* row_gate;       // gather_x: gate of each permuted row

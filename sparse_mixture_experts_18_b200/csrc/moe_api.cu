@@ -112,6 +112,7 @@ Workspace carve(const Plan& p, void* base) {
   Workspace w;
   w.status = reinterpret_cast<uint32_t*>(b + p.o_status);
   w.ticket = reinterpret_cast<unsigned int*>(b + p.o_status + 64);
+  w.scan_ticket = reinterpret_cast<unsigned int*>(b + p.o_status + 128);
   w.rpart = reinterpret_cast<float*>(b + p.o_rpart);
   w.row_tok = reinterpret_cast<int32_t*>(b + p.o_rowtok);
   w.row_gate = reinterpret_cast<float*>(b + p.o_rowgate);

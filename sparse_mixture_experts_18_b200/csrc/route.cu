@@ -10,6 +10,8 @@
 //                 is how experts with zero gate are skipped (Indonesian news summary,
 //                 section on how the MoE layer is computed) while each expert sees a
 //                 variable number of tokens (same page, implementation notes).
+#include <type_traits>
+
 #include "internal.h"
 
 namespace moe {
@@ -58,6 +60,14 @@ struct GroupSync {
   }
 };
 
+// Shared-memory copy of W_g for the persistent router: row j (n floats) starts at
+// j*n + 4*(j/8).  The skew of four floats per eight rows spreads the rows that the lanes of a
+// warp read together (eight rows apart) over all banks.
+__host__ __device__ __forceinline__ int wg_smem_index(int j, int n) { return j * n + 4 * (j >> 3); }
+__host__ __device__ __forceinline__ size_t wg_smem_bytes(int d, int n) {
+  return ((size_t)d * n + 4 * (size_t)(d >> 3)) * sizeof(float);
+}
+
 // Router, TopK and softmax of tokens [t0, t0 + ntok), ntok <= RT_TOK, by ROUTE_THREADS
 // threads (tid = 0..255).  Experts are taken eight at a time: each thread accumulates the
 // logits of the block's tokens for eight experts over its 8-element chunks of the hidden
@@ -65,7 +75,8 @@ struct GroupSync {
 // are summed in a fixed order.  hist (shared, may be null) counts selections.
 constexpr int RT_TOK = 8;
 
-template <typename Tin, typename Sync>
+// W_SMEM: Wg is a shared-memory copy in the skewed layout of wg_smem_index (and w_vec holds).
+template <typename Tin, bool W_SMEM, typename Sync>
 __device__ __forceinline__ void route_token_block(
     const Tin* __restrict__ x, const float* __restrict__ Wg, bool w_vec, int64_t t0, int ntok,
     int d, int n, int K, int tid, float (*red)[64], float (*logits)[MAX_EXPERTS], int* hist,
@@ -88,13 +99,21 @@ __device__ __forceinline__ void route_token_block(
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float w[8];
-        const float* wr = Wg + (int64_t)(j0 + i) * n + eg;
-        if (w_vec) {  // eight experts of one row: two aligned float4 loads
-          const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr));
-          const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr) + 1);
+        if (W_SMEM || w_vec) {  // eight experts of one row: two aligned float4 loads
+          float4 w0, w1;
+          if (W_SMEM) {
+            const float* wr = Wg + wg_smem_index(j0 + i, n) + eg;
+            w0 = *reinterpret_cast<const float4*>(wr);
+            w1 = *reinterpret_cast<const float4*>(wr + 4);
+          } else {
+            const float* wr = Wg + (int64_t)(j0 + i) * n + eg;
+            w0 = __ldg(reinterpret_cast<const float4*>(wr));
+            w1 = __ldg(reinterpret_cast<const float4*>(wr) + 1);
+          }
           w[0] = w0.x; w[1] = w0.y; w[2] = w0.z; w[3] = w0.w;
           w[4] = w1.x; w[5] = w1.y; w[6] = w1.z; w[7] = w1.w;
         } else {
+          const float* wr = Wg + (int64_t)(j0 + i) * n + eg;
 #pragma unroll
           for (int e = 0; e < 8; ++e) w[e] = eg + e < n ? __ldg(wr + e) : 0.f;
         }
@@ -188,9 +207,52 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
   const int ntok = (int)(T - t0 < tokb ? T - t0 : tokb);
   if (threadIdx.x < MAX_EXPERTS) hist[threadIdx.x] = 0;
   __syncthreads();
-  route_token_block<Tin>(x, Wg, w_vec, t0, ntok, d, n, K, threadIdx.x, red, logits, hist, idx,
-                         gate, CtaSync{});
+  route_token_block<Tin, false>(x, Wg, w_vec, t0, ntok, d, n, K, threadIdx.x, red, logits, hist,
+                                idx, gate, CtaSync{});
   if (threadIdx.x < n) blk_counts[(int64_t)blockIdx.x * n + threadIdx.x] = hist[threadIdx.x];
+}
+
+// Large batches whose router matrix fits in shared memory: each CTA copies W_g once (skewed
+// layout, wg_smem_index) and its two 256-thread groups route token blocks b = 2*CTA + group,
+// then b + 2*grid, ... (same per-block arithmetic, histogram and outputs as
+// router_topk_kernel), so W_g crosses from L2 once per SM instead of once per token block,
+// and two blocks' load latencies overlap on each SM.
+constexpr int RT_SMEM_MAX = 200 * 1024;
+
+template <typename Tin>
+__global__ void __launch_bounds__(2 * ROUTE_THREADS, 1)
+    router_topk_smem_kernel(const Tin* __restrict__ x, const float* __restrict__ Wg, int64_t T,
+                            int d, int n, int K, int tokb, int64_t nblk,
+                            int32_t* __restrict__ idx, float* __restrict__ gate,
+                            int32_t* __restrict__ blk_counts) {
+  extern __shared__ float4 wg_raw[];
+  float* sw = reinterpret_cast<float*>(wg_raw);
+  __shared__ float red[2][ROUTE_THREADS / 32][64];
+  __shared__ float logits[2][RT_TOK][MAX_EXPERTS];
+  __shared__ int hist[2][MAX_EXPERTS];
+  // W_g rows as float4 quarters (n % 8 == 0): row j, quarter q -> skewed row start + 4q
+  const int q4 = n / 4;
+  for (int i = threadIdx.x; i < d * q4; i += blockDim.x) {
+    const int j = i / q4, q = i % q4;
+    *reinterpret_cast<float4*>(sw + wg_smem_index(j, n) + 4 * q) =
+        __ldg(reinterpret_cast<const float4*>(Wg) + i);
+  }
+  // W_g is the caller's; x and the outputs are ordered after the previous kernel
+  pdl_wait();
+  pdl_trigger();
+  __syncthreads();
+  const int grp = threadIdx.x / ROUTE_THREADS, gt = threadIdx.x % ROUTE_THREADS;
+  const GroupSync sync{1 + grp};
+  for (int64_t b = (int64_t)blockIdx.x * 2 + grp; b < nblk; b += (int64_t)gridDim.x * 2) {
+    if (gt < MAX_EXPERTS) hist[grp][gt] = 0;
+    sync();
+    const int64_t t0 = b * tokb;
+    const int ntok = (int)(T - t0 < tokb ? T - t0 : tokb);
+    route_token_block<Tin, true>(x, sw, true, t0, ntok, d, n, K, gt, red[grp], logits[grp],
+                                 hist[grp], idx, gate, sync);
+    if (gt < n) blk_counts[b * n + gt] = hist[grp][gt];
+    sync();
+  }
 }
 
 // Copy the x rows of `E` entries (entry i = (token t0 + i / K, slot i % K)) to their
@@ -414,55 +476,78 @@ __global__ void __launch_bounds__(RS_THREADS)
   gather_rows(x, 0, d, K, E, s_row, xperm, tid, RS_THREADS);
 }
 
-// One CTA: for every expert, exclusive prefix of the block histograms over blocks, the
-// expert's total, and the start row of its group (groups padded to row_align rows).  The
-// experts are scanned side by side: G = 1024 / n' threads per expert (n' = n rounded up to a
-// power of two), each summing a contiguous range of blocks, then a shared-memory scan.
-__global__ void __launch_bounds__(1024)
+// One CTA per expert e: exclusive prefix over router blocks of the block histograms
+// (blk_base[b][e]) and the expert's total (counts[e]).  Each thread takes a contiguous run of
+// blocks; the runs' sums are scanned across the CTA (warp shuffles, then the 32 warp sums).
+// The last CTA to finish (a ticket that wraps back to 0) lays out the groups: offsets[e] =
+// sum over e' < e of counts[e'] rounded up to row_align.
+constexpr int SCAN_THREADS = 1024;
+constexpr int SCAN_RUN = 8;  // blocks per thread held in registers per pass
+
+__global__ void __launch_bounds__(SCAN_THREADS)
     route_scan_kernel(const int32_t* __restrict__ blk_counts, int64_t nblk, int n,
                       int row_align, int64_t rows_max, int32_t* __restrict__ blk_base,
                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                      uint32_t* status) {
+                      unsigned int* ticket, uint32_t* status) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int part[1024];
-  __shared__ int total[MAX_EXPERTS];
-  int np = 1;
-  while (np < n) np <<= 1;
-  const int G = 1024 / np;                      // threads per expert (>= 16)
-  const int e = threadIdx.x / G, i = threadIdx.x % G;
-  const int64_t chunk = (nblk + G - 1) / G;
-  const int64_t b0 = i * chunk, b1 = b0 + chunk < nblk ? b0 + chunk : nblk;
+  __shared__ int wsum[SCAN_THREADS / 32];
+  __shared__ int s_last;
+  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t run = (nblk + SCAN_THREADS - 1) / SCAN_THREADS;
+  const int64_t b0 = tid * run, b1 = b0 + run < nblk ? b0 + run : nblk;
   int local = 0;
-  if (e < n) {
-#pragma unroll 8
-    for (int64_t b = b0; b < b1; ++b) local += blk_counts[b * n + e];
+  for (int64_t b = b0; b < b1; b += SCAN_RUN) {
+    int v[SCAN_RUN];
+#pragma unroll
+    for (int j = 0; j < SCAN_RUN; ++j) v[j] = b + j < b1 ? blk_counts[(b + j) * n + e] : 0;
+#pragma unroll
+    for (int j = 0; j < SCAN_RUN; ++j) local += v[j];
   }
-  part[threadIdx.x] = local;
+  // inclusive scan of the per-thread sums: within each warp, then over the warps
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  // inclusive Hillis-Steele scan inside each expert's G-thread segment
-  for (int off = 1; off < G; off <<= 1) {
-    const int v = i >= off ? part[threadIdx.x - off] : 0;
-    __syncthreads();
-    part[threadIdx.x] += v;
-    __syncthreads();
-  }
-  if (e < n) {
-    int run = part[threadIdx.x] - local;  // exclusive prefix of this thread's range
-#pragma unroll 8
-    for (int64_t b = b0; b < b1; ++b) {
-      blk_base[b * n + e] = run;
-      run += blk_counts[b * n + e];
+  if (warp == 0) {
+    int ws = wsum[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ws, off);
+      if (lane >= off) ws += y;
     }
-    if (i == G - 1) total[e] = part[threadIdx.x];
+    wsum[lane] = ws;  // inclusive over warps
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  int prefix = incl - local + (warp > 0 ? wsum[warp - 1] : 0);
+  for (int64_t b = b0; b < b1; b += SCAN_RUN) {
+    int v[SCAN_RUN];
+#pragma unroll
+    for (int j = 0; j < SCAN_RUN; ++j) v[j] = b + j < b1 ? blk_counts[(b + j) * n + e] : 0;
+#pragma unroll
+    for (int j = 0; j < SCAN_RUN; ++j)
+      if (b + j < b1) {
+        blk_base[(b + j) * n + e] = prefix;
+        prefix += v[j];
+      }
+  }
+  if (tid == SCAN_THREADS - 1) {
+    counts[e] = wsum[31];
+    __threadfence();
+    s_last = atomicInc(ticket, (unsigned)gridDim.x - 1u) == (unsigned)gridDim.x - 1u;
+  }
+  __syncthreads();
+  if (s_last && tid == 0) {
+    __threadfence();
     int64_t off = 0;
     for (int x = 0; x < n; ++x) {
-      counts[x] = total[x];
+      const int c = *(volatile const int32_t*)&counts[x];
       offsets[x] = (int32_t)off;
-      off += (int64_t)(total[x] + row_align - 1) / row_align * row_align;
+      off += (int64_t)(c + row_align - 1) / row_align * row_align;
     }
     offsets[n] = (int32_t)off;
     if (off > rows_max) set_status(status, DEV_ERR_ROW);
@@ -531,10 +616,32 @@ static cudaError_t launch_router_t(const Tin* x, const float* Wg, int64_t T, int
                                    int K, int32_t* idx, float* gate, int32_t* blk_counts,
                                    cudaStream_t s) {
   const int tokb = route_tokens_per_block(K);
-  const unsigned grid = (unsigned)((T + tokb - 1) / tokb);
+  const int64_t nblk = (T + tokb - 1) / tokb;
   const bool w_vec = n % 8 == 0 && (reinterpret_cast<uintptr_t>(Wg) & 15u) == 0;
-  pdl(router_topk_kernel<Tin>, grid, ROUTE_THREADS, 0, s)(x, Wg, w_vec, T, d, n, K, tokb, idx,
-                                                          gate, blk_counts);
+  const size_t wbytes = wg_smem_bytes(d, n);
+  const int sms = num_sms();
+  // bf16 activations only: with fp32 rows (32 bytes per 8 elements) the two-group kernel
+  // would not fit its registers
+  if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+  if (w_vec && wbytes <= (size_t)RT_SMEM_MAX && nblk >= 2 * (int64_t)sms) {
+    auto kern = router_topk_smem_kernel<Tin>;
+    static int configured = 0;  // per instantiation
+    if (configured < (int)wbytes) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wbytes);
+      if (e != cudaSuccess) return e;
+      configured = (int)wbytes;
+    }
+    const int64_t want = (nblk + 1) / 2;
+    const unsigned grid = (unsigned)(want < sms ? want : sms);
+    pdl(kern, grid, 2 * ROUTE_THREADS, wbytes, s)(x, Wg, T, d, n, K, tokb, nblk, idx, gate,
+                                                  blk_counts);
+    return cudaGetLastError();
+  }
+  }
+  pdl(router_topk_kernel<Tin>, (unsigned)nblk, ROUTE_THREADS, 0, s)(x, Wg, w_vec, T, d, n, K,
+                                                                    tokb, idx, gate,
+                                                                    blk_counts);
   return cudaGetLastError();
 }
 
@@ -562,8 +669,9 @@ cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Wo
     err = launch_router_t(static_cast<const float*>(x), Wg, p.T, (int)p.d, p.n, p.K, w.idx,
                           w.gate, w.blk_counts, s);
   if (err != cudaSuccess) return err;
-  pdl(route_scan_kernel, 1, 1024, 0, s)(w.blk_counts, p.nblk, p.n, p.row_align, p.rows_max,
-                                       w.blk_base, w.counts, w.offsets, w.status);
+  pdl(route_scan_kernel, (unsigned)p.n, SCAN_THREADS, 0, s)(
+      w.blk_counts, p.nblk, p.n, p.row_align, p.rows_max, w.blk_base, w.counts, w.offsets,
+      w.scan_ticket, w.status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int tokb = route_tokens_per_block(p.K);
   if (p.dt == 1)
