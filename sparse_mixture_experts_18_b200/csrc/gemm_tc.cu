@@ -356,7 +356,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 // meantime.  A tile whose second block lies past the last column block computes one block.  Expert groups are padded to 256 rows on this path.
 constexpr int PAIR_ROWS = 256;
 constexpr int PAIR_THREADS = 320;
-constexpr int PAIR_PF = 8;  // K blocks between an L2 prefetch and the load of the same tile
 
 struct PairCtrl {
   uint64_t full[MAX_STAGES];   // leader: the stage's bytes of both CTAs have landed
@@ -484,27 +483,12 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
     const uint64_t pol_w = policy_evict_normal();
     const uint64_t pol_x = policy_evict_last();
     const uint32_t full0 = map_to_rank(&c->full[0], 0);
-    // L2 prefetch of the tiles PAIR_PF K blocks ahead (of this work unit or the next), so
-    // that a weight tile's first touch from DRAM is not on the MMA's critical path
-    auto prefetch = [&](const Work& w, int kb) {
-      const int k = kb * 64;
-      if (!gather) tma_prefetch_2d(&tmX, k, w.row0 + (int)rank * (w.m >> 1));
-      for (int j = 0; j < w.count; ++j) {
-        const int cb = w.s + j;
-        if (KIND == KIND_G13)
-          tma_prefetch_2d(rank == 0 ? &tmW0 : &tmW1, k, w.e * a.nw + cb * 128);
-        else
-          tma_prefetch_2d(&tmW0, k, w.e * a.nw + cb * 256 + (int)rank * 128);
-      }
-    };
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int id = pair; id < total && ok && (gather || lane == 0); id += npairs) {
       const Work w = decode_pair_work(a, c, ps, id);
       if (w.count == 0) continue;
-      const Work wn = decode_pair_work(a, c, ps, id + npairs < total ? id + npairs : id);
-      const bool has_next = id + npairs < total && wn.count > 0;
       const int rows_cta = w.m >> 1;
       const int row = w.row0 + (int)rank * rows_cta;
       int tok[4] = {0, 0, 0, 0};
@@ -543,13 +527,6 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
         }
         if (gather)
           tma_gather4_pair(st + lane * 512, &tmX, fb, k, tok[0], tok[1], tok[2], tok[3], pol_x);
-        if (lane == 0) {
-          const int pkb = kb + PAIR_PF;
-          if (pkb < a.num_kb)
-            prefetch(w, pkb);
-          else if (has_next && pkb - a.num_kb < a.num_kb)
-            prefetch(wn, pkb - a.num_kb);
-        }
         if (++stage == a.stages) { stage = 0; phase ^= 1u; }
       }
     }
