@@ -34,6 +34,12 @@
  *    of 64 on the bf16 path and of 8 on the fp32 path; otherwise MOE_ERR_UNSUPPORTED.
  *  - out must not alias x.  Calls sharing one workspace must not overlap on the GPU.
  *  - Thread safety: no mutable global state; concurrent calls need separate workspaces.
+ *  - Environment: MOE_GATHER_X=1 (read at every call) switches large batches (T*K >= 640 n,
+ *    bf16) to an alternative data path: the up-projection gathers its activation rows from x
+ *    by token (TMA tile::gather4) instead of reading a permuted copy, and the
+ *    down-projection applies the gates.  Same results within rounding, same workspace size;
+ *    slower on B200 (the default is the permuted copy).  The pages describe grouping the
+ *    tokens per expert but fix no data path between the grouping and the expert GEMMs.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
