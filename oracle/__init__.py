@@ -62,6 +62,15 @@ def lib():
         L.oracle_block_forward.restype = I32
         L.oracle_block_forward.argtypes = [I64, I64, I64, I32, I32, I32, D, P, P, P, P, P, P,
                                            P]
+        L.oracle_e4m3_value.restype = D
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_code.restype = ctypes.c_uint8
+        L.oracle_e4m3_code.argtypes = [ctypes.c_float]
+        L.oracle_quantize_rows_e4m3.restype = None
+        L.oracle_quantize_rows_e4m3.argtypes = [I64, I64, I32, P, P, P]
+        L.oracle_moe_forward_fp8.restype = I32
+        L.oracle_moe_forward_fp8.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, P, P,
+                                             I64, P, P, P, P]
         _lib = L
     return _lib
 
@@ -233,3 +242,54 @@ def tie_band(logits_row: np.ndarray, K: int, rel: float = 1e-4):
     sure = [i for i in order[:K] if i not in near]
     sets = [tuple(sorted(sure + list(c))) for c in itertools.combinations(near, K - len(sure))]
     return True, sets
+
+
+# ------------------------------------------------------------------ FP8 expert weights
+
+def e4m3_value(code: int) -> float:
+    """Value of an OCP FP8 E4M3 code (NaN for S.1111.111)."""
+    return lib().oracle_e4m3_value(int(code) & 0xFF)
+
+
+def e4m3_code(v: float) -> int:
+    """Nearest E4M3 code to the binary32 value v (ties to even, saturating at 448)."""
+    return int(lib().oracle_e4m3_code(float(v)))
+
+
+def quantize_rows_e4m3(v):
+    """Per-row E4M3 quantisation of a [rows][cols] bf16/fp32 tensor: s = max|v| / 448 (1 for a
+    zero row), q = E4M3(v / s), both in binary32.  Returns (q uint8 [rows, cols], s f32)."""
+    a, dt = _raw(v)
+    a = a.reshape(-1, a.shape[-1])
+    rows, cols = a.shape
+    q = np.zeros((rows, cols), np.uint8)
+    sc = np.zeros(rows, np.float32)
+    lib().oracle_quantize_rows_e4m3(rows, cols, dt, _ptr(a), _ptr(q), _ptr(sc))
+    return q, sc
+
+
+def moe_forward_fp8(x, Wg, W1q, W3q, W2q, s1, s3, s2, n: int, K: int, tokens=None):
+    """Block output (unrounded, f64) with E4M3 expert weights and binary32 row scales for the
+    given token rows: W1q/W3q [n,F,d] and W2q [n,d,F] uint8 codes, s1/s3 [n,F], s2 [n,d].
+    Returns (y [len, d] f64, idx [len, K] i32, gate [len, K] f64)."""
+    xa, dt = _raw(x)
+    if dt != BF16:
+        raise TypeError("the FP8-weight block takes bf16 activations")
+    T, d = xa.shape
+    w1 = np.ascontiguousarray(W1q, np.uint8)
+    w3 = np.ascontiguousarray(W3q, np.uint8)
+    w2 = np.ascontiguousarray(W2q, np.uint8)
+    F = w1.shape[1]
+    a1 = np.ascontiguousarray(s1, np.float32)
+    a3 = np.ascontiguousarray(s3, np.float32)
+    a2 = np.ascontiguousarray(s2, np.float32)
+    tok = np.arange(T, dtype=np.int64) if tokens is None else np.asarray(tokens, np.int64)
+    y = np.zeros((len(tok), d), np.float64)
+    idx = np.zeros((len(tok), K), np.int32)
+    gate = np.zeros((len(tok), K), np.float64)
+    rc = lib().oracle_moe_forward_fp8(T, d, F, n, K, _ptr(xa), _ptr(_wg(Wg)), _ptr(w1),
+                                      _ptr(w3), _ptr(w2), _ptr(a1), _ptr(a3), _ptr(a2),
+                                      len(tok), _ptr(tok), _ptr(y), _ptr(idx), _ptr(gate))
+    if rc:
+        raise ValueError(f"oracle_moe_forward_fp8 failed ({rc})")
+    return y, idx, gate

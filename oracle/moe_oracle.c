@@ -34,7 +34,9 @@
  * Layouts (row-major): x [T][d]; W_g [d][n] fp32; W1, W3 [n][F][d]; W2 [n][d][F].
  *
  * Parity status: every function here is pinned by tests against closed forms, brute force
- * or library routines (see tests/test_oracle.py); none is "parity unpinned".
+ * or library routines (see tests/test_oracle.py); none is "parity unpinned".  The FP8
+ * functions at the end (E4M3 codes, row quantisation, the FP8-weight block) are pinned
+ * against the format's defining values and torch's float8_e4m3fn conversion.
  */
 #include <math.h>
 #include <stdint.h>
@@ -327,5 +329,154 @@ int oracle_block_forward(int64_t rows, int64_t d, int64_t F, int n, int K, int d
     free(yr);
   }
   free(xn);
+  return fail ? 3 : 0;
+}
+
+/* ---------------------------------------------------------------- FP8 expert weights
+ *
+ * The low-precision-weights variant (the pages mention only quantised community builds of
+ * the model, so the format below is this library's own reading, the plainest one):
+ *   - OCP FP8 E4M3 ("fn" flavour): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
+ *     no infinities, S.1111.111 is NaN, largest finite value 448, smallest subnormal 2^-9;
+ *   - one binary32 scale per row of every weight matrix (W1, W3 rows f of [F][d], W2 rows i
+ *     of [d][F]), per activation row (token) and per row of h:
+ *       s = max_j |v_j| / 448  (s = 1 for an all-zero row),   q_j = E4M3(v_j / s)
+ *     with E4M3 the nearest code, ties to the even mantissa, |v| > 448 clamped to 448;
+ *     s and v_j / s are computed in binary32, as the kernels do, so that both sides decide
+ *     the integer codes in the same precision;
+ *   - a_f = s_x s1_f sum_j q_x,j q1_f,j and b_f likewise with W3 (the code products summed
+ *     exactly, in double); h_f = silu(a_f) b_f rounded to binary32 and quantised per row
+ *     (s_h, q_h); y_i = s_h s2_i sum_f q_h,f q2_i,f; out = sum_k G_k y_{e_k}, rounded once.
+ *   Routing is the bf16 block's (the router reads the bf16 activations and fp32 W_g).
+ */
+
+/* Value of an E4M3 code. */
+double oracle_e4m3_value(uint8_t c) {
+  const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -v : v;
+}
+
+/* Nearest E4M3 code to v (ties to the even code, i.e. the even mantissa), saturating.  The
+ * non-negative finite codes 0..126 are in increasing order of value, so the nearest one is
+ * found by a plain search. */
+uint8_t oracle_e4m3_code(float v) {
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  const double a = fabs((double)v);
+  if (a >= 448.0) return sign | 126;
+  int best = 0;
+  double bd = a;
+  for (int c = 1; c <= 126; ++c) {
+    const double dist = fabs(oracle_e4m3_value((uint8_t)c) - a);
+    if (dist < bd || (dist == bd && (c & 1) == 0)) { best = c; bd = dist; }
+  }
+  return sign | (uint8_t)best;
+}
+
+/* Row scale in binary32: max |v| / 448, or 1 for an all-zero row. */
+static float e4m3_row_scale(const float* v, int64_t cols) {
+  float amax = 0.0f;
+  for (int64_t j = 0; j < cols; ++j) {
+    const float a = fabsf(v[j]);
+    if (a > amax) amax = a;
+  }
+  return amax > 0.0f ? amax / 448.0f : 1.0f;
+}
+
+static void e4m3_quantize_row(const float* v, int64_t cols, uint8_t* q, float* s) {
+  const volatile float sc = e4m3_row_scale(v, cols);
+  *s = sc;
+  for (int64_t j = 0; j < cols; ++j) {
+    const volatile float r = v[j] / sc;
+    q[j] = oracle_e4m3_code(r);
+  }
+}
+
+/* Per-row quantisation of a [rows][cols] matrix of dtype (bf16 or fp32) values. */
+void oracle_quantize_rows_e4m3(int64_t rows, int64_t cols, int dtype, const void* v,
+                               uint8_t* q, float* scales) {
+#pragma omp parallel
+  {
+    float* row = (float*)malloc(sizeof(float) * cols);
+#pragma omp for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+      if (!row) continue;
+      for (int64_t j = 0; j < cols; ++j) row[j] = (float)elem(v, dtype, r * cols + j);
+      e4m3_quantize_row(row, cols, q + r * cols, scales + r);
+    }
+    free(row);
+  }
+}
+
+/* The block with FP8 expert weights for the tokens tok[0..n_tok): y[r][0..d) in double
+ * (unrounded).  x bf16 [T][d]; W1q, W3q [n][F][d] and W2q [n][d][F] E4M3 codes; s1, s3
+ * [n][F] and s2 [n][d] binary32 row scales. */
+int oracle_moe_forward_fp8(int64_t T, int64_t d, int64_t F, int n, int K, const void* x,
+                           const float* Wg, const uint8_t* W1q, const uint8_t* W3q,
+                           const uint8_t* W2q, const float* s1, const float* s3,
+                           const float* s2, int64_t n_tok, const int64_t* tok, double* y,
+                           int32_t* idx_out, double* gate_out) {
+  if (n < 1 || n > 256 || K < 1 || K > n) return 1;
+  for (int64_t r = 0; r < n_tok; ++r) if (tok[r] < 0 || tok[r] >= T) return 2;
+  double lut[256];
+  for (int c = 0; c < 256; ++c) lut[c] = oracle_e4m3_value((uint8_t)c);
+  int fail = 0;
+#pragma omp parallel
+  {
+    float* xf = (float*)malloc(sizeof(float) * d);
+    uint8_t* qx = (uint8_t*)malloc(d);
+    float* hf = (float*)malloc(sizeof(float) * F);
+    uint8_t* qh = (uint8_t*)malloc(F);
+    if (!xf || !qx || !hf || !qh) {
+#pragma omp atomic write
+      fail = 1;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_tok; ++r) {
+      if (!xf || !qx || !hf || !qh) continue;
+      const int64_t t = tok[r];
+      double l[256], gate[256];
+      int32_t idx[256];
+      router_logits(d, n, ORACLE_BF16, x, t, Wg, l);
+      topk_softmax(n, K, l, idx, gate);
+      for (int64_t j = 0; j < d; ++j) xf[j] = (float)elem(x, ORACLE_BF16, t * d + j);
+      float sx;
+      e4m3_quantize_row(xf, d, qx, &sx);
+      double* yr = y + r * d;
+      for (int64_t i = 0; i < d; ++i) yr[i] = 0.0;
+      for (int k = 0; k < K; ++k) {
+        const int e = idx[k];
+        for (int64_t f = 0; f < F; ++f) {
+          const uint8_t* w1 = W1q + ((int64_t)e * F + f) * d;
+          const uint8_t* w3 = W3q + ((int64_t)e * F + f) * d;
+          double sa = 0.0, sb = 0.0;
+          for (int64_t j = 0; j < d; ++j) {
+            sa += lut[qx[j]] * lut[w1[j]];
+            sb += lut[qx[j]] * lut[w3[j]];
+          }
+          const double a = (double)sx * (double)s1[(int64_t)e * F + f] * sa;
+          const double b = (double)sx * (double)s3[(int64_t)e * F + f] * sb;
+          hf[f] = (float)(oracle_silu(a) * b);
+        }
+        float sh;
+        e4m3_quantize_row(hf, F, qh, &sh);
+        for (int64_t i = 0; i < d; ++i) {
+          const uint8_t* w2 = W2q + ((int64_t)e * d + i) * F;
+          double sy = 0.0;
+          for (int64_t f = 0; f < F; ++f) sy += lut[qh[f]] * lut[w2[f]];
+          yr[i] += gate[k] * ((double)sh * (double)s2[(int64_t)e * d + i] * sy);
+        }
+      }
+      for (int k = 0; k < K; ++k) {
+        if (idx_out) idx_out[r * K + k] = idx[k];
+        if (gate_out) gate_out[r * K + k] = gate[k];
+      }
+    }
+    free(xf);
+    free(qx);
+    free(hf);
+    free(qh);
+  }
   return fail ? 3 : 0;
 }

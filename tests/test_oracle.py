@@ -283,3 +283,127 @@ def test_block_forward_is_residual_plus_moe_of_norm(oracle_lib):
     got, idx, _ = oracle_lib.block_forward(x64, Wg, W1, W3, W2, n, 2, eps)
     assert np.array_equal(idx, idx_ref)
     assert np.allclose(got, ref, rtol=0, atol=0)
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) expert weights
+
+E4M3 = torch.float8_e4m3fn
+
+
+def _e4m3_codes_torch(v):
+    """E4M3 codes of binary32 values by torch's own float8 conversion (a library routine)."""
+    return v.to(torch.float32).to(E4M3).view(torch.uint8)
+
+
+def test_e4m3_table_closed_forms(oracle_lib):
+    # the format's defining points: 448 largest finite, 2^-9 smallest subnormal, 2^-6
+    # smallest normal, 1.0 = exponent 7, NaN at S.1111.111, sign bit 0x80
+    assert oracle_lib.e4m3_value(0x7E) == 448.0
+    assert oracle_lib.e4m3_value(0x01) == 2.0 ** -9
+    assert oracle_lib.e4m3_value(0x08) == 2.0 ** -6
+    assert oracle_lib.e4m3_value(0x07) == 7 * 2.0 ** -9
+    assert oracle_lib.e4m3_value(0x38) == 1.0
+    assert oracle_lib.e4m3_value(0xB8) == -1.0
+    assert math.isnan(oracle_lib.e4m3_value(0x7F)) and math.isnan(oracle_lib.e4m3_value(0xFF))
+    # every finite code is its own nearest code; codes increase with value
+    vals = [oracle_lib.e4m3_value(c) for c in range(127)]
+    assert all(b > a for a, b in zip(vals, vals[1:]))
+    for c in list(range(127)) + list(range(128, 255)):
+        assert oracle_lib.e4m3_code(oracle_lib.e4m3_value(c)) == c
+    # saturation
+    assert oracle_lib.e4m3_code(1e30) == 0x7E and oracle_lib.e4m3_code(-500.0) == 0xFE
+
+
+def test_e4m3_rounding_matches_torch(oracle_lib):
+    # nearest code, ties to even: every midpoint between neighbouring codes, points just
+    # beside them, and a dense random set, against torch's float8_e4m3fn conversion
+    vals = [oracle_lib.e4m3_value(c) for c in range(127)]
+    pts = []
+    for a, b in zip(vals, vals[1:]):
+        m = (a + b) / 2
+        pts += [m, np.nextafter(np.float32(m), np.float32(0)), np.nextafter(np.float32(m),
+                                                                            np.float32(1e9))]
+    g = torch.Generator().manual_seed(7)
+    rnd = torch.randn(4000, generator=g) * torch.exp(torch.randn(4000, generator=g) * 3)
+    pts = torch.tensor(np.array(pts, np.float32))
+    pts = torch.cat([pts, -pts, rnd.clamp(-448, 448)])
+    ours = np.array([oracle_lib.e4m3_code(float(v)) for v in pts], np.uint8)
+    assert np.array_equal(ours, _e4m3_codes_torch(pts).numpy())
+
+
+def test_quantize_rows_e4m3(oracle_lib):
+    # s = max|v| / 448 in binary32, codes = E4M3(v / s): the largest element maps to +-448,
+    # an all-zero row gets s = 1 and zero codes, and codes match torch's conversion of v / s
+    g = torch.Generator().manual_seed(11)
+    v = (torch.randn(6, 300, generator=g) * torch.tensor([1e-3, 1, 3, 50, 1e3, 0])[:, None]
+         ).to(torch.bfloat16)
+    q, s = oracle_lib.quantize_rows_e4m3(v)
+    vf = v.float()
+    amax = vf.abs().amax(dim=1)
+    assert s[5] == 1.0 and np.all((q[5] & 0x7F) == 0)  # signed zeros keep their sign
+    np.testing.assert_array_equal(s[:5], (amax[:5] / 448.0).numpy())
+    for r in range(5):
+        ref = _e4m3_codes_torch(vf[r] / torch.tensor(s[r])).numpy()
+        assert np.array_equal(q[r], ref)
+        j = int(vf[r].abs().argmax())
+        assert abs(oracle_lib.e4m3_value(int(q[r, j]))) == 448.0
+
+
+def _fp8_layer(T, d, F, n, seed):
+    x, Wg, W1, W3, W2 = _layer(T, d, F, n, seed=seed, dtype=torch.bfloat16)
+    W1q, s1 = oracle_lib_module().quantize_rows_e4m3(W1.reshape(n * F, d))
+    W3q, s3 = oracle_lib_module().quantize_rows_e4m3(W3.reshape(n * F, d))
+    W2q, s2 = oracle_lib_module().quantize_rows_e4m3(W2.reshape(n * d, F))
+    return (x, Wg, W1q.reshape(n, F, d), W3q.reshape(n, F, d), W2q.reshape(n, d, F),
+            s1.reshape(n, F), s3.reshape(n, F), s2.reshape(n, d))
+
+
+def oracle_lib_module():
+    import oracle
+    return oracle
+
+
+def _fp8_reference_torch(x, Wg, W1q, W3q, W2q, s1, s3, s2, K):
+    """The FP8-weight block from torch library steps: float8_e4m3fn conversions for every
+    quantisation, float64 matmuls for the code products."""
+    T, d = x.shape
+    xf = x.float()
+    sx = xf.abs().amax(dim=1) / 448.0
+    xq = (xf / sx[:, None]).to(E4M3).to(torch.float64)
+    l = x.double() @ Wg.double()
+    top = torch.topk(l, K, dim=1)
+    G = torch.softmax(top.values, dim=1)
+    val = lambda q: torch.from_numpy(q).view(E4M3).to(torch.float64)
+    y = torch.zeros(T, d, dtype=torch.float64)
+    for t in range(T):
+        for k in range(K):
+            e = int(top.indices[t, k])
+            a = sx[t].double() * torch.from_numpy(s1[e]).double() * (val(W1q[e]) @ xq[t])
+            b = sx[t].double() * torch.from_numpy(s3[e]).double() * (val(W3q[e]) @ xq[t])
+            h = (torch.nn.functional.silu(a) * b).float()
+            sh = h.abs().amax() / 448.0
+            hq = (h / sh).to(E4M3).to(torch.float64)
+            y[t] += G[t, k] * (sh.double() * torch.from_numpy(s2[e]).double() *
+                               (val(W2q[e]) @ hq))
+    return y.numpy(), top.indices.numpy()
+
+
+def test_fp8_block_matches_library_reference(oracle_lib):
+    T, d, F, n, K = 6, 64, 96, 4, 2
+    L = _fp8_layer(T, d, F, n, seed=71)
+    y, idx, gate = oracle_lib.moe_forward_fp8(*L, n, K)
+    ref, ridx = _fp8_reference_torch(*L, K)
+    assert np.array_equal(idx, ridx)
+    assert np.allclose(y, ref, rtol=1e-9, atol=1e-12)
+
+
+def test_fp8_block_routing_and_scale_linearity(oracle_lib):
+    # routing is the bf16 block's, and y is linear in the W2 row scales: doubling s2 (a power
+    # of two) doubles y bit for bit
+    T, d, F, n, K = 5, 64, 64, 8, 2
+    x, Wg, W1q, W3q, W2q, s1, s3, s2 = _fp8_layer(T, d, F, n, seed=81)
+    y, idx, gate = oracle_lib.moe_forward_fp8(x, Wg, W1q, W3q, W2q, s1, s3, s2, n, K)
+    _, ridx, rgate = oracle_lib.route(x, Wg, n, K)
+    assert np.array_equal(idx, ridx) and np.array_equal(gate, rgate)
+    y2, _, _ = oracle_lib.moe_forward_fp8(x, Wg, W1q, W3q, W2q, s1, s3, 2 * s2, n, K)
+    assert np.array_equal(y2, 2 * y)

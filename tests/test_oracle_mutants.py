@@ -32,6 +32,16 @@ MUTANTS = [
     ("bf16_one_bit_short", "int q = e - 8;", "int q = e - 7;"),
     ("rmsnorm_eps_dropped", "1.0 / sqrt(ss / (double)d + eps);", "1.0 / sqrt(ss / (double)d);"),
     ("residual_dropped", "round_to(x[r * d + i] + yr[i], dtype);", "round_to(yr[i], dtype);"),
+    ("e4m3_ties_to_odd", "(dist == bd && (c & 1) == 0)", "(dist == bd && (c & 1) == 1)"),
+    ("e4m3_wrong_max", "return amax > 0.0f ? amax / 448.0f : 1.0f;",
+     "return amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    ("e4m3_subnormal_step", "ldexp((double)m, -9)", "ldexp((double)m, -10)"),
+    ("fp8_x_scale_dropped", "const double a = (double)sx * (double)s1[(int64_t)e * F + f] * sa;",
+     "const double a = (double)s1[(int64_t)e * F + f] * sa;"),
+    ("fp8_h_scale_dropped",
+     "yr[i] += gate[k] * ((double)sh * (double)s2[(int64_t)e * d + i] * sy);",
+     "yr[i] += gate[k] * ((double)s2[(int64_t)e * d + i] * sy);"),
+    ("fp8_w3_uses_w1", "sb += lut[qx[j]] * lut[w3[j]];", "sb += lut[qx[j]] * lut[w1[j]];"),
 ]
 
 
