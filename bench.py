@@ -331,6 +331,142 @@ def run_gpu(args, w):
     return line
 
 
+def run_gpu_fp8(args, w):
+    """The FP8-weight variant (E4M3 expert weights with row scales) on a small-batch workload:
+    same step, timing and JSON line as run_gpu, one GPU (replicas as run_gpu for N > 1)."""
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_18_b200 as moe
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=300))
+    peaks = _peaks()
+    wr = replica_workload(w, rank)
+    x = moe_inputs.make_x(wr, device=dev)
+    layer = moe_inputs.make_layer(wr, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        q = {k: moe.moe_quantize_rows_e4m3(layer[k], stream=stream) for k in ("W1", "W3", "W2")}
+    Wg = layer["Wg"]
+    del layer
+    args_q = (q["W1"][0], q["W3"][0], q["W2"][0], q["W1"][1], q["W3"][1], q["W2"][1])
+    nbytes = moe.moe_workspace_bytes_fp8(w.T, w.d, w.F, w.n, w.K)
+    if nbytes == 0:
+        raise SystemExit(f"{w.name}: the FP8-weight block covers small-batch shapes only")
+    ws = moe.alloc_workspace(nbytes, dev, stream)
+    out = torch.empty_like(x)
+    plan = moe.moe_plan_info(w.T, w.d, w.F, w.n, w.K)
+
+    def step():
+        moe.moe_forward_fp8(x, Wg, *args_q, w.K, out=out, workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+        ms = ev0.elapsed_time(ev1)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)]
+               for _ in range(args.steps)]
+        for i in range(args.steps):
+            for e in evs[i]:
+                e.record(stream)
+            moe.moe_forward_fp8(x, Wg, *args_q, w.K, out=out, workspace=ws, stream=stream,
+                                events=evs[i])
+        barrier()
+        stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
+                    for i in range(args.steps)]
+        xh = x.cpu().pin_memory()
+        oh = torch.empty_like(xh).pin_memory()
+        xd = torch.empty_like(x)
+
+        def e2e_step():  # pinned host x in, the block, host out back
+            with torch.cuda.stream(stream):
+                xd.copy_(xh, non_blocking=True)
+            moe.moe_forward_fp8(xd, Wg, *args_q, w.K, out=out, workspace=ws, stream=stream)
+            with torch.cuda.stream(stream):
+                oh.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+            stream.synchronize()
+        ev1.record(stream)
+        barrier()
+        e2e_ms = ev0.elapsed_time(ev1)
+    code, raw = moe.moe_workspace_status(ws, stream)
+    if code != 0:
+        raise RuntimeError(f"device status {code} ({raw:#x})")
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    # active experts of this batch, from the bf16 router on the host (routing is shared)
+    l = x.float().cpu() @ Wg.float().cpu()
+    n_active = int(torch.unique(torch.topk(l, w.K, dim=1).indices).numel())
+    ms_step = ms / args.steps
+    tok_s = world * w.T * args.steps / (ms / 1e3)
+    g13 = statistics.mean(st[1] for st in stage_ms)
+    stage_avg = [statistics.mean(st[j] for st in stage_ms) for j in range(5)]
+    bytes13 = n_active * 2 * w.F * (w.d + 4) + w.T * w.K * (w.d + 4)
+    step_bytes = n_active * 3 * w.F * w.d + n_active * (2 * w.F + w.d) * 4 + w.d * w.n * 4 \
+        + 2 * w.T * w.d * 2
+    achieved = bytes13 / (g13 / 1e3) / 1e9
+    line = {
+        "metric": METRIC + " -- FP8 (E4M3) expert-weight variant", "value": round(tok_s, 2),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 weights and activations, fp32 accumulate, bf16 out",
+        "data": "synthetic (seeded N(0,1) activations, RMS-normalised; N(0,1/fan_in) weights "
+                "quantised per row to E4M3 on the device)",
+        "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K}, "
+                               "E4M3 expert weights",
+                   "tokens_per_rank": w.T,
+                   "l2": f"inputs larger than L2 ({3 * w.n * w.F * w.d / 1e9:.2f} GB of E4M3 "
+                         "expert weights)",
+                   "parallelism": f"replicas x{world}",
+                   "tiling": f"small-batch swap-AB split-K {plan['split13']}/{plan['split2']}, "
+                             "tcgen05 kind::f8f6f4", "active_experts": n_active},
+        "pct_roofline": {"bound": "hbm", "frac": round(step_bytes / (ms_step / 1e3) / 1e9 /
+                                                       peaks["hbm_gbs"], 4),
+                         "basis": "E4M3 weight bytes (+ row scales) of selected experts per "
+                                  "step / measured HBM copy GB/s"},
+        "roofline": {"bound": "hbm", "kernel": "tc_grouped_gemm G13 (E4M3)",
+                     "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": peaks["source"],
+                     "launch_ms": round(g13, 5)},
+        "stage_ms": {"route": round(stage_avg[0], 5), "gemm13": round(stage_avg[1], 5),
+                     "swiglu_quantize": round(stage_avg[2], 5),
+                     "gemm2": round(stage_avg[3], 5), "combine": round(stage_avg[4], 5)},
+        "e2e": {"value": round(world * w.T * args.steps / (e2e_ms / 1e3), 2),
+                "unit": "tokens/s", "h2d_bytes_per_step": w.T * w.d * 2,
+                "d2h_bytes_per_step": w.T * w.d * 2},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return line
+
+
 def cpu_baseline(w, x, layer, ntok):
     """The oracle as it stands on the host cores, on a bounded sample of tokens."""
     import oracle
@@ -402,6 +538,8 @@ def main(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=4,
                     help="tokens per oracle sample (CPU baseline / reference arm)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "e4m3"],
+                    help="e4m3: the FP8 expert-weight variant (small-batch workloads)")
     ap.add_argument("--gather-x", action="store_true",
                     help="CTA-pair path: gather G13's A rows from x (TMA gather4) instead of "
                          "X_perm, gates applied in G2 (sets MOE_GATHER_X=1)")
@@ -415,6 +553,8 @@ def main(argv=None):
         ap.error("the bench measures the bf16 path")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.weights == "e4m3":
+        return run_gpu_fp8(args, w)
     return run_gpu(args, w)
 
 

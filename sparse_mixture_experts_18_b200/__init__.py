@@ -4,11 +4,13 @@ The computation lives in libmoe.so (hand-written CUDA kernels behind the C ABI d
 include/moe.h); this package is its build script and a ctypes binding.
 """
 from .moe import (MOE_BF16, MOE_F32, MoeError, alloc_workspace, lib, moe_forward,
-                  moe_forward_debug, moe_forward_host_io,
-                  moe_forward_noalloc, moe_forward_profiled, moe_plan_info, moe_stack_forward,
-                  moe_stack_workspace_bytes, moe_workspace_bytes, moe_workspace_status)
+                  moe_forward_debug, moe_forward_fp8, moe_forward_host_io,
+                  moe_forward_noalloc, moe_forward_profiled, moe_plan_info,
+                  moe_quantize_rows_e4m3, moe_stack_forward, moe_stack_workspace_bytes,
+                  moe_workspace_bytes, moe_workspace_bytes_fp8, moe_workspace_status)
 
 __all__ = ["MOE_BF16", "MOE_F32", "MoeError", "alloc_workspace", "lib", "moe_forward",
-           "moe_forward_debug", "moe_forward_host_io", "moe_forward_noalloc", "moe_forward_profiled",
-           "moe_plan_info", "moe_stack_forward",
-           "moe_stack_workspace_bytes", "moe_workspace_bytes", "moe_workspace_status"]
+           "moe_forward_debug", "moe_forward_fp8", "moe_forward_host_io",
+           "moe_forward_noalloc", "moe_forward_profiled", "moe_plan_info",
+           "moe_quantize_rows_e4m3", "moe_stack_forward", "moe_stack_workspace_bytes",
+           "moe_workspace_bytes", "moe_workspace_bytes_fp8", "moe_workspace_status"]

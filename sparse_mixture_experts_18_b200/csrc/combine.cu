@@ -76,11 +76,14 @@ struct Out4<float> {
   }
 };
 
-template <typename Tout, bool RESID>
+// SCALED (FP8-weight block): the expert outputs are code sums, scaled here by the row's h
+// scale row_scale[row] and the W2 row scales col_scale[e][column] of the slot's expert.
+template <typename Tout, bool RESID, bool SCALED = false>
 __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ Y, int S, int64_t split_stride, int64_t T, int d,
                    int K, const int32_t* __restrict__ inv, const float* __restrict__ gate,
-                   Tout* out, const Tout* resid) {
+                   Tout* out, const Tout* resid, const float* __restrict__ row_scale,
+                   const float* __restrict__ col_scale, const int32_t* __restrict__ expert) {
   pdl_wait();
   pdl_trigger();
   const int vpr = d / 4;
@@ -105,6 +108,12 @@ __global__ void __launch_bounds__(256)
         if (s < S) {
           yk.x += part[s].x; yk.y += part[s].y; yk.z += part[s].z; yk.w += part[s].w;
         }
+      if (SCALED) {
+        const float rs = row_scale[row];
+        const float4 cs = __ldg(reinterpret_cast<const float4*>(
+            col_scale + (int64_t)expert[t * K + k] * d + c));
+        yk.x *= rs * cs.x; yk.y *= rs * cs.y; yk.z *= rs * cs.z; yk.w *= rs * cs.w;
+      }
       acc[0] = fmaf(g, yk.x, acc[0]);
       acc[1] = fmaf(g, yk.y, acc[1]);
       acc[2] = fmaf(g, yk.z, acc[2]);
@@ -185,10 +194,19 @@ __global__ void __launch_bounds__(256)
 }
 
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
-                           cudaStream_t s) {
+                           cudaStream_t s, const float* s2) {
   const int S = p.swap ? p.s2 : 1;
   const int64_t split_stride = p.rows_max * p.d;
   const float* gates = p.gather_x ? nullptr : w.gate;  // gather_x: G2 applied the gates
+  if (p.fp8) {  // small batches only (T <= 64), bf16 out, no residual
+    const int64_t total = p.T * (p.d / 4);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks < 1) blocks = 1;
+    pdl(combine_kernel<__nv_bfloat16, false, true>, (unsigned)blocks, 256, 0, s)(
+        w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate,
+        static_cast<__nv_bfloat16*>(out), nullptr, w.sh, s2, w.idx);
+    return cudaGetLastError();
+  }
   if (p.T >= 1024) {  // enough tokens for one warp each
     const int64_t blocks = (p.T + 7) / 8;
     const unsigned g = (unsigned)(blocks < ((int64_t)1 << 30) ? blocks : ((int64_t)1 << 30));
@@ -223,19 +241,21 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
     if (resid)
       pdl(combine_kernel<__nv_bfloat16, true>, (unsigned)blocks, 256, 0, s)(
           w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o,
-          static_cast<const __nv_bfloat16*>(resid));
+          static_cast<const __nv_bfloat16*>(resid), nullptr, nullptr, nullptr);
     else
       pdl(combine_kernel<__nv_bfloat16, false>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr);
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr, nullptr, nullptr,
+          nullptr);
   } else {
     auto* o = static_cast<float*>(out);
     if (resid)
       pdl(combine_kernel<float, true>, (unsigned)blocks, 256, 0, s)(
           w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o,
-          static_cast<const float*>(resid));
+          static_cast<const float*>(resid), nullptr, nullptr, nullptr);
     else
       pdl(combine_kernel<float, false>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr);
+          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr, nullptr, nullptr,
+          nullptr);
   }
   return cudaGetLastError();
 }

@@ -118,7 +118,19 @@ __device__ __forceinline__ bool wait_short(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-template <int KIND, bool SWAP>
+// One MMA of the kernel's operand kind: bf16 (kind::f16) or E4M3 (kind::f8f6f4).
+template <bool E4M3>
+__device__ __forceinline__ void umma_kind(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  if constexpr (E4M3)
+    umma_e4m3(tmem_d, adesc, bdesc, idesc, accumulate);
+  else
+    umma_bf16(tmem_d, adesc, bdesc, idesc, accumulate);
+}
+
+// E4M3: operands are FP8 codes (128 per 128-byte row, so a K block is 128 elements wide);
+// the accumulators hold the code products, scaled later by the row scales.
+template <int KIND, bool SWAP, bool E4M3 = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                            const __grid_constant__ CUtensorMap tmW0,
@@ -182,7 +194,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint8_t* st = smem + (size_t)stage * a.stage_bytes;
           uint64_t* fb = &c->full[stage];
           mbar_arrive_expect_tx(fb, a.tx_bytes);
-          const int k = (SWAP ? w.s * a.num_kb + kb : kb) * 64;
+          const int k = (SWAP ? w.s * a.num_kb + kb : kb) * (E4M3 ? 128 : 64);
           if (!SWAP) {
             tma_load_2d(st, &tmX, fb, k, w.mt * TILE_M, pol_x);
             if (KIND == KIND_G13) {
@@ -212,7 +224,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16(128, SWAP ? a.tok_tile : 256);
+      const uint32_t idesc = E4M3 ? umma_idesc_e4m3(128, SWAP ? a.tok_tile : 256)
+                                  : umma_idesc_bf16(128, SWAP ? a.tok_tile : 256);
       int stage = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -228,17 +241,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t sb = smem_u32(smem + (size_t)stage * a.stage_bytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t kofs = kk * 32;  // 16 bf16 along K inside the 128-byte row
+            const uint32_t kofs = kk * 32;  // 16 bf16 / 32 E4M3 along K in the 128-byte row
             const uint32_t accum = (kb | kk) != 0;
             if (!SWAP) {
-              umma_bf16(dtm, umma_desc_k128(sb + kofs), umma_desc_k128(sb + TILE_BYTES + kofs),
-                        idesc, accum);
+              umma_kind<E4M3>(dtm, umma_desc_k128(sb + kofs),
+                              umma_desc_k128(sb + TILE_BYTES + kofs), idesc, accum);
             } else {
               const uint64_t bd = umma_desc_k128(sb + a.x_off + kofs);
-              umma_bf16(dtm, umma_desc_k128(sb + kofs), bd, idesc, accum);
+              umma_kind<E4M3>(dtm, umma_desc_k128(sb + kofs), bd, idesc, accum);
               if (KIND == KIND_G13)
-                umma_bf16(dtm + a.tok_tile, umma_desc_k128(sb + TILE_BYTES + kofs), bd, idesc,
-                          accum);
+                umma_kind<E4M3>(dtm + a.tok_tile, umma_desc_k128(sb + TILE_BYTES + kofs), bd,
+                                idesc, accum);
             }
           }
           umma_commit(&c->empty[stage]);  // frees the stage once these MMAs have read it
@@ -766,6 +779,102 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ---------------------------------------------------------------- FP8 (E4M3) weights
+// Row scale in binary32 as the E4M3 format is used here: max |v| / 448 (1 for a zero row),
+// codes E4M3(v / s), nearest with ties to even, saturating.
+constexpr int Q_THREADS = 512;
+
+__device__ __forceinline__ float block_max(float v, float* wmax) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
+  return m;
+}
+
+// One CTA per row of a [rows][cols] bf16 matrix (cols % 4 == 0).
+__global__ void __launch_bounds__(Q_THREADS)
+    quantize_rows_e4m3_kernel(const __nv_bfloat16* __restrict__ v, int64_t cols,
+                              uint8_t* __restrict__ q, float* __restrict__ scales) {
+  __shared__ float wmax[Q_THREADS / 32];
+  const __nv_bfloat16* row = v + (int64_t)blockIdx.x * cols;
+  float amax = 0.f;
+  for (int64_t c = threadIdx.x * 4; c < cols; c += Q_THREADS * 4) {
+    const uint2 r = *reinterpret_cast<const uint2*>(row + c);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(r.x)), fabsf(bf16_hi(r.x))),
+                             fmaxf(fabsf(bf16_lo(r.y)), fabsf(bf16_hi(r.y)))));
+  }
+  const float s = e4m3_scale(block_max(amax, wmax));
+  if (threadIdx.x == 0) scales[blockIdx.x] = s;
+  uint8_t* qr = q + (int64_t)blockIdx.x * cols;
+  for (int64_t c = threadIdx.x * 4; c < cols; c += Q_THREADS * 4) {
+    const uint2 r = *reinterpret_cast<const uint2*>(row + c);
+    *reinterpret_cast<uint32_t*>(qr + c) =
+        e4m3x4(bf16_lo(r.x), bf16_hi(r.x), bf16_lo(r.y), bf16_hi(r.y), s);
+  }
+}
+
+// FP8 small batch, one CTA per permuted row r of expert e (rows grouped by offsets):
+//   a_f = (s_x[r] s1[e][f]) sum_s A_s,  b_f = (s_x[r] s3[e][f]) sum_s B_s  (splits in order),
+//   h_f = silu(a_f) b_f in binary32, then the row is quantised: s_h[r], hq[r][f].
+// h is kept in shared memory (F floats) between the two passes.
+__global__ void __launch_bounds__(Q_THREADS)
+    swiglu_reduce_e4m3_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
+                              int F, int n, const int32_t* __restrict__ offsets,
+                              const float* __restrict__ sx, const float* __restrict__ s1,
+                              const float* __restrict__ s3, uint8_t* __restrict__ hq,
+                              float* __restrict__ sh) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ float hbuf[];
+  __shared__ float wmax[Q_THREADS / 32];
+  __shared__ int s_e;
+  const int64_t r = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int e = 0;
+    while (e + 1 < n && r >= offsets[e + 1]) ++e;
+    s_e = e;
+  }
+  __syncthreads();
+  const int e = s_e;
+  const float xs = sx[r];
+  const float* pa = p13 + r * 2 * F;
+  float amax = 0.f;
+  for (int c = threadIdx.x * 4; c < F; c += Q_THREADS * 4) {
+    float4 ta[REDUCE_MAX_S], tb[REDUCE_MAX_S];
+#pragma unroll
+    for (int k = 0; k < REDUCE_MAX_S; ++k)
+      if (k < S) {
+        ta[k] = __ldg(reinterpret_cast<const float4*>(pa + k * split_stride + c));
+        tb[k] = __ldg(reinterpret_cast<const float4*>(pa + k * split_stride + F + c));
+      }
+    float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
+#pragma unroll
+    for (int k = 0; k < REDUCE_MAX_S; ++k)
+      if (k < S) {
+        sa.x += ta[k].x; sa.y += ta[k].y; sa.z += ta[k].z; sa.w += ta[k].w;
+        sb.x += tb[k].x; sb.y += tb[k].y; sb.z += tb[k].z; sb.w += tb[k].w;
+      }
+    const float4 w1 = __ldg(reinterpret_cast<const float4*>(s1 + (int64_t)e * F + c));
+    const float4 w3 = __ldg(reinterpret_cast<const float4*>(s3 + (int64_t)e * F + c));
+    float4 h;
+    h.x = silu_epilogue((xs * w1.x) * sa.x) * ((xs * w3.x) * sb.x);
+    h.y = silu_epilogue((xs * w1.y) * sa.y) * ((xs * w3.y) * sb.y);
+    h.z = silu_epilogue((xs * w1.z) * sa.z) * ((xs * w3.z) * sb.z);
+    h.w = silu_epilogue((xs * w1.w) * sa.w) * ((xs * w3.w) * sb.w);
+    *reinterpret_cast<float4*>(hbuf + c) = h;
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h.x), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w))));
+  }
+  const float s = e4m3_scale(block_max(amax, wmax));  // (its barrier also orders hbuf)
+  if (threadIdx.x == 0) sh[r] = s;
+  for (int c = threadIdx.x * 4; c < F; c += Q_THREADS * 4) {
+    const float4 h = *reinterpret_cast<const float4*>(hbuf + c);
+    *reinterpret_cast<uint32_t*>(hq + r * F + c) = e4m3x4(h.x, h.y, h.z, h.w, s);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -803,13 +912,28 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D E4M3 tensor [outer][inner] of bytes, box = box_rows x 128 codes, 128-byte swizzle.
+static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                        uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 constexpr uint32_t SMEM_STAGE_BUDGET = 200 * 1024;
 
-template <int KIND, bool SWAP>
+template <int KIND, bool SWAP, bool E4M3 = false>
 static cudaError_t launch_one(const CUtensorMap& mx, const CUtensorMap& mw0,
                               const CUtensorMap& mw1, TcArgs a, int max_work, cudaStream_t s) {
   const size_t smem = (size_t)a.stages * a.stage_bytes + sizeof(Ctrl) + 1024;
-  auto kern = tc_grouped_gemm_kernel<KIND, SWAP>;
+  auto kern = tc_grouped_gemm_kernel<KIND, SWAP, E4M3>;
   static int configured = 0;
   if (configured < (int)smem) {
     cudaError_t e =
@@ -1031,6 +1155,90 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   a.out_ld = d;
   a.split_stride = p.rows_max * (int64_t)d;
   if ((err = launch_one<KIND_G2, true>(mH, mW2, mW2, a, n * a.wb * a.splits, s)) !=
+      cudaSuccess)
+    return err;
+  return record(ev, 2, s);
+}
+
+cudaError_t launch_quantize_rows_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
+                                      float* scales, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  quantize_rows_e4m3_kernel<<<(unsigned)rows, Q_THREADS, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(v), cols, q, scales);
+  return cudaGetLastError();
+}
+
+// The small-batch tiling of launch_expert_gemms_tc on E4M3 codes: G13 partial sums, the
+// scaled SwiGLU with h quantised per row, G2 partial sums (scaled in the combine).
+cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const uint8_t* W3q,
+                                     const uint8_t* W2q, const float* s1, const float* s3,
+                                     const Workspace& w, cudaStream_t s,
+                                     cudaEvent_t const* ev) {
+  CUtensorMap mX, mW1, mW3, mH, mW2;
+  const int d = (int)p.d, F = (int)p.F, n = p.n;
+  const int tok = p.tok_tile;
+  const uint32_t xbytes = (uint32_t)tok * 128;
+  const uint32_t xslot = (xbytes + 1023u) & ~1023u;
+  if (!make_map_u8(&mX, w.xperm, d, p.rows_max, tok) ||
+      !make_map_u8(&mW1, W1q, d, (uint64_t)n * F, 128) ||
+      !make_map_u8(&mW3, W3q, d, (uint64_t)n * F, 128) ||
+      !make_map_u8(&mH, w.h, F, p.rows_max, tok) ||
+      !make_map_u8(&mW2, W2q, F, (uint64_t)n * d, 128))
+    return cudaErrorInvalidValue;
+  cudaError_t err;
+  TcArgs a{};
+  a.offsets = w.offsets;
+  a.n = n;
+  a.tok_tile = tok;
+  a.status = w.status;
+  a.splits = p.s13;
+  a.num_kb = d / 128 / p.s13;
+  a.nw = F;
+  a.wb = (F + 127) / 128;
+  a.x_off = 2 * TILE_BYTES;
+  a.stage_bytes = 2 * TILE_BYTES + xslot;
+  a.tx_bytes = 2 * TILE_BYTES + xbytes;
+  a.stages = stages_for(a.stage_bytes);
+  a.acc_cols = 2 * tok;
+  a.nacc = 2 * a.acc_cols <= 512 ? 2 : 1;
+  a.tmem_cols = pow2_cols(a.nacc * a.acc_cols);
+  a.out = w.p13;
+  a.out_ld = 2 * (int64_t)F;
+  a.split_stride = p.rows_max * 2 * (int64_t)F;
+  if ((err = launch_one<KIND_G13, true, true>(mX, mW1, mW3, a, n * a.wb * a.splits, s)) !=
+      cudaSuccess)
+    return err;
+  if ((err = record(ev, 0, s)) != cudaSuccess) return err;
+  const size_t hsmem = (size_t)F * sizeof(float);
+  static size_t configured = 0;
+  if (configured < hsmem) {
+    if ((err = cudaFuncSetAttribute(swiglu_reduce_e4m3_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem)) !=
+        cudaSuccess)
+      return err;
+    configured = hsmem;
+  }
+  const int rows = (int)(p.T * p.K);
+  pdl(swiglu_reduce_e4m3_kernel, rows > 0 ? rows : 1, Q_THREADS, hsmem, s)(
+      w.p13, p.s13, a.split_stride, F, n, w.offsets, w.sx, s1, s3,
+      static_cast<uint8_t*>(w.h), w.sh);
+  if ((err = cudaGetLastError()) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
+    return err;
+  a.splits = p.s2;
+  a.num_kb = F / 128 / p.s2;
+  a.nw = d;
+  a.wb = (d + 127) / 128;
+  a.x_off = TILE_BYTES;
+  a.stage_bytes = TILE_BYTES + xslot;
+  a.tx_bytes = TILE_BYTES + xbytes;
+  a.stages = stages_for(a.stage_bytes);
+  a.acc_cols = tok;
+  a.nacc = 2 * a.acc_cols <= 512 ? 2 : 1;
+  a.tmem_cols = pow2_cols(a.nacc * a.acc_cols);
+  a.out = w.y;
+  a.out_ld = d;
+  a.split_stride = p.rows_max * (int64_t)d;
+  if ((err = launch_one<KIND_G2, true, true>(mH, mW2, mW2, a, n * a.wb * a.splits, s)) !=
       cudaSuccess)
     return err;
   return record(ev, 2, s);

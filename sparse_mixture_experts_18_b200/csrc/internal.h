@@ -33,10 +33,12 @@ struct Plan {
   int tok_tile = 0;        // swap: MMA N (tokens per expert tile), multiple of 16
   int s13 = 1, s2 = 1;     // swap: split-K factors of the two expert GEMMs
   bool stack = false;      // workspace also holds the normalised activations
+  bool fp8 = false;        // E4M3 expert weights with row scales (small batch only)
   // workspace byte offsets
   size_t o_rpart;          // small batch: partial router logits [ceil(d/64)][T][n]
   size_t o_rowtok;         // token of each permuted row [rows_max] (small batch, gather_x)
   size_t o_rowgate;        // gather_x: gate of each permuted row [rows_max]
+  size_t o_sx, o_sh;       // fp8: scales of the X_perm rows and of the h rows [rows_max]
   size_t o_status, o_idx, o_gate, o_blk_counts, o_blk_base, o_counts, o_offsets, o_inv,
       o_xperm, o_h, o_y, o_p13, o_xn, total;
 };
@@ -49,6 +51,8 @@ struct Workspace {
   float* rpart;          // small-batch routing: partial logits
   int32_t* row_tok;      // token of each permuted row (small batch, gather_x)
   float* row_gate;       // gather_x: gate of each permuted row
+  float* sx;             // fp8: scale of each X_perm row (its token's)
+  float* sh;             // fp8: scale of each h row
   int32_t *idx, *blk_counts, *blk_base, *counts, *offsets, *inv;
   float* gate;
   void* xperm;  // [rows_max][d] activations in permuted order
@@ -87,7 +91,8 @@ PdlLaunch<KArgs...> pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
   return PdlLaunch<KArgs...>{kern, grid, block, smem, s};
 }
 
-bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p);
+bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p,
+               bool fp8 = false);
 Workspace carve(const Plan& p, void* base);
 
 int route_tokens_per_block(int K);
@@ -97,11 +102,21 @@ cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Wo
 cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
                                    const void* W3, const void* W2, const Workspace& w,
                                    cudaStream_t s, cudaEvent_t const* ev = nullptr);
+// fp8: the small-batch GEMMs on E4M3 codes; W1q/W3q [n][F][d], W2q [n][d][F]; s1/s3 [n][F]
+// and s2 [n][d] row scales.  ev as for launch_expert_gemms_tc.
+cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const uint8_t* W3q,
+                                     const uint8_t* W2q, const float* s1, const float* s3,
+                                     const Workspace& w, cudaStream_t s,
+                                     cudaEvent_t const* ev = nullptr);
+// Per-row E4M3 quantisation of a [rows][cols] bf16 matrix (cols % 4 == 0).
+cudaError_t launch_quantize_rows_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
+                                      float* scales, cudaStream_t s);
 cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float* W3,
                                      const float* W2, const Workspace& w, cudaStream_t s,
                                      cudaEvent_t const* ev = nullptr);
+// fp8 (p.fp8): s2 [n][d] are the W2 row scales; expert outputs are scaled by s_h[row] s2[e][i]
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
-                           cudaStream_t s);
+                           cudaStream_t s, const float* s2 = nullptr);
 cudaError_t launch_rmsnorm(const void* x, void* xn, int64_t T, int64_t d, float eps,
                            cudaStream_t s);
 int num_sms();

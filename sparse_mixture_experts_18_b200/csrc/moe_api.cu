@@ -52,8 +52,10 @@ static bool gather_x_requested() {
   return v != nullptr && v[0] == '1';
 }
 
-bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p) {
+bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p,
+               bool fp8) {
   if (T < 0 || d <= 0 || F <= 0 || n < 1 || n > MAX_EXPERTS || K < 1 || K > n) return false;
+  if (fp8 && (dt != 1 || stack || d % 128 || F % 128)) return false;
   if (dt == 1) {
     if (d % 64 || F % 64) return false;
   } else if (dt == 0) {
@@ -76,11 +78,15 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   const int tokb = route_tokens_per_block(K);
   q.nblk = (T + tokb - 1) / tokb;
   q.fused_route = T <= 64 && T * K <= 1024;  // limits of route_split_kernel
+  // FP8 expert weights: the small-batch path with its one-launch routing only
+  q.fp8 = fp8;
+  if (fp8 && !(q.swap && q.fused_route)) return false;
+  const int kbw = fp8 ? 128 : 64;  // elements per 128-byte K block
   if (q.swap) {
     q.tok_tile = (int)((T + 15) / 16 * 16);
     const int sms = num_sms();
-    q.s13 = choose_split((int)(d / 64), n * (int)((F + 127) / 128), sms);
-    q.s2 = choose_split((int)(F / 64), n * (int)((d + 127) / 128), sms);
+    q.s13 = choose_split((int)(d / kbw), n * (int)((F + 127) / 128), sms);
+    q.s2 = choose_split((int)(F / kbw), n * (int)((d + 127) / 128), sms);
   }
   const size_t es = dt == 1 ? 2 : 4;
   size_t o = 0;
@@ -102,6 +108,8 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   // (the layout does not depend on gather_x, so a workspace sized earlier stays valid)
   q.o_rowtok = take(q.fused_route || q.pair ? (size_t)q.rows_max * 4 : 0);
   q.o_rowgate = take(q.pair ? (size_t)q.rows_max * 4 : 0);
+  q.o_sx = take(fp8 ? (size_t)q.rows_max * 4 : 0);  // X_perm and h hold E4M3 codes then
+  q.o_sh = take(fp8 ? (size_t)q.rows_max * 4 : 0);
   q.total = o;
   *p = q;
   return true;
@@ -116,6 +124,8 @@ Workspace carve(const Plan& p, void* base) {
   w.rpart = reinterpret_cast<float*>(b + p.o_rpart);
   w.row_tok = reinterpret_cast<int32_t*>(b + p.o_rowtok);
   w.row_gate = reinterpret_cast<float*>(b + p.o_rowgate);
+  w.sx = reinterpret_cast<float*>(b + p.o_sx);
+  w.sh = reinterpret_cast<float*>(b + p.o_sh);
   w.idx = reinterpret_cast<int32_t*>(b + p.o_idx);
   w.gate = reinterpret_cast<float*>(b + p.o_gate);
   w.blk_counts = reinterpret_cast<int32_t*>(b + p.o_blk_counts);
@@ -238,6 +248,58 @@ moe_status moe_forward(const void* x, const float* W_g, const void* W1, const vo
   if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
   const Workspace w = carve(p, workspace);
   return forward_impl(p, x, W_g, W1, W3, W2, out, nullptr, w, static_cast<cudaStream_t>(stream));
+}
+
+size_t moe_workspace_bytes_fp8(int64_t T, int64_t d, int64_t F, int n, int K) {
+  Plan p;
+  if (!make_plan(T, d, F, n, K, 1, false, &p, true)) return 0;
+  return p.total;
+}
+
+moe_status moe_quantize_rows_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
+                                  float* scales, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 4) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!v || !q || !scales || !aligned(v, 8) || !aligned(q, 4)) return MOE_ERR_INVALID_ARG;
+  if (rows > ((int64_t)1 << 31) - 1) return MOE_ERR_UNSUPPORTED;
+  return launch_quantize_rows_e4m3(v, rows, cols, q, scales, static_cast<cudaStream_t>(stream))
+                 == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_forward_fp8(const void* x, const float* W_g, const uint8_t* W1q,
+                           const uint8_t* W3q, const uint8_t* W2q, const float* s1,
+                           const float* s3, const float* s2, int64_t T, int64_t d, int64_t F,
+                           int n, int K, void* out, void* workspace, size_t workspace_bytes,
+                           void* stream, void* const* events, int n_events) {
+  Plan p;
+  if (!make_plan(T, d, F, n, K, 1, false, &p, true)) {
+    const moe_status st = shape_status(T, d, F, n, K, MOE_BF16);
+    return st == MOE_ERR_INVALID_ARG ? st : MOE_ERR_UNSUPPORTED;
+  }
+  if (n_events != 0 && (n_events != 6 || !events)) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  moe_status st = check_common(x, W_g, W1q, W3q, W2q, out, workspace);
+  if (st != MOE_OK) return st;
+  if (!s1 || !s3 || !s2 || !aligned(s1, 16) || !aligned(s3, 16) || !aligned(s2, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (out == x) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  const Workspace w = carve(p, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev[6];
+  for (int i = 0; i < n_events; ++i) ev[i] = static_cast<cudaEvent_t>(events[i]);
+  cudaEvent_t const* evp = n_events ? ev : nullptr;
+  if (evp && cudaEventRecord(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_route(p, x, W_g, w, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (evp && cudaEventRecord(ev[1], s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_expert_gemms_e4m3(p, W1q, W3q, W2q, s1, s3, w, s, evp ? ev + 2 : nullptr) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_combine(p, w, out, nullptr, s, s2) != cudaSuccess) return MOE_ERR_CUDA;
+  if (evp && cudaEventRecord(ev[5], s) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 moe_status moe_forward_profiled(const void* x, const float* W_g, const void* W1,

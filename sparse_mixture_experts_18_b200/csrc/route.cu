@@ -212,6 +212,38 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
   if (threadIdx.x < n) blk_counts[(int64_t)blockIdx.x * n + threadIdx.x] = hist[threadIdx.x];
 }
 
+// FP8-weight block: entry i (token i / K) -> permuted row row[i]: the token's bf16 x row as
+// E4M3 codes with its own scale (max |x| / 448), one warp per entry, two passes over the row.
+__device__ __forceinline__ void gather_rows_e4m3(const __nv_bfloat16* __restrict__ x, int d,
+                                                 int K, int E, const int* row,
+                                                 uint8_t* __restrict__ xq,
+                                                 float* __restrict__ sx, int tid,
+                                                 int nthreads) {
+  const int lane = tid & 31, nwarps = nthreads >> 5;
+  for (int i = tid >> 5; i < E; i += nwarps) {
+    const int r = row[i];
+    if (r < 0) continue;
+    const __nv_bfloat16* src = x + (int64_t)(i / K) * d;
+    float amax = 0.f;
+    for (int c = lane * 4; c < d; c += 128) {
+      const uint2 v = *reinterpret_cast<const uint2*>(src + c);
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
+                               fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float s = e4m3_scale(amax);
+    if (lane == 0) sx[r] = s;
+    uint8_t* dst = xq + (int64_t)r * d;
+    for (int c = lane * 4; c < d; c += 128) {
+      const uint2 v = *reinterpret_cast<const uint2*>(src + c);
+      *reinterpret_cast<uint32_t*>(dst + c) =
+          e4m3x4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y), s);
+    }
+  }
+}
+
 // Large batches whose router matrix fits in shared memory: each CTA copies W_g once (skewed
 // layout, wg_smem_index) and its two 256-thread groups route token blocks b = 2*CTA + group,
 // then b + 2*grid, ... (same per-block arithmetic, histogram and outputs as
@@ -303,7 +335,8 @@ __global__ void __launch_bounds__(RS_THREADS)
                        int32_t* __restrict__ idx, float* __restrict__ gate,
                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                        int32_t* __restrict__ inv, int32_t* __restrict__ row_tok,
-                       Tact* __restrict__ xperm, uint32_t* status) {
+                       Tact* __restrict__ xperm, uint32_t* status,
+                       uint8_t* __restrict__ xq, float* __restrict__ sx) {
   pdl_wait();
   pdl_trigger();
   constexpr int PER = RS_MAX_ENTRIES / RS_THREADS;  // entries per thread in the rank phase
@@ -470,6 +503,13 @@ __global__ void __launch_bounds__(RS_THREADS)
     s_row[i] = row;
     inv[i] = row;
     if (row >= 0) row_tok[row] = i / K;
+  }
+  if (xq != nullptr) {  // FP8-weight block: quantised rows and their scales
+    if constexpr (std::is_same<Tact, __nv_bfloat16>::value) {
+      __syncthreads();
+      gather_rows_e4m3(x, d, K, E, s_row, xq, sx, tid, RS_THREADS);
+    }
+    return;
   }
   if (xperm == nullptr) return;  // the GEMM loads token rows straight from x
   __syncthreads();
@@ -652,7 +692,8 @@ static cudaError_t launch_route_small_t(const Plan& p, const Tact* x, const floa
   pdl(route_split_kernel<Tact>, G, RS_THREADS, 0, s)(
       x, Wg, (int)p.T, (int)p.d, p.n, p.K, p.row_align, p.rows_max, w.rpart, w.ticket, w.idx,
       w.gate, w.counts, w.offsets, w.inv, w.row_tok,
-      static_cast<Tact*>(w.xperm), w.status);
+      static_cast<Tact*>(w.xperm), w.status,
+      p.fp8 ? static_cast<uint8_t*>(w.xperm) : nullptr, p.fp8 ? w.sx : nullptr);
   return cudaGetLastError();
 }
 

@@ -68,6 +68,13 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.argtypes = [I32]
         L.moe_abi_version.restype = I32
         L.moe_abi_version.argtypes = []
+        L.moe_quantize_rows_e4m3.restype = I32
+        L.moe_quantize_rows_e4m3.argtypes = [P, I64, I64, P, P, P]
+        L.moe_workspace_bytes_fp8.restype = SZ
+        L.moe_workspace_bytes_fp8.argtypes = [I64, I64, I64, I32, I32]
+        L.moe_forward_fp8.restype = I32
+        L.moe_forward_fp8.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, P, P, SZ,
+                                      P, ctypes.POINTER(P), I32]
         _lib = L
     return _lib
 
@@ -232,3 +239,45 @@ def moe_stack_forward(x, layers, K: int, eps: float = 1e-5, workspace=None, stre
         _ptr(x), pg, p1, p3, p2, L, T, d, F, n, K, dt, float(eps), _ptr(workspace),
         workspace.numel(), _stream(stream)))
     return x
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) expert weights
+
+def moe_quantize_rows_e4m3(v: torch.Tensor, stream=None):
+    """Per-row E4M3 codes (uint8, same shape) and fp32 scales (one per row) of a bf16 CUDA
+    tensor whose last dimension is the row: s = max|v| / 448, code = E4M3(v / s)."""
+    if v.dtype != torch.bfloat16 or not v.is_cuda:
+        raise TypeError("moe_quantize_rows_e4m3 takes a bf16 CUDA tensor")
+    v = v.contiguous()
+    cols = v.shape[-1]
+    rows = v.numel() // cols
+    q = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
+    s = torch.empty(v.shape[:-1], dtype=torch.float32, device=v.device)
+    _check("moe_quantize_rows_e4m3", lib().moe_quantize_rows_e4m3(
+        _ptr(v), rows, cols, _ptr(q), _ptr(s), _stream(stream)))
+    return q, s
+
+
+def moe_workspace_bytes_fp8(T, d, F, n, K) -> int:
+    return int(lib().moe_workspace_bytes_fp8(T, d, F, n, K))
+
+
+def moe_forward_fp8(x, W_g, W1q, W3q, W2q, s1, s3, s2, K: int, out=None, workspace=None,
+                    stream=None, events=None):
+    """The block with E4M3 expert weights (codes W1q/W3q [n,F,d], W2q [n,d,F]; fp32 row scales
+    s1/s3 [n,F], s2 [n,d]); x and out bf16.  events: None or six torch.cuda.Event recorded at
+    the stage boundaries by the library.  Returns out."""
+    T, d = x.shape
+    n, F, _ = W1q.shape
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = alloc_workspace(moe_workspace_bytes_fp8(T, d, F, n, K), x.device, stream)
+    ev, nev = None, 0
+    if events is not None:
+        ev = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        nev = 6
+    _check("moe_forward_fp8", lib().moe_forward_fp8(
+        _ptr(x), _ptr(W_g), _ptr(W1q), _ptr(W3q), _ptr(W2q), _ptr(s1), _ptr(s3), _ptr(s2),
+        T, d, F, n, K, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream), ev, nev))
+    return out

@@ -160,3 +160,40 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     with pytest.raises(ImportError):
         binding.lib()
     importlib.reload(binding)
+
+
+def _fwd8(L, x=0x1000, wg=0x2000, w1=0x3000, w3=0x4000, w2=0x5000, s1=0x7000, s3=0x8000,
+          s2=0x9000, T=16, d=256, F=384, n=8, K=2, out=0x6000, ws=0x10000, ws_bytes=1 << 40,
+          events=None, n_events=0):
+    return L.moe_forward_fp8(P(x), P(wg), P(w1), P(w3), P(w2), P(s1), P(s3), P(s2), T, d, F, n,
+                             K, P(out), P(ws), ws_bytes, None, events, n_events)
+
+
+def test_fp8_workspace_and_supported_shapes(L):
+    ws8 = L.moe_workspace_bytes_fp8
+    assert ws8(16, 4096, 14336, 8, 2) > 0                        # Mixtral decode
+    assert ws8(64, 4096, 14336, 8, 2) > 0
+    assert ws8(65, 4096, 14336, 8, 2) == 0                       # past the one-launch routing
+    assert ws8(16, 4032, 14336, 8, 2) == 0                       # d % 128
+    assert ws8(16, 4096, 14272, 8, 2) == 0                       # F % 128
+    assert ws8(64, 256, 384, 1, 1) == 0                          # T*K >= 64 n: not small batch
+    assert ws8(0, 4096, 14336, 8, 2) > 0
+
+
+def test_fp8_forward_rejects_bad_arguments_before_launch(L):
+    assert _fwd8(L, x=0) == INVALID and _fwd8(L, w2=0) == INVALID
+    assert _fwd8(L, s1=0) == INVALID and _fwd8(L, s2=0x9004) == INVALID   # null / misaligned
+    assert _fwd8(L, out=0x1000) == INVALID                                # aliases x
+    assert _fwd8(L, d=192) == UNSUPPORTED and _fwd8(L, T=100) == UNSUPPORTED
+    assert _fwd8(L, K=9) == INVALID
+    assert _fwd8(L, ws_bytes=4096) == WORKSPACE
+    assert _fwd8(L, n_events=5, events=(P * 6)(*([P(0x1)] * 6))) == INVALID
+    assert _fwd8(L, T=0, x=0, out=0) == OK
+
+
+def test_quantize_rows_validation(L):
+    q = L.moe_quantize_rows_e4m3
+    assert q(P(0x1000), 4, 6, P(0x2000), P(0x3000), None) == INVALID      # cols % 4
+    assert q(None, 4, 8, P(0x2000), P(0x3000), None) == INVALID
+    assert q(P(0x1004), 4, 8, P(0x2000), P(0x3000), None) == INVALID      # v not 8-byte aligned
+    assert q(P(0x1000), 0, 8, None, None, None) == OK                     # no rows: no-op

@@ -1,0 +1,92 @@
+"""GPU parity of the FP8-weight variant (E4M3 expert weights with per-row scales, on the
+small-batch decode path) against the oracle's FP8 block: quantisation codes and scales bit
+for bit, block outputs within the bf16 bars."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+cuda = pytest.importorskip("torch").cuda
+if not cuda.is_available():  # pragma: no cover - the driver runs this file on a B200 only
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import sparse_mixture_experts_18_b200 as moe  # noqa: E402
+
+
+def _quantize_layer(L, n, F, d):
+    W1q, s1 = moe.moe_quantize_rows_e4m3(L["W1"])
+    W3q, s3 = moe.moe_quantize_rows_e4m3(L["W3"])
+    W2q, s2 = moe.moe_quantize_rows_e4m3(L["W2"])
+    return W1q, W3q, W2q, s1, s3, s2
+
+
+def _run_fp8(w, gen_device="cpu", budget=None):
+    x = moe_inputs.make_x(w, device=gen_device)
+    layer = moe_inputs.make_layer(w, device=gen_device)
+    xd = x.cuda()
+    L = {k: v.cuda() for k, v in layer.items()}
+    W1q, W3q, W2q, s1, s3, s2 = _quantize_layer(L, w.n, w.F, w.d)
+    out = moe.moe_forward_fp8(xd, L["Wg"], W1q, W3q, W2q, s1, s3, s2, w.K)
+    torch.cuda.synchronize()
+    xc = x.cpu()
+    wg = layer["Wg"].cpu()
+    q = [t.cpu().numpy() for t in (W1q, W3q, W2q, s1, s3, s2)]
+    del L
+    logits, _, _ = parity.oracle.route(xc, wg, w.n, w.K)
+    exempt = {t for t in range(w.T) if parity.oracle.tie_band(logits[t], w.K,
+                                                               parity.TIE_REL)[0]}
+    tokens = [t for t in range(w.T) if t not in exempt]
+    if budget is not None:
+        tokens = tokens[:budget]
+    y, _, _ = parity.oracle.moe_forward_fp8(xc, wg, *q, w.n, w.K, tokens=tokens)
+    ref = parity.oracle.round_array(y, parity.oracle.BF16)
+    got = out.float().cpu().numpy()[tokens]
+    rep = parity.compare_outputs(got, ref, torch.bfloat16)
+    rep.update(exempt=len(exempt), tokens=len(tokens))
+    assert rep["ok"], rep
+    return rep
+
+
+def test_quantize_rows_bit_exact():
+    g = torch.Generator().manual_seed(5)
+    scales = torch.tensor([1e-4, 0.01, 1.0, 7.0, 300.0, 0.0, 1e3, 2.5])[:, None]
+    v = (torch.randn(8, 1024, generator=g) * scales).to(torch.bfloat16)
+    v[3, 17] = -v[3, 17].abs().max() * 4          # a dominant negative element
+    q, s = moe.moe_quantize_rows_e4m3(v.cuda())
+    torch.cuda.synchronize()
+    qo, so = parity.oracle.quantize_rows_e4m3(v)
+    np.testing.assert_array_equal(q.cpu().numpy(), qo)
+    np.testing.assert_array_equal(s.cpu().numpy(), so)
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 37, 64])
+def test_fp8_small_batch(T):
+    _run_fp8(moe_inputs.small(T=T, d=512, F=768))
+
+
+@pytest.mark.parametrize("n,K", [(16, 4), (64, 2), (1, 1), (8, 1)])
+def test_fp8_expert_counts(n, K):
+    _run_fp8(moe_inputs.small(T=12, d=256, F=384, n=n, K=K))
+
+
+def test_fp8_decode_t16_full():
+    # Mixtral shapes: 1.4 GB of E4M3 expert weights instead of 2.8 GB of bf16
+    rep = _run_fp8(moe_inputs.WORKLOADS["decode_t16"], gen_device="cuda")
+    assert rep["tokens"] + rep["exempt"] == 16
+
+
+def test_fp8_repeat_calls_bitwise():
+    w = moe_inputs.small(T=16, d=512, F=768)
+    x = moe_inputs.make_x(w).cuda()
+    L = {k: v.cuda() for k, v in moe_inputs.make_layer(w).items()}
+    qs = _quantize_layer(L, w.n, w.F, w.d)
+    ws = moe.alloc_workspace(moe.moe_workspace_bytes_fp8(w.T, w.d, w.F, w.n, w.K))
+    a = moe.moe_forward_fp8(x, L["Wg"], *qs, w.K, workspace=ws).clone()
+    b = moe.moe_forward_fp8(x, L["Wg"], *qs, w.K, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert moe.moe_workspace_status(ws)[0] == 0
