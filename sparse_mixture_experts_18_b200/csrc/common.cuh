@@ -286,7 +286,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
-// Every thread of both CTAs: makes barrier initialisation visible cluster-wide.
+// Load a float from shared memory of a CTA of this cluster (address from map_to_rank).
+__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+// Every thread of every CTA of the cluster: makes prior shared-memory writes (barrier
+// initialisation included) visible cluster-wide.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");

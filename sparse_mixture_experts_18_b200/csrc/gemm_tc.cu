@@ -816,10 +816,14 @@ __global__ void __launch_bounds__(Q_THREADS)
   }
 }
 
-// FP8 small batch, one CTA per permuted row r of expert e (rows grouped by offsets):
+// FP8 small batch: permuted row r of expert e (rows grouped by offsets) is handled by a
+// cluster of RQ_CLUSTER CTAs, each taking F / RQ_CLUSTER columns:
 //   a_f = (s_x[r] s1[e][f]) sum_s A_s,  b_f = (s_x[r] s3[e][f]) sum_s B_s  (splits in order),
-//   h_f = silu(a_f) b_f in binary32, then the row is quantised: s_h[r], hq[r][f].
-// h is kept in shared memory (F floats) between the two passes.
+//   h_f = silu(a_f) b_f in binary32; the row's max |h| is combined across the cluster through
+//   distributed shared memory, then each CTA quantises its columns: s_h[r], hq[r][f].
+// h stays in shared memory between the two passes.
+constexpr int RQ_CLUSTER = 4;
+
 __global__ void __launch_bounds__(Q_THREADS)
     swiglu_reduce_e4m3_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
                               int F, int n, const int32_t* __restrict__ offsets,
@@ -828,10 +832,13 @@ __global__ void __launch_bounds__(Q_THREADS)
                               float* __restrict__ sh) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ float hbuf[];
+  extern __shared__ float hbuf[];  // F / RQ_CLUSTER floats
   __shared__ float wmax[Q_THREADS / 32];
+  __shared__ float cta_max;
   __shared__ int s_e;
-  const int64_t r = blockIdx.x;
+  const uint32_t rank = cluster_ctarank();
+  const int64_t r = blockIdx.x / RQ_CLUSTER;
+  const int fc = F / RQ_CLUSTER, f0 = (int)rank * fc;
   if (threadIdx.x == 0) {
     int e = 0;
     while (e + 1 < n && r >= offsets[e + 1]) ++e;
@@ -842,7 +849,8 @@ __global__ void __launch_bounds__(Q_THREADS)
   const float xs = sx[r];
   const float* pa = p13 + r * 2 * F;
   float amax = 0.f;
-  for (int c = threadIdx.x * 4; c < F; c += Q_THREADS * 4) {
+  for (int cl = threadIdx.x * 4; cl < fc; cl += Q_THREADS * 4) {
+    const int c = f0 + cl;
     float4 ta[REDUCE_MAX_S], tb[REDUCE_MAX_S];
 #pragma unroll
     for (int k = 0; k < REDUCE_MAX_S; ++k)
@@ -864,15 +872,23 @@ __global__ void __launch_bounds__(Q_THREADS)
     h.y = silu_epilogue((xs * w1.y) * sa.y) * ((xs * w3.y) * sb.y);
     h.z = silu_epilogue((xs * w1.z) * sa.z) * ((xs * w3.z) * sb.z);
     h.w = silu_epilogue((xs * w1.w) * sa.w) * ((xs * w3.w) * sb.w);
-    *reinterpret_cast<float4*>(hbuf + c) = h;
+    *reinterpret_cast<float4*>(hbuf + cl) = h;
     amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h.x), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w))));
   }
-  const float s = e4m3_scale(block_max(amax, wmax));  // (its barrier also orders hbuf)
-  if (threadIdx.x == 0) sh[r] = s;
-  for (int c = threadIdx.x * 4; c < F; c += Q_THREADS * 4) {
-    const float4 h = *reinterpret_cast<const float4*>(hbuf + c);
-    *reinterpret_cast<uint32_t*>(hq + r * F + c) = e4m3x4(h.x, h.y, h.z, h.w, s);
+  const float m = block_max(amax, wmax);  // (its barrier also orders hbuf)
+  if (threadIdx.x == 0) cta_max = m;
+  cluster_sync_all();  // every CTA's maximum is in its shared memory
+  float rmax = 0.f;
+#pragma unroll
+  for (int q = 0; q < RQ_CLUSTER; ++q)
+    rmax = fmaxf(rmax, ld_cluster_f32(map_to_rank(&cta_max, (uint32_t)q)));
+  const float s = e4m3_scale(rmax);
+  if (threadIdx.x == 0 && rank == 0) sh[r] = s;
+  for (int cl = threadIdx.x * 4; cl < fc; cl += Q_THREADS * 4) {
+    const float4 h = *reinterpret_cast<const float4*>(hbuf + cl);
+    *reinterpret_cast<uint32_t*>(hq + r * F + f0 + cl) = e4m3x4(h.x, h.y, h.z, h.w, s);
   }
+  cluster_sync_all();  // no CTA leaves while a peer may still read its maximum
 }
 
 // ---------------------------------------------------------------- host side
@@ -1209,19 +1225,36 @@ cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const ui
       cudaSuccess)
     return err;
   if ((err = record(ev, 0, s)) != cudaSuccess) return err;
-  const size_t hsmem = (size_t)F * sizeof(float);
-  static size_t configured = 0;
-  if (configured < hsmem) {
-    if ((err = cudaFuncSetAttribute(swiglu_reduce_e4m3_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem)) !=
-        cudaSuccess)
+  const size_t hsmem = (size_t)(F / RQ_CLUSTER) * sizeof(float);
+  {
+    static size_t configured = 0;
+    if (configured < hsmem) {
+      if ((err = cudaFuncSetAttribute(swiglu_reduce_e4m3_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)hsmem)) != cudaSuccess)
+        return err;
+      configured = hsmem;
+    }
+    const int rows = (int)(p.T * p.K);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = RQ_CLUSTER;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)(RQ_CLUSTER * (rows > 0 ? rows : 1)), 1, 1);
+    cfg.blockDim = dim3(Q_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = hsmem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if ((err = cudaLaunchKernelEx(&cfg, swiglu_reduce_e4m3_kernel, w.p13, p.s13, a.split_stride,
+                                  F, n, static_cast<const int32_t*>(w.offsets), w.sx, s1, s3,
+                                  static_cast<uint8_t*>(w.h), w.sh)) != cudaSuccess)
       return err;
-    configured = hsmem;
   }
-  const int rows = (int)(p.T * p.K);
-  pdl(swiglu_reduce_e4m3_kernel, rows > 0 ? rows : 1, Q_THREADS, hsmem, s)(
-      w.p13, p.s13, a.split_stride, F, n, w.offsets, w.sx, s1, s3,
-      static_cast<uint8_t*>(w.h), w.sh);
   if ((err = cudaGetLastError()) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
     return err;
   a.splits = p.s2;

@@ -219,27 +219,45 @@ __device__ __forceinline__ void gather_rows_e4m3(const __nv_bfloat16* __restrict
                                                  uint8_t* __restrict__ xq,
                                                  float* __restrict__ sx, int tid,
                                                  int nthreads) {
+  constexpr int U = 4;  // 16-byte loads in flight per lane
   const int lane = tid & 31, nwarps = nthreads >> 5;
   for (int i = tid >> 5; i < E; i += nwarps) {
     const int r = row[i];
     if (r < 0) continue;
-    const __nv_bfloat16* src = x + (int64_t)(i / K) * d;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(i / K) * d);
+    const int nv = d / 8;  // 8 bf16 per 16-byte vector
     float amax = 0.f;
-    for (int c = lane * 4; c < d; c += 128) {
-      const uint2 v = *reinterpret_cast<const uint2*>(src + c);
-      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
-                               fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+    for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+      uint4 t[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (v0 + 32 * u < nv) t[u] = __ldg(src + v0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (v0 + 32 * u < nv) {
+          const uint32_t w[4] = {t[u].x, t[u].y, t[u].z, t[u].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[k])), fabsf(bf16_hi(w[k]))));
+        }
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1)
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const float s = e4m3_scale(amax);
     if (lane == 0) sx[r] = s;
-    uint8_t* dst = xq + (int64_t)r * d;
-    for (int c = lane * 4; c < d; c += 128) {
-      const uint2 v = *reinterpret_cast<const uint2*>(src + c);
-      *reinterpret_cast<uint32_t*>(dst + c) =
-          e4m3x4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y), s);
+    uint2* dst = reinterpret_cast<uint2*>(xq + (int64_t)r * d);
+    for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+      uint4 t[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (v0 + 32 * u < nv) t[u] = __ldg(src + v0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (v0 + 32 * u < nv)
+          dst[v0 + 32 * u] = make_uint2(
+              e4m3x4(bf16_lo(t[u].x), bf16_hi(t[u].x), bf16_lo(t[u].y), bf16_hi(t[u].y), s),
+              e4m3x4(bf16_lo(t[u].z), bf16_hi(t[u].z), bf16_lo(t[u].w), bf16_hi(t[u].w), s));
     }
   }
 }
