@@ -313,6 +313,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// Four rows y0..y3 of a 2-D tensor whose map has a one-row box (64 bf16, 128-byte swizzle)
+// into 512 consecutive bytes of this CTA's shared memory, completion on its barrier `bar`.
+// Rows outside the tensor arrive as zeros.  No multicast.
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* map,
+                                            uint64_t* bar, int32_t x, int32_t y0, int32_t y1,
+                                            int32_t y2, int32_t y3, uint64_t cache_hint) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+      "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "l"(cache_hint)
+      : "memory");
+}
+
 // Four rows y0..y3 of a 2-D bf16 tensor whose map has a one-row box (64 elements, 128-byte
 // swizzle) into 512 consecutive bytes of shared memory, by either CTA of a pair; completion
 // is counted on the leader's barrier.  Rows outside the tensor (e.g. y = number of rows)

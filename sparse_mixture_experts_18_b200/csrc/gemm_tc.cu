@@ -56,6 +56,7 @@ struct TcArgs {
   const int32_t* counts;   // [n] rows routed to each expert
   int gather_T;            // rows of x (a row index past the end reads zeros)
   const float* row_gate;   // gate of each permuted row
+  int gather_rows;         // small batch gathering from x: permuted rows (T*K)
 };
 
 struct Ctrl {
@@ -70,6 +71,7 @@ struct Ctrl {
   int nact;
   int off[MAX_EXPERTS + 1];
   int act[MAX_EXPERTS];
+  int gtok[SMALL_ROUTE_MAX_ROWS];  // small batch gathering from x: token of each row
 };
 
 struct Work {
@@ -166,6 +168,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   pdl_wait();  // expert offsets and operands come from the previous kernels
   pdl_trigger();
   if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
+  const bool gather = SWAP && KIND == KIND_G13 && a.row_tok != nullptr;
+  if (gather)
+    for (int i = threadIdx.x; i < a.gather_rows; i += blockDim.x) c->gtok[i] = a.row_tok[i];
   __syncthreads();
   if (threadIdx.x == 0) {
     int na = 0;
@@ -208,7 +213,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int wr = w.e * a.nw + w.wblk * 128;
             tma_load_2d(st, &tmW0, fb, k, wr, pol_w);
             if (KIND == KIND_G13) tma_load_2d(st + TILE_BYTES, &tmW1, fb, k, wr, pol_w);
-            tma_load_2d(st + a.x_off, &tmX, fb, k, w.row0, pol_x);
+            if (gather) {  // the expert's token rows straight from x, four per gather
+              for (int g = 0; g < a.tok_tile / 4; ++g) {
+                int tk[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  tk[j] = 4 * g + j < w.count ? c->gtok[w.row0 + 4 * g + j] : a.gather_T;
+                tma_gather4(st + a.x_off + g * 512, &tmX, fb, k, tk[0], tk[1], tk[2], tk[3],
+                            pol_x);
+              }
+            } else {
+              tma_load_2d(st + a.x_off, &tmX, fb, k, w.row0, pol_x);
+            }
           }
           c->issued[stage] += 1;
           if (++stage == a.stages) { stage = 0; phase ^= 1u; }
@@ -1119,7 +1135,9 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   const int tok = p.tok_tile;
   const uint32_t xbytes = (uint32_t)tok * 128;
   const uint32_t xslot = (xbytes + 1023u) & ~1023u;
-  if (!make_map(&mX, w.xperm, d, p.rows_max, tok) ||
+  // gather_small: G13's token rows come from x by token (one-row boxes), else from X_perm
+  if (!(p.gather_small ? make_map(&mX, x, d, (uint64_t)p.T, 1)
+                       : make_map(&mX, w.xperm, d, p.rows_max, tok)) ||
       !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||
       !make_map(&mW3, W3, d, (uint64_t)n * F, 128) || !make_map(&mH, w.h, F, p.rows_max, tok) ||
       !make_map(&mW2, W2, F, (uint64_t)n * d, 128))
@@ -1144,9 +1162,15 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   a.out = w.p13;
   a.out_ld = 2 * (int64_t)F;
   a.split_stride = p.rows_max * 2 * (int64_t)F;
+  if (p.gather_small) {
+    a.row_tok = w.row_tok;
+    a.gather_T = (int)p.T;
+    a.gather_rows = (int)(p.T * p.K);
+  }
   if ((err = launch_one<KIND_G13, true>(mX, mW1, mW3, a, n * a.wb * a.splits, s)) !=
       cudaSuccess)
     return err;
+  a.row_tok = nullptr;
   if ((err = record(ev, 0, s)) != cudaSuccess) return err;
   const int64_t rows = p.T * p.K;
   const int64_t vec = rows * F / 4;

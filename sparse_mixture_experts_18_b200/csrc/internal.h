@@ -16,6 +16,7 @@ namespace moe {
 constexpr int TILE_M = 128;       // rows of one tensor-core accumulator tile
 constexpr int SIMT_TILE = 64;     // rows of one fp32 SIMT tile
 constexpr int MAX_EXPERTS = 64;
+constexpr int SMALL_ROUTE_MAX_ROWS = 1024;  // T*K limit of the one-launch routing
 
 // Everything about a forward call that depends only on its shape.
 struct Plan {
@@ -30,6 +31,8 @@ struct Plan {
   int64_t rows_max = 0;    // upper bound of permuted rows (T*K plus padding)
   int64_t nblk = 0;        // router / permute blocks
   bool fused_route = false;  // small batch: routing in one launch (route_split_kernel)
+  bool gather_small = false; // small batch (bf16, fused routing): G13 gathers its token rows
+                             // from x (TMA gather4); routing writes no X_perm
   int tok_tile = 0;        // swap: MMA N (tokens per expert tile), multiple of 16
   int s13 = 1, s2 = 1;     // swap: split-K factors of the two expert GEMMs
   bool stack = false;      // workspace also holds the normalised activations

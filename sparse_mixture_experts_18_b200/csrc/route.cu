@@ -343,7 +343,7 @@ __device__ __forceinline__ void gather_rows(const Tact* __restrict__ x, int64_t 
 // rows.
 constexpr int RS_THREADS = 1024;
 constexpr int RS_MAX_T = 64;
-constexpr int RS_MAX_ENTRIES = 1024;
+constexpr int RS_MAX_ENTRIES = SMALL_ROUTE_MAX_ROWS;
 
 template <typename Tact>
 __global__ void __launch_bounds__(RS_THREADS)
@@ -364,6 +364,7 @@ __global__ void __launch_bounds__(RS_THREADS)
   __shared__ int s_off[MAX_EXPERTS + 1];
   __shared__ int s_row[RS_MAX_ENTRIES];
   __shared__ int s_idx[RS_MAX_ENTRIES];
+  __shared__ float s_sel[RS_THREADS / 32][MAX_EXPERTS];  // per warp: the kept logits
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, c = blockIdx.x;
@@ -444,30 +445,40 @@ __global__ void __launch_bounds__(RS_THREADS)
     if (v < T * n && sub8 == 0) logit[v] = sum;
   }
   __syncthreads();
-  if (tid < T) {  // TopK by repeated arg-max (ties -> lower index), softmax over the kept;
-                  // the selection is run twice (normaliser, then output) to stay in registers
-    const float* l = logit + tid * n;
+  // TopK by repeated arg-max (ties -> lower index), one warp per token with the n <= 64
+  // logits spread over the lanes (lane e holds experts e and e + 32); then the softmax over
+  // the kept logits shifted by the largest, summed in slot order
+  for (int t = warp; t < T; t += RS_THREADS / 32) {
+    const float* l = logit + t * n;
+    const float v0 = lane < n ? l[lane] : -INFINITY;
+    const float v1 = lane + 32 < n ? l[lane + 32] : -INFINITY;
+    bool u0 = lane >= n, u1 = lane + 32 >= n;
     float top = 0.f, z = 0.f;
-    for (int pass = 0; pass < 2; ++pass) {
-      uint64_t used = 0;
-      for (int k = 0; k < K; ++k) {
-        int best = -1;
-        float bv = 0.f;
-        for (int e = 0; e < n; ++e) {
-          if ((used >> e) & 1ull) continue;
-          if (best < 0 || l[e] > bv) { best = e; bv = l[e]; }
-        }
-        used |= 1ull << best;
-        if (pass == 0) {
-          if (k == 0) top = bv;
-          z += expf(bv - top);
-        } else {
-          idx[tid * K + k] = best;
-          s_idx[tid * K + k] = best;
-          gate[tid * K + k] = expf(bv - top) / z;
-        }
+    for (int k = 0; k < K; ++k) {
+      float bv;
+      int bi;
+      if (!u0 && (u1 || !(v1 > v0))) { bv = v0; bi = lane; }
+      else if (!u1) { bv = v1; bi = lane + 32; }
+      else { bv = -INFINITY; bi = 64 + lane; }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if (bi == lane) u0 = true;
+      if (bi == lane + 32) u1 = true;
+      if (k == 0) top = bv;
+      z += expf(bv - top);
+      if (lane == 0) {
+        idx[t * K + k] = bi;
+        s_idx[t * K + k] = bi;
+        s_sel[warp][k] = bv;
       }
     }
+    __syncwarp();
+    for (int k = lane; k < K; k += 32) gate[t * K + k] = expf(s_sel[warp][k] - top) / z;
+    __syncwarp();
   }
   __syncthreads();
   const int E = T * K;
@@ -710,7 +721,7 @@ static cudaError_t launch_route_small_t(const Plan& p, const Tact* x, const floa
   pdl(route_split_kernel<Tact>, G, RS_THREADS, 0, s)(
       x, Wg, (int)p.T, (int)p.d, p.n, p.K, p.row_align, p.rows_max, w.rpart, w.ticket, w.idx,
       w.gate, w.counts, w.offsets, w.inv, w.row_tok,
-      static_cast<Tact*>(w.xperm), w.status,
+      p.gather_small ? nullptr : static_cast<Tact*>(w.xperm), w.status,
       p.fp8 ? static_cast<uint8_t*>(w.xperm) : nullptr, p.fp8 ? w.sx : nullptr);
   return cudaGetLastError();
 }
