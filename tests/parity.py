@@ -1,7 +1,7 @@
 """Comparison of the CUDA library against the CPU oracle (shared by the GPU tests and the
 smoke check).
 
-Bars (from the method's contract for this build):
+Bars (the parity contract of the block):
   - routing: selected experts equal the oracle's exactly, ties to the lower index; the only
     exempt tokens are those whose K-th and (K+1)-th oracle logits are within 1e-4 relative
     (for them the GPU's set must be one of the admissible sets); slot order is checked where

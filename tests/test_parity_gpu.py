@@ -12,7 +12,7 @@ from tests import parity
 pytestmark = pytest.mark.gpu
 
 cuda = pytest.importorskip("torch").cuda
-if not cuda.is_available():  # pragma: no cover - the driver runs this file on a B200 only
+if not cuda.is_available():  # pragma: no cover - these tests need a B200
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 import sparse_mixture_experts_18_b200 as moe  # noqa: E402
