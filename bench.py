@@ -45,8 +45,8 @@ DEFAULT_WORKLOAD = "decode_t16"
 # captures summarised in profiles/tc_grouped_gemm_<workload>.md, valid only for the kernel
 # source they were taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "decode_t16": {"bytes": 1886803232, "src": "e854547ffc04"},
-    "prefill_t4096": {"bytes": 2495925680, "src": "e854547ffc04"},
+    "decode_t16": {"bytes": 1887145816, "src": "d6fe4cf56c17"},
+    "prefill_t4096": {"bytes": 2552105840, "src": "d6fe4cf56c17"},
 }
 
 
