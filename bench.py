@@ -509,7 +509,8 @@ def run_reference(args, w):
     oracle.build()
     x = moe_inputs.make_x(w)
     layer = moe_inputs.make_layer(w)
-    per_step = min(w.T, args.cpu_tokens)
+    threads = _omp_threads()
+    per_step = min(w.T, max(args.cpu_tokens, threads))  # a token for every host thread
     for i in range(args.warmup):
         oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
                            tokens=[i % w.T])
@@ -528,8 +529,9 @@ def run_reference(args, w):
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K}"},
-            "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": _omp_threads(),
-                             "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s",
+                             "cores": min(per_step, threads), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
