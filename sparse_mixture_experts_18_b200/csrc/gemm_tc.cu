@@ -7,19 +7,22 @@
 //   G2:   Y = h_e . W2_e^T                              kept in fp32
 // where X_e are the rows routed to expert e (grouped by the permute kernel).
 //
-// One persistent kernel per GEMM, one CTA per SM, 6 warps:
-//   warp 0      TMA producer (one thread) filling a ring of shared-memory stages,
+// Persistent kernels, one CTA (or CTA pair) per SM, warp-specialised:
+//   warp 0      TMA producer filling a ring of shared-memory stages,
 //   warp 1      owns the TMEM allocation; one thread issues tcgen05.mma,
-//   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulator, SwiGLU / store.
-// Accumulators are double-buffered in TMEM so the epilogue of one tile overlaps the MMAs
-// of the next.  All waits are bounded (see common.cuh).
+//   the rest    epilogue: tcgen05.ld of the fp32 accumulators, SwiGLU / store.
+// All waits are bounded (see common.cuh).
 //
-// Two tilings:
-//   prefill (!SWAP): tile = 128 permuted rows x (G13: 128 columns of W1 and the same 128 of
-//     W3, stacked into one N = 256 MMA operand | G2: 256 columns of W2), full K per tile.
-//   small batch (SWAP): the weights are the 128-row MMA operand and the expert's tokens the
-//     N dimension (16..256), K split into `splits` ranges so that every SM streams weights;
-//     fp32 partial sums go to per-split slabs reduced in a fixed order afterwards.
+// Tilings (chosen per call from the shape, see make_plan):
+//   128-row tiles (tc_grouped_gemm_kernel, !SWAP): tile = 128 permuted rows x (G13: 128
+//     columns of W1 and the same 128 of W3, stacked into one N = 256 MMA operand | G2: 256
+//     columns of W2), full K per tile, accumulators double-buffered in TMEM.
+//   small batch (tc_grouped_gemm_kernel, SWAP): the weights are the 128-row MMA operand and
+//     the expert's tokens the N dimension (16..256), K split into `splits` ranges so that
+//     every SM streams weights; fp32 partial sums go to per-split slabs reduced in a fixed
+//     order afterwards.  With E4M3 the operands are FP8 codes (kind::f8f6f4).
+//   CTA pairs (tc_pair_gemm_kernel): cta_group::2 tiles of 256 rows x two 256-column blocks,
+//     M = 128 tiles for an expert's last 128 rows (see the section below).
 #include <stdio.h>
 
 #include "internal.h"
