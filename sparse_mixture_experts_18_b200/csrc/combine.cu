@@ -6,9 +6,10 @@
 //            Indonesian news summary's expert-parallelism notes put it).  fp32 sum over the
 //            K slots in slot order (and over split slabs in split order), rounded once;
 //            16-byte vectorised loads and stores.  With a residual input, out = resid + sum,
-//            also in fp32 before the single rounding (the stacked-block workload).  On the
-//            CTA-pair path the down-projection epilogue has already multiplied each row by
-//            its gate, and the combine only sums the K rows.
+//            also in fp32 before the single rounding (the stacked-block workload).  With the
+//            gather-from-x option of the CTA-pair path (MOE_GATHER_X=1) the down-projection
+//            epilogue has already multiplied each row by its gate, and the combine only sums
+//            the K rows; with FP8 expert weights it applies the h and W2 row scales.
 //  rmsnorm:  xn = x / sqrt(mean(x^2) + eps) with unit gain, fp32 math, bf16 result.
 #include "internal.h"
 

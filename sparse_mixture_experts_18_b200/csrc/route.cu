@@ -339,8 +339,9 @@ __device__ __forceinline__ void gather_rows(const Tact* __restrict__ x, int64_t 
 // atomicInc so it is back at 0 for the next call) sums the partials in CTA order, then does
 // TopK and softmax, the expert counts, group offsets (padded to row_align), the stable rank
 // of every (token, slot) (per-warp match + per-expert prefix over 32-entry chunks), the
-// inverse map token -> row, the map row -> token, and (if xperm is given) the gather of x
-// rows.
+// inverse map token -> row and the map row -> token.  Then, if xq is given (FP8 weights), the
+// rows as E4M3 codes with their scales; else, if xperm is given, the bf16 rows (without
+// either, the G13 kernel gathers the token rows from x itself).
 constexpr int RS_THREADS = 1024;
 constexpr int RS_MAX_T = 64;
 constexpr int RS_MAX_ENTRIES = SMALL_ROUTE_MAX_ROWS;
@@ -540,7 +541,7 @@ __global__ void __launch_bounds__(RS_THREADS)
     }
     return;
   }
-  if (xperm == nullptr) return;  // the GEMM loads token rows straight from x
+  if (xperm == nullptr) return;  // the G13 kernel gathers the token rows from x
   __syncthreads();
   gather_rows(x, 0, d, K, E, s_row, xperm, tid, RS_THREADS);
 }
