@@ -73,6 +73,10 @@ def test_fp8_expert_counts(n, K):
     _run_fp8(moe_inputs.small(T=12, d=256, F=384, n=n, K=K))
 
 
+def test_fp8_one_launch_routing_at_its_limit():
+    _run_fp8(moe_inputs.small(T=64, d=256, F=384, n=64, K=16))
+
+
 def test_fp8_decode_t16_full():
     # Mixtral shapes: 1.4 GB of E4M3 expert weights instead of 2.8 GB of bf16
     rep = _run_fp8(moe_inputs.WORKLOADS["decode_t16"], gen_device="cuda")

@@ -98,6 +98,14 @@ def test_expert_counts(n, K):
     _run(moe_inputs.small(T=24, d=256, F=256, n=n, K=K))
 
 
+def test_one_launch_routing_at_its_limit():
+    # T = 64 tokens x K = 16 of n = 64: 1024 (token, slot) entries, the most the one-launch
+    # router takes; up to 64 tokens per expert in the gathered small-batch tiles
+    w = moe_inputs.small(T=64, d=256, F=384, n=64, K=16)
+    assert moe.moe_plan_info(w.T, w.d, w.F, w.n, w.K)["small_batch"] is True
+    _run(w)
+
+
 @pytest.mark.parametrize("T", [7, 200, 1100])
 def test_f32_path_ragged(T):
     _run(moe_inputs.small(T=T, d=136, F=200, dtype="f32", rms_x=False))
