@@ -45,8 +45,8 @@ DEFAULT_WORKLOAD = "decode_t16"
 # captures summarised in profiles/tc_grouped_gemm_<workload>.md, valid only for the kernel
 # source they were taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "decode_t16": {"bytes": 1887145816, "src": "3d29c3997808"},
-    "prefill_t4096": {"bytes": 2552105840, "src": "3d29c3997808"},
+    "decode_t16": {"bytes": 1886786272, "src": "9c8fdd53d8eb"},
+    "prefill_t4096": {"bytes": 2523485256, "src": "9c8fdd53d8eb"},
 }
 
 

@@ -837,8 +837,9 @@ __global__ void __launch_bounds__(Q_THREADS)
 
 // FP8 small batch: permuted row r of expert e (rows grouped by offsets) is handled by a
 // cluster of RQ_CLUSTER CTAs, each taking F / RQ_CLUSTER columns:
-//   a_f = (s_x[r] s1[e][f]) sum_s A_s,  b_f = (s_x[r] s3[e][f]) sum_s B_s  (splits in order),
-//   h_f = silu(a_f) b_f in binary32; the row's max |h| is combined across the cluster through
+//   a_f = (s_x s1[e][f]) sum_s A_s,  b_f = (s_x s3[e][f]) sum_s B_s  (splits in order; s_x the
+//   scale of the row's token), h_f = silu(a_f) b_f in binary32; the row's max |h| is combined
+//   across the cluster through
 //   distributed shared memory, then each CTA quantises its columns: s_h[r], hq[r][f].
 // h stays in shared memory between the two passes.
 constexpr int RQ_CLUSTER = 4;
@@ -846,6 +847,7 @@ constexpr int RQ_CLUSTER = 4;
 __global__ void __launch_bounds__(Q_THREADS)
     swiglu_reduce_e4m3_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
                               int F, int n, const int32_t* __restrict__ offsets,
+                              const int32_t* __restrict__ row_tok,
                               const float* __restrict__ sx, const float* __restrict__ s1,
                               const float* __restrict__ s3, uint8_t* __restrict__ hq,
                               float* __restrict__ sh) {
@@ -865,7 +867,7 @@ __global__ void __launch_bounds__(Q_THREADS)
   }
   __syncthreads();
   const int e = s_e;
-  const float xs = sx[r];
+  const float xs = sx[row_tok[r]];  // the scale of the row's token
   const float* pa = p13 + r * 2 * F;
   float amax = 0.f;
   for (int cl = threadIdx.x * 4; cl < fc; cl += Q_THREADS * 4) {
@@ -1222,7 +1224,8 @@ cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const ui
   const int tok = p.tok_tile;
   const uint32_t xbytes = (uint32_t)tok * 128;
   const uint32_t xslot = (xbytes + 1023u) & ~1023u;
-  if (!make_map_u8(&mX, w.xperm, d, p.rows_max, tok) ||
+  // the expert's token rows are gathered from the per-token E4M3 rows (one-row boxes)
+  if (!make_map_u8(&mX, w.xperm, d, (uint64_t)p.T, 1) ||
       !make_map_u8(&mW1, W1q, d, (uint64_t)n * F, 128) ||
       !make_map_u8(&mW3, W3q, d, (uint64_t)n * F, 128) ||
       !make_map_u8(&mH, w.h, F, p.rows_max, tok) ||
@@ -1248,9 +1251,13 @@ cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const ui
   a.out = w.p13;
   a.out_ld = 2 * (int64_t)F;
   a.split_stride = p.rows_max * 2 * (int64_t)F;
+  a.row_tok = w.row_tok;
+  a.gather_T = (int)p.T;
+  a.gather_rows = (int)(p.T * p.K);
   if ((err = launch_one<KIND_G13, true, true>(mX, mW1, mW3, a, n * a.wb * a.splits, s)) !=
       cudaSuccess)
     return err;
+  a.row_tok = nullptr;
   if ((err = record(ev, 0, s)) != cudaSuccess) return err;
   const size_t hsmem = (size_t)(F / RQ_CLUSTER) * sizeof(float);
   {
@@ -1278,7 +1285,8 @@ cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const ui
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     if ((err = cudaLaunchKernelEx(&cfg, swiglu_reduce_e4m3_kernel, w.p13, p.s13, a.split_stride,
-                                  F, n, static_cast<const int32_t*>(w.offsets), w.sx, s1, s3,
+                                  F, n, static_cast<const int32_t*>(w.offsets),
+                                  static_cast<const int32_t*>(w.row_tok), w.sx, s1, s3,
                                   static_cast<uint8_t*>(w.h), w.sh)) != cudaSuccess)
       return err;
   }

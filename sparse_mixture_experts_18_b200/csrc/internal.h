@@ -41,7 +41,7 @@ struct Plan {
   size_t o_rpart;          // small batch: partial router logits [ceil(d/64)][T][n]
   size_t o_rowtok;         // token of each permuted row [rows_max] (small batch, gather_x)
   size_t o_rowgate;        // gather_x: gate of each permuted row [rows_max]
-  size_t o_sx, o_sh;       // fp8: scales of the X_perm rows and of the h rows [rows_max]
+  size_t o_sx, o_sh;       // fp8: token-row scales [T] and h-row scales [rows_max]
   size_t o_status, o_idx, o_gate, o_blk_counts, o_blk_base, o_counts, o_offsets, o_inv,
       o_xperm, o_h, o_y, o_p13, o_xn, total;
 };
@@ -54,7 +54,7 @@ struct Workspace {
   float* rpart;          // small-batch routing: partial logits
   int32_t* row_tok;      // token of each permuted row (small batch, gather_x)
   float* row_gate;       // gather_x: gate of each permuted row
-  float* sx;             // fp8: scale of each X_perm row (its token's)
+  float* sx;             // fp8: scale of each token's row (the E4M3 rows are per token)
   float* sh;             // fp8: scale of each h row
   int32_t *idx, *blk_counts, *blk_base, *counts, *offsets, *inv;
   float* gate;

@@ -81,7 +81,7 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   // FP8 expert weights: the small-batch path with its one-launch routing only
   q.fp8 = fp8;
   if (fp8 && !(q.swap && q.fused_route)) return false;
-  q.gather_small = q.swap && q.fused_route && !fp8 && dt == 1;
+  q.gather_small = q.swap && q.fused_route && dt == 1;  // (FP8: from the quantised rows)
   const int kbw = fp8 ? 128 : 64;  // elements per 128-byte K block
   if (q.swap) {
     q.tok_tile = (int)((T + 15) / 16 * 16);

@@ -212,19 +212,17 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
   if (threadIdx.x < n) blk_counts[(int64_t)blockIdx.x * n + threadIdx.x] = hist[threadIdx.x];
 }
 
-// FP8-weight block: entry i (token i / K) -> permuted row row[i]: the token's bf16 x row as
-// E4M3 codes with its own scale (max |x| / 448), one warp per entry, two passes over the row.
-__device__ __forceinline__ void gather_rows_e4m3(const __nv_bfloat16* __restrict__ x, int d,
-                                                 int K, int E, const int* row,
-                                                 uint8_t* __restrict__ xq,
-                                                 float* __restrict__ sx, int tid,
-                                                 int nthreads) {
+// FP8-weight block: every token's bf16 x row as E4M3 codes with its own scale (max |x| /
+// 448) into xq[t] and sx[t]; one warp per token, two passes over the row.  The G13 kernel
+// gathers the rows of each expert from xq by token.
+__device__ __forceinline__ void quantize_tokens_e4m3(const __nv_bfloat16* __restrict__ x,
+                                                     int d, int T, uint8_t* __restrict__ xq,
+                                                     float* __restrict__ sx, int tid,
+                                                     int nthreads) {
   constexpr int U = 4;  // 16-byte loads in flight per lane
   const int lane = tid & 31, nwarps = nthreads >> 5;
-  for (int i = tid >> 5; i < E; i += nwarps) {
-    const int r = row[i];
-    if (r < 0) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(i / K) * d);
+  for (int r = tid >> 5; r < T; r += nwarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * d);
     const int nv = d / 8;  // 8 bf16 per 16-byte vector
     float amax = 0.f;
     for (int v0 = lane; v0 < nv; v0 += 32 * U) {
@@ -340,8 +338,8 @@ __device__ __forceinline__ void gather_rows(const Tact* __restrict__ x, int64_t 
 // TopK and softmax, the expert counts, group offsets (padded to row_align), the stable rank
 // of every (token, slot) (per-warp match + per-expert prefix over 32-entry chunks), the
 // inverse map token -> row and the map row -> token.  Then, if xq is given (FP8 weights), the
-// rows as E4M3 codes with their scales; else, if xperm is given, the bf16 rows (without
-// either, the G13 kernel gathers the token rows from x itself).
+// token rows as E4M3 codes with their scales; else, if xperm is given, the bf16 rows in
+// permuted order.  The G13 kernel gathers token rows from x (bf16) or xq (FP8) otherwise.
 constexpr int RS_THREADS = 1024;
 constexpr int RS_MAX_T = 64;
 constexpr int RS_MAX_ENTRIES = SMALL_ROUTE_MAX_ROWS;
@@ -534,11 +532,9 @@ __global__ void __launch_bounds__(RS_THREADS)
     inv[i] = row;
     if (row >= 0) row_tok[row] = i / K;
   }
-  if (xq != nullptr) {  // FP8-weight block: quantised rows and their scales
-    if constexpr (std::is_same<Tact, __nv_bfloat16>::value) {
-      __syncthreads();
-      gather_rows_e4m3(x, d, K, E, s_row, xq, sx, tid, RS_THREADS);
-    }
+  if (xq != nullptr) {  // FP8-weight block: quantised token rows and their scales
+    if constexpr (std::is_same<Tact, __nv_bfloat16>::value)
+      quantize_tokens_e4m3(x, d, T, xq, sx, tid, RS_THREADS);
     return;
   }
   if (xperm == nullptr) return;  // the G13 kernel gathers the token rows from x
