@@ -171,9 +171,10 @@ MOE_API moe_status moe_forward_profiled(const void* x, const float* W_g, const v
 
 /* Work plan chosen for a shape (for reports): *small_batch = 1 if the weights are the MMA's
  * 128-row operand (small token counts), 0 otherwise; *split13 / *split2 = K-splits of the
- * two expert GEMMs on that path (1 otherwise); *launches = kernels one forward launches. */
+ * two expert GEMMs on that path (1 otherwise); *launches = kernels one forward launches;
+ * *pair = 1 if the expert GEMMs run on CTA pairs (256-row tiles).  Any output may be NULL. */
 MOE_API moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt,
-                                 int* small_batch, int* split13, int* split2, int* launches);
+                                 int* small_batch, int* split13, int* split2, int* launches, int* pair);
 
 /* Stack of L blocks on a residual stream (attention omitted), in place on x [T][d]:
  *   for l in 0..L-1:  x <- round(x + MoE_l(RMSNorm(x)))

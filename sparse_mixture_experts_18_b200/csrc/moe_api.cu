@@ -326,13 +326,14 @@ moe_status moe_forward_profiled(const void* x, const float* W_g, const void* W1,
 }
 
 moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt,
-                         int* small_batch, int* split13, int* split2, int* launches) {
+                         int* small_batch, int* split13, int* split2, int* launches, int* pair) {
   Plan p;
   if (!make_plan(T, d, F, n, K, (int)dt, false, &p)) return shape_status(T, d, F, n, K, dt);
   if (small_batch) *small_batch = p.swap ? 1 : 0;
   if (split13) *split13 = p.swap ? p.s13 : 1;
   if (split2) *split2 = p.swap ? p.s2 : 1;
   if (launches) *launches = T == 0 ? 0 : (p.fused_route ? 1 : 3) + (p.swap ? 3 : 2) + 1;
+  if (pair) *pair = p.pair ? 1 : 0;
   return MOE_OK;
 }
 

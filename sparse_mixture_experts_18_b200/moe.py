@@ -61,7 +61,7 @@ def lib() -> ctypes.CDLL:
                                            P, ctypes.POINTER(P), I32]
         IP = ctypes.POINTER(ctypes.c_int)
         L.moe_plan_info.restype = I32
-        L.moe_plan_info.argtypes = [I64, I64, I64, I32, I32, I32, IP, IP, IP, IP]
+        L.moe_plan_info.argtypes = [I64, I64, I64, I32, I32, I32, IP, IP, IP, IP, IP]
         L.moe_forward_noalloc.restype = I32
         L.moe_forward_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P, P]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -181,11 +181,10 @@ def moe_forward_profiled(x, W_g, W1, W3, W2, K: int, events, out=None, workspace
 def moe_plan_info(T, d, F, n, K, dtype=torch.bfloat16) -> dict:
     """The work plan the library picks for a shape."""
     dt = MOE_BF16 if dtype in (torch.bfloat16, MOE_BF16) else MOE_F32
-    v = [ctypes.c_int(0) for _ in range(4)]
+    v = [ctypes.c_int(0) for _ in range(5)]
     _check("moe_plan_info", lib().moe_plan_info(T, d, F, n, K, dt, *[ctypes.byref(i) for i in v]))
-    pair = not v[0].value and dt == MOE_BF16 and T * K >= 640 * n  # same rule as the plan
     return {"small_batch": bool(v[0].value), "split13": v[1].value, "split2": v[2].value,
-            "launches": v[3].value, "pair": bool(pair)}
+            "launches": v[3].value, "pair": bool(v[4].value)}
 
 
 def moe_forward_debug(x, W_g, W1, W3, W2, K: int, out=None, workspace=None, stream=None):

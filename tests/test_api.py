@@ -69,19 +69,22 @@ def test_workspace_bytes(L):
 
 
 def _plan(L, T, d, F, n, K, dt=BF16):
-    v = [ctypes.c_int(-1) for _ in range(4)]
+    v = [ctypes.c_int(-1) for _ in range(5)]
     rc = L.moe_plan_info(T, d, F, n, K, dt, *[ctypes.byref(i) for i in v])
     return rc, [i.value for i in v]
 
 
 def test_plan_selection(L):
-    rc, (small, s13, s2, launches) = _plan(L, 16, 4096, 14336, 8, 2)
+    rc, (small, s13, s2, launches, pair) = _plan(L, 16, 4096, 14336, 8, 2)
     assert rc == OK and small == 1 and s13 >= 1 and s2 >= 1 and launches == 5  # fused route
-    assert 4096 // 64 % s13 == 0 and 14336 // 64 % s2 == 0
-    rc, (small, s13, s2, launches) = _plan(L, 4096, 4096, 14336, 8, 2)
-    assert rc == OK and small == 0 and s13 == 1 and s2 == 1 and launches == 6
-    rc, (small, _, _, _) = _plan(L, 64, 128, 256, 8, 2, F32)
-    assert rc == OK and small == 0
+    assert pair == 0 and 4096 // 64 % s13 == 0 and 14336 // 64 % s2 == 0
+    rc, (small, s13, s2, launches, pair) = _plan(L, 4096, 4096, 14336, 8, 2)
+    assert rc == OK and small == 0 and s13 == 1 and s2 == 1 and launches == 6 and pair == 1
+    rc, (small, _, _, _, pair) = _plan(L, 1024, 4096, 14336, 8, 2)   # 128-row tiles
+    assert rc == OK and small == 0 and pair == 0
+    rc, (small, _, _, _, pair) = _plan(L, 64, 128, 256, 8, 2, F32)
+    assert rc == OK and small == 0 and pair == 0
+    assert L.moe_plan_info(16, 4096, 14336, 8, 2, BF16, None, None, None, None, None) == OK
     assert _plan(L, 16, 100, 256, 8, 2)[0] == UNSUPPORTED
     assert _plan(L, 16, 128, 256, 8, 9)[0] == INVALID
 
