@@ -2,18 +2,23 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-A step is one pass of the whole block (router + TopK + softmax, permute, both expert GEMMs,
-gated combine) over one batch of seeded synthetic input of the workload's shapes.  Default
-workload: Mixtral-shaped decode batch (T=16, d=4096, F=14336, n=8, K=2, bf16).
+A step is one pass of the whole hot path (router + TopK + softmax, permute, both expert GEMMs,
+gated combine; for stacked workloads RMSNorm and the residual add, in every block) over one
+batch of seeded synthetic input of the workload's shapes.  Default workload: the largest
+single-GPU configuration, 32 stacked Mixtral MoE blocks (RMSNorm -> MoE -> residual,
+attention omitted) on T=8192 tokens, d=4096, F=14336, n=8, K=2, bf16, ~90 GB of weights.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a device
 synchronisation, timed with CUDA events on the launching stream, max over ranks.  The expert
 weights (2.8 GB per layer) exceed the 126 MB L2, so no flush is needed between steps.
-  value   tokens/s of all ranks with inputs resident in HBM (moe_forward);
-  e2e     the same through moe_forward_host_io with pinned host x / out, host<->device
-          copies and a per-step synchronisation inside the timed region;
+  value   tokens/s of all ranks with inputs resident in HBM (moe_forward / moe_stack_forward);
+  e2e     the same through the host-I/O entry points (moe_forward_host_io /
+          moe_stack_forward_host_io) with pinned host x / out, host<->device copies and a
+          per-step synchronisation inside the timed region;
   roofline  the dominant kernel (the gate/up expert GEMM), its duration from events the
-          library records on its own stream around each stage.
+          library records on its own stream around each stage (of every block);
+  parity  the benched workload's GPU result against the oracle on the CPU-baseline leg's
+          token sample (for the stack: block 1 on the GPU's own input).
 With N > 1 (torchrun) every rank runs an independent replica on its own batch (the block
 has no exchange step on one node's data-parallel path): weak scaling.
 
@@ -39,11 +44,11 @@ import torch  # noqa: E402
 import moe_inputs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and TFLOP/s (bf16, top-2 of 8) as % of B200 roofline"
-DEFAULT_WORKLOAD = "decode_t16"
+DEFAULT_WORKLOAD = "stack32_t8192"
 
-# DRAM bytes (read + write) of one launch of the dominant kernel (G13), from the ncu
-# captures summarised in profiles/tc_grouped_gemm_<workload>.md, valid only for the kernel
-# source they were taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
+# DRAM bytes (read + write) of one launch of the dominant kernel (G13), from one ncu capture
+# of that kernel on the workload's shapes (for the stack: one T=8192 block), valid only for
+# the kernel source it was taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
     "decode_t16": {"bytes": 1886786272, "src": "9c8fdd53d8eb"},
     "prefill_t4096": {"bytes": 2523485256, "src": "9c8fdd53d8eb"},
@@ -174,24 +179,24 @@ def run_gpu(args, w):
     layers = [moe_inputs.make_layer(wr, layer=l, device=dev) for l in range(w.layers)]
     layer = layers[0]
     stream = torch.cuda.Stream(device=dev)
-    ws = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K, torch.bfloat16),
-                             dev, stream)
-    out = torch.empty_like(x)
     plan = moe.moe_plan_info(w.T, w.d, w.F, w.n, w.K)
     small_batch, s13, s2, launches = (plan["small_batch"], plan["split13"], plan["split2"],
                                       plan["launches"])
     stacked = w.layers > 1
+    out = torch.empty_like(x)
     if stacked:  # x is the residual stream: every step restarts from the same input
-        ws_stack = moe.alloc_workspace(
-            moe.moe_stack_workspace_bytes(w.T, w.d, w.F, w.n, w.K), dev, stream)
-        xs = torch.empty_like(x)
-        launches = w.layers * (1 + launches) + 1  # RMSNorm per block, the restart copy
+        ws = moe.alloc_workspace(moe.moe_stack_workspace_bytes(w.T, w.d, w.F, w.n, w.K), dev,
+                                 stream)
+        launches = w.layers * (1 + launches)  # each block: RMSNorm, then the MoE block
+    else:
+        ws = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K,
+                                                         torch.bfloat16), dev, stream)
 
     def step():
         if stacked:
             with torch.cuda.stream(stream):
-                xs.copy_(x, non_blocking=True)
-            moe.moe_stack_forward(xs, layers, w.K, workspace=ws_stack, stream=stream)
+                out.copy_(x, non_blocking=True)
+            moe.moe_stack_forward(out, layers, w.K, workspace=ws, stream=stream)
         else:
             moe.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.K, out=out,
                             workspace=ws, stream=stream)
@@ -204,9 +209,13 @@ def run_gpu(args, w):
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
+    # routing of the (first) block on this batch, for the report and the roofline bytes
+    ws1 = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K, torch.bfloat16),
+                              dev, stream)
     _, idx, _, counts, _, _ = moe.moe_forward_debug(x, layer["Wg"], layer["W1"], layer["W3"],
-                                                    layer["W2"], w.K, workspace=ws,
+                                                    layer["W2"], w.K, workspace=ws1,
                                                     stream=stream)
+    del ws1
     torch.cuda.synchronize(dev)
     counts = counts.cpu().tolist()
     n_active = sum(1 for c in counts if c > 0)
@@ -222,28 +231,35 @@ def run_gpu(args, w):
         barrier()
         ms = ev0.elapsed_time(ev1)
         # ---- per-stage durations from events recorded by the library on its stream
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        # (stacked: six per block); stage_ms[i] lists (route, G13, reduce, G2, combine) per block
+        nev = 6 * w.layers
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)]
                for _ in range(args.steps)]
         for i in range(args.steps):
             for e in evs[i]:
                 e.record(stream)  # creates the cudaEvent_t; the library re-records it
-            moe.moe_forward_profiled(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.K,
-                                     evs[i], out=out, workspace=ws, stream=stream)
+            if stacked:
+                with torch.cuda.stream(stream):
+                    out.copy_(x, non_blocking=True)
+                moe.moe_stack_forward_profiled(out, layers, w.K, evs[i], workspace=ws,
+                                               stream=stream)
+            else:
+                moe.moe_forward_profiled(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"],
+                                         w.K, evs[i], out=out, workspace=ws, stream=stream)
         barrier()
-        stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)]
-                    for i in range(args.steps)]
-        # ---- e2e: pinned host x in, host out back, every step
+        stage_ms = [[evs[i][6 * b + j].elapsed_time(evs[i][6 * b + j + 1]) for j in range(5)]
+                    for i in range(args.steps) for b in range(w.layers)]
+        del evs
+        # ---- e2e: pinned host x in, host out back, every step, through the C-ABI host-I/O
+        # entry points
         xh = x.cpu().pin_memory()
         oh = torch.empty_like(xh).pin_memory()
         xd, od = torch.empty_like(x), torch.empty_like(x)
 
         def e2e_step():
-            if stacked:  # host -> device, the 32-block stack in place, device -> host
-                with torch.cuda.stream(stream):
-                    xd.copy_(xh, non_blocking=True)
-                moe.moe_stack_forward(xd, layers, w.K, workspace=ws_stack, stream=stream)
-                with torch.cuda.stream(stream):
-                    oh.copy_(xd, non_blocking=True)
+            if stacked:
+                moe.moe_stack_forward_host_io(xh, xd, layers, w.K, oh, workspace=ws,
+                                              stream=stream)
             else:
                 moe.moe_forward_host_io(xh, xd, layer["Wg"], layer["W1"], layer["W3"],
                                         layer["W2"], w.K, od, oh, ws, stream=stream)
@@ -271,8 +287,8 @@ def run_gpu(args, w):
     ms_step = ms / args.steps
     tok_s = world * w.T * args.steps / (ms / 1e3)
     tflops = tok_s * w.layers * _flops_per_token(w) / 1e12
-    g13 = statistics.mean(s[1] for s in stage_ms)          # gate/up GEMM (dominant kernel)
-    stage_avg = [statistics.mean(s[j] for s in stage_ms) for j in range(5)]
+    g13 = statistics.mean(st[1] for st in stage_ms)       # gate/up GEMM (dominant kernel)
+    stage_avg = [statistics.mean(st[j] for st in stage_ms) for j in range(5)]
     es = 2
     timed_s = ms / 1e3
     bf16_peak = peaks["bf16_sustained"] if timed_s > 1.0 else peaks["bf16"]
@@ -296,14 +312,13 @@ def run_gpu(args, w):
               "CTA-pair 256-row tiles" if plan["pair"] else "128-row tiles")
     cap = TRAFFIC.get(w.name)
     traffic = cap["bytes"] if cap and cap["src"] == kernel_source_hash() else None
+    workload = workload_label(w)
     line = {
         "metric": METRIC, "value": round(tok_s, 2), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations, RMS-normalised; N(0,1/fan_in) weights)",
-        "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K} bf16"
-                               + (f", {w.layers} x (RMSNorm -> MoE -> residual)" if stacked
-                                  else ""),
+        "config": {"workload": workload,
                    "tokens_per_rank": w.T, "l2": "inputs larger than L2 "
                    f"({w.layers * 3 * w.n * w.F * w.d * es / 1e9:.2f} GB of expert weights)",
                    "parallelism": f"replicas x{world}",
@@ -315,28 +330,50 @@ def run_gpu(args, w):
                          "frac": round(step_frac, 4),
                          "basis": "unique expert-weight bytes of selected experts per step / "
                                   "measured HBM copy GB/s" if step_hbm else
-                                  "routed FLOPs per step / measured bf16 GEMM TFLOP/s"},
+                                  "routed FLOPs per step / measured bf16 GEMM TFLOP/s"
+                                  + (" (sustained)" if bf16_peak == peaks["bf16_sustained"]
+                                     else " (burst)")},
         "roofline": {"bound": bound,
                      "kernel": ("tc_pair_gemm" if plan["pair"] else "tc_grouped_gemm")
-                               + " G13 (gate/up + SwiGLU)",
+                               + " G13 (gate/up + SwiGLU)"
+                               + (f", every block of {w.layers}" if stacked else ""),
                      "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": peaks["source"], "launch_ms": round(g13, 5)},
+                     "peak_source": peaks["source"]
+                     + (" (sustained)" if unit == "TFLOP/s" and peak == peaks["bf16_sustained"]
+                        else " (burst)" if unit == "TFLOP/s" else ""),
+                     "launch_ms": round(g13, 5),
+                     "launches_timed": len(stage_ms)},
         "stage_ms": {"route": round(stage_avg[0], 5), "gemm13": round(stage_avg[1], 5),
                      "splitk_reduce": round(stage_avg[2], 5), "gemm2": round(stage_avg[3], 5),
                      "combine": round(stage_avg[4], 5)},
         "e2e": {"value": round(world * w.T * args.steps / (e2e_ms / 1e3), 2),
                 "unit": "tokens/s", "h2d_bytes_per_step": w.T * w.d * es,
-                "d2h_bytes_per_step": w.T * w.d * es},
+                "d2h_bytes_per_step": w.T * w.d * es,
+                "api": "moe_stack_forward_host_io" if stacked else "moe_forward_host_io"},
         "gpu_launches": launches * args.steps,
         "clocks": clocks.summary(),
     }
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, x.cpu(), {k: v.cpu() for k, v in layer.items()},
-                                            args.cpu_tokens)
+        # GPU result the CPU-baseline leg checks its oracle sample against: the first block
+        if stacked:
+            gpu1 = x.clone()
+            moe.moe_stack_forward(gpu1, layers[:1], w.K, workspace=ws, stream=stream)
+        else:
+            gpu1 = out
+        torch.cuda.synchronize(dev)
+        line["cpu_baseline"], line["parity"] = cpu_baseline(
+            w, x.cpu(), {k: v.cpu() for k, v in layer.items()}, args.cpu_tokens,
+            gpu_out=gpu1.float().cpu())
     del layers
     print(json.dumps(line), flush=True)
     return line
+
+
+def workload_label(w) -> str:
+    """config.workload string, shared by both arms of the benchmark."""
+    return (f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K} bf16"
+            + (f", {w.layers} x (RMSNorm -> MoE -> residual)" if w.layers > 1 else ""))
 
 
 def run_gpu_fp8(args, w):
@@ -475,30 +512,83 @@ def run_gpu_fp8(args, w):
     return line
 
 
-def cpu_baseline(w, x, layer, ntok, seconds: float = 10.0):
+def _oracle_block(oracle, w, x, layer, toks):
+    """The oracle's result for token rows `toks` of the workload's (first) block, rounded to
+    bf16 as the GPU's output is: the MoE block, or for stacked workloads one whole block
+    x + MoE(RMSNorm(x)).  Also the oracle's router logits of those rows."""
+    import numpy as np
+    xs = x[toks]
+    if w.layers > 1:
+        xin = xs.double().numpy()
+        ref, _, _ = oracle.block_forward(xin, layer["Wg"], layer["W1"], layer["W3"], layer["W2"],
+                                         w.n, w.K, 1e-5)
+        xn = torch.from_numpy(oracle.rmsnorm(xin, 1e-5, oracle.BF16)).to(torch.bfloat16)
+        logits, _, _ = oracle.route(xn, layer["Wg"], w.n, w.K)
+        return ref, logits
+    y, _, _ = oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
+                                 tokens=np.asarray(toks, np.int64))
+    logits, _, _ = oracle.route(xs, layer["Wg"], w.n, w.K)
+    return oracle.round_array(y, oracle.BF16), logits
+
+
+def cpu_baseline(w, x, layer, ntok, seconds: float = 10.0, gpu_out=None):
     """The oracle as it stands on the host cores, on a bounded sample of the workload: calls
-    of max(ntok, threads) tokens (cycling through the batch) repeated for about `seconds`."""
+    of max(ntok, threads) tokens (cycling through the batch) repeated for about `seconds`;
+    for stacked workloads the oracle runs one whole block and the rate is divided by the
+    number of blocks.  Returns (baseline dict, parity dict): the parity dict compares the
+    oracle's results for the tokens it evaluated with gpu_out (the GPU's result of the same
+    block on the same input) -- max-abs and relative L2 error over the tokens whose K-th and
+    (K+1)-th oracle logits are more than 1e-4 apart (relative), and the count of those that
+    are not (exempt near-ties, whose expert set either way is correct)."""
+    import numpy as np
+
     import oracle
     oracle.build()
     threads = _omp_threads()
     chunk = max(1, min(max(ntok, threads), w.T))
     done, start = 0, 0
+    refs = {}
     t0 = time.perf_counter()
     while True:
         toks = [(start + j) % w.T for j in range(chunk)]
-        oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
-                           tokens=toks)
+        ref, logits = _oracle_block(oracle, w, x, layer, toks)
+        for j, t in enumerate(toks):
+            refs.setdefault(t, (ref[j], logits[j]))
         done += chunk
         start = (start + chunk) % w.T
         dt = time.perf_counter() - t0
         if dt >= seconds:
             break
-    per_block = f", one of the {w.layers} blocks (rate divided by {w.layers})" \
+    blocks = f", one whole block of the {w.layers} (rate divided by {w.layers})" \
         if w.layers > 1 else ""
-    return {"value": round(done / dt / w.layers, 4), "unit": "tokens/s",
+    base = {"value": round(done / dt / w.layers, 4), "unit": "tokens/s",
             "cores": min(chunk, threads), "kind": "oracle",
             "sample": f"{done} token evaluations in calls of {chunk} (cycling over the {w.T} "
-                      f"tokens of {w.name}){per_block}, {dt:.1f} s (fp64 C, OpenMP over tokens)"}
+                      f"tokens of {w.name}){blocks}, {dt:.1f} s (fp64 C, OpenMP over tokens)"}
+    if gpu_out is None:
+        return base, None
+    toks = sorted(refs)
+    exempt, err, refn = 0, [], []
+    for t in toks:
+        r, l = refs[t]
+        srt = np.sort(l)[::-1]
+        a, b = srt[w.K - 1], srt[w.K] if w.K < w.n else -np.inf
+        if w.K < w.n and abs(a - b) <= 1e-4 * max(abs(a), abs(b)):
+            exempt += 1
+            continue
+        err.append(gpu_out[t].double().numpy() - r)
+        refn.append(r)
+    err, refn = np.array(err), np.array(refn)
+    max_abs = float(np.max(np.abs(err))) if err.size else 0.0
+    rel_l2 = float(np.linalg.norm(err) / max(np.linalg.norm(refn), 1e-300)) if err.size else 0.0
+    allow = 2e-2 + (2.0 ** -7 * np.abs(refn) if w.layers > 1 else 0.0)
+    par = {"what": ("block 1 of the stack (RMSNorm -> MoE -> residual) on the GPU's input"
+                    if w.layers > 1 else "the block's output") + ", oracle in fp64",
+           "tokens": len(toks), "exempt": exempt, "max_abs": max_abs, "rel_l2": rel_l2,
+           "ok": bool(err.size == 0 or (np.all(np.abs(err) <= allow) and rel_l2 <= 5e-3)),
+           "bars": "max-abs 2e-2" + (" + 2^-7 |ref|" if w.layers > 1 else "")
+                   + ", rel-L2 5e-3; exempt: 2nd-vs-3rd logit gap <= 1e-4 relative"}
+    return base, par
 
 
 def _omp_threads():
@@ -509,7 +599,10 @@ def _omp_threads():
 
 
 def run_reference(args, w):
-    """Reference arm: the CPU oracle timed on the host cores (rank 0 only)."""
+    """Reference arm: the CPU oracle timed on the host cores (rank 0 only), on the same
+    workload, metric and unit as the GPU arm; each step a bounded sample of tokens of the
+    (first) block, for stacked workloads one whole block with the rate divided by the number
+    of blocks."""
     world, rank, _ = _dist()
     if rank != 0:
         return None
@@ -520,23 +613,21 @@ def run_reference(args, w):
     threads = _omp_threads()
     per_step = min(w.T, max(args.cpu_tokens, threads))  # a token for every host thread
     for i in range(args.warmup):
-        oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
-                           tokens=[i % w.T])
+        _oracle_block(oracle, w, x, layer, [i % w.T])
     t0 = time.perf_counter()
     for i in range(args.steps):
         toks = [(i * per_step + j) % w.T for j in range(per_step)]
-        oracle.moe_forward(x, layer["Wg"], layer["W1"], layer["W3"], layer["W2"], w.n, w.K,
-                           tokens=toks)
+        _oracle_block(oracle, w, x, layer, toks)
     dt = time.perf_counter() - t0
     v = per_step * args.steps / dt / w.layers
     sample = (f"{per_step} of {w.T} tokens of {w.name} per step "
               "(fp64 C oracle, OpenMP over tokens)"
-              + (f"; one block, rate divided by {w.layers} blocks" if w.layers > 1 else ""))
+              + (f"; one whole block, rate divided by {w.layers} blocks" if w.layers > 1 else ""))
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K}"},
+            "config": {"workload": workload_label(w)},
             "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s",
                              "cores": min(per_step, threads), "kind": "oracle",
                              "sample": sample},
@@ -558,6 +649,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "e4m3"],
                     help="e4m3: the FP8 expert-weight variant (small-batch workloads)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="run only the first N blocks of a stacked workload (N=1: one MoE "
+                         "block of its shape), e.g. for an ncu capture of a few GB")
     ap.add_argument("--gather-x", action="store_true",
                     help="CTA-pair path: gather G13's A rows from x (TMA gather4) instead of "
                          "X_perm, gates applied in G2 (sets MOE_GATHER_X=1)")
@@ -567,6 +661,10 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = moe_inputs.WORKLOADS[args.workload]
+    if args.layers is not None:
+        if not 1 <= args.layers <= w.layers:
+            ap.error(f"--layers must be in 1..{w.layers} for {w.name}")
+        w = w.replace(layers=args.layers)
     if w.dtype != "bf16":
         ap.error("the bench measures the bf16 path")
     if args.impl == "reference":

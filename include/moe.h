@@ -2,16 +2,20 @@
  * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts block library (libmoe.so).
  *
  * What is computed, per token x (a row of the activation matrix), as defined in
- * "Mixtral of Experts" (arXiv 2401.04088), method section, equations G(x) and y:
+ * "Mixtral of Experts" (arXiv 2401.04088; the xyznot.com summary page of that title, method
+ * section, equations G(x) and y):
  *
  *   l    = x . W_g                         router logits over n experts, fp32, no bias
  *   G(x) = Softmax(TopK(l))                TopK keeps the K largest logits (others -inf);
  *                                          Mixtral uses K = 2 of n = 8
  *   y    = sum_i G(x)_i * SwiGLU_i(x),     SwiGLU_i(x) = W2_i . (silu(W1_i . x) * (W3_i . x))
  *
- * Experts whose gate is zero are not evaluated (the Indonesian news summary, section on how
- * the MoE layer is computed, notes this is exact); tokens are grouped per expert instead
- * (the same page's implementation notes: variable token counts per expert).
+ * Experts whose gate is zero are not evaluated ("Mixtral 8x7B: Model Bahasa Sparse Mixture of
+ * Experts", id.news.hada.io, section "Cara Komputasi Layer MoE": outputs of zero-gate experts
+ * need not be computed); tokens are grouped per expert instead (same page, section
+ * "Implementasi dan Efisiensi Inferensi": the number of tokens per expert varies).
+ * Below, "the method section" is the xyznot.com page's and "the hada.io page" is the
+ * Indonesian summary.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -69,21 +73,28 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
-/* Bytes of device workspace moe_forward / moe_forward_debug need for this shape
+/* Workspace plumbing (the pages have no counterpart: the caller-owned scratch memory of the
+ * grouping and expert stages below).
+ * Bytes of device workspace moe_forward / moe_forward_debug need for this shape
  * (0 if the shape is unsupported).  moe_stack_forward needs moe_stack_workspace_bytes(). */
 MOE_API size_t moe_workspace_bytes(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt);
 
-/* Zero the workspace's status word and counters; call once after allocating it. */
+/* Zero the workspace's status word and counters (enqueued on `stream`); call once after
+ * allocating it, and again after any error that moe_workspace_status() reports. */
 MOE_API moe_status moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
-/* Synchronise `stream`, then read and clear the workspace status word written by kernels.
- * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded wait ran out), MOE_ERR_DEVICE (an index out
- * of range) or MOE_ERR_CUDA (the stream reported an error).  *raw (may be NULL) receives
- * the raw bit mask.  After any error, call moe_workspace_init() again before reusing the
- * workspace (an interrupted call can leave its counters mid-count). */
+/* Synchronise `stream`, then read the workspace status word written by kernels and, if it is
+ * not zero, clear it (the clear is enqueued on `stream`).  Returns MOE_OK, MOE_ERR_TIMEOUT (a
+ * bounded wait ran out), MOE_ERR_DEVICE (an index out of range) or MOE_ERR_CUDA (the stream
+ * reported an error).  *raw (may be NULL) receives the raw bit mask (bit 0: a wait ran out;
+ * bit 1: an expert index outside [0, n); bit 2: a permuted row outside the workspace).
+ * After any error, call moe_workspace_init() again before reusing the workspace (an
+ * interrupted call can leave its counters mid-count). */
 MOE_API moe_status moe_workspace_status(void* workspace, void* stream, uint32_t* raw);
 
-/* One MoE block forward:  out[t] = sum_k G(x_t)_k * SwiGLU_{e_k}(x_t).
+/* One MoE block forward:  out[t] = sum_k G(x_t)_k * SwiGLU_{e_k}(x_t)
+ * (the method section, equations G(x) = Softmax(TopK(x . W_g)) and y; the hada.io page,
+ * "Cara Komputasi Layer MoE": softmax over the top-K logits of a linear layer, K = 2).
  *   x    [T][d]   dt           token activations
  *   W_g  [d][n]   fp32         router weight
  *   W1   [n][F][d] dt          gate projection of each expert
@@ -96,7 +107,9 @@ MOE_API moe_status moe_forward(const void* x, const float* W_g, const void* W1, 
                        moe_dtype dt, void* out, void* workspace, size_t workspace_bytes,
                        void* stream);
 
-/* moe_forward, then copies of the routing state into caller buffers (each may be NULL):
+/* moe_forward, then copies of the routing state into caller buffers (each may be NULL) --
+ * the router's choice G(x) (method section, equation G(x)) and the per-expert grouping of
+ * the tokens (hada.io page, "Implementasi dan Efisiensi Inferensi"):
  *   topk_idx [T][K] int32      selected experts, slot 0 = larger logit
  *   topk_gate [T][K] fp32      G(x) over the kept experts (rows sum to 1)
  *   expert_counts [n] int32    tokens routed to each expert
@@ -111,7 +124,8 @@ MOE_API moe_status moe_forward_debug(const void* x, const float* W_g, const void
                              int32_t* token_rows);
 
 /* ---- FP8 expert weights (a variant for decode bandwidth; the pages only mention quantised
- * community builds, so the format is this library's plain reading):
+ * community builds -- the reader comments on the hada.io page -- and fix no format, so the
+ * format is this library's plain reading; it is not the hardware's block-scaled MX format):
  * OCP FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
  * largest finite 448) with one fp32 scale per row of each weight matrix:
  *   s = max_j |w_j| / 448 (1 for a zero row), code_j = E4M3(w_j / s), nearest, ties to even,
@@ -146,7 +160,8 @@ MOE_API moe_status moe_forward_fp8(const void* x, const float* W_g, const uint8_
                                    size_t workspace_bytes, void* stream, void* const* events,
                                    int n_events);
 
-/* moe_forward with HOST input and output: copies x_host (pinned recommended) to x_dev,
+/* moe_forward with HOST input and output (the block as in moe_forward; the host copies are
+ * plumbing with no counterpart in the pages): copies x_host (pinned recommended) to x_dev,
  * runs the block into out_dev and copies it back to out_host, all on `stream`; returns
  * after enqueueing (synchronise the stream before reading out_host).  x_dev and out_dev
  * are caller-owned device buffers of T*d elements. */
@@ -157,7 +172,8 @@ MOE_API moe_status moe_forward_host_io(const void* x_host, void* x_dev, const fl
                                size_t workspace_bytes, void* stream);
 
 /* moe_forward that also records caller-created CUDA events (cudaEvent_t, passed as void*)
- * on `stream` at the stage boundaries, for timing each kernel live:
+ * on `stream` at the stage boundaries, for timing each kernel live (measurement plumbing; the
+ * stages are those of moe_forward):
  *   events[0] before routing            events[1] after router, scan and permute
  *   events[2] after the gate/up GEMM    events[3] after the split-K reduction (== [2] when
  *                                                  the small-batch tiling is not used)
@@ -169,7 +185,7 @@ MOE_API moe_status moe_forward_profiled(const void* x, const float* W_g, const v
                                         void* workspace, size_t workspace_bytes, void* stream,
                                         void* const* events, int n_events);
 
-/* Work plan chosen for a shape (for reports): *small_batch = 1 if the weights are the MMA's
+/* Work plan chosen for a shape (for reports; no counterpart in the pages): *small_batch = 1 if the weights are the MMA's
  * 128-row operand (small token counts), 0 otherwise; *split13 / *split2 = K-splits of the
  * two expert GEMMs on that path (1 otherwise); *launches = kernels one forward launches;
  * *pair = 1 if the expert GEMMs run on CTA pairs (256-row tiles).  Any output may be NULL. */
@@ -178,15 +194,58 @@ MOE_API moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, 
 
 /* Stack of L blocks on a residual stream (attention omitted), in place on x [T][d]:
  *   for l in 0..L-1:  x <- round(x + MoE_l(RMSNorm(x)))
- * RMSNorm has unit gain: x / sqrt(mean(x^2) + eps), rounded to dt; the residual sum is
- * taken in fp32 and rounded once.  W_g, W1, W3, W2 are HOST arrays of L device pointers
- * (per-layer weights, layouts as above).  Only the bf16 path is supported. */
+ * The pages say only that every one of Mixtral's 32 layers replaces its feed-forward block
+ * with this MoE block (hada.io page, "Arsitektur Sparse Mixture of Experts"); the RMSNorm ->
+ * MoE -> residual stacking with attention left out is the library's stacked-block workload,
+ * not a passage of the pages.  RMSNorm has unit gain: x / sqrt(mean(x^2) + eps), rounded to
+ * dt; the residual sum is taken in fp32 and rounded once.  W_g, W1, W3, W2 are HOST arrays
+ * of L device pointers (per-layer weights, layouts as above).  Only the bf16 path is
+ * supported. */
 MOE_API size_t moe_stack_workspace_bytes(int64_t T, int64_t d, int64_t F, int n, int K,
                                  moe_dtype dt);
 MOE_API moe_status moe_stack_forward(void* x, const float* const* W_g, const void* const* W1,
                              const void* const* W3, const void* const* W2, int L, int64_t T,
                              int64_t d, int64_t F, int n, int K, moe_dtype dt, float eps,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* moe_stack_forward that records caller-created CUDA events at every block's stage
+ * boundaries (measurement plumbing): events[6*l + j] is block l's event j as in
+ * moe_forward_profiled (the block's RMSNorm runs just before events[6*l]).
+ * n_events must be 6*L. */
+MOE_API moe_status moe_stack_forward_profiled(void* x, const float* const* W_g,
+                                              const void* const* W1, const void* const* W3,
+                                              const void* const* W2, int L, int64_t T,
+                                              int64_t d, int64_t F, int n, int K, moe_dtype dt,
+                                              float eps, void* workspace,
+                                              size_t workspace_bytes, void* stream,
+                                              void* const* events, int n_events);
+
+/* moe_stack_forward with HOST input and output (host copies are plumbing): copies x_host
+ * (T*d bf16, pinned recommended) to the caller's device buffer x_dev, runs the L blocks in
+ * place on x_dev and copies the result to out_host, all enqueued on `stream`; returns after
+ * enqueueing (synchronise the stream before reading out_host). */
+MOE_API moe_status moe_stack_forward_host_io(const void* x_host, void* x_dev,
+                                             const float* const* W_g, const void* const* W1,
+                                             const void* const* W3, const void* const* W2,
+                                             int L, int64_t T, int64_t d, int64_t F, int n,
+                                             int K, moe_dtype dt, float eps, void* out_host,
+                                             void* workspace, size_t workspace_bytes,
+                                             void* stream);
+
+/* Test hook for the failure path (no counterpart in the pages): moe_forward, except that the
+ * one-CTA tensor-core kernel of the gate/up projection issues none of its loads, so its
+ * tensor-core thread waits on a barrier that nothing will complete; that wait, and the other
+ * pipeline waits of the kernel, give up after wait_limit_cycles (1 .. 4e9 SM clock cycles).
+ * The kernel then records bit 0 in the status word, lets nothing in flight outlive it, frees
+ * its tensor memory and returns; the rest of the block runs on undefined values.  Expect
+ * moe_workspace_status() == MOE_ERR_TIMEOUT afterwards, then call moe_workspace_init().
+ * Shapes that take the CTA-pair or fp32 kernels return MOE_ERR_UNSUPPORTED. */
+MOE_API moe_status moe_debug_forward_withheld(const void* x, const float* W_g, const void* W1,
+                                              const void* W3, const void* W2, int64_t T,
+                                              int64_t d, int64_t F, int n, int K, moe_dtype dt,
+                                              void* out, void* workspace,
+                                              size_t workspace_bytes, void* stream,
+                                              int64_t wait_limit_cycles);
 
 /* moe_forward without a caller-supplied workspace, for callers that cannot allocate device
  * memory (e.g. a plugin inside an application whose own pool owns every allocation, or a
@@ -196,17 +255,27 @@ MOE_API moe_status moe_stack_forward(void* x, const float* const* W_g, const voi
  *     library; every GPU that loads the library holds it until the process exits.  Shapes
  *     whose moe_workspace_bytes() exceeds it return MOE_ERR_WORKSPACE (at Mixtral's sizes it
  *     fits decode batches of up to 24 tokens).
- *   - The first call on a device, with that device current, looks up the array's address
- *     and zeroes its status word (synchronously); make that first call before any stream
- *     capture.  Nothing is allocated, and nothing is freed.
+ *   - Every call looks up the array's device address on the current device.  The first call
+ *     on a device (and the first after the context was re-created) also zeroes the array's
+ *     256-byte header with an asynchronous memset enqueued on `stream`, ahead of that call's
+ *     kernels; make that first call before any stream capture.  Nothing is allocated, and
+ *     nothing is freed.
  *   - All calls share the one array and it keeps the last call's contents: calls that
  *     overlap on the GPU (other streams, other threads) race on it.
+ *   - Faults that kernels detect go to the array's status word: read them with
+ *     moe_noalloc_status().
  * Arguments, layouts and errors otherwise as moe_forward. */
 #define MOE_NOALLOC_WORKSPACE_BYTES (32u << 20)
 MOE_API moe_status moe_forward_noalloc(const void* x, const float* W_g, const void* W1,
                                        const void* W3, const void* W2, int64_t T, int64_t d,
                                        int64_t F, int n, int K, moe_dtype dt, void* out,
                                        void* stream);
+
+/* moe_workspace_status() for the array moe_forward_noalloc uses (the paper has no
+ * counterpart): synchronises `stream`, reads and clears the status word.  On an error it
+ * also zeroes the array's header (status word and counters) on `stream` and synchronises,
+ * so the next moe_forward_noalloc starts clean. */
+MOE_API moe_status moe_noalloc_status(void* stream, uint32_t* raw);
 
 /* Short description of a status code (static string). */
 MOE_API const char* moe_status_string(moe_status s);

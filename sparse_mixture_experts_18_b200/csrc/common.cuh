@@ -87,17 +87,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the barrier's phase with the given parity has completed.  Gives up after
-// WAIT_LIMIT_CYCLES (or at once if *abort is set while waiting), records DEV_ERR_TIMEOUT and
-// returns false; the caller then unwinds without issuing further work.
+// `limit` cycles (WAIT_LIMIT_CYCLES unless a caller passes a shorter one), or at once if
+// *abort is set while waiting, records DEV_ERR_TIMEOUT and returns false; the caller then
+// unwinds without issuing further work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                          volatile int* abort) {
+                                          volatile int* abort,
+                                          long long limit = WAIT_LIMIT_CYCLES) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort) return false;
-      if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+      if (clock64() - t0 > limit) {
         set_status(status, DEV_ERR_TIMEOUT);
         *abort = 1;
         return false;

@@ -60,6 +60,12 @@ struct TcArgs {
   int gather_T;            // rows of x (a row index past the end reads zeros)
   const float* row_gate;   // gate of each permuted row
   int gather_rows;         // small batch gathering from x: permuted rows (T*K)
+  // one-CTA kernel: cycles a pipeline wait may last before the kernel gives up
+  // (WAIT_LIMIT_CYCLES), and the failure-path test hook: withhold_loads = 1 makes the
+  // producer issue no load at all, so the MMA thread's first wait is on a barrier nothing
+  // will complete and runs out after wait_limit cycles (0 on every forward call)
+  long long wait_limit = WAIT_LIMIT_CYCLES;
+  int withhold_loads = 0;
 };
 
 struct Ctrl {
@@ -194,11 +200,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const uint64_t pol_x = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
-      for (int id = blockIdx.x; id < total; id += gridDim.x) {
+      for (int id = blockIdx.x; id < total && !a.withhold_loads; id += gridDim.x) {
         const Work w = decode_work<SWAP>(a, c, id);
         bool ok = true;
         for (int kb = 0; kb < a.num_kb; ++kb) {
-          if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort)) { ok = false; break; }
+          if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort, a.wait_limit)) {
+            ok = false;
+            break;
+          }
           uint8_t* st = smem + (size_t)stage * a.stage_bytes;
           uint64_t* fb = &c->full[stage];
           mbar_arrive_expect_tx(fb, a.tx_bytes);
@@ -251,11 +260,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++it) {
         const uint32_t acc = (uint32_t)it % a.nacc;
         const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
-        if (!mbar_wait(&c->tempty[acc], aph ^ 1u, a.status, &c->abort)) break;
+        if (!mbar_wait(&c->tempty[acc], aph ^ 1u, a.status, &c->abort, a.wait_limit)) break;
         tc_fence_after();
         const uint32_t dtm = tmem_base + acc * a.acc_cols;
         for (int kb = 0; kb < a.num_kb; ++kb) {
-          if (!mbar_wait(&c->full[stage], phase, a.status, &c->abort)) { ok = false; break; }
+          if (!mbar_wait(&c->full[stage], phase, a.status, &c->abort, a.wait_limit)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t sb = smem_u32(smem + (size_t)stage * a.stage_bytes);
 #pragma unroll
@@ -294,7 +306,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const Work w = decode_work<SWAP>(a, c, id);
       const uint32_t acc = (uint32_t)it % a.nacc;
       const uint32_t aph = ((uint32_t)it / a.nacc) & 1u;
-      const bool ok = mbar_wait(&c->tfull[acc], aph, a.status, &c->abort);
+      const bool ok = mbar_wait(&c->tfull[acc], aph, a.status, &c->abort, a.wait_limit);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * a.acc_cols;
@@ -1120,9 +1132,15 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
     a.n_tiles = (F + 127) / 128;
     a.out = w.h;
     a.out_ld = F;
+    if (p.g13_withhold) {
+      a.withhold_loads = 1;
+      a.wait_limit = p.g13_wait_limit;
+    }
     if ((err = launch_one<KIND_G13, false>(mX, mW1, mW3, a, m_tiles_max * a.n_tiles, s)) !=
         cudaSuccess)
       return err;
+    a.withhold_loads = 0;
+    a.wait_limit = WAIT_LIMIT_CYCLES;
     if ((err = record(ev, 0, s)) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
       return err;
     // G2
@@ -1172,10 +1190,16 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
     a.gather_T = (int)p.T;
     a.gather_rows = (int)(p.T * p.K);
   }
+  if (p.g13_withhold) {
+    a.withhold_loads = 1;
+    a.wait_limit = p.g13_wait_limit;
+  }
   if ((err = launch_one<KIND_G13, true>(mX, mW1, mW3, a, n * a.wb * a.splits, s)) !=
       cudaSuccess)
     return err;
   a.row_tok = nullptr;
+  a.withhold_loads = 0;
+  a.wait_limit = WAIT_LIMIT_CYCLES;
   if ((err = record(ev, 0, s)) != cudaSuccess) return err;
   const int64_t rows = p.T * p.K;
   const int64_t vec = rows * F / 4;

@@ -37,6 +37,10 @@ struct Plan {
   int s13 = 1, s2 = 1;     // swap: split-K factors of the two expert GEMMs
   bool stack = false;      // workspace also holds the normalised activations
   bool fp8 = false;        // E4M3 expert weights with row scales (small batch only)
+  // failure-path test hook (moe_debug_forward_withheld only): the one-CTA G13 kernel issues
+  // no loads and its pipeline waits give up after g13_wait_limit cycles
+  bool g13_withhold = false;
+  long long g13_wait_limit = 0;
   // workspace byte offsets
   size_t o_rpart;          // small batch: partial router logits [ceil(d/64)][T][n]
   size_t o_rowtok;         // token of each permuted row [rows_max] (small batch, gather_x)

@@ -188,7 +188,7 @@ using namespace moe;
 
 extern "C" {
 
-int moe_abi_version(void) { return 1; }
+int moe_abi_version(void) { return 2; }
 
 const char* moe_status_string(moe_status s) {
   switch (s) {
@@ -227,9 +227,11 @@ moe_status moe_workspace_status(void* workspace, void* stream, uint32_t* raw) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t bits = 0;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaMemcpy(&bits, workspace, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaMemcpyAsync(&bits, workspace, sizeof bits, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (cudaMemset(workspace, 0, sizeof bits) != cudaSuccess) return MOE_ERR_CUDA;
+  // cleared on the same stream, so the next call enqueued there sees zero
+  if (bits && cudaMemsetAsync(workspace, 0, sizeof bits, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (raw) *raw = bits;
   if (bits & DEV_ERR_TIMEOUT) return MOE_ERR_TIMEOUT;
   if (bits) return MOE_ERR_DEVICE;
@@ -385,6 +387,36 @@ moe_status moe_forward_host_io(const void* x_host, void* x_dev, const float* W_g
   return MOE_OK;
 }
 
+// Validation shared by the stack entry points (bf16 only; x is updated in place).
+static moe_status stack_check(const Plan& p, const void* x, const float* const* W_g,
+                              const void* const* W1, const void* const* W3,
+                              const void* const* W2, int L, float eps, size_t workspace_bytes,
+                              const void* workspace) {
+  if (L < 0 || !W_g || !W1 || !W3 || !W2 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (p.T == 0 || L == 0) return MOE_OK;
+  for (int l = 0; l < L; ++l) {
+    moe_status st = check_common(x, W_g[l], W1[l], W3[l], W2[l], x, workspace);
+    if (st != MOE_OK) return st;
+  }
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// L blocks in place on x; ev (may be null): 6 events per block, as moe_forward_profiled.
+static moe_status stack_impl(const Plan& p, void* x, const float* const* W_g,
+                             const void* const* W1, const void* const* W3,
+                             const void* const* W2, int L, float eps, void* workspace,
+                             cudaStream_t s, cudaEvent_t const* ev) {
+  const Workspace w = carve(p, workspace);
+  for (int l = 0; l < L; ++l) {
+    if (launch_rmsnorm(x, w.xn, p.T, p.d, eps, s) != cudaSuccess) return MOE_ERR_CUDA;
+    moe_status st = forward_impl(p, w.xn, W_g[l], W1[l], W3[l], W2[l], x, x, w, s,
+                                 ev ? ev + 6 * (size_t)l : nullptr);
+    if (st != MOE_OK) return st;
+  }
+  return MOE_OK;
+}
+
 moe_status moe_stack_forward(void* x, const float* const* W_g, const void* const* W1,
                              const void* const* W3, const void* const* W2, int L, int64_t T,
                              int64_t d, int64_t F, int n, int K, moe_dtype dt, float eps,
@@ -392,21 +424,73 @@ moe_status moe_stack_forward(void* x, const float* const* W_g, const void* const
   if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   Plan p;
   if (!make_plan(T, d, F, n, K, (int)dt, true, &p)) return shape_status(T, d, F, n, K, dt);
-  if (L < 0 || !W_g || !W1 || !W3 || !W2 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
-  if (T == 0 || L == 0) return MOE_OK;
-  for (int l = 0; l < L; ++l) {
-    moe_status st = check_common(x, W_g[l], W1[l], W3[l], W2[l], x, workspace);
-    if (st != MOE_OK) return st;
-  }
-  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  moe_status st = stack_check(p, x, W_g, W1, W3, W2, L, eps, workspace_bytes, workspace);
+  if (st != MOE_OK || T == 0 || L == 0) return st;
+  return stack_impl(p, x, W_g, W1, W3, W2, L, eps, workspace,
+                    static_cast<cudaStream_t>(stream), nullptr);
+}
+
+moe_status moe_stack_forward_profiled(void* x, const float* const* W_g, const void* const* W1,
+                                      const void* const* W3, const void* const* W2, int L,
+                                      int64_t T, int64_t d, int64_t F, int n, int K,
+                                      moe_dtype dt, float eps, void* workspace,
+                                      size_t workspace_bytes, void* stream,
+                                      void* const* events, int n_events) {
+  if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, true, &p)) return shape_status(T, d, F, n, K, dt);
+  if (L < 0 || n_events != 6 * L || (L > 0 && !events)) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_events; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARG;
+  moe_status st = stack_check(p, x, W_g, W1, W3, W2, L, eps, workspace_bytes, workspace);
+  if (st != MOE_OK || T == 0 || L == 0) return st;
+  return stack_impl(p, x, W_g, W1, W3, W2, L, eps, workspace,
+                    static_cast<cudaStream_t>(stream),
+                    reinterpret_cast<cudaEvent_t const*>(events));
+}
+
+moe_status moe_stack_forward_host_io(const void* x_host, void* x_dev, const float* const* W_g,
+                                     const void* const* W1, const void* const* W3,
+                                     const void* const* W2, int L, int64_t T, int64_t d,
+                                     int64_t F, int n, int K, moe_dtype dt, float eps,
+                                     void* out_host, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (dt != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, true, &p)) return shape_status(T, d, F, n, K, dt);
+  if (T > 0 && (!x_host || !out_host)) return MOE_ERR_INVALID_ARG;
+  moe_status st = stack_check(p, x_dev, W_g, W1, W3, W2, L, eps, workspace_bytes, workspace);
+  if (st != MOE_OK || T == 0) return st;
+  if (!x_dev) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const Workspace w = carve(p, workspace);
-  for (int l = 0; l < L; ++l) {
-    if (launch_rmsnorm(x, w.xn, T, d, eps, s) != cudaSuccess) return MOE_ERR_CUDA;
-    moe_status st = forward_impl(p, w.xn, W_g[l], W1[l], W3[l], W2[l], x, x, w, s);
-    if (st != MOE_OK) return st;
-  }
+  const size_t bytes = (size_t)T * d * 2;
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = stack_impl(p, x_dev, W_g, W1, W3, W2, L, eps, workspace, s, nullptr);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(out_host, x_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+moe_status moe_debug_forward_withheld(const void* x, const float* W_g, const void* W1,
+                                      const void* W3, const void* W2, int64_t T, int64_t d,
+                                      int64_t F, int n, int K, moe_dtype dt, void* out,
+                                      void* workspace, size_t workspace_bytes, void* stream,
+                                      int64_t wait_limit_cycles) {
+  Plan p;
+  if (!make_plan(T, d, F, n, K, (int)dt, false, &p)) return shape_status(T, d, F, n, K, dt);
+  if (wait_limit_cycles < 1 || wait_limit_cycles > WAIT_LIMIT_CYCLES) return MOE_ERR_INVALID_ARG;
+  if (p.dt != 1 || p.pair) return MOE_ERR_UNSUPPORTED;  // the one-CTA tensor-core kernel only
+  if (T == 0) return MOE_OK;
+  moe_status st = check_common(x, W_g, W1, W3, W2, out, workspace);
+  if (st != MOE_OK) return st;
+  if (out == x) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  p.g13_withhold = true;
+  p.g13_wait_limit = wait_limit_cycles;
+  const Workspace w = carve(p, workspace);
+  return forward_impl(p, x, W_g, W1, W3, W2, out, nullptr, w, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -64,6 +64,18 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_info.argtypes = [I64, I64, I64, I32, I32, I32, IP, IP, IP, IP, IP]
         L.moe_forward_noalloc.restype = I32
         L.moe_forward_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P, P]
+        L.moe_noalloc_status.restype = I32
+        L.moe_noalloc_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+        L.moe_stack_forward_profiled.restype = I32
+        L.moe_stack_forward_profiled.argtypes = [P, P, P, P, P, I32, I64, I64, I64, I32, I32,
+                                                 I32, ctypes.c_float, P, SZ, P,
+                                                 ctypes.POINTER(P), I32]
+        L.moe_stack_forward_host_io.restype = I32
+        L.moe_stack_forward_host_io.argtypes = [P, P, P, P, P, P, I32, I64, I64, I64, I32, I32,
+                                                I32, ctypes.c_float, P, P, SZ, P]
+        L.moe_debug_forward_withheld.restype = I32
+        L.moe_debug_forward_withheld.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P,
+                                                 P, SZ, P, I64]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [I32]
         L.moe_abi_version.restype = I32
@@ -220,24 +232,78 @@ def moe_forward_host_io(x_host, x_dev, W_g, W1, W3, W2, K: int, out_dev, out_hos
     return out_host
 
 
-def moe_stack_forward(x, layers, K: int, eps: float = 1e-5, workspace=None, stream=None):
-    """In place on x: for each layer dict (W_g, W1, W3, W2), x <- x + MoE(RMSNorm(x))."""
-    L = len(layers)
+def _layer_ptrs(layers):
+    arr = ctypes.c_void_p * max(len(layers), 1)
+    return tuple(arr(*[l[k].data_ptr() for l in layers]) for k in ("Wg", "W1", "W3", "W2"))
+
+
+def _stack_ws(x, layers, K, workspace, stream):
     T, d = x.shape
     n, F, _ = layers[0]["W1"].shape
-    dt = _dt(x)
     if workspace is None:
-        workspace = alloc_workspace(moe_stack_workspace_bytes(T, d, F, n, K, dt), x.device,
+        workspace = alloc_workspace(moe_stack_workspace_bytes(T, d, F, n, K, _dt(x)), x.device,
                                     stream)
-    arr = ctypes.c_void_p * max(L, 1)
-    pg = arr(*[l["Wg"].data_ptr() for l in layers])
-    p1 = arr(*[l["W1"].data_ptr() for l in layers])
-    p3 = arr(*[l["W3"].data_ptr() for l in layers])
-    p2 = arr(*[l["W2"].data_ptr() for l in layers])
+    return T, d, F, n, workspace
+
+
+def moe_stack_forward(x, layers, K: int, eps: float = 1e-5, workspace=None, stream=None):
+    """In place on x: for each layer dict (W_g, W1, W3, W2), x <- x + MoE(RMSNorm(x))."""
+    T, d, F, n, workspace = _stack_ws(x, layers, K, workspace, stream)
+    pg, p1, p3, p2 = _layer_ptrs(layers)
     _check("moe_stack_forward", lib().moe_stack_forward(
-        _ptr(x), pg, p1, p3, p2, L, T, d, F, n, K, dt, float(eps), _ptr(workspace),
-        workspace.numel(), _stream(stream)))
+        _ptr(x), pg, p1, p3, p2, len(layers), T, d, F, n, K, _dt(x), float(eps),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
     return x
+
+
+def moe_stack_forward_profiled(x, layers, K: int, events, eps: float = 1e-5, workspace=None,
+                               stream=None):
+    """moe_stack_forward recording six torch.cuda.Event per block (a list of 6*L events, each
+    recorded once beforehand so that it exists) at the stage boundaries."""
+    T, d, F, n, workspace = _stack_ws(x, layers, K, workspace, stream)
+    pg, p1, p3, p2 = _layer_ptrs(layers)
+    handles = (ctypes.c_void_p * max(len(events), 1))(
+        *[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check("moe_stack_forward_profiled", lib().moe_stack_forward_profiled(
+        _ptr(x), pg, p1, p3, p2, len(layers), T, d, F, n, K, _dt(x), float(eps),
+        _ptr(workspace), workspace.numel(), _stream(stream), handles, len(events)))
+    return x
+
+
+def moe_stack_forward_host_io(x_host, x_dev, layers, K: int, out_host, eps: float = 1e-5,
+                              workspace=None, stream=None):
+    """Host x in, host out: H2D copy into x_dev, the L blocks in place on x_dev, D2H copy to
+    out_host, all enqueued on the stream (synchronise before reading out_host)."""
+    T, d, F, n, workspace = _stack_ws(x_dev, layers, K, workspace, stream)
+    pg, p1, p3, p2 = _layer_ptrs(layers)
+    _check("moe_stack_forward_host_io", lib().moe_stack_forward_host_io(
+        _ptr(x_host), _ptr(x_dev), pg, p1, p3, p2, len(layers), T, d, F, n, K, _dt(x_dev),
+        float(eps), _ptr(out_host), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out_host
+
+
+def moe_noalloc_status(stream=None) -> tuple[int, int]:
+    """Status code and raw bits of the array moe_forward_noalloc uses (read and cleared)."""
+    raw = ctypes.c_uint32(0)
+    code = lib().moe_noalloc_status(_stream(stream), ctypes.byref(raw))
+    return code, raw.value
+
+
+def moe_debug_forward_withheld(x, W_g, W1, W3, W2, K: int, wait_limit_cycles: int, out=None,
+                               workspace=None, stream=None):
+    """Failure-path test hook: the block with the gate/up kernel's loads withheld so that its
+    pipeline wait runs out after wait_limit_cycles (see include/moe.h).  Returns out (its
+    values are undefined)."""
+    T, d, F, n = _dims(x, W1, W_g)
+    dt = _dt(x)
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = alloc_workspace(moe_workspace_bytes(T, d, F, n, K, dt), x.device, stream)
+    _check("moe_debug_forward_withheld", lib().moe_debug_forward_withheld(
+        _ptr(x), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt, _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream(stream), int(wait_limit_cycles)))
+    return out
 
 
 # ------------------------------------------------------------------ FP8 (E4M3) expert weights

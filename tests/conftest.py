@@ -30,3 +30,21 @@ def oracle_lib():
         import oracle as mod
     mod.build()
     return mod
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print the parity reports the GPU tests recorded: tokens compared, near-tie tokens
+    exempted from the routing check, max-abs and relative L2 error against the oracle."""
+    try:
+        from tests import parity
+    except ImportError:  # pragma: no cover
+        return
+    if not parity.REPORTS:
+        return
+    tr = terminalreporter
+    tr.write_line("parity against the oracle (tokens compared, exempt near-ties, max-abs, "
+                  "rel-L2):")
+    for name, r in parity.REPORTS:
+        tr.write_line(f"  {name}: tokens={r.get('tokens')} exempt={r.get('exempt')} "
+                      f"max_abs={r.get('max_abs', float('nan')):.3g} "
+                      f"rel_l2={r.get('rel_l2', float('nan')):.3g} ok={r.get('ok')}")

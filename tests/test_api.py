@@ -32,7 +32,9 @@ def test_header_declares_entry_points():
     names = _declared()
     for want in ("moe_forward", "moe_forward_debug", "moe_workspace_bytes", "moe_stack_forward",
                  "moe_status_string", "moe_forward_host_io", "moe_workspace_init",
-                 "moe_workspace_status", "moe_forward_profiled", "moe_plan_info"):
+                 "moe_workspace_status", "moe_forward_profiled", "moe_plan_info",
+                 "moe_stack_forward_profiled", "moe_stack_forward_host_io",
+                 "moe_debug_forward_withheld", "moe_forward_noalloc", "moe_noalloc_status"):
         assert want in names
 
 
@@ -134,6 +136,38 @@ def test_stack_validation(L):
                                ctypes.c_float(1e-5), P(0x10000), 1 << 40, None) == INVALID
     assert L.moe_stack_forward(P(0x1000), arr, arr, arr, arr, 2, 16, 256, 256, 8, 2, BF16,
                                ctypes.c_float(1e-5), P(0x10000), 1024, None) == WORKSPACE
+
+
+def test_stack_profiled_and_host_io_validation(L):
+    arr = (P * 2)(P(0x3000), P(0x3000))
+    evs = (P * 12)(*([P(0x1)] * 12))
+    prof = L.moe_stack_forward_profiled
+    args = (P(0x1000), arr, arr, arr, arr, 2, 16, 256, 256, 8, 2, BF16, ctypes.c_float(1e-5),
+            P(0x10000), 1 << 40, None)
+    assert prof(*args, evs, 11) == INVALID                   # six events per block
+    assert prof(*args, None, 12) == INVALID
+    assert prof(*args[:11], F32, *args[12:], evs, 12) == UNSUPPORTED
+    assert prof(P(0x1000), arr, arr, arr, arr, 2, 16, 256, 256, 8, 2, BF16,
+                ctypes.c_float(1e-5), P(0x10000), 1024, None, evs, 12) == WORKSPACE
+    hio = L.moe_stack_forward_host_io
+    assert hio(None, P(0x1000), arr, arr, arr, arr, 2, 16, 256, 256, 8, 2, BF16,
+               ctypes.c_float(1e-5), P(0x7000), P(0x10000), 1 << 40, None) == INVALID
+    assert hio(P(0x8000), P(0x1000), arr, arr, arr, arr, 2, 16, 256, 256, 8, 2, BF16,
+               ctypes.c_float(1e-5), None, P(0x10000), 1 << 40, None) == INVALID
+    assert hio(P(0x8000), P(0x1000), arr, arr, arr, arr, 2, 16, 256, 256, 8, 2, F32,
+               ctypes.c_float(1e-5), P(0x7000), P(0x10000), 1 << 40, None) == UNSUPPORTED
+
+
+def test_withheld_hook_validation(L):
+    def call(T=16, d=256, F=256, dt=BF16, limit=1000):
+        return L.moe_debug_forward_withheld(P(0x1000), P(0x2000), P(0x3000), P(0x4000),
+                                            P(0x5000), T, d, F, 8, 2, dt, P(0x6000),
+                                            P(0x10000), 1 << 40, None, limit)
+    assert call(limit=0) == INVALID and call(limit=-5) == INVALID
+    assert call(limit=5_000_000_000) == INVALID              # above the kernels' own limit
+    assert call(dt=F32) == UNSUPPORTED                       # the fp32 kernel has no pipeline
+    assert call(T=4096) == UNSUPPORTED                       # CTA-pair tiling
+    assert call(T=0) == OK
 
 
 def test_host_io_validation(L):
