@@ -232,6 +232,60 @@ MOE_API moe_status moe_stack_forward_host_io(const void* x_host, void* x_dev,
                                              void* workspace, size_t workspace_bytes,
                                              void* stream);
 
+/* ---- Expert parallelism: the block's stages as separate calls, so that the experts can be
+ * spread over GPUs with an exchange between them ("Mixtral 8x7B: Model Bahasa Sparse Mixture
+ * of Experts", id.news.hada.io, section "Implementasi dan Efisiensi Inferensi": tokens are
+ * sent to the GPU that holds their expert and the expert outputs return to the tokens'
+ * original positions).  The exchanges themselves are the caller's (e.g. NCCL all-to-alls);
+ * moe_route -> [dispatch] -> moe_experts_forward -> [return] -> moe_combine on one GPU gives
+ * moe_forward's result within rounding.
+ *
+ * Workspace bytes of moe_route (0 if unsupported). */
+MOE_API size_t moe_route_workspace_bytes(int64_t T, int64_t d, int n, int K, moe_dtype dt);
+
+/* The router, TopK and softmax of every token (method section, equation G(x)) and the
+ * grouping of the T*K (token, slot) rows by expert, unpadded and stable (by token, then
+ * slot): expert e's rows are x_grouped[o_e .. o_e + expert_counts[e]), o_e = sum of the
+ * counts of the experts before e.
+ *   x [T][d] dt, W_g [d][n] fp32            inputs (x 16-byte aligned)
+ *   x_grouped [T*K][d] dt                   the token rows in grouped order (must not alias x)
+ *   topk_idx, token_rows [T][K] int32       selected experts; row of each (token, slot)
+ *   topk_gate [T][K] fp32                   G(x) over the kept experts
+ *   expert_counts [n] int32
+ * Requirements as moe_forward (d a multiple of 64 for bf16, 8 for fp32). */
+MOE_API moe_status moe_route(const void* x, const float* W_g, int64_t T, int64_t d, int n,
+                             int K, moe_dtype dt, void* x_grouped, int32_t* topk_idx,
+                             float* topk_gate, int32_t* expert_counts, int32_t* token_rows,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of moe_experts_forward for `rows` received rows (0 if unsupported). */
+MOE_API size_t moe_experts_workspace_bytes(int64_t rows, int64_t d, int64_t F, int n_local,
+                                           moe_dtype dt);
+
+/* The SwiGLU experts (method section, equation y; W2 . (silu(W1 . x) * (W3 . x))) of one
+ * GPU's n_local experts on rows received from S sources:
+ *   x_rows [rows][d] dt         S segments in source order; segment s holds seg_counts[s][e]
+ *                               rows for local expert e = 0 .. n_local-1, in expert order
+ *   seg_counts [S][n_local]     int32, device (S * n_local <= 2048; they must add up to rows,
+ *                               else bit 2 of the status word is set and nothing is computed)
+ *   W1, W3 [n_local][F][d], W2 [n_local][d][F] dt   the local experts' weights
+ *   y_rows [rows][d] fp32       y_rows[r] = SwiGLU_e(x_rows[r]), same row order, no gate
+ * The rows are regrouped on the device into the padded per-expert layout of the grouped
+ * GEMMs (the same kernels and tilings as moe_forward for `rows` rows over n_local experts). */
+MOE_API moe_status moe_experts_forward(const void* x_rows, int64_t rows,
+                                       const int32_t* seg_counts, int S, const void* W1,
+                                       const void* W3, const void* W2, int64_t d, int64_t F,
+                                       int n_local, moe_dtype dt, float* y_rows, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/* The gate-weighted combine back to token order (method section, equation y):
+ *   out[t] = sum_k topk_gate[t][k] * y_rows[token_rows[t][k]]
+ * summed in fp32 in slot order and rounded once to dt (out [T][d], 16-byte aligned; y_rows
+ * fp32, 16-byte aligned; d a multiple of 4).  No workspace. */
+MOE_API moe_status moe_combine(const float* y_rows, const int32_t* token_rows,
+                               const float* topk_gate, int64_t T, int64_t d, int K, moe_dtype dt,
+                               void* out, void* stream);
+
 /* Test hook for the failure path (no counterpart in the pages): moe_forward, except that the
  * one-CTA tensor-core kernel of the gate/up projection issues none of its loads, so its
  * tensor-core thread waits on a barrier that nothing will complete; that wait, and the other

@@ -194,6 +194,47 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// out[t] = (resid[t] +) sum_k gate[t][k] * sum_s Y[s][inv[t][k]] for T tokens, Tout = bf16
+// or fp32 (gate null: 1), picking the one-warp-per-token kernel for T >= 1024.
+template <typename Tout>
+static cudaError_t combine_rows_t(const float* Y, int S, int64_t split_stride, int64_t T, int d,
+                                  int K, const int32_t* inv, const float* gate, Tout* out,
+                                  const Tout* resid, cudaStream_t s) {
+  if (T >= 1024) {  // enough tokens for one warp each
+    const int64_t blocks = (T + 7) / 8;
+    const unsigned g = (unsigned)(blocks < ((int64_t)1 << 30) ? blocks : ((int64_t)1 << 30));
+    if (resid)
+      pdl(combine_rows_kernel<Tout, true>, g, 256, 0, s)(Y, S, split_stride, T, d, K, inv, gate,
+                                                         out, resid);
+    else
+      pdl(combine_rows_kernel<Tout, false>, g, 256, 0, s)(Y, S, split_stride, T, d, K, inv,
+                                                          gate, out, nullptr);
+    return cudaGetLastError();
+  }
+  const int64_t total = T * (d / 4);
+  int64_t blocks = (total + 255) / 256;  // one 4-column item per thread: all loads in flight
+  if (blocks > ((int64_t)1 << 30)) blocks = (int64_t)1 << 30;
+  if (blocks < 1) blocks = 1;
+  if (resid)
+    pdl(combine_kernel<Tout, true>, (unsigned)blocks, 256, 0, s)(
+        Y, S, split_stride, T, d, K, inv, gate, out, resid, nullptr, nullptr, nullptr);
+  else
+    pdl(combine_kernel<Tout, false>, (unsigned)blocks, 256, 0, s)(
+        Y, S, split_stride, T, d, K, inv, gate, out, nullptr, nullptr, nullptr, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_rows(const float* Y, int S, int64_t split_stride, int64_t T, int d,
+                                int K, const int32_t* inv, const float* gate, void* out,
+                                const void* resid, bool out_f32, cudaStream_t s) {
+  if (out_f32)
+    return combine_rows_t(Y, S, split_stride, T, d, K, inv, gate, static_cast<float*>(out),
+                          static_cast<const float*>(resid), s);
+  return combine_rows_t(Y, S, split_stride, T, d, K, inv, gate,
+                        static_cast<__nv_bfloat16*>(out),
+                        static_cast<const __nv_bfloat16*>(resid), s);
+}
+
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
                            cudaStream_t s, const float* s2) {
   const int S = p.swap ? p.s2 : 1;
@@ -208,57 +249,8 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
         static_cast<__nv_bfloat16*>(out), nullptr, w.sh, s2, w.idx);
     return cudaGetLastError();
   }
-  if (p.T >= 1024) {  // enough tokens for one warp each
-    const int64_t blocks = (p.T + 7) / 8;
-    const unsigned g = (unsigned)(blocks < ((int64_t)1 << 30) ? blocks : ((int64_t)1 << 30));
-    if (p.dt == 1) {
-      auto* o = static_cast<__nv_bfloat16*>(out);
-      if (resid)
-        pdl(combine_rows_kernel<__nv_bfloat16, true>, g, 256, 0, s)(
-            w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o,
-            static_cast<const __nv_bfloat16*>(resid));
-      else
-        pdl(combine_rows_kernel<__nv_bfloat16, false>, g, 256, 0, s)(
-            w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr);
-    } else {
-      auto* o = static_cast<float*>(out);
-      if (resid)
-        pdl(combine_rows_kernel<float, true>, g, 256, 0, s)(w.y, S, split_stride, p.T, (int)p.d,
-                                                           p.K, w.inv, gates, o,
-                                                           static_cast<const float*>(resid));
-      else
-        pdl(combine_rows_kernel<float, false>, g, 256, 0, s)(w.y, S, split_stride, p.T,
-                                                            (int)p.d, p.K, w.inv, gates, o,
-                                                            nullptr);
-    }
-    return cudaGetLastError();
-  }
-  const int64_t total = p.T * (p.d / 4);
-  int64_t blocks = (total + 255) / 256;  // one 4-column item per thread: all loads in flight
-  if (blocks > ((int64_t)1 << 30)) blocks = (int64_t)1 << 30;
-  if (blocks < 1) blocks = 1;
-  if (p.dt == 1) {
-    auto* o = static_cast<__nv_bfloat16*>(out);
-    if (resid)
-      pdl(combine_kernel<__nv_bfloat16, true>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o,
-          static_cast<const __nv_bfloat16*>(resid), nullptr, nullptr, nullptr);
-    else
-      pdl(combine_kernel<__nv_bfloat16, false>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr, nullptr, nullptr,
-          nullptr);
-  } else {
-    auto* o = static_cast<float*>(out);
-    if (resid)
-      pdl(combine_kernel<float, true>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o,
-          static_cast<const float*>(resid), nullptr, nullptr, nullptr);
-    else
-      pdl(combine_kernel<float, false>, (unsigned)blocks, 256, 0, s)(
-          w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, o, nullptr, nullptr, nullptr,
-          nullptr);
-  }
-  return cudaGetLastError();
+  return launch_combine_rows(w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, out, resid,
+                             p.dt == 0, s);
 }
 
 // One warp per row: sum of squares in fp32 (lane-strided 8-element chunks, then a shuffle

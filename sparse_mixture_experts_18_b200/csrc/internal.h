@@ -98,8 +98,10 @@ PdlLaunch<KArgs...> pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
   return PdlLaunch<KArgs...>{kern, grid, block, smem, s};
 }
 
+// route_only: the plan of moe_route (routing and unpadded grouping into a caller buffer; no
+// expert stages, F unused).
 bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p,
-               bool fp8 = false);
+               bool fp8 = false, bool route_only = false);
 Workspace carve(const Plan& p, void* base);
 
 int route_tokens_per_block(int K);
@@ -124,6 +126,17 @@ cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float
 // fp8 (p.fp8): s2 [n][d] are the W2 row scales; expert outputs are scaled by s_h[row] s2[e][i]
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
                            cudaStream_t s, const float* s2 = nullptr);
+// out[t] = (resid[t] +) sum_k gate[t][k] * sum_{s < S} Y[s * split_stride + inv[t][k] row]
+// (gate null: weight 1), fp32 sums in split then slot order, rounded once to bf16, or kept
+// fp32 (out_f32).
+cudaError_t launch_combine_rows(const float* Y, int S, int64_t split_stride, int64_t T, int d,
+                                int K, const int32_t* inv, const float* gate, void* out,
+                                const void* resid, bool out_f32, cudaStream_t s);
+// Expert-parallel local stage: rows received from S sources, each source's rows grouped by
+// the nl local experts (seg_counts [S][nl] on the device), are placed in the padded
+// per-expert layout of the plan (X_perm, counts, offsets, inv = padded row of each row).
+cudaError_t launch_ep_regroup(const Plan& p, const void* x_rows, const int32_t* seg_counts,
+                              int S, const Workspace& w, cudaStream_t s);
 cudaError_t launch_rmsnorm(const void* x, void* xn, int64_t T, int64_t d, float eps,
                            cudaStream_t s);
 int num_sms();

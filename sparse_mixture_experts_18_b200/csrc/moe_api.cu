@@ -53,7 +53,7 @@ static bool gather_x_requested() {
 }
 
 bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack, Plan* p,
-               bool fp8) {
+               bool fp8, bool route_only) {
   if (T < 0 || d <= 0 || F <= 0 || n < 1 || n > MAX_EXPERTS || K < 1 || K > n) return false;
   if (fp8 && (dt != 1 || stack || d % 128 || F % 128)) return false;
   if (dt == 1) {
@@ -71,6 +71,10 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   q.pair = dt == 1 && !q.swap && T * K >= 640 * (int64_t)n;
   q.row_align = dt == 0 ? SIMT_TILE : (q.swap ? 1 : TILE_M);
   q.gather_x = q.pair && gather_x_requested();
+  if (route_only) {  // experts' rows contiguous and unpadded, in the caller's buffer
+    q.swap = q.pair = q.gather_x = false;
+    q.row_align = 1;
+  }
   const int64_t P = T * K;
   q.rows_max = (P + (int64_t)n * (q.row_align - 1) + q.row_align - 1) / q.row_align * q.row_align;
   if (q.swap) q.rows_max = (P + 15) / 16 * 16;  // >= tok_tile rows for the token TMA box
@@ -82,6 +86,7 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   q.fp8 = fp8;
   if (fp8 && !(q.swap && q.fused_route)) return false;
   q.gather_small = q.swap && q.fused_route && dt == 1;  // (FP8: from the quantised rows)
+  if (route_only) q.rows_max = P;
   const int kbw = fp8 ? 128 : 64;  // elements per 128-byte K block
   if (q.swap) {
     q.tok_tile = (int)((T + 15) / 16 * 16);
@@ -100,9 +105,9 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   q.o_counts = take((size_t)n * 4);
   q.o_offsets = take((size_t)(n + 1) * 4);
   q.o_inv = take((size_t)P * 4);
-  q.o_xperm = take((size_t)q.rows_max * d * es);
-  q.o_h = take((size_t)q.rows_max * F * es);
-  q.o_y = take((size_t)(q.swap ? q.s2 : 1) * q.rows_max * d * 4);
+  q.o_xperm = take(route_only ? 0 : (size_t)q.rows_max * d * es);
+  q.o_h = take(route_only ? 0 : (size_t)q.rows_max * F * es);
+  q.o_y = take(route_only ? 0 : (size_t)(q.swap ? q.s2 : 1) * q.rows_max * d * 4);
   q.o_p13 = take(q.swap ? (size_t)q.s13 * q.rows_max * 2 * F * 4 : 0);
   q.o_xn = take(stack ? (size_t)T * d * es : 0);
   q.o_rpart = take(q.fused_route ? (size_t)((d + 63) / 64) * T * n * 4 : 0);
@@ -471,6 +476,96 @@ moe_status moe_stack_forward_host_io(const void* x_host, void* x_dev, const floa
   if (cudaMemcpyAsync(out_host, x_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+// ---------------------------------------------------------------- expert parallelism
+size_t moe_route_workspace_bytes(int64_t T, int64_t d, int n, int K, moe_dtype dt) {
+  Plan p;
+  if (!make_plan(T, d, 64, n, K, (int)dt, false, &p, false, true)) return 0;
+  return p.total;
+}
+
+moe_status moe_route(const void* x, const float* W_g, int64_t T, int64_t d, int n, int K,
+                     moe_dtype dt, void* x_grouped, int32_t* topk_idx, float* topk_gate,
+                     int32_t* expert_counts, int32_t* token_rows, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  Plan p;
+  if (!make_plan(T, d, 64, n, K, (int)dt, false, &p, false, true))
+    return shape_status(T, d, 64, n, K, dt);
+  if (T == 0) return MOE_OK;
+  if (!x || !W_g || !x_grouped || !topk_idx || !topk_gate || !expert_counts || !token_rows ||
+      !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(W_g, 16) || !aligned(x_grouped, 16) || !aligned(workspace, 256) ||
+      !aligned(topk_idx, 4) || !aligned(topk_gate, 4) || !aligned(expert_counts, 4) ||
+      !aligned(token_rows, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (x_grouped == x) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  Workspace w = carve(p, workspace);
+  w.idx = topk_idx;
+  w.gate = topk_gate;
+  w.counts = expert_counts;
+  w.inv = token_rows;
+  w.xperm = x_grouped;
+  return launch_route(p, x, W_g, w, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+size_t moe_experts_workspace_bytes(int64_t rows, int64_t d, int64_t F, int n_local,
+                                   moe_dtype dt) {
+  Plan p;
+  if (!make_plan(rows, d, F, n_local, 1, (int)dt, false, &p)) return 0;
+  return p.total;
+}
+
+moe_status moe_experts_forward(const void* x_rows, int64_t rows, const int32_t* seg_counts,
+                               int S, const void* W1, const void* W3, const void* W2, int64_t d,
+                               int64_t F, int n_local, moe_dtype dt, float* y_rows,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  Plan p;
+  if (!make_plan(rows, d, F, n_local, 1, (int)dt, false, &p))
+    return shape_status(rows, d, F, n_local, 1, dt);
+  if (S < 1 || (int64_t)S * n_local > 2048) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!x_rows || !seg_counts || !W1 || !W3 || !W2 || !y_rows || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x_rows, 16) || !aligned(W1, 16) || !aligned(W3, 16) || !aligned(W2, 16) ||
+      !aligned(y_rows, 16) || !aligned(workspace, 256) || !aligned(seg_counts, 4))
+    return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
+  p.gather_small = false;  // the rows are regrouped into X_perm below
+  p.gather_x = false;
+  const Workspace w = carve(p, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_ep_regroup(p, x_rows, seg_counts, S, w, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaError_t err =
+      p.dt == 1 ? launch_expert_gemms_tc(p, x_rows, W1, W3, W2, w, s)
+                : launch_expert_gemms_simt(p, static_cast<const float*>(W1),
+                                           static_cast<const float*>(W3),
+                                           static_cast<const float*>(W2), w, s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  // back to the received order, splits summed, kept in fp32 (no gate: the sender applies it)
+  if (launch_combine_rows(w.y, p.swap ? p.s2 : 1, p.rows_max * d, rows, (int)d, 1, w.inv,
+                          nullptr, y_rows, nullptr, true, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_combine(const float* y_rows, const int32_t* token_rows, const float* topk_gate,
+                       int64_t T, int64_t d, int K, moe_dtype dt, void* out, void* stream) {
+  if (T < 0 || d <= 0 || K < 1 || K > MAX_EXPERTS || (dt != MOE_F32 && dt != MOE_BF16))
+    return MOE_ERR_INVALID_ARG;
+  if (d % 4 || d > (1 << 20)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!y_rows || !token_rows || !topk_gate || !out || !aligned(y_rows, 16) || !aligned(out, 16) ||
+      !aligned(token_rows, 4) || !aligned(topk_gate, 4))
+    return MOE_ERR_INVALID_ARG;
+  return launch_combine_rows(y_rows, 1, 0, T, (int)d, K, token_rows, topk_gate, out, nullptr,
+                             dt == MOE_F32, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 moe_status moe_debug_forward_withheld(const void* x, const float* W_g, const void* W1,

@@ -48,18 +48,6 @@ struct Vec8<float> {
   }
 };
 
-// Synchronisation of the threads that route one token block: the whole CTA, or one
-// 256-thread group of a larger CTA (named barrier 1 + group).
-struct CtaSync {
-  __device__ __forceinline__ void operator()() const { __syncthreads(); }
-};
-struct GroupSync {
-  int id;
-  __device__ __forceinline__ void operator()() const {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(ROUTE_THREADS) : "memory");
-  }
-};
-
 // Shared-memory copy of W_g for the persistent router: row j (n floats) starts at
 // j*n + 4*(j/8).  The skew of four floats per eight rows spreads the rows that the lanes of a
 // warp read together (eight rows apart) over all banks.
@@ -74,13 +62,16 @@ __host__ __device__ __forceinline__ size_t wg_smem_bytes(int d, int n) {
 // dimension (so each W_g row segment is loaded once per RT_TOK tokens); lanes and then warps
 // are summed in a fixed order.  hist (shared, may be null) counts selections.
 constexpr int RT_TOK = 8;
+// W_g bytes up to which the large-batch router keeps it in shared memory (the rest of its
+// 227 KB holds the per-team sums and logits)
+constexpr int RT_SMEM_MAX = 176 * 1024;
 
-// W_SMEM: Wg is a shared-memory copy in the skewed layout of wg_smem_index (and w_vec holds).
-template <typename Tin, bool W_SMEM, typename Sync>
+// w_vec: W_g rows are 16-byte aligned and n % 8 == 0 (eight experts per two float4 loads).
+template <typename Tin>
 __device__ __forceinline__ void route_token_block(
     const Tin* __restrict__ x, const float* __restrict__ Wg, bool w_vec, int64_t t0, int ntok,
     int d, int n, int K, int tid, float (*red)[64], float (*logits)[MAX_EXPERTS], int* hist,
-    int32_t* __restrict__ idx, float* __restrict__ gate, Sync sync) {
+    int32_t* __restrict__ idx, float* __restrict__ gate) {
   const int warp = tid >> 5, lane = tid & 31;
   for (int eg = 0; eg < n; eg += 8) {
     float acc[RT_TOK][8];
@@ -99,17 +90,10 @@ __device__ __forceinline__ void route_token_block(
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float w[8];
-        if (W_SMEM || w_vec) {  // eight experts of one row: two aligned float4 loads
-          float4 w0, w1;
-          if (W_SMEM) {
-            const float* wr = Wg + wg_smem_index(j0 + i, n) + eg;
-            w0 = *reinterpret_cast<const float4*>(wr);
-            w1 = *reinterpret_cast<const float4*>(wr + 4);
-          } else {
-            const float* wr = Wg + (int64_t)(j0 + i) * n + eg;
-            w0 = __ldg(reinterpret_cast<const float4*>(wr));
-            w1 = __ldg(reinterpret_cast<const float4*>(wr) + 1);
-          }
+        if (w_vec) {  // eight experts of one row: two aligned float4 loads
+          const float* wr = Wg + (int64_t)(j0 + i) * n + eg;
+          const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr));
+          const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr) + 1);
           w[0] = w0.x; w[1] = w0.y; w[2] = w0.z; w[3] = w0.w;
           w[4] = w1.x; w[5] = w1.y; w[6] = w1.z; w[7] = w1.w;
         } else {
@@ -149,14 +133,14 @@ __device__ __forceinline__ void route_token_block(
     }
     red[warp][base] = v[0];
     red[warp][base + 1] = v[1];
-    sync();
+    __syncthreads();
     if (tid < 64 && eg + (tid & 7) < n) {
       float sum = 0.f;
 #pragma unroll
       for (int w = 0; w < ROUTE_THREADS / 32; ++w) sum += red[w][tid];
       logits[tid >> 3][eg + (tid & 7)] = sum;
     }
-    sync();
+    __syncthreads();
   }
 
   // TopK by repeated arg-max (strict '>' keeps the lower index on ties), then Softmax over
@@ -188,7 +172,7 @@ __device__ __forceinline__ void route_token_block(
       }
     }
   }
-  sync();
+  __syncthreads();
 }
 
 // Block b routes tokens [b*tokb, b*tokb + tokb) (tokb <= RT_TOK) and writes its expert
@@ -207,8 +191,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
   const int ntok = (int)(T - t0 < tokb ? T - t0 : tokb);
   if (threadIdx.x < MAX_EXPERTS) hist[threadIdx.x] = 0;
   __syncthreads();
-  route_token_block<Tin, false>(x, Wg, w_vec, t0, ntok, d, n, K, threadIdx.x, red, logits, hist,
-                                idx, gate, CtaSync{});
+  route_token_block<Tin>(x, Wg, w_vec, t0, ntok, d, n, K, threadIdx.x, red, logits, hist, idx,
+                         gate);
   if (threadIdx.x < n) blk_counts[(int64_t)blockIdx.x * n + threadIdx.x] = hist[threadIdx.x];
 }
 
@@ -260,26 +244,55 @@ __device__ __forceinline__ void quantize_tokens_e4m3(const __nv_bfloat16* __rest
   }
 }
 
-// Large batches whose router matrix fits in shared memory: each CTA copies W_g once (skewed
-// layout, wg_smem_index) and its two 256-thread groups route token blocks b = 2*CTA + group,
-// then b + 2*grid, ... (same per-block arithmetic, histogram and outputs as
-// router_topk_kernel), so W_g crosses from L2 once per SM instead of once per token block,
-// and two blocks' load latencies overlap on each SM.
-constexpr int RT_SMEM_MAX = 200 * 1024;
+// Large batches whose router matrix fits in shared memory: one persistent CTA of 16 warps per
+// SM copies W_g once (skewed layout, wg_smem_index); then "teams" of S warps (S = 1 .. 16,
+// chosen by the host so that one wave of teams covers the token blocks) route token blocks
+// b = team, team + teams, ... independently of each other, with no CTA-wide barrier after
+// the copy.  The S warps of a team split the hidden dimension: warp w takes the 8-element
+// chunks c = 32 w + lane, 32 w + lane + 32 S, ...  Each lane accumulates the logits of the
+// block's tokens for eight experts at a time in fp32 (the eight experts as four packed pairs,
+// fma.rn.f32x2: two independent IEEE fmas per instruction, which halves the issue slots of
+// the multiply-adds), the 64 partial sums are reduce-scattered over the warp's lanes, the S
+// warps' sums are added in warp order by the team's first warp, which then runs TopK and the
+// softmax (one lane per token) and writes the block's expert histogram.  Outputs and their
+// layout are those of router_topk_kernel.
+constexpr int RW_THREADS = 512;
 
-template <typename Tin>
-__global__ void __launch_bounds__(2 * ROUTE_THREADS, 1)
-    router_topk_smem_kernel(const Tin* __restrict__ x, const float* __restrict__ Wg, int64_t T,
-                            int d, int n, int K, int tokb, int64_t nblk,
-                            int32_t* __restrict__ idx, float* __restrict__ gate,
-                            int32_t* __restrict__ blk_counts) {
+__device__ __forceinline__ void ffma2(float2& acc, float a, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %2};\n\t"
+      "mov.b64 rb, {%3, %4};\n\t"
+      "mov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "f"(a), "f"(b0), "f"(b1));
+}
+
+template <int S>
+struct TeamSync {  // the S warps of one team: named barrier 1 + team (a warp barrier if S = 1)
+  int id;
+  __device__ __forceinline__ void operator()() const {
+    if (S == 1)
+      __syncwarp();
+    else
+      asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(32 * S) : "memory");
+  }
+};
+
+template <int S>
+__global__ void __launch_bounds__(RW_THREADS, 1)
+    router_team_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ Wg,
+                       int64_t T, int d, int n, int K, int tokb, int64_t nblk,
+                       int32_t* __restrict__ idx, float* __restrict__ gate,
+                       int32_t* __restrict__ blk_counts) {
+  constexpr int TEAMS = RW_THREADS / 32 / S;
   extern __shared__ float4 wg_raw[];
   float* sw = reinterpret_cast<float*>(wg_raw);
-  __shared__ float red[2][ROUTE_THREADS / 32][64];
-  __shared__ float logits[2][RT_TOK][MAX_EXPERTS];
-  __shared__ int hist[2][MAX_EXPERTS];
-  // W_g rows as float4 quarters (n % 8 == 0): row j, quarter q -> skewed row start + 4q
-  const int q4 = n / 4;
+  __shared__ float red[TEAMS][S][64];                 // each warp's 64 sums of one expert group
+  __shared__ float logits[TEAMS][RT_TOK][MAX_EXPERTS];
+  __shared__ int sel[TEAMS][64];                      // the block's K * ntok selections
+  const int q4 = n / 4;  // W_g rows as float4 quarters (n % 8 == 0)
   for (int i = threadIdx.x; i < d * q4; i += blockDim.x) {
     const int j = i / q4, q = i % q4;
     *reinterpret_cast<float4*>(sw + wg_smem_index(j, n) + 4 * q) =
@@ -289,17 +302,111 @@ __global__ void __launch_bounds__(2 * ROUTE_THREADS, 1)
   pdl_wait();
   pdl_trigger();
   __syncthreads();
-  const int grp = threadIdx.x / ROUTE_THREADS, gt = threadIdx.x % ROUTE_THREADS;
-  const GroupSync sync{1 + grp};
-  for (int64_t b = (int64_t)blockIdx.x * 2 + grp; b < nblk; b += (int64_t)gridDim.x * 2) {
-    if (gt < MAX_EXPERTS) hist[grp][gt] = 0;
-    sync();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int team = warp / S, tw = warp % S;
+  const TeamSync<S> sync{1 + team};
+  const int nchunk = d / 8;
+  for (int64_t b = (int64_t)blockIdx.x * TEAMS + team; b < nblk; b += (int64_t)gridDim.x * TEAMS) {
     const int64_t t0 = b * tokb;
     const int ntok = (int)(T - t0 < tokb ? T - t0 : tokb);
-    route_token_block<Tin, true>(x, sw, true, t0, ntok, d, n, K, gt, red[grp], logits[grp],
-                                 hist[grp], idx, gate, sync);
-    if (gt < n) blk_counts[b * n + gt] = hist[grp][gt];
-    sync();
+    for (int eg = 0; eg < n; eg += 8) {
+      float2 acc[RT_TOK][4];
+#pragma unroll
+      for (int a = 0; a < RT_TOK; ++a)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[a][e] = make_float2(0.f, 0.f);
+      for (int ci = tw * 32 + lane; ci < nchunk; ci += 32 * S) {
+        const int j0 = ci * 8;
+        Vec8<__nv_bfloat16> xv[RT_TOK];
+#pragma unroll
+        for (int a = 0; a < RT_TOK; ++a)
+          if (a < ntok) xv[a].load(x + (t0 + a) * (int64_t)d + j0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float* wr = sw + wg_smem_index(j0 + i, n) + eg;
+          const float4 w0 = *reinterpret_cast<const float4*>(wr);
+          const float4 w1 = *reinterpret_cast<const float4*>(wr + 4);
+#pragma unroll
+          for (int a = 0; a < RT_TOK; ++a) {
+            if (a < ntok) {
+              const float xa = xv[a].get(i);
+              ffma2(acc[a][0], xa, w0.x, w0.y);
+              ffma2(acc[a][1], xa, w0.z, w0.w);
+              ffma2(acc[a][2], xa, w1.x, w1.y);
+              ffma2(acc[a][3], xa, w1.z, w1.w);
+            }
+          }
+        }
+      }
+      // butterfly reduce-scatter of the 64 partial sums over the lanes (value a*8 + e)
+      float v[64];
+#pragma unroll
+      for (int a = 0; a < RT_TOK; ++a)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[a * 8 + 2 * e] = acc[a][e].x;
+          v[a * 8 + 2 * e + 1] = acc[a][e].y;
+        }
+      int base = 0;
+#pragma unroll
+      for (int half = 32, off = 16; off >= 1; half >>= 1, off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = upper ? v[i] : v[half + i];
+          const float keep = upper ? v[half + i] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+        if (upper) base += half;
+      }
+      red[team][tw][base] = v[0];
+      red[team][tw][base + 1] = v[1];
+      sync();
+      if (tw == 0) {  // lane l: values 2l and 2l + 1, summed over the team's warps in order
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int vi = 2 * lane + h;
+          float sum = 0.f;
+#pragma unroll
+          for (int w = 0; w < S; ++w) sum += red[team][w][vi];
+          if (eg + (vi & 7) < n) logits[team][vi >> 3][eg + (vi & 7)] = sum;
+        }
+      }
+      sync();  // red is rewritten by the next expert group or block
+    }
+    if (tw == 0) {
+      __syncwarp();
+      // TopK by repeated arg-max (strict '>' keeps the lower index on ties), then Softmax
+      // over the kept logits shifted by the largest, summed in slot order; lane a = token a
+      if (lane < ntok) {
+        const float* l = logits[team][lane];
+        const int64_t t = t0 + lane;
+        uint64_t used = 0;
+        float top = 0.f, z = 0.f;
+        for (int k = 0; k < K; ++k) {
+          int best = -1;
+          float bv = 0.f;
+          for (int e = 0; e < n; ++e) {
+            if ((used >> e) & 1ull) continue;
+            if (best < 0 || l[e] > bv) { best = e; bv = l[e]; }
+          }
+          used |= 1ull << best;
+          if (k == 0) top = bv;
+          z += expf(bv - top);
+          sel[team][lane * K + k] = best;
+          idx[t * K + k] = best;
+        }
+        for (int k = 0; k < K; ++k)
+          gate[t * K + k] = expf(l[sel[team][lane * K + k]] - top) / z;
+      }
+      __syncwarp();
+      for (int e = lane; e < n; e += 32) {  // the block's histogram
+        int c = 0;
+        for (int i = 0; i < ntok * K; ++i) c += sel[team][i] == e;
+        blk_counts[b * n + e] = c;
+      }
+      __syncwarp();
+    }
   }
 }
 
@@ -671,11 +778,139 @@ __global__ void __launch_bounds__(256)
   gather_rows(x, t0, d, K, E, ent_row, xperm, threadIdx.x, blockDim.x);
 }
 
+// ---------------------------------------------------------------- expert-parallel regroup
+// The rows a rank receives for its nl local experts arrive from S sources (ranks), each
+// source's rows grouped by local expert in expert order, with seg_counts[s][e] rows in
+// segment (s, e).  This kernel places them in the per-expert layout the grouped GEMMs take:
+// expert e's group is padded to row_align rows and holds the segments (0, e), (1, e), ...
+// in source order.  Every CTA recomputes the segment starts in shared memory (S * nl <= 2048
+// entries); CTA 0 also writes counts and offsets.  Then one warp per received row r finds its
+// segment (binary search over the segment starts), writes inv[r] = its padded row and copies
+// the row into X_perm.  The counts must add up to `rows` (else DEV_ERR_ROW, nothing copied).
+constexpr int EP_MAX_SEGS = 2048;
+
+template <typename Tact>
+__global__ void __launch_bounds__(256)
+    ep_regroup_kernel(const Tact* __restrict__ xr, int64_t rows, int d,
+                      const int32_t* __restrict__ seg_counts, int S, int nl, int row_align,
+                      int64_t rows_max, int32_t* __restrict__ counts,
+                      int32_t* __restrict__ offsets, int32_t* __restrict__ inv,
+                      Tact* __restrict__ xperm, uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int s_cnt[EP_MAX_SEGS];    // segment (s, e) at s * nl + e: its count
+  __shared__ int s_start[EP_MAX_SEGS];  // its first received row
+  __shared__ int s_base[EP_MAX_SEGS];   // its first row in the padded layout
+  __shared__ int s_off[MAX_EXPERTS + 1];
+  __shared__ int s_ok;
+  const int nseg = S * nl;
+  for (int i = threadIdx.x; i < nseg; i += blockDim.x) s_cnt[i] = seg_counts[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int64_t off = 0, start = 0;
+    bool ok = true;
+    for (int e = 0; e < nl; ++e) {  // expert groups: segments of expert e in source order
+      s_off[e] = (int)off;
+      int64_t c = 0;
+      for (int q = 0; q < S; ++q) {
+        const int v = s_cnt[q * nl + e];
+        ok = ok && v >= 0;
+        s_base[q * nl + e] = (int)(off + c);
+        c += v;
+      }
+      if (blockIdx.x == 0) counts[e] = (int32_t)c;
+      off += (c + row_align - 1) / row_align * row_align;
+    }
+    s_off[nl] = (int)off;
+    for (int i = 0; i < nseg; ++i) {  // received order: source-major, then expert
+      s_start[i] = (int)start;
+      start += s_cnt[i];
+    }
+    ok = ok && start == rows && off <= rows_max;
+    if (blockIdx.x == 0) {
+      for (int e = 0; e <= nl; ++e) offsets[e] = s_off[e];
+      if (!ok) set_status(status, DEV_ERR_ROW);
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const int lane = threadIdx.x & 31;
+  const int vpr = d * (int)sizeof(Tact) / 16;
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    int lo = 0, hi = nseg - 1;  // last segment starting at or before r (it is not empty)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_start[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    const int64_t dst = s_base[lo] + (r - s_start[lo]);
+    if (lane == 0) inv[r] = (int32_t)dst;
+    const uint4* src = reinterpret_cast<const uint4*>(xr + r * d);
+    uint4* out = reinterpret_cast<uint4*>(xperm + dst * d);
+    for (int c = lane; c < vpr; c += 32) out[c] = __ldg(src + c);
+  }
+}
+
+cudaError_t launch_ep_regroup(const Plan& p, const void* x_rows, const int32_t* seg_counts,
+                              int S, const Workspace& w, cudaStream_t s) {
+  const int64_t rows = p.T;  // the received rows are the plan's tokens (K = 1)
+  int64_t blocks = (rows + 7) / 8;
+  const int64_t cap = 4 * (int64_t)num_sms();
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  if (p.dt == 1)
+    pdl(ep_regroup_kernel<__nv_bfloat16>, (unsigned)blocks, 256, 0, s)(
+        static_cast<const __nv_bfloat16*>(x_rows), rows, (int)p.d, seg_counts, S, p.n,
+        p.row_align, p.rows_max, w.counts, w.offsets, w.inv,
+        static_cast<__nv_bfloat16*>(w.xperm), w.status);
+  else
+    pdl(ep_regroup_kernel<float>, (unsigned)blocks, 256, 0, s)(
+        static_cast<const float*>(x_rows), rows, (int)p.d, seg_counts, S, p.n, p.row_align,
+        p.rows_max, w.counts, w.offsets, w.inv, static_cast<float*>(w.xperm), w.status);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- host launchers
 
 // Tokens per router / permute block: eight, or fewer when K > 8 so that a block's
 // (token, slot) entries stay within 64.
 int route_tokens_per_block(int K) { return K <= 8 ? RT_TOK : (64 / K > 0 ? 64 / K : 1); }
+
+// Warps per token block of router_team_kernel: the S (1 .. 16) that minimises the time of
+// ceil(nblk * S / warp slots) rounds of 1/S of a block's work each; ties go to the smaller S
+// (fewer partial sums to add).
+static int router_team_size(int64_t nblk, int sms, int d) {
+  const int64_t slots = (int64_t)sms * (RW_THREADS / 32);
+  int best = 1;
+  double best_t = 1e30;
+  for (int S = 1; S <= 16; S <<= 1) {
+    if (S > 1 && d / 8 < 32 * S) break;  // every warp of a team needs a chunk per lane
+    const double t = (double)((nblk * S + slots - 1) / slots) / S;
+    if (t < best_t * 0.99) { best_t = t; best = S; }
+  }
+  return best;
+}
+
+template <int S>
+static cudaError_t launch_router_team(const __nv_bfloat16* x, const float* Wg, int64_t T, int d,
+                                      int n, int K, int tokb, int64_t nblk, size_t wbytes,
+                                      int sms, int32_t* idx, float* gate, int32_t* blk_counts,
+                                      cudaStream_t s) {
+  auto kern = router_team_kernel<S>;
+  static int configured = 0;  // per instantiation
+  if (configured < (int)wbytes) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wbytes);
+    if (e != cudaSuccess) return e;
+    configured = (int)wbytes;
+  }
+  constexpr int TEAMS = RW_THREADS / 32 / S;
+  const int64_t want = (nblk + TEAMS - 1) / TEAMS;
+  const unsigned grid = (unsigned)(want < sms ? want : sms);
+  pdl(kern, grid, RW_THREADS, wbytes, s)(x, Wg, T, d, n, K, tokb, nblk, idx, gate, blk_counts);
+  return cudaGetLastError();
+}
 
 template <typename Tin>
 static cudaError_t launch_router_t(const Tin* x, const float* Wg, int64_t T, int d, int n,
@@ -686,24 +921,23 @@ static cudaError_t launch_router_t(const Tin* x, const float* Wg, int64_t T, int
   const bool w_vec = n % 8 == 0 && (reinterpret_cast<uintptr_t>(Wg) & 15u) == 0;
   const size_t wbytes = wg_smem_bytes(d, n);
   const int sms = num_sms();
-  // bf16 activations only: with fp32 rows (32 bytes per 8 elements) the two-group kernel
-  // would not fit its registers
+  // bf16 activations, W_g in shared memory, and enough token blocks to pay for copying W_g
+  // to every SM
   if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
-  if (w_vec && wbytes <= (size_t)RT_SMEM_MAX && nblk >= 2 * (int64_t)sms) {
-    auto kern = router_topk_smem_kernel<Tin>;
-    static int configured = 0;  // per instantiation
-    if (configured < (int)wbytes) {
-      const cudaError_t e =
-          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wbytes);
-      if (e != cudaSuccess) return e;
-      configured = (int)wbytes;
+    if (w_vec && wbytes <= (size_t)RT_SMEM_MAX && nblk >= (int64_t)sms) {
+      switch (router_team_size(nblk, sms, d)) {
+        case 1: return launch_router_team<1>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
+                                             gate, blk_counts, s);
+        case 2: return launch_router_team<2>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
+                                             gate, blk_counts, s);
+        case 4: return launch_router_team<4>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
+                                             gate, blk_counts, s);
+        case 8: return launch_router_team<8>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
+                                             gate, blk_counts, s);
+        default: return launch_router_team<16>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
+                                               gate, blk_counts, s);
+      }
     }
-    const int64_t want = (nblk + 1) / 2;
-    const unsigned grid = (unsigned)(want < sms ? want : sms);
-    pdl(kern, grid, 2 * ROUTE_THREADS, wbytes, s)(x, Wg, T, d, n, K, tokb, nblk, idx, gate,
-                                                  blk_counts);
-    return cudaGetLastError();
-  }
   }
   pdl(router_topk_kernel<Tin>, (unsigned)nblk, ROUTE_THREADS, 0, s)(x, Wg, w_vec, T, d, n, K,
                                                                     tokb, idx, gate,

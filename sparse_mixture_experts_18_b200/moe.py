@@ -76,6 +76,17 @@ def lib() -> ctypes.CDLL:
         L.moe_debug_forward_withheld.restype = I32
         L.moe_debug_forward_withheld.argtypes = [P, P, P, P, P, I64, I64, I64, I32, I32, I32, P,
                                                  P, SZ, P, I64]
+        L.moe_route_workspace_bytes.restype = SZ
+        L.moe_route_workspace_bytes.argtypes = [I64, I64, I32, I32, I32]
+        L.moe_route.restype = I32
+        L.moe_route.argtypes = [P, P, I64, I64, I32, I32, I32, P, P, P, P, P, P, SZ, P]
+        L.moe_experts_workspace_bytes.restype = SZ
+        L.moe_experts_workspace_bytes.argtypes = [I64, I64, I64, I32, I32]
+        L.moe_experts_forward.restype = I32
+        L.moe_experts_forward.argtypes = [P, I64, P, I32, P, P, P, I64, I64, I32, I32, P, P, SZ,
+                                          P]
+        L.moe_combine.restype = I32
+        L.moe_combine.argtypes = [P, P, P, I64, I64, I32, I32, P, P]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [I32]
         L.moe_abi_version.restype = I32
@@ -303,6 +314,57 @@ def moe_debug_forward_withheld(x, W_g, W1, W3, W2, K: int, wait_limit_cycles: in
     _check("moe_debug_forward_withheld", lib().moe_debug_forward_withheld(
         _ptr(x), _ptr(W_g), _ptr(W1), _ptr(W3), _ptr(W2), T, d, F, n, K, dt, _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(stream), int(wait_limit_cycles)))
+    return out
+
+
+# ------------------------------------------------------------------ expert parallelism stages
+
+def moe_route(x, W_g, K: int, workspace=None, stream=None):
+    """Router, TopK, softmax and the grouping of the (token, slot) rows by expert, unpadded:
+    returns (x_grouped [T*K, d], topk_idx [T, K], topk_gate [T, K], expert_counts [n],
+    token_rows [T, K]); expert e's rows are x_grouped[sum(counts[:e]) : sum(counts[:e+1])]."""
+    T, d = x.shape
+    n = W_g.shape[1]
+    dt = _dt(x)
+    dev = x.device
+    if workspace is None:
+        workspace = alloc_workspace(int(lib().moe_route_workspace_bytes(T, d, n, K, dt)), dev,
+                                    stream)
+    xg = torch.empty((T * K, d), dtype=x.dtype, device=dev)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    gate = torch.empty((T, K), dtype=torch.float32, device=dev)
+    counts = torch.empty((n,), dtype=torch.int32, device=dev)
+    rows = torch.empty((T, K), dtype=torch.int32, device=dev)
+    _check("moe_route", lib().moe_route(
+        _ptr(x), _ptr(W_g), T, d, n, K, dt, _ptr(xg), _ptr(idx), _ptr(gate), _ptr(counts),
+        _ptr(rows), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return xg, idx, gate, counts, rows
+
+
+def moe_experts_forward(x_rows, seg_counts, W1, W3, W2, workspace=None, stream=None):
+    """y_rows[r] = SwiGLU_e(x_rows[r]) in fp32 for rows that arrive in S segments, each grouped
+    by the n_local experts of W1/W3/W2 (seg_counts: int32 [S, n_local] on the device)."""
+    rows, d = x_rows.shape
+    nl, F, _ = W1.shape
+    S = seg_counts.shape[0]
+    dt = _dt(x_rows)
+    if workspace is None:
+        workspace = alloc_workspace(
+            int(lib().moe_experts_workspace_bytes(rows, d, F, nl, dt)), x_rows.device, stream)
+    y = torch.empty((rows, d), dtype=torch.float32, device=x_rows.device)
+    _check("moe_experts_forward", lib().moe_experts_forward(
+        _ptr(x_rows), rows, _ptr(seg_counts.contiguous()), S, _ptr(W1), _ptr(W3), _ptr(W2), d,
+        F, nl, dt, _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return y
+
+
+def moe_combine(y_rows, token_rows, topk_gate, out, stream=None):
+    """out[t] = sum_k topk_gate[t, k] * y_rows[token_rows[t, k]] (fp32 sum, one rounding)."""
+    T, K = token_rows.shape
+    d = y_rows.shape[1]
+    _check("moe_combine", lib().moe_combine(
+        _ptr(y_rows), _ptr(token_rows), _ptr(topk_gate), T, d, K, _dt(out), _ptr(out),
+        _stream(stream)))
     return out
 
 

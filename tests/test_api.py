@@ -34,7 +34,9 @@ def test_header_declares_entry_points():
                  "moe_status_string", "moe_forward_host_io", "moe_workspace_init",
                  "moe_workspace_status", "moe_forward_profiled", "moe_plan_info",
                  "moe_stack_forward_profiled", "moe_stack_forward_host_io",
-                 "moe_debug_forward_withheld", "moe_forward_noalloc", "moe_noalloc_status"):
+                 "moe_debug_forward_withheld", "moe_forward_noalloc", "moe_noalloc_status",
+                 "moe_route", "moe_route_workspace_bytes", "moe_experts_forward",
+                 "moe_experts_workspace_bytes", "moe_combine"):
         assert want in names
 
 
@@ -168,6 +170,37 @@ def test_withheld_hook_validation(L):
     assert call(dt=F32) == UNSUPPORTED                       # the fp32 kernel has no pipeline
     assert call(T=4096) == UNSUPPORTED                       # CTA-pair tiling
     assert call(T=0) == OK
+
+
+def test_expert_parallel_stage_validation(L):
+    rb = L.moe_route_workspace_bytes
+    assert rb(16, 4096, 8, 2, BF16) > 0 and rb(16, 4000, 8, 2, BF16) == 0
+    # the route-only workspace holds no expert stages: far smaller than the block's
+    assert rb(4096, 4096, 8, 2, BF16) < moe.moe_workspace_bytes(4096, 4096, 14336, 8, 2, BF16) / 50
+    route = L.moe_route
+    args = [P(0x1000), P(0x2000), 16, 256, 8, 2, BF16, P(0x3000), P(0x4000), P(0x5000),
+            P(0x6000), P(0x7000), P(0x10000), 1 << 40, None]
+    assert route(*args[:7], P(0x1000), *args[8:]) == INVALID     # x_grouped aliases x
+    assert route(*args[:7], None, *args[8:]) == INVALID
+    assert route(*args[:13], 64, None) == WORKSPACE
+    assert route(*args[:5], 9, *args[6:]) == INVALID               # K > n
+    assert route(P(0), P(0), 0, 256, 8, 2, BF16, *([P(0)] * 6), 0, None) == OK   # T = 0
+    eb = L.moe_experts_workspace_bytes
+    assert eb(100, 4096, 14336, 4, BF16) > 0 and eb(100, 4096, 14300, 4, BF16) == 0
+    exf = L.moe_experts_forward
+    eargs = [P(0x1000), 100, P(0x2000), 2, P(0x3000), P(0x4000), P(0x5000), 256, 256, 4, BF16,
+             P(0x6000), P(0x10000), 1 << 40, None]
+    assert exf(*eargs[:3], 0, *eargs[4:]) == INVALID                # no source
+    assert exf(*eargs[:3], 1024, *eargs[4:]) == INVALID             # S * n_local > 2048
+    assert exf(*eargs[:2], None, *eargs[3:]) == INVALID
+    assert exf(*eargs[:13], 512, None) == WORKSPACE
+    assert exf(*eargs[:7], 200, *eargs[8:]) == UNSUPPORTED          # d % 64
+    assert exf(P(0), 0, P(0), 2, P(0), P(0), P(0), 256, 256, 4, BF16, P(0), P(0), 0, None) == OK
+    comb = L.moe_combine
+    assert comb(P(0x1000), P(0x2000), P(0x3000), 16, 256, 0, BF16, P(0x4000), None) == INVALID
+    assert comb(P(0x1000), P(0x2000), P(0x3000), 16, 250, 2, BF16, P(0x4000), None) == UNSUPPORTED
+    assert comb(P(0x1008), P(0x2000), P(0x3000), 16, 256, 2, BF16, P(0x4000), None) == INVALID
+    assert comb(None, None, None, 0, 256, 2, BF16, None, None) == OK
 
 
 def test_host_io_validation(L):
