@@ -50,10 +50,8 @@ DEFAULT_WORKLOAD = "stack32_t8192"
 # of that kernel on the workload's shapes (for the stack: one T=8192 block), valid only for
 # the kernel source it was taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "decode_t16": {"bytes": 1886786272, "src": "9c8fdd53d8eb"},
-    "prefill_t4096": {"bytes": 2523485256, "src": "9c8fdd53d8eb"},
+    "stack32_t8192": {"bytes": 3175285736, "src": "12bfa10d6348"},
 }
-
 
 def kernel_source_hash() -> str:
     """Hash of the GEMM kernels' code (csrc/gemm_tc.cu + csrc/common.cuh) with comments and

@@ -194,6 +194,65 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// combine_rows_kernel for K = 2 without split slabs (the large-batch tilings): both slots'
+// loads and the residual's are issued together before any is used, so a lane has 2 x 8
+// float4 plus 8 residual vectors in flight; same arithmetic and result as combine_rows_kernel
+// (acc = fma(g1, y1, fma(g0, y0, 0)), then resid + acc, rounded once).
+template <typename Tout, bool RESID>
+__global__ void __launch_bounds__(256)
+    combine_rows_k2_kernel(const float* __restrict__ Y, int64_t T, int d,
+                           const int32_t* __restrict__ inv, const float* __restrict__ gate,
+                           Tout* out, const Tout* resid) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
+       t += nwarps) {
+    const int2 rows = *reinterpret_cast<const int2*>(inv + 2 * t);
+    float g0 = 1.f, g1 = 1.f;  // null gate: rows already gated
+    if (gate) {
+      const float2 g = *reinterpret_cast<const float2*>(gate + 2 * t);
+      g0 = g.x;
+      g1 = g.y;
+    }
+    const float* y0 = Y + (int64_t)(rows.x < 0 ? 0 : rows.x) * d;
+    const float* y1 = Y + (int64_t)(rows.y < 0 ? 0 : rows.y) * d;
+    for (int c0 = lane * 4; c0 < d; c0 += 128 * COMBINE_U) {
+      float4 a[COMBINE_U], b[COMBINE_U];
+      float r[COMBINE_U][4];
+#pragma unroll
+      for (int u = 0; u < COMBINE_U; ++u) {
+        const int c = c0 + 128 * u;
+        if (c < d) {
+          a[u] = __ldg(reinterpret_cast<const float4*>(y0 + c));
+          b[u] = __ldg(reinterpret_cast<const float4*>(y1 + c));
+          if (RESID) Out4<Tout>::load(resid + t * d + c, r[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < COMBINE_U; ++u) {
+        const int c = c0 + 128 * u;
+        if (c >= d) continue;
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
+        if (rows.x >= 0) {
+          o[0] = fmaf(g0, a[u].x, o[0]); o[1] = fmaf(g0, a[u].y, o[1]);
+          o[2] = fmaf(g0, a[u].z, o[2]); o[3] = fmaf(g0, a[u].w, o[3]);
+        }
+        if (rows.y >= 0) {
+          o[0] = fmaf(g1, b[u].x, o[0]); o[1] = fmaf(g1, b[u].y, o[1]);
+          o[2] = fmaf(g1, b[u].z, o[2]); o[3] = fmaf(g1, b[u].w, o[3]);
+        }
+        if (RESID) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[i] = r[u][i] + o[i];
+        }
+        Out4<Tout>::store(out + t * d + c, o);
+      }
+    }
+  }
+}
+
 // out[t] = (resid[t] +) sum_k gate[t][k] * sum_s Y[s][inv[t][k]] for T tokens, Tout = bf16
 // or fp32 (gate null: 1), picking the one-warp-per-token kernel for T >= 1024.
 template <typename Tout>
@@ -203,6 +262,16 @@ static cudaError_t combine_rows_t(const float* Y, int S, int64_t split_stride, i
   if (T >= 1024) {  // enough tokens for one warp each
     const int64_t blocks = (T + 7) / 8;
     const unsigned g = (unsigned)(blocks < ((int64_t)1 << 30) ? blocks : ((int64_t)1 << 30));
+    const bool k2 = K == 2 && S == 1 && (reinterpret_cast<uintptr_t>(inv) & 7u) == 0 &&
+                    (!gate || (reinterpret_cast<uintptr_t>(gate) & 7u) == 0);
+    if (k2) {
+      if (resid)
+        pdl(combine_rows_k2_kernel<Tout, true>, g, 256, 0, s)(Y, T, d, inv, gate, out, resid);
+      else
+        pdl(combine_rows_k2_kernel<Tout, false>, g, 256, 0, s)(Y, T, d, inv, gate, out,
+                                                               nullptr);
+      return cudaGetLastError();
+    }
     if (resid)
       pdl(combine_rows_kernel<Tout, true>, g, 256, 0, s)(Y, S, split_stride, T, d, K, inv, gate,
                                                          out, resid);

@@ -292,11 +292,20 @@ __global__ void __launch_bounds__(RW_THREADS, 1)
   __shared__ float red[TEAMS][S][64];                 // each warp's 64 sums of one expert group
   __shared__ float logits[TEAMS][RT_TOK][MAX_EXPERTS];
   __shared__ int sel[TEAMS][64];                      // the block's K * ntok selections
-  const int q4 = n / 4;  // W_g rows as float4 quarters (n % 8 == 0)
-  for (int i = threadIdx.x; i < d * q4; i += blockDim.x) {
-    const int j = i / q4, q = i % q4;
-    *reinterpret_cast<float4*>(sw + wg_smem_index(j, n) + 4 * q) =
-        __ldg(reinterpret_cast<const float4*>(Wg) + i);
+  // W_g rows as float4 quarters (n % 8 == 0), eight loads in flight per thread
+  const int q4 = n / 4, total4 = d * q4;
+  for (int i0 = threadIdx.x; i0 < total4; i0 += 8 * RW_THREADS) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (i0 + u * RW_THREADS < total4)
+        v[u] = __ldg(reinterpret_cast<const float4*>(Wg) + i0 + u * RW_THREADS);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * RW_THREADS;
+      if (i < total4)
+        *reinterpret_cast<float4*>(sw + wg_smem_index(i / q4, n) + 4 * (i % q4)) = v[u];
+    }
   }
   // W_g is the caller's; x and the outputs are ordered after the previous kernel
   pdl_wait();
@@ -877,16 +886,17 @@ cudaError_t launch_ep_regroup(const Plan& p, const void* x_rows, const int32_t* 
 // (token, slot) entries stay within 64.
 int route_tokens_per_block(int K) { return K <= 8 ? RT_TOK : (64 / K > 0 ? 64 / K : 1); }
 
-// Warps per token block of router_team_kernel: the S (1 .. 16) that minimises the time of
-// ceil(nblk * S / warp slots) rounds of 1/S of a block's work each; ties go to the smaller S
-// (fewer partial sums to add).
+// Warps per token block of router_team_kernel: the S (1 .. 16) that minimises the estimated
+// time ceil(nblk * S / warp slots) * (1/S + 0.1), i.e. rounds of a team's share of a block
+// plus a per-block cost of the cross-warp sums, barriers and TopK (0.1 of a block's work at
+// Mixtral's width); ties go to the smaller S.
 static int router_team_size(int64_t nblk, int sms, int d) {
   const int64_t slots = (int64_t)sms * (RW_THREADS / 32);
   int best = 1;
   double best_t = 1e30;
   for (int S = 1; S <= 16; S <<= 1) {
     if (S > 1 && d / 8 < 32 * S) break;  // every warp of a team needs a chunk per lane
-    const double t = (double)((nblk * S + slots - 1) / slots) / S;
+    const double t = (double)((nblk * S + slots - 1) / slots) * (1.0 / S + 0.1);
     if (t < best_t * 0.99) { best_t = t; best = S; }
   }
   return best;

@@ -94,3 +94,30 @@ def test_fp8_repeat_calls_bitwise():
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert moe.moe_workspace_status(ws)[0] == 0
+
+
+def test_fp8_decode_error_against_the_bf16_block():
+    """How far the FP8 variant's output is from the exact block on the unquantised bf16
+    weights (the oracle's bf16 block), on the Mixtral decode shape.  Reported in the run's
+    parity summary.  E4M3's nearest rounding errs by at most 2^-4 relative (3 mantissa bits),
+    about 0.02-0.03 RMS for values spread over the binade; four quantisations lie on the path
+    (x, W1/W3, h, W2), so the expected relative L2 error is a few 1e-2.  The bar, 0.1, only
+    catches a lost scale or a wrong code (errors of order 1)."""
+    w = moe_inputs.WORKLOADS["decode_t16"]
+    x = moe_inputs.make_x(w, device="cuda")
+    L = moe_inputs.make_layer(w, device="cuda")
+    qs = _quantize_layer(L, w.n, w.F, w.d)
+    out = moe.moe_forward_fp8(x, L["Wg"], *qs, w.K)
+    torch.cuda.synchronize()
+    xc = x.cpu()
+    lc = {k: v.cpu() for k, v in L.items()}
+    del L, qs
+    logits, idx, _ = parity.oracle.route(xc, lc["Wg"], w.n, w.K)
+    ref = parity.oracle_outputs(xc, lc["Wg"], lc["W1"], lc["W3"], lc["W2"], w.n, w.K,
+                                np.arange(w.T), idx, [])
+    err = out.float().cpu().numpy().astype(np.float64) - ref
+    rep = {"tokens": w.T, "exempt": 0, "max_abs": float(np.max(np.abs(err))),
+           "rel_l2": float(np.linalg.norm(err) / np.linalg.norm(ref)), "ok": True}
+    rep["ok"] = rep["rel_l2"] <= 0.1
+    parity.record("decode_t16 FP8 (E4M3) weights vs the bf16 block (error of the format)", rep)
+    assert rep["ok"], rep

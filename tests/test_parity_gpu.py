@@ -92,6 +92,14 @@ def test_all_tokens_to_two_experts_gather_x(monkeypatch, T):
     test_all_tokens_to_two_experts(T)
 
 
+@pytest.mark.parametrize("T", [1180, 1200, 2400, 2501])
+def test_router_team_sizes(T):
+    # Mixtral's hidden size with W_g in shared memory: the large-batch router splits each
+    # 8-token block over 16 (T = 1180), 8 (T = 1200) or 4 (T = 2400) warps, and T = 2501 ends
+    # in a ragged block; a narrow expert width keeps the oracle quick
+    _run(moe_inputs.small(T=T, d=4096, F=128), budget=300)
+
+
 @pytest.mark.parametrize("T", [1, 5, 16, 37, 100, 255])
 def test_small_batch_tiling(T):
     # T <= 256 and T*K < 64*n: weights as the 128-row MMA operand, split-K
