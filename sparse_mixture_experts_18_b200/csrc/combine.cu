@@ -194,15 +194,43 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// RMSNorm of one row by one warp, in the column order of the large-batch combine (lane l takes
+// columns l*4 + 128 u + 1024 p, four at a time): the sum of squares is accumulated in that
+// order with fmaf and reduced by a fixed xor tree, so that the combine that fuses the next
+// block's RMSNorm (combine_rows_k2_kernel with NORM) produces bit for bit the same result.
+__device__ __forceinline__ float rms_inv_from_sumsq(float ss, int d, float eps) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  return 1.0f / sqrtf(ss / (float)d + eps);
+}
+
+__device__ __forceinline__ void rms_scale_row(const __nv_bfloat16* xr, __nv_bfloat16* xnr, int d,
+                                              int lane, float inv) {
+  for (int c0 = lane * 4; c0 < d; c0 += 128 * COMBINE_U) {
+#pragma unroll
+    for (int u = 0; u < COMBINE_U; ++u) {
+      const int c = c0 + 128 * u;
+      if (c >= d) continue;
+      float v[4];
+      Out4<__nv_bfloat16>::load(xr + c, v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] *= inv;
+      Out4<__nv_bfloat16>::store(xnr + c, v);
+    }
+  }
+}
+
 // combine_rows_kernel for K = 2 without split slabs (the large-batch tilings): both slots'
 // loads and the residual's are issued together before any is used, so a lane has 2 x 8
 // float4 plus 8 residual vectors in flight; same arithmetic and result as combine_rows_kernel
 // (acc = fma(g1, y1, fma(g0, y0, 0)), then resid + acc, rounded once).
-template <typename Tout, bool RESID>
+// NORM (bf16 only, with the residual): the kernel also writes the RMSNorm of each result row
+// (the next stacked block's input) to xn, exactly as rmsnorm_kernel would from the stored row.
+template <typename Tout, bool RESID, bool NORM = false>
 __global__ void __launch_bounds__(256)
     combine_rows_k2_kernel(const float* __restrict__ Y, int64_t T, int d,
                            const int32_t* __restrict__ inv, const float* __restrict__ gate,
-                           Tout* out, const Tout* resid) {
+                           Tout* out, const Tout* resid, __nv_bfloat16* xn, float eps) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -218,6 +246,7 @@ __global__ void __launch_bounds__(256)
     }
     const float* y0 = Y + (int64_t)(rows.x < 0 ? 0 : rows.x) * d;
     const float* y1 = Y + (int64_t)(rows.y < 0 ? 0 : rows.y) * d;
+    float ss = 0.f;  // NORM: sum of squares of the stored (rounded) row
     for (int c0 = lane * 4; c0 < d; c0 += 128 * COMBINE_U) {
       float4 a[COMBINE_U], b[COMBINE_U];
       float r[COMBINE_U][4];
@@ -248,9 +277,25 @@ __global__ void __launch_bounds__(256)
           for (int i = 0; i < 4; ++i) o[i] = r[u][i] + o[i];
         }
         Out4<Tout>::store(out + t * d + c, o);
+        if constexpr (NORM) {
+          const uint32_t lo = pack_bf16x2(o[0], o[1]), hi = pack_bf16x2(o[2], o[3]);
+          const float q[4] = {bf16_lo(lo), bf16_hi(lo), bf16_lo(hi), bf16_hi(hi)};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ss = fmaf(q[i], q[i], ss);
+        }
       }
     }
+    if constexpr (NORM) {
+      // this lane re-reads only the columns it stored itself (plain loads, program order)
+      rms_scale_row(reinterpret_cast<const __nv_bfloat16*>(out) + t * d, xn + t * d, d, lane,
+                    rms_inv_from_sumsq(ss, d, eps));
+    }
   }
+}
+
+static bool combine_k2_fits(int64_t T, int K, int S, const int32_t* inv, const float* gate) {
+  return T >= 1024 && K == 2 && S == 1 && (reinterpret_cast<uintptr_t>(inv) & 7u) == 0 &&
+         (!gate || (reinterpret_cast<uintptr_t>(gate) & 7u) == 0);
 }
 
 // out[t] = (resid[t] +) sum_k gate[t][k] * sum_s Y[s][inv[t][k]] for T tokens, Tout = bf16
@@ -262,14 +307,13 @@ static cudaError_t combine_rows_t(const float* Y, int S, int64_t split_stride, i
   if (T >= 1024) {  // enough tokens for one warp each
     const int64_t blocks = (T + 7) / 8;
     const unsigned g = (unsigned)(blocks < ((int64_t)1 << 30) ? blocks : ((int64_t)1 << 30));
-    const bool k2 = K == 2 && S == 1 && (reinterpret_cast<uintptr_t>(inv) & 7u) == 0 &&
-                    (!gate || (reinterpret_cast<uintptr_t>(gate) & 7u) == 0);
-    if (k2) {
+    if (combine_k2_fits(T, K, S, inv, gate)) {
       if (resid)
-        pdl(combine_rows_k2_kernel<Tout, true>, g, 256, 0, s)(Y, T, d, inv, gate, out, resid);
+        pdl(combine_rows_k2_kernel<Tout, true>, g, 256, 0, s)(Y, T, d, inv, gate, out, resid,
+                                                              nullptr, 0.f);
       else
         pdl(combine_rows_k2_kernel<Tout, false>, g, 256, 0, s)(Y, T, d, inv, gate, out,
-                                                               nullptr);
+                                                               nullptr, nullptr, 0.f);
       return cudaGetLastError();
     }
     if (resid)
@@ -305,7 +349,20 @@ cudaError_t launch_combine_rows(const float* Y, int S, int64_t split_stride, int
 }
 
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
-                           cudaStream_t s, const float* s2) {
+                           cudaStream_t s, const float* s2, void* norm_out, float eps,
+                           bool* normed) {
+  if (normed) *normed = false;
+  const float* g2 = p.gather_x ? nullptr : w.gate;
+  if (norm_out && resid && p.dt == 1 && !p.fp8 && !p.swap &&
+      combine_k2_fits(p.T, p.K, 1, w.inv, g2)) {
+    const int64_t blocks = (p.T + 7) / 8;
+    const unsigned g = (unsigned)(blocks < ((int64_t)1 << 30) ? blocks : ((int64_t)1 << 30));
+    pdl(combine_rows_k2_kernel<__nv_bfloat16, true, true>, g, 256, 0, s)(
+        w.y, p.T, (int)p.d, w.inv, g2, static_cast<__nv_bfloat16*>(out),
+        static_cast<const __nv_bfloat16*>(resid), static_cast<__nv_bfloat16*>(norm_out), eps);
+    if (normed) *normed = true;
+    return cudaGetLastError();
+  }
   const int S = p.swap ? p.s2 : 1;
   const int64_t split_stride = p.rows_max * p.d;
   const float* gates = p.gather_x ? nullptr : w.gate;  // gather_x: G2 applied the gates
@@ -322,8 +379,6 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
                              p.dt == 0, s);
 }
 
-// One warp per row: sum of squares in fp32 (lane-strided 8-element chunks, then a shuffle
-// tree), then x / sqrt(mean + eps) rounded to bf16.
 __global__ void __launch_bounds__(256)
     rmsnorm_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ xn,
                    int64_t T, int d, float eps) {
@@ -334,22 +389,18 @@ __global__ void __launch_bounds__(256)
   if (row >= T) return;
   const __nv_bfloat16* xr = x + row * d;
   float ss = 0.f;
-  for (int c = lane * 8; c < d; c += 256) {
-    float v[8];
-    Out8<__nv_bfloat16>::load(xr + c, v);
+  for (int c0 = lane * 4; c0 < d; c0 += 128 * COMBINE_U) {
+    float v[COMBINE_U][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) ss = fmaf(v[i], v[i], ss);
+    for (int u = 0; u < COMBINE_U; ++u)
+      if (c0 + 128 * u < d) Out4<__nv_bfloat16>::load(xr + c0 + 128 * u, v[u]);
+#pragma unroll
+    for (int u = 0; u < COMBINE_U; ++u)
+      if (c0 + 128 * u < d)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ss = fmaf(v[u][i], v[u][i], ss);
   }
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
-  for (int c = lane * 8; c < d; c += 256) {
-    float v[8];
-    Out8<__nv_bfloat16>::load(xr + c, v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] *= inv;
-    Out8<__nv_bfloat16>::store(xn + row * d + c, v);
-  }
+  rms_scale_row(xr, xn + row * d, d, lane, rms_inv_from_sumsq(ss, d, eps));
 }
 
 cudaError_t launch_rmsnorm(const void* x, void* xn, int64_t T, int64_t d, float eps,

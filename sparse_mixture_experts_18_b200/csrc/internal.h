@@ -124,8 +124,12 @@ cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float
                                      const float* W2, const Workspace& w, cudaStream_t s,
                                      cudaEvent_t const* ev = nullptr);
 // fp8 (p.fp8): s2 [n][d] are the W2 row scales; expert outputs are scaled by s_h[row] s2[e][i]
+// norm_out (may be null; bf16 with a residual): when the large-batch K = 2 combine applies,
+// it also writes the RMSNorm (unit gain, eps) of every result row there -- the next stacked
+// block's input -- and sets *normed; otherwise the caller runs launch_rmsnorm.
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
-                           cudaStream_t s, const float* s2 = nullptr);
+                           cudaStream_t s, const float* s2 = nullptr, void* norm_out = nullptr,
+                           float eps = 0.f, bool* normed = nullptr);
 // out[t] = (resid[t] +) sum_k gate[t][k] * sum_{s < S} Y[s * split_stride + inv[t][k] row]
 // (gate null: weight 1), fp32 sums in split then slot order, rounded once to bf16, or kept
 // fp32 (out_f32).

@@ -168,10 +168,13 @@ static moe_status shape_status(int64_t T, int64_t d, int64_t F, int n, int K, in
 
 // The kernel sequence of one block on already-validated arguments.
 // ev (may be null): six events recorded at the stage boundaries (see moe_forward_profiled).
+// norm_out (stacked blocks): where the combine may also write the next block's RMSNorm input
+// (*normed tells whether it did; see launch_combine).
 static moe_status forward_impl(const Plan& p, const void* x, const float* W_g, const void* W1,
                                const void* W3, const void* W2, void* out, const void* resid,
                                const Workspace& w, cudaStream_t s,
-                               cudaEvent_t const* ev = nullptr) {
+                               cudaEvent_t const* ev = nullptr, void* norm_out = nullptr,
+                               float eps = 0.f, bool* normed = nullptr) {
   if (ev && cudaEventRecord(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_route(p, x, W_g, w, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -182,7 +185,8 @@ static moe_status forward_impl(const Plan& p, const void* x, const float* W_g, c
                                            static_cast<const float*>(W2), w, s,
                                            ev ? ev + 2 : nullptr);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_combine(p, w, out, resid, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_combine(p, w, out, resid, s, nullptr, norm_out, eps, normed) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (ev && cudaEventRecord(ev[5], s) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
@@ -413,10 +417,13 @@ static moe_status stack_impl(const Plan& p, void* x, const float* const* W_g,
                              const void* const* W2, int L, float eps, void* workspace,
                              cudaStream_t s, cudaEvent_t const* ev) {
   const Workspace w = carve(p, workspace);
+  bool have_xn = false;  // the previous block's combine already wrote this block's input
   for (int l = 0; l < L; ++l) {
-    if (launch_rmsnorm(x, w.xn, p.T, p.d, eps, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!have_xn && launch_rmsnorm(x, w.xn, p.T, p.d, eps, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
     moe_status st = forward_impl(p, w.xn, W_g[l], W1[l], W3[l], W2[l], x, x, w, s,
-                                 ev ? ev + 6 * (size_t)l : nullptr);
+                                 ev ? ev + 6 * (size_t)l : nullptr,
+                                 l + 1 < L ? w.xn : nullptr, eps, &have_xn);
     if (st != MOE_OK) return st;
   }
   return MOE_OK;

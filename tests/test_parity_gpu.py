@@ -288,10 +288,13 @@ def test_stack_host_io_and_profiled_match_the_device_path():
         assert g13 > 0.0
 
 
-def test_stack_small():
-    """Four stacked blocks (RMSNorm -> MoE -> residual) on 300 tokens, every token of every
-    block checked against the oracle block on the GPU's own input."""
-    w = moe_inputs.small(T=300, d=256, F=512, layers=4)
+@pytest.mark.parametrize("T", [300, 1100])
+def test_stack_small(T):
+    """Four stacked blocks (RMSNorm -> MoE -> residual), every token of every block checked
+    against the oracle block on the GPU's own input.  At T = 1100 the combine also writes the
+    next block's RMSNorm (the fused path), which must equal the separate RMSNorm bit for bit
+    (one 4-block call against four 1-block calls)."""
+    w = moe_inputs.small(T=T, d=256, F=512, layers=4)
     x = moe_inputs.make_x(w).cuda()
     layers = [{k: v.cuda() for k, v in moe_inputs.make_layer(w, layer=l).items()}
               for l in range(w.layers)]
