@@ -185,7 +185,10 @@ def run_gpu(args, w):
     if stacked:  # x is the residual stream: every step restarts from the same input
         ws = moe.alloc_workspace(moe.moe_stack_workspace_bytes(w.T, w.d, w.F, w.n, w.K), dev,
                                  stream)
-        launches = w.layers * (1 + launches)  # each block: RMSNorm, then the MoE block
+        # each block: the MoE block and its input's RMSNorm, which the previous block's K = 2
+        # combine writes on the large-batch tilings (only the first block launches it then)
+        fused_norm = not small_batch and w.T >= 1024 and w.K == 2
+        launches = w.layers * launches + (1 if fused_norm else w.layers)
     else:
         ws = moe.alloc_workspace(moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K,
                                                          torch.bfloat16), dev, stream)

@@ -116,9 +116,10 @@ MOE_API moe_status moe_forward(const void* x, const float* W_g, const void* W1, 
  *   expert_offsets [n+1] int32 first row of each expert's group in the permuted layout
  *   token_rows [T][K] int32    permuted row of each (token, slot)
  * Enqueued on `stream` like moe_forward (no synchronisation). */
-MOE_API moe_status moe_forward_debug(const void* x, const float* W_g, const void* W1, const void* W3,
-                             const void* W2, int64_t T, int64_t d, int64_t F, int n, int K,
-                             moe_dtype dt, void* out, void* workspace, size_t workspace_bytes,
+MOE_API moe_status moe_forward_debug(const void* x, const float* W_g, const void* W1,
+                             const void* W3, const void* W2, int64_t T, int64_t d, int64_t F,
+                             int n, int K, moe_dtype dt, void* out, void* workspace,
+                             size_t workspace_bytes,
                              void* stream, int32_t* topk_idx, float* topk_gate,
                              int32_t* expert_counts, int32_t* expert_offsets,
                              int32_t* token_rows);
@@ -185,12 +186,16 @@ MOE_API moe_status moe_forward_profiled(const void* x, const float* W_g, const v
                                         void* workspace, size_t workspace_bytes, void* stream,
                                         void* const* events, int n_events);
 
-/* Work plan chosen for a shape (for reports; no counterpart in the pages): *small_batch = 1 if the weights are the MMA's
- * 128-row operand (small token counts), 0 otherwise; *split13 / *split2 = K-splits of the
- * two expert GEMMs on that path (1 otherwise); *launches = kernels one forward launches;
- * *pair = 1 if the expert GEMMs run on CTA pairs (256-row tiles).  Any output may be NULL. */
+/* Work plan chosen for a shape (for reports; no counterpart in the pages):
+ *   *small_batch = 1 if the weights are the MMA's 128-row operand (small token counts);
+ *   *split13 / *split2 = K-splits of the two expert GEMMs on that path (1 otherwise);
+ *   *launches = kernels one forward launches (a stack of them launches one more, the first
+ *              block's RMSNorm, on the large-batch tilings);
+ *   *pair = 1 if the expert GEMMs run on CTA pairs (256-row tiles).
+ * Any output may be NULL. */
 MOE_API moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt,
-                                 int* small_batch, int* split13, int* split2, int* launches, int* pair);
+                                 int* small_batch, int* split13, int* split2, int* launches,
+                                 int* pair);
 
 /* Stack of L blocks on a residual stream (attention omitted), in place on x [T][d]:
  *   for l in 0..L-1:  x <- round(x + MoE_l(RMSNorm(x)))

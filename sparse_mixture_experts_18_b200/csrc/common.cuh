@@ -108,6 +108,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
+// Wait (at most WAIT_LIMIT_CYCLES / 16) for a phase on the unwind path of a kernel that
+// already gave up, e.g. for its own copies in flight to land before it exits.
+__device__ __forceinline__ bool wait_short(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > (WAIT_LIMIT_CYCLES >> 4)) return false;
+  return true;
+}
+
 // ---------------------------------------------------------------- TMA (no multicast)
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

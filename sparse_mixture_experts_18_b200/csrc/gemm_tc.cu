@@ -122,13 +122,6 @@ __device__ __forceinline__ Work decode_work(const TcArgs& a, const Ctrl* c, int 
   return w;
 }
 
-__device__ __forceinline__ bool wait_short(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > (WAIT_LIMIT_CYCLES >> 4)) return false;
-  return true;
-}
-
 // One MMA of the kernel's operand kind: bf16 (kind::f16) or E4M3 (kind::f8f6f4).
 template <bool E4M3>
 __device__ __forceinline__ void umma_kind(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
@@ -974,6 +967,11 @@ static bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                   uint32_t box_rows) {
+  return make_map(m, base, inner, outer, box_rows);
 }
 
 constexpr uint32_t SMEM_STAGE_BUDGET = 200 * 1024;

@@ -46,6 +46,7 @@ struct Plan {
   size_t o_rowtok;         // token of each permuted row [rows_max] (small batch, gather_x)
   size_t o_rowgate;        // gather_x: gate of each permuted row [rows_max]
   size_t o_sx, o_sh;       // fp8: token-row scales [T] and h-row scales [rows_max]
+  size_t o_wparts;         // tensor-core router: W_g as three bf16 parts [3n padded][d]
   size_t o_status, o_idx, o_gate, o_blk_counts, o_blk_base, o_counts, o_offsets, o_inv,
       o_xperm, o_h, o_y, o_p13, o_xn, total;
 };
@@ -60,6 +61,7 @@ struct Workspace {
   float* row_gate;       // gather_x: gate of each permuted row
   float* sx;             // fp8: scale of each token's row (the E4M3 rows are per token)
   float* sh;             // fp8: scale of each h row
+  __nv_bfloat16* wparts; // tensor-core router: the W_g parts
   int32_t *idx, *blk_counts, *blk_base, *counts, *offsets, *inv;
   float* gate;
   void* xperm;  // [rows_max][d] activations in permuted order
@@ -105,6 +107,16 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
 Workspace carve(const Plan& p, void* base);
 
 int route_tokens_per_block(int K);
+// The router of large batches on the tensor cores (route_tc.cu): taken for bf16, T >= 1024,
+// n <= 16, K <= 8; writes idx, gate and the 8-token block histograms like the CUDA-core
+// router.
+bool router_tc_applies(const Plan& p);
+size_t router_tc_parts_bytes(int64_t d, int n);
+cudaError_t launch_router_tc(const Plan& p, const void* x, const float* Wg, const Workspace& w,
+                             cudaStream_t s);
+// 2-D bf16 tensor map [outer][inner], box box_rows x 64 elements, 128-byte swizzle.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                   uint32_t box_rows);
 cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Workspace& w,
                          cudaStream_t s);
 // ev (may be null): events recorded after G13, after the split-K reduction, after G2.

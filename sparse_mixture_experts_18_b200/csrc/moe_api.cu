@@ -116,6 +116,7 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   q.o_rowgate = take(q.pair ? (size_t)q.rows_max * 4 : 0);
   q.o_sx = take(fp8 ? (size_t)q.rows_max * 4 : 0);  // X_perm and h hold E4M3 codes then
   q.o_sh = take(fp8 ? (size_t)q.rows_max * 4 : 0);
+  q.o_wparts = take(router_tc_applies(q) ? router_tc_parts_bytes(d, n) : 0);
   q.total = o;
   *p = q;
   return true;
@@ -132,6 +133,7 @@ Workspace carve(const Plan& p, void* base) {
   w.row_gate = reinterpret_cast<float*>(b + p.o_rowgate);
   w.sx = reinterpret_cast<float*>(b + p.o_sx);
   w.sh = reinterpret_cast<float*>(b + p.o_sh);
+  w.wparts = reinterpret_cast<__nv_bfloat16*>(b + p.o_wparts);
   w.idx = reinterpret_cast<int32_t*>(b + p.o_idx);
   w.gate = reinterpret_cast<float*>(b + p.o_gate);
   w.blk_counts = reinterpret_cast<int32_t*>(b + p.o_blk_counts);
@@ -343,7 +345,10 @@ moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtyp
   if (small_batch) *small_batch = p.swap ? 1 : 0;
   if (split13) *split13 = p.swap ? p.s13 : 1;
   if (split2) *split2 = p.swap ? p.s2 : 1;
-  if (launches) *launches = T == 0 ? 0 : (p.fused_route ? 1 : 3) + (p.swap ? 3 : 2) + 1;
+  if (launches)
+    *launches = T == 0 ? 0
+                       : (p.fused_route ? 1 : 3) + (router_tc_applies(p) ? 1 : 0) +
+                             (p.swap ? 3 : 2) + 1;
   if (pair) *pair = p.pair ? 1 : 0;
   return MOE_OK;
 }

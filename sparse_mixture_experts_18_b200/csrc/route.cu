@@ -973,7 +973,9 @@ cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Wo
     return p.dt == 1 ? launch_route_small_t(p, static_cast<const __nv_bfloat16*>(x), Wg, w, s)
                      : launch_route_small_t(p, static_cast<const float*>(x), Wg, w, s);
   cudaError_t err;
-  if (p.dt == 1)
+  if (router_tc_applies(p))
+    err = launch_router_tc(p, x, Wg, w, s);
+  else if (p.dt == 1)
     err = launch_router_t(static_cast<const __nv_bfloat16*>(x), Wg, p.T, (int)p.d, p.n, p.K,
                           w.idx, w.gate, w.blk_counts, s);
   else

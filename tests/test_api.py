@@ -83,7 +83,10 @@ def test_plan_selection(L):
     assert rc == OK and small == 1 and s13 >= 1 and s2 >= 1 and launches == 5  # fused route
     assert pair == 0 and 4096 // 64 % s13 == 0 and 14336 // 64 % s2 == 0
     rc, (small, s13, s2, launches, pair) = _plan(L, 4096, 4096, 14336, 8, 2)
-    assert rc == OK and small == 0 and s13 == 1 and s2 == 1 and launches == 6 and pair == 1
+    # W_g split, tensor-core router, scan, permute, G13, G2, combine
+    assert rc == OK and small == 0 and s13 == 1 and s2 == 1 and launches == 7 and pair == 1
+    rc, (_, _, _, launches, _) = _plan(L, 512, 4096, 14336, 8, 2)   # CUDA-core router
+    assert rc == OK and launches == 6
     rc, (small, _, _, _, pair) = _plan(L, 1024, 4096, 14336, 8, 2)   # 128-row tiles
     assert rc == OK and small == 0 and pair == 0
     rc, (small, _, _, _, pair) = _plan(L, 64, 128, 256, 8, 2, F32)
