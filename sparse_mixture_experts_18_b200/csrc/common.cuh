@@ -304,6 +304,17 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
   return v;
 }
 
+// Four floats from shared memory of a CTA of this cluster (16-byte aligned address).  Issue
+// several of these back to back before using any: they complete in parallel.
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
 // Every thread of every CTA of the cluster: makes prior shared-memory writes (barrier
 // initialisation included) visible cluster-wide.
 __device__ __forceinline__ void cluster_sync_all() {

@@ -25,9 +25,11 @@ namespace moe {
 
 constexpr int RTC_THREADS = 192;
 constexpr int RTC_TILE = 128;         // tokens per tile (MMA M)
-constexpr int RTC_STAGES = 6;
+constexpr int RTC_MAX_STAGES = 12;
 constexpr int RTC_MAX_N = 16;         // experts
 constexpr int RTC_MAX_NPAD = 48;      // 3 * 16 accumulator columns
+constexpr int RTC_PSTRIDE = 52;       // floats per row of partial sums (16-byte rows)
+constexpr uint32_t RTC_SMEM_BUDGET = 200 * 1024;
 
 __host__ __device__ constexpr int rtc_npad(int n) { return (3 * n + 15) / 16 * 16; }
 
@@ -58,11 +60,11 @@ __global__ void __launch_bounds__(256)
 }
 
 struct RtcCtrl {
-  uint64_t full[RTC_STAGES];
-  uint64_t empty[RTC_STAGES];
+  uint64_t full[RTC_MAX_STAGES];
+  uint64_t empty[RTC_MAX_STAGES];
   uint64_t tfull;
   uint64_t mma_done;
-  uint32_t issued[RTC_STAGES];
+  uint32_t issued[RTC_MAX_STAGES];
   uint32_t tmem_slot;
   int abort;
 };
@@ -71,15 +73,18 @@ template <int CS>
 __global__ void __launch_bounds__(RTC_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmW, int64_t T, int n, int K,
-                     int npad, int kb_per_cta, int64_t nblk, int32_t* __restrict__ idx,
+                     int npad, int kb_per_cta, int stages, int64_t nblk,
+                     int32_t* __restrict__ idx,
                      float* __restrict__ gate, int32_t* __restrict__ blk_counts,
                      uint32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t a_bytes = RTC_TILE * 128, b_bytes = (uint32_t)npad * 128;
   const uint32_t stage_bytes = (a_bytes + b_bytes + 1023u) & ~1023u;
-  RtcCtrl* c = reinterpret_cast<RtcCtrl*>(smem + (size_t)RTC_STAGES * stage_bytes);
-  float* part = reinterpret_cast<float*>(c + 1);  // [RTC_TILE][RTC_MAX_NPAD + 1] partial sums
+  RtcCtrl* c = reinterpret_cast<RtcCtrl*>(smem + (size_t)stages * stage_bytes);
+  // [RTC_TILE][RTC_PSTRIDE] partial sums, 16-byte aligned rows
+  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(c) +
+                                         ((sizeof(RtcCtrl) + 15) & ~(size_t)15));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CS > 1 ? cluster_ctarank() : 0;
   const int64_t tile = blockIdx.x / CS;
@@ -87,7 +92,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
   const int kb0 = (int)rank * kb_per_cta;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < RTC_STAGES; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(&c->full[s], 1);
       mbar_init(&c->empty[s], 1);
       c->issued[s] = 0;
@@ -117,8 +122,8 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     if (lane == 0) {  // ------------------------------------------------ TMA producer
       const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
       for (int kb = 0; kb < kb_per_cta; ++kb) {
-        const int stage = kb % RTC_STAGES;
-        const uint32_t phase = (uint32_t)(kb / RTC_STAGES) & 1u;
+        const int stage = kb % stages;
+        const uint32_t phase = (uint32_t)(kb / stages) & 1u;
         if (!mbar_wait(&c->empty[stage], phase ^ 1u, status, &c->abort)) break;
         uint8_t* st = smem + (size_t)stage * stage_bytes;
         mbar_arrive_expect_tx(&c->full[stage], a_bytes + b_bytes);
@@ -128,7 +133,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         c->issued[stage] += 1;
       }
       if (c->abort)  // let every issued copy land before the shared memory goes away
-        for (int s = 0; s < RTC_STAGES; ++s)
+        for (int s = 0; s < stages; ++s)
           if (c->issued[s]) wait_short(&c->full[s], (c->issued[s] - 1u) & 1u);
     }
     __syncwarp();
@@ -137,8 +142,8 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
       const uint32_t idesc = umma_idesc_bf16(RTC_TILE, npad);
       bool ok = true;
       for (int kb = 0; kb < kb_per_cta && ok; ++kb) {
-        const int stage = kb % RTC_STAGES;
-        const uint32_t phase = (uint32_t)(kb / RTC_STAGES) & 1u;
+        const int stage = kb % stages;
+        const uint32_t phase = (uint32_t)(kb / stages) & 1u;
         if (!mbar_wait(&c->full[stage], phase, status, &c->abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sb = smem_u32(smem + (size_t)stage * stage_bytes);
@@ -159,7 +164,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     // this thread's token (TMEM lane / accumulator row r): its npad partial sums go to its
     // row of `part` (zeros if a wait ran out; the status word then reports it)
     const int q = warp & 3, r = q * 32 + lane;
-    float* mine = part + r * (RTC_MAX_NPAD + 1);
+    float4* mine = reinterpret_cast<float4*>(part + r * RTC_PSTRIDE);
     const bool ok = mbar_wait(&c->tfull, 0, status, &c->abort);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
@@ -168,16 +173,22 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
       tmem_ld32(tb, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) mine[i] = __uint_as_float(v[i]);
+      for (int i = 0; i < 8; ++i)
+        mine[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                              __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
       if (npad > 32) {
         uint32_t w16[16];
         tmem_ld16(tb + 32, w16);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) mine[32 + i] = __uint_as_float(w16[i]);
+        for (int i = 0; i < 4; ++i)
+          mine[8 + i] = make_float4(__uint_as_float(w16[4 * i]), __uint_as_float(w16[4 * i + 1]),
+                                    __uint_as_float(w16[4 * i + 2]),
+                                    __uint_as_float(w16[4 * i + 3]));
       }
     } else {
-      for (int i = 0; i < npad; ++i) mine[i] = 0.f;
+#pragma unroll
+      for (int i = 0; i < RTC_MAX_NPAD / 4; ++i) mine[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 
@@ -185,12 +196,26 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
   if (warp >= 2 && rank == 0) {
     const int q = warp & 3, r = q * 32 + lane;
     const int64_t t = t0 + r;
-    float* mine = part + r * (RTC_MAX_NPAD + 1);
-    if (CS > 1) {  // add the other CTAs' K ranges in rank order
+    float* mine = part + r * RTC_PSTRIDE;
+    if (CS > 1) {  // add the other CTAs' K ranges in rank order; a peer's row in one batch
+      float4* m4 = reinterpret_cast<float4*>(mine);
+      float4 sum[RTC_MAX_NPAD / 4];
+#pragma unroll
+      for (int i = 0; i < RTC_MAX_NPAD / 4; ++i) sum[i] = m4[i];
       for (uint32_t p = 1; p < (uint32_t)CS; ++p) {
         const uint32_t base = map_to_rank(mine, p);
-        for (int i = 0; i < npad; ++i) mine[i] += ld_cluster_f32(base + 4u * (uint32_t)i);
+        float4 t4[RTC_MAX_NPAD / 4];
+#pragma unroll
+        for (int i = 0; i < RTC_MAX_NPAD / 4; ++i)
+          if (4 * i < npad) t4[i] = ld_cluster_v4(base + 16u * (uint32_t)i);
+#pragma unroll
+        for (int i = 0; i < RTC_MAX_NPAD / 4; ++i)
+          if (4 * i < npad) {
+            sum[i].x += t4[i].x; sum[i].y += t4[i].y; sum[i].z += t4[i].z; sum[i].w += t4[i].w;
+          }
       }
+#pragma unroll
+      for (int i = 0; i < RTC_MAX_NPAD / 4; ++i) m4[i] = sum[i];
     }
     float l[RTC_MAX_N];
 #pragma unroll
@@ -263,8 +288,11 @@ template <int CS>
 static cudaError_t launch_rtc(const CUtensorMap& mx, const CUtensorMap& mw, const Plan& p,
                               int npad, int64_t tiles, const Workspace& w, cudaStream_t s) {
   const uint32_t stage_bytes = (uint32_t)((RTC_TILE * 128 + npad * 128 + 1023) / 1024 * 1024);
-  const size_t smem = (size_t)RTC_STAGES * stage_bytes + sizeof(RtcCtrl) +
-                      (size_t)RTC_TILE * (RTC_MAX_NPAD + 1) * 4 + 1024;
+  const size_t fixed = ((sizeof(RtcCtrl) + 15) & ~(size_t)15) +
+                       (size_t)RTC_TILE * RTC_PSTRIDE * 4 + 1024;
+  int stages = (int)((RTC_SMEM_BUDGET - fixed) / stage_bytes);
+  if (stages > RTC_MAX_STAGES) stages = RTC_MAX_STAGES;
+  const size_t smem = (size_t)stages * stage_bytes + fixed;
   auto kern = router_tc_kernel<CS>;
   static int configured = 0;
   if (configured < (int)smem) {
@@ -288,8 +316,8 @@ static cudaError_t launch_rtc(const CUtensorMap& mx, const CUtensorMap& mw, cons
   cfg.attrs = attr;
   cfg.numAttrs = CS > 1 ? 2 : 1;
   const int kb_per_cta = (int)(p.d / 64 / CS);
-  return cudaLaunchKernelEx(&cfg, kern, mx, mw, p.T, p.n, p.K, npad, kb_per_cta, p.nblk, w.idx,
-                            w.gate, w.blk_counts, w.status);
+  return cudaLaunchKernelEx(&cfg, kern, mx, mw, p.T, p.n, p.K, npad, kb_per_cta, stages, p.nblk,
+                            w.idx, w.gate, w.blk_counts, w.status);
 }
 
 cudaError_t launch_router_tc(const Plan& p, const void* x, const float* Wg, const Workspace& w,
@@ -306,14 +334,15 @@ cudaError_t launch_router_tc(const Plan& p, const void* x, const float* Wg, cons
   if (!make_map_bf16(&mx, x, (uint64_t)d, (uint64_t)p.T, RTC_TILE) ||
       !make_map_bf16(&mw, w.wparts, (uint64_t)d, (uint64_t)npad, (uint32_t)npad))
     return cudaErrorInvalidValue;
-  // cluster size: the smallest of 1, 2, 4 (dividing d / 64) that fills the SMs best
+  // cluster size c of 1, 2 or 4 (dividing d / 64) minimising the estimated time: waves of
+  // CTAs times (1/c of a tile's stream + a fixed cost per CTA of 0.15 of it)
   const int64_t tiles = (p.T + RTC_TILE - 1) / RTC_TILE;
   const int sms = num_sms();
   int cs = 1;
   double best = 1e30;
   for (int c = 1; c <= 4; c <<= 1) {
     if ((d / 64) % c) break;
-    const double t = (double)((tiles * c + sms - 1) / sms) / c;
+    const double t = (double)((tiles * c + sms - 1) / sms) * (1.0 / c + 0.15);
     if (t < best * 0.99) { best = t; cs = c; }
   }
   switch (cs) {
