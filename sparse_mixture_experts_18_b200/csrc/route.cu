@@ -2,14 +2,16 @@
 //
 //  router_topk:   l = x . W_g (fp32 accumulation), TopK (ties -> lower expert index) and
 //                 Softmax over the K kept logits ("Mixtral of Experts", method section,
-//                 equation G(x)); also a per-block expert histogram.
+//                 equation G(x)); also a per-block expert histogram.  Large bf16 batches
+//                 with n <= 16 take the tensor-core router of route_tc.cu instead.
 //  route_scan:    per-expert exclusive prefix over router blocks and the row offsets of each
 //                 expert's group (each group padded to `row_align` rows).
 //  permute:       stable placement of every (token, slot) in its expert's group, the
 //                 inverse map token -> row, and the gather of x rows into that order.  This
-//                 is how experts with zero gate are skipped (Indonesian news summary,
-//                 section on how the MoE layer is computed) while each expert sees a
-//                 variable number of tokens (same page, implementation notes).
+//                 is how experts with zero gate are skipped ("Mixtral 8x7B: Model Bahasa
+//                 Sparse Mixture of Experts", hada.io, section "Cara Komputasi Layer MoE")
+//                 while each expert sees a variable number of tokens (same page, section
+//                 "Implementasi dan Efisiensi Inferensi").
 #include <type_traits>
 
 #include "internal.h"
@@ -48,23 +50,12 @@ struct Vec8<float> {
   }
 };
 
-// Shared-memory copy of W_g for the persistent router: row j (n floats) starts at
-// j*n + 4*(j/8).  The skew of four floats per eight rows spreads the rows that the lanes of a
-// warp read together (eight rows apart) over all banks.
-__host__ __device__ __forceinline__ int wg_smem_index(int j, int n) { return j * n + 4 * (j >> 3); }
-__host__ __device__ __forceinline__ size_t wg_smem_bytes(int d, int n) {
-  return ((size_t)d * n + 4 * (size_t)(d >> 3)) * sizeof(float);
-}
-
 // Router, TopK and softmax of tokens [t0, t0 + ntok), ntok <= RT_TOK, by ROUTE_THREADS
 // threads (tid = 0..255).  Experts are taken eight at a time: each thread accumulates the
 // logits of the block's tokens for eight experts over its 8-element chunks of the hidden
 // dimension (so each W_g row segment is loaded once per RT_TOK tokens); lanes and then warps
 // are summed in a fixed order.  hist (shared, may be null) counts selections.
 constexpr int RT_TOK = 8;
-// W_g bytes up to which the large-batch router keeps it in shared memory (the rest of its
-// 227 KB holds the per-team sums and logits)
-constexpr int RT_SMEM_MAX = 176 * 1024;
 
 // w_vec: W_g rows are 16-byte aligned and n % 8 == 0 (eight experts per two float4 loads).
 template <typename Tin>
@@ -240,181 +231,6 @@ __device__ __forceinline__ void quantize_tokens_e4m3(const __nv_bfloat16* __rest
           dst[v0 + 32 * u] = make_uint2(
               e4m3x4(bf16_lo(t[u].x), bf16_hi(t[u].x), bf16_lo(t[u].y), bf16_hi(t[u].y), s),
               e4m3x4(bf16_lo(t[u].z), bf16_hi(t[u].z), bf16_lo(t[u].w), bf16_hi(t[u].w), s));
-    }
-  }
-}
-
-// Large batches whose router matrix fits in shared memory: one persistent CTA of 16 warps per
-// SM copies W_g once (skewed layout, wg_smem_index); then "teams" of S warps (S = 1 .. 16,
-// chosen by the host so that one wave of teams covers the token blocks) route token blocks
-// b = team, team + teams, ... independently of each other, with no CTA-wide barrier after
-// the copy.  The S warps of a team split the hidden dimension: warp w takes the 8-element
-// chunks c = 32 w + lane, 32 w + lane + 32 S, ...  Each lane accumulates the logits of the
-// block's tokens for eight experts at a time in fp32 (the eight experts as four packed pairs,
-// fma.rn.f32x2: two independent IEEE fmas per instruction, which halves the issue slots of
-// the multiply-adds), the 64 partial sums are reduce-scattered over the warp's lanes, the S
-// warps' sums are added in warp order by the team's first warp, which then runs TopK and the
-// softmax (one lane per token) and writes the block's expert histogram.  Outputs and their
-// layout are those of router_topk_kernel.
-constexpr int RW_THREADS = 512;
-
-__device__ __forceinline__ void ffma2(float2& acc, float a, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-      "mov.b64 ra, {%2, %2};\n\t"
-      "mov.b64 rb, {%3, %4};\n\t"
-      "mov.b64 rc, {%0, %1};\n\t"
-      "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
-      "mov.b64 {%0, %1}, rc;\n\t}"
-      : "+f"(acc.x), "+f"(acc.y)
-      : "f"(a), "f"(b0), "f"(b1));
-}
-
-template <int S>
-struct TeamSync {  // the S warps of one team: named barrier 1 + team (a warp barrier if S = 1)
-  int id;
-  __device__ __forceinline__ void operator()() const {
-    if (S == 1)
-      __syncwarp();
-    else
-      asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(32 * S) : "memory");
-  }
-};
-
-template <int S>
-__global__ void __launch_bounds__(RW_THREADS, 1)
-    router_team_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ Wg,
-                       int64_t T, int d, int n, int K, int tokb, int64_t nblk,
-                       int32_t* __restrict__ idx, float* __restrict__ gate,
-                       int32_t* __restrict__ blk_counts) {
-  constexpr int TEAMS = RW_THREADS / 32 / S;
-  extern __shared__ float4 wg_raw[];
-  float* sw = reinterpret_cast<float*>(wg_raw);
-  __shared__ float red[TEAMS][S][64];                 // each warp's 64 sums of one expert group
-  __shared__ float logits[TEAMS][RT_TOK][MAX_EXPERTS];
-  __shared__ int sel[TEAMS][64];                      // the block's K * ntok selections
-  // W_g rows as float4 quarters (n % 8 == 0), eight loads in flight per thread
-  const int q4 = n / 4, total4 = d * q4;
-  for (int i0 = threadIdx.x; i0 < total4; i0 += 8 * RW_THREADS) {
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (i0 + u * RW_THREADS < total4)
-        v[u] = __ldg(reinterpret_cast<const float4*>(Wg) + i0 + u * RW_THREADS);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * RW_THREADS;
-      if (i < total4)
-        *reinterpret_cast<float4*>(sw + wg_smem_index(i / q4, n) + 4 * (i % q4)) = v[u];
-    }
-  }
-  // W_g is the caller's; x and the outputs are ordered after the previous kernel
-  pdl_wait();
-  pdl_trigger();
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int team = warp / S, tw = warp % S;
-  const TeamSync<S> sync{1 + team};
-  const int nchunk = d / 8;
-  for (int64_t b = (int64_t)blockIdx.x * TEAMS + team; b < nblk; b += (int64_t)gridDim.x * TEAMS) {
-    const int64_t t0 = b * tokb;
-    const int ntok = (int)(T - t0 < tokb ? T - t0 : tokb);
-    for (int eg = 0; eg < n; eg += 8) {
-      float2 acc[RT_TOK][4];
-#pragma unroll
-      for (int a = 0; a < RT_TOK; ++a)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[a][e] = make_float2(0.f, 0.f);
-      for (int ci = tw * 32 + lane; ci < nchunk; ci += 32 * S) {
-        const int j0 = ci * 8;
-        Vec8<__nv_bfloat16> xv[RT_TOK];
-#pragma unroll
-        for (int a = 0; a < RT_TOK; ++a)
-          if (a < ntok) xv[a].load(x + (t0 + a) * (int64_t)d + j0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float* wr = sw + wg_smem_index(j0 + i, n) + eg;
-          const float4 w0 = *reinterpret_cast<const float4*>(wr);
-          const float4 w1 = *reinterpret_cast<const float4*>(wr + 4);
-#pragma unroll
-          for (int a = 0; a < RT_TOK; ++a) {
-            if (a < ntok) {
-              const float xa = xv[a].get(i);
-              ffma2(acc[a][0], xa, w0.x, w0.y);
-              ffma2(acc[a][1], xa, w0.z, w0.w);
-              ffma2(acc[a][2], xa, w1.x, w1.y);
-              ffma2(acc[a][3], xa, w1.z, w1.w);
-            }
-          }
-        }
-      }
-      // butterfly reduce-scatter of the 64 partial sums over the lanes (value a*8 + e)
-      float v[64];
-#pragma unroll
-      for (int a = 0; a < RT_TOK; ++a)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[a * 8 + 2 * e] = acc[a][e].x;
-          v[a * 8 + 2 * e + 1] = acc[a][e].y;
-        }
-      int base = 0;
-#pragma unroll
-      for (int half = 32, off = 16; off >= 1; half >>= 1, off >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float send = upper ? v[i] : v[half + i];
-          const float keep = upper ? v[half + i] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-        if (upper) base += half;
-      }
-      red[team][tw][base] = v[0];
-      red[team][tw][base + 1] = v[1];
-      sync();
-      if (tw == 0) {  // lane l: values 2l and 2l + 1, summed over the team's warps in order
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int vi = 2 * lane + h;
-          float sum = 0.f;
-#pragma unroll
-          for (int w = 0; w < S; ++w) sum += red[team][w][vi];
-          if (eg + (vi & 7) < n) logits[team][vi >> 3][eg + (vi & 7)] = sum;
-        }
-      }
-      sync();  // red is rewritten by the next expert group or block
-    }
-    if (tw == 0) {
-      __syncwarp();
-      // TopK by repeated arg-max (strict '>' keeps the lower index on ties), then Softmax
-      // over the kept logits shifted by the largest, summed in slot order; lane a = token a
-      if (lane < ntok) {
-        const float* l = logits[team][lane];
-        const int64_t t = t0 + lane;
-        uint64_t used = 0;
-        float top = 0.f, z = 0.f;
-        for (int k = 0; k < K; ++k) {
-          int best = -1;
-          float bv = 0.f;
-          for (int e = 0; e < n; ++e) {
-            if ((used >> e) & 1ull) continue;
-            if (best < 0 || l[e] > bv) { best = e; bv = l[e]; }
-          }
-          used |= 1ull << best;
-          if (k == 0) top = bv;
-          z += expf(bv - top);
-          sel[team][lane * K + k] = best;
-          idx[t * K + k] = best;
-        }
-        for (int k = 0; k < K; ++k)
-          gate[t * K + k] = expf(l[sel[team][lane * K + k]] - top) / z;
-      }
-      __syncwarp();
-      for (int e = lane; e < n; e += 32) {  // the block's histogram
-        int c = 0;
-        for (int i = 0; i < ntok * K; ++i) c += sel[team][i] == e;
-        blk_counts[b * n + e] = c;
-      }
-      __syncwarp();
     }
   }
 }
@@ -886,42 +702,6 @@ cudaError_t launch_ep_regroup(const Plan& p, const void* x_rows, const int32_t* 
 // (token, slot) entries stay within 64.
 int route_tokens_per_block(int K) { return K <= 8 ? RT_TOK : (64 / K > 0 ? 64 / K : 1); }
 
-// Warps per token block of router_team_kernel: the S (1 .. 16) that minimises the estimated
-// time ceil(nblk * S / warp slots) * (1/S + 0.1), i.e. rounds of a team's share of a block
-// plus a per-block cost of the cross-warp sums, barriers and TopK (0.1 of a block's work at
-// Mixtral's width); ties go to the smaller S.
-static int router_team_size(int64_t nblk, int sms, int d) {
-  const int64_t slots = (int64_t)sms * (RW_THREADS / 32);
-  int best = 1;
-  double best_t = 1e30;
-  for (int S = 1; S <= 16; S <<= 1) {
-    if (S > 1 && d / 8 < 32 * S) break;  // every warp of a team needs a chunk per lane
-    const double t = (double)((nblk * S + slots - 1) / slots) * (1.0 / S + 0.1);
-    if (t < best_t * 0.99) { best_t = t; best = S; }
-  }
-  return best;
-}
-
-template <int S>
-static cudaError_t launch_router_team(const __nv_bfloat16* x, const float* Wg, int64_t T, int d,
-                                      int n, int K, int tokb, int64_t nblk, size_t wbytes,
-                                      int sms, int32_t* idx, float* gate, int32_t* blk_counts,
-                                      cudaStream_t s) {
-  auto kern = router_team_kernel<S>;
-  static int configured = 0;  // per instantiation
-  if (configured < (int)wbytes) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wbytes);
-    if (e != cudaSuccess) return e;
-    configured = (int)wbytes;
-  }
-  constexpr int TEAMS = RW_THREADS / 32 / S;
-  const int64_t want = (nblk + TEAMS - 1) / TEAMS;
-  const unsigned grid = (unsigned)(want < sms ? want : sms);
-  pdl(kern, grid, RW_THREADS, wbytes, s)(x, Wg, T, d, n, K, tokb, nblk, idx, gate, blk_counts);
-  return cudaGetLastError();
-}
-
 template <typename Tin>
 static cudaError_t launch_router_t(const Tin* x, const float* Wg, int64_t T, int d, int n,
                                    int K, int32_t* idx, float* gate, int32_t* blk_counts,
@@ -929,26 +709,6 @@ static cudaError_t launch_router_t(const Tin* x, const float* Wg, int64_t T, int
   const int tokb = route_tokens_per_block(K);
   const int64_t nblk = (T + tokb - 1) / tokb;
   const bool w_vec = n % 8 == 0 && (reinterpret_cast<uintptr_t>(Wg) & 15u) == 0;
-  const size_t wbytes = wg_smem_bytes(d, n);
-  const int sms = num_sms();
-  // bf16 activations, W_g in shared memory, and enough token blocks to pay for copying W_g
-  // to every SM
-  if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
-    if (w_vec && wbytes <= (size_t)RT_SMEM_MAX && nblk >= (int64_t)sms) {
-      switch (router_team_size(nblk, sms, d)) {
-        case 1: return launch_router_team<1>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
-                                             gate, blk_counts, s);
-        case 2: return launch_router_team<2>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
-                                             gate, blk_counts, s);
-        case 4: return launch_router_team<4>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
-                                             gate, blk_counts, s);
-        case 8: return launch_router_team<8>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
-                                             gate, blk_counts, s);
-        default: return launch_router_team<16>(x, Wg, T, d, n, K, tokb, nblk, wbytes, sms, idx,
-                                               gate, blk_counts, s);
-      }
-    }
-  }
   pdl(router_topk_kernel<Tin>, (unsigned)nblk, ROUTE_THREADS, 0, s)(x, Wg, w_vec, T, d, n, K,
                                                                     tokb, idx, gate,
                                                                     blk_counts);

@@ -15,8 +15,7 @@
 //
 // One CTA per 128-token tile and K range: a cluster of CS CTAs (CS = 1, 2 or 4) splits the
 // hidden dimension, and the leader adds the others' partial sums in rank order through
-// distributed shared memory.  Each tile walks its K range from a staggered start (a fixed,
-// tile-dependent order of the fp32 sums).  Warp 0 streams x and the W_g parts with TMA (no multicast), one
+// distributed shared memory.  Warp 0 streams x and the W_g parts with TMA (no multicast), one
 // thread of warp 1 issues the MMAs, warps 2-5 read the accumulators (one token per thread) and
 // run TopK (ties to the lower index) and the softmax over the kept logits, and write the
 // token block histograms the scan kernel takes (8-token blocks, as router_topk_kernel).
@@ -122,17 +121,13 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {  // ------------------------------------------------ TMA producer
       const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
-      // tiles start at staggered K blocks, so that concurrent CTAs read different column
-      // windows of their rows rather than the same one
-      const int kb_first = (int)((tile * 7) % kb_per_cta);
       for (int kb = 0; kb < kb_per_cta; ++kb) {
         const int stage = kb % stages;
         const uint32_t phase = (uint32_t)(kb / stages) & 1u;
         if (!mbar_wait(&c->empty[stage], phase ^ 1u, status, &c->abort)) break;
         uint8_t* st = smem + (size_t)stage * stage_bytes;
         mbar_arrive_expect_tx(&c->full[stage], a_bytes + b_bytes);
-        const int kbs = kb + kb_first < kb_per_cta ? kb + kb_first : kb + kb_first - kb_per_cta;
-        const int k = (kb0 + kbs) * 64;
+        const int k = (kb0 + kb) * 64;
         tma_load_2d(st, &tmX, &c->full[stage], k, (int32_t)t0, pol_x);  // rows >= T: zeros
         tma_load_2d(st + a_bytes, &tmW, &c->full[stage], k, 0, pol_w);
         c->issued[stage] += 1;

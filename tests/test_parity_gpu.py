@@ -92,12 +92,13 @@ def test_all_tokens_to_two_experts_gather_x(monkeypatch, T):
     test_all_tokens_to_two_experts(T)
 
 
-@pytest.mark.parametrize("T", [1180, 1200, 2400, 2501])
-def test_router_team_sizes(T):
-    # Mixtral's hidden size with W_g in shared memory: the large-batch router splits each
-    # 8-token block over 16 (T = 1180), 8 (T = 1200) or 4 (T = 2400) warps, and T = 2501 ends
-    # in a ragged block; a narrow expert width keeps the oracle quick
-    _run(moe_inputs.small(T=T, d=4096, F=128), budget=300)
+@pytest.mark.parametrize("T,d,n,K", [(1024, 4096, 8, 2), (1100, 4096, 8, 2), (2501, 4096, 8, 2),
+                                     (1500, 256, 5, 2), (1300, 320, 12, 3), (1030, 512, 16, 8)])
+def test_router_tc_tiles(T, d, n, K):
+    # the tensor-core router (T >= 1024, n <= 16, K <= 8): an exact multiple of its 128-token
+    # tile, ragged last tiles, clusters of 4 splitting d, and accumulators of 16 (n = 5), 48
+    # (n = 12, 16) columns; a narrow expert width keeps the oracle quick
+    _run(moe_inputs.small(T=T, d=d, F=128, n=n, K=K), budget=300)
 
 
 @pytest.mark.parametrize("T", [1, 5, 16, 37, 100, 255])
