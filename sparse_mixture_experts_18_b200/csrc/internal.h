@@ -108,7 +108,7 @@ Workspace carve(const Plan& p, void* base);
 
 int route_tokens_per_block(int K);
 // The router of large batches on the tensor cores (route_tc.cu): taken for bf16, T >= 1024,
-// n <= 16, K <= 8; writes idx, gate and the 8-token block histograms like the CUDA-core
+// n <= 64, K <= 8; writes idx, gate and the 8-token block histograms like the CUDA-core
 // router.
 bool router_tc_applies(const Plan& p);
 size_t router_tc_parts_bytes(int64_t d, int n);

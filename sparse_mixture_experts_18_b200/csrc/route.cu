@@ -3,7 +3,7 @@
 //  router_topk:   l = x . W_g (fp32 accumulation), TopK (ties -> lower expert index) and
 //                 Softmax over the K kept logits ("Mixtral of Experts", method section,
 //                 equation G(x)); also a per-block expert histogram.  Large bf16 batches
-//                 with n <= 16 take the tensor-core router of route_tc.cu instead.
+//                 with n <= 64 take the tensor-core router of route_tc.cu instead.
 //  route_scan:    per-expert exclusive prefix over router blocks and the row offsets of each
 //                 expert's group (each group padded to `row_align` rows).
 //  permute:       stable placement of every (token, slot) in its expert's group, the

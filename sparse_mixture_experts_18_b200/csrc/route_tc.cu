@@ -26,12 +26,19 @@ namespace moe {
 constexpr int RTC_THREADS = 192;
 constexpr int RTC_TILE = 128;         // tokens per tile (MMA M)
 constexpr int RTC_MAX_STAGES = 12;
-constexpr int RTC_MAX_N = 16;         // experts
-constexpr int RTC_MAX_NPAD = 48;      // 3 * 16 accumulator columns
-constexpr int RTC_PSTRIDE = 52;       // floats per row of partial sums (16-byte rows)
+constexpr int RTC_MAX_N = 64;         // experts
+constexpr int RTC_MAX_NPAD = 192;     // 3 * 64 accumulator columns
+// one CTA per SM with as many stages in flight as shared memory holds (two CTAs per SM with
+// half the stages each measured slower)
 constexpr uint32_t RTC_SMEM_BUDGET = 200 * 1024;
 
 __host__ __device__ constexpr int rtc_npad(int n) { return (3 * n + 15) / 16 * 16; }
+// floats per row of partial sums: 16-byte rows, and four banks apart from row to row so that
+// the 16-byte accesses of eight consecutive rows fall in different banks
+__host__ __device__ constexpr int rtc_pstride(int npad) { return npad + 4; }
+__host__ __device__ constexpr uint32_t rtc_tmem_cols(int npad) {
+  return npad <= 32 ? 32 : npad <= 64 ? 64 : npad <= 128 ? 128 : 256;
+}
 
 // W_g [d][n] fp32 -> parts [npad][d] bf16: row e = hi of column e, n + e = mid, 2n + e = lo,
 // rows from 3n on are zero.
@@ -69,7 +76,8 @@ struct RtcCtrl {
   int abort;
 };
 
-template <int CS>
+// MAXN: 16 or 64, the most experts the instance handles (its TopK loops are unrolled to it)
+template <int CS, int MAXN>
 __global__ void __launch_bounds__(RTC_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmW, int64_t T, int n, int K,
@@ -82,9 +90,9 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
   const uint32_t a_bytes = RTC_TILE * 128, b_bytes = (uint32_t)npad * 128;
   const uint32_t stage_bytes = (a_bytes + b_bytes + 1023u) & ~1023u;
   RtcCtrl* c = reinterpret_cast<RtcCtrl*>(smem + (size_t)stages * stage_bytes);
-  // [RTC_TILE][RTC_PSTRIDE] partial sums, 16-byte aligned rows
-  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(c) +
-                                         ((sizeof(RtcCtrl) + 15) & ~(size_t)15));
+  // [RTC_TILE][pstride] partial sums, 16-byte aligned rows: in the stages' memory, which
+  // is idle once the accumulator is complete (every load issued has been consumed by then)
+  float* part = reinterpret_cast<float*>(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CS > 1 ? cluster_ctarank() : 0;
   const int64_t tile = blockIdx.x / CS;
@@ -106,7 +114,8 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
   }
-  const uint32_t tmem_cols = npad <= 32 ? 32 : 64;
+  const uint32_t tmem_cols = rtc_tmem_cols(npad);
+  const int pstride = rtc_pstride(npad);
   if (warp == 1) {
     tmem_alloc(&c->tmem_slot, tmem_cols);
     tmem_relinquish();
@@ -164,31 +173,34 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     // this thread's token (TMEM lane / accumulator row r): its npad partial sums go to its
     // row of `part` (zeros if a wait ran out; the status word then reports it)
     const int q = warp & 3, r = q * 32 + lane;
-    float4* mine = reinterpret_cast<float4*>(part + r * RTC_PSTRIDE);
+    float4* mine = reinterpret_cast<float4*>(part + r * pstride);
     const bool ok = mbar_wait(&c->tfull, 0, status, &c->abort);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
-      uint32_t v[32];
-      tmem_ld32(tb, v);
-      tmem_ld_wait();
+      for (int c0 = 0; c0 < npad; c0 += 32) {  // npad is a multiple of 16
+        if (c0 + 32 <= npad) {
+          uint32_t v[32];
+          tmem_ld32(tb + c0, v);
+          tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        mine[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                              __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-      if (npad > 32) {
-        uint32_t w16[16];
-        tmem_ld16(tb + 32, w16);
-        tmem_ld_wait();
+          for (int i = 0; i < 8; ++i)
+            mine[c0 / 4 + i] =
+                make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                            __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        } else {
+          uint32_t v[16];
+          tmem_ld16(tb + c0, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          mine[8 + i] = make_float4(__uint_as_float(w16[4 * i]), __uint_as_float(w16[4 * i + 1]),
-                                    __uint_as_float(w16[4 * i + 2]),
-                                    __uint_as_float(w16[4 * i + 3]));
+          for (int i = 0; i < 4; ++i)
+            mine[c0 / 4 + i] =
+                make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                            __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
       }
     } else {
-#pragma unroll
-      for (int i = 0; i < RTC_MAX_NPAD / 4; ++i) mine[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < npad / 4; ++i) mine[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 
@@ -196,37 +208,42 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
   if (warp >= 2 && rank == 0) {
     const int q = warp & 3, r = q * 32 + lane;
     const int64_t t = t0 + r;
-    float* mine = part + r * RTC_PSTRIDE;
-    if (CS > 1) {  // add the other CTAs' K ranges in rank order; a peer's row in one batch
+    float* mine = part + r * pstride;
+    if (CS > 1) {  // add the other CTAs' K ranges in rank order, 48 columns per batch of loads
       float4* m4 = reinterpret_cast<float4*>(mine);
-      float4 sum[RTC_MAX_NPAD / 4];
+      constexpr int CH = 12;  // float4 per batch
+      for (int c4 = 0; c4 < npad / 4; c4 += CH) {
+        float4 sum[CH];
 #pragma unroll
-      for (int i = 0; i < RTC_MAX_NPAD / 4; ++i) sum[i] = m4[i];
-      for (uint32_t p = 1; p < (uint32_t)CS; ++p) {
-        const uint32_t base = map_to_rank(mine, p);
-        float4 t4[RTC_MAX_NPAD / 4];
+        for (int i = 0; i < CH; ++i)
+          if (c4 + i < npad / 4) sum[i] = m4[c4 + i];
+        for (uint32_t p = 1; p < (uint32_t)CS; ++p) {
+          const uint32_t base = map_to_rank(mine, p) + 16u * (uint32_t)c4;
+          float4 t4[CH];
 #pragma unroll
-        for (int i = 0; i < RTC_MAX_NPAD / 4; ++i)
-          if (4 * i < npad) t4[i] = ld_cluster_v4(base + 16u * (uint32_t)i);
+          for (int i = 0; i < CH; ++i)
+            if (c4 + i < npad / 4) t4[i] = ld_cluster_v4(base + 16u * (uint32_t)i);
 #pragma unroll
-        for (int i = 0; i < RTC_MAX_NPAD / 4; ++i)
-          if (4 * i < npad) {
-            sum[i].x += t4[i].x; sum[i].y += t4[i].y; sum[i].z += t4[i].z; sum[i].w += t4[i].w;
-          }
+          for (int i = 0; i < CH; ++i)
+            if (c4 + i < npad / 4) {
+              sum[i].x += t4[i].x; sum[i].y += t4[i].y; sum[i].z += t4[i].z; sum[i].w += t4[i].w;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < CH; ++i)
+          if (c4 + i < npad / 4) m4[c4 + i] = sum[i];
       }
-#pragma unroll
-      for (int i = 0; i < RTC_MAX_NPAD / 4; ++i) m4[i] = sum[i];
     }
-    float l[RTC_MAX_N];
+    float l[MAXN];
 #pragma unroll
-    for (int e = 0; e < RTC_MAX_N; ++e)
+    for (int e = 0; e < MAXN; ++e)
       l[e] = e < n ? (mine[e] + mine[n + e]) + mine[2 * n + e] : -INFINITY;
     // TopK by repeated arg-max (strict '>' keeps the lower index on ties), then Softmax over
     // the kept logits shifted by the largest, summed in slot order
     int sel[8];
     float kept[8];
     const bool valid = t < T;
-    uint32_t used = 0;
+    uint64_t used = 0;
     float top = 0.f, z = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -236,11 +253,11 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
       float bv = -INFINITY;
       bool any = false;
 #pragma unroll
-      for (int e = 0; e < RTC_MAX_N; ++e) {
-        if (e >= n || ((used >> e) & 1u)) continue;
+      for (int e = 0; e < MAXN; ++e) {
+        if (e >= n || ((used >> e) & 1ull)) continue;
         if (!any || l[e] > bv) { best = e; bv = l[e]; any = true; }
       }
-      used |= 1u << best;
+      used |= 1ull << best;
       if (k == 0) top = bv;
       z += expf(bv - top);
       sel[k] = best;
@@ -284,16 +301,25 @@ bool router_tc_applies(const Plan& p) {
 
 size_t router_tc_parts_bytes(int64_t d, int n) { return (size_t)rtc_npad(n) * d * 2; }
 
-template <int CS>
-static cudaError_t launch_rtc(const CUtensorMap& mx, const CUtensorMap& mw, const Plan& p,
-                              int npad, int64_t tiles, const Workspace& w, cudaStream_t s) {
+// Pipeline stages and dynamic shared memory of the router for npad accumulator columns.
+static size_t rtc_smem(int npad, int* stages_out) {
   const uint32_t stage_bytes = (uint32_t)((RTC_TILE * 128 + npad * 128 + 1023) / 1024 * 1024);
-  const size_t fixed = ((sizeof(RtcCtrl) + 15) & ~(size_t)15) +
-                       (size_t)RTC_TILE * RTC_PSTRIDE * 4 + 1024;
+  const size_t fixed = sizeof(RtcCtrl) + 1024;
   int stages = (int)((RTC_SMEM_BUDGET - fixed) / stage_bytes);
   if (stages > RTC_MAX_STAGES) stages = RTC_MAX_STAGES;
-  const size_t smem = (size_t)stages * stage_bytes + fixed;
-  auto kern = router_tc_kernel<CS>;
+  if (stages < 2) stages = 2;
+  // the partial sums [RTC_TILE][pstride] reuse the stages' memory
+  while ((size_t)stages * stage_bytes < (size_t)RTC_TILE * rtc_pstride(npad) * 4) ++stages;
+  *stages_out = stages;
+  return (size_t)stages * stage_bytes + fixed;
+}
+
+template <int CS, int MAXN>
+static cudaError_t launch_rtc(const CUtensorMap& mx, const CUtensorMap& mw, const Plan& p,
+                              int npad, int64_t tiles, const Workspace& w, cudaStream_t s) {
+  int stages = 0;
+  const size_t smem = rtc_smem(npad, &stages);
+  auto kern = router_tc_kernel<CS, MAXN>;
   static int configured = 0;
   if (configured < (int)smem) {
     const cudaError_t e =
@@ -335,20 +361,30 @@ cudaError_t launch_router_tc(const Plan& p, const void* x, const float* Wg, cons
       !make_map_bf16(&mw, w.wparts, (uint64_t)d, (uint64_t)npad, (uint32_t)npad))
     return cudaErrorInvalidValue;
   // cluster size c of 1, 2 or 4 (dividing d / 64) minimising the estimated time: waves of
-  // CTAs times (1/c of a tile's stream + a fixed cost per CTA of 0.15 of it)
+  // CTAs (two per SM when their shared memory allows) times (1/c of a tile's stream + a fixed
+  // cost per CTA of 0.15 of it)
   const int64_t tiles = (p.T + RTC_TILE - 1) / RTC_TILE;
-  const int sms = num_sms();
+  int stages = 0;
+  const size_t smem = rtc_smem(npad, &stages);
+  const int64_t slots = (2 * (smem + 1024) <= 228 * 1024 ? 2 : 1) * (int64_t)num_sms();
   int cs = 1;
   double best = 1e30;
   for (int c = 1; c <= 4; c <<= 1) {
     if ((d / 64) % c) break;
-    const double t = (double)((tiles * c + sms - 1) / sms) * (1.0 / c + 0.15);
+    const double t = (double)((tiles * c + slots - 1) / slots) * (1.0 / c + 0.15);
     if (t < best * 0.99) { best = t; cs = c; }
   }
+  if (p.n <= 16) {
+    switch (cs) {
+      case 1: return launch_rtc<1, 16>(mx, mw, p, npad, tiles, w, s);
+      case 2: return launch_rtc<2, 16>(mx, mw, p, npad, tiles, w, s);
+      default: return launch_rtc<4, 16>(mx, mw, p, npad, tiles, w, s);
+    }
+  }
   switch (cs) {
-    case 1: return launch_rtc<1>(mx, mw, p, npad, tiles, w, s);
-    case 2: return launch_rtc<2>(mx, mw, p, npad, tiles, w, s);
-    default: return launch_rtc<4>(mx, mw, p, npad, tiles, w, s);
+    case 1: return launch_rtc<1, 64>(mx, mw, p, npad, tiles, w, s);
+    case 2: return launch_rtc<2, 64>(mx, mw, p, npad, tiles, w, s);
+    default: return launch_rtc<4, 64>(mx, mw, p, npad, tiles, w, s);
   }
 }
 

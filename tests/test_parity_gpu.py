@@ -93,11 +93,13 @@ def test_all_tokens_to_two_experts_gather_x(monkeypatch, T):
 
 
 @pytest.mark.parametrize("T,d,n,K", [(1024, 4096, 8, 2), (1100, 4096, 8, 2), (2501, 4096, 8, 2),
-                                     (1500, 256, 5, 2), (1300, 320, 12, 3), (1030, 512, 16, 8)])
+                                     (1500, 256, 5, 2), (1300, 320, 12, 3), (1030, 512, 16, 8),
+                                     (1100, 256, 32, 3), (1500, 512, 48, 2), (1024, 256, 64, 4)])
 def test_router_tc_tiles(T, d, n, K):
-    # the tensor-core router (T >= 1024, n <= 16, K <= 8): an exact multiple of its 128-token
-    # tile, ragged last tiles, clusters of 4 splitting d, and accumulators of 16 (n = 5), 48
-    # (n = 12, 16) columns; a narrow expert width keeps the oracle quick
+    # the tensor-core router (T >= 1024, n <= 64, K <= 8): an exact multiple of its 128-token
+    # tile, ragged last tiles, clusters splitting d (4 where d / 64 allows, 1 at d = 320), and
+    # accumulators of 16 (n = 5) to 192 (n = 64) columns; a narrow expert width keeps the
+    # oracle quick
     _run(moe_inputs.small(T=T, d=d, F=128, n=n, K=K), budget=300)
 
 
