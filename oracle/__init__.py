@@ -66,8 +66,12 @@ def lib():
         L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_code.restype = ctypes.c_uint8
         L.oracle_e4m3_code.argtypes = [ctypes.c_float]
-        L.oracle_quantize_rows_e4m3.restype = None
-        L.oracle_quantize_rows_e4m3.argtypes = [I64, I64, I32, P, P, P]
+        L.oracle_e8m0_value.restype = D
+        L.oracle_e8m0_value.argtypes = [ctypes.c_uint8]
+        L.oracle_mx_scale_code.restype = ctypes.c_uint8
+        L.oracle_mx_scale_code.argtypes = [P, I32]
+        L.oracle_quantize_mx_e4m3.restype = None
+        L.oracle_quantize_mx_e4m3.argtypes = [I64, I64, I32, P, P, P]
         L.oracle_moe_forward_fp8.restype = I32
         L.oracle_moe_forward_fp8.argtypes = [I64, I64, I64, I32, I32, P, P, P, P, P, P, P, P,
                                              I64, P, P, P, P]
@@ -256,22 +260,38 @@ def e4m3_code(v: float) -> int:
     return int(lib().oracle_e4m3_code(float(v)))
 
 
-def quantize_rows_e4m3(v):
-    """Per-row E4M3 quantisation of a [rows][cols] bf16/fp32 tensor: s = max|v| / 448 (1 for a
-    zero row), q = E4M3(v / s), both in binary32.  Returns (q uint8 [rows, cols], s f32)."""
+def e8m0_value(code: int) -> float:
+    """Value of an E8M0 scale code, 2^(code - 127) (NaN for 255)."""
+    return lib().oracle_e8m0_value(int(code) & 0xFF)
+
+
+def mx_scale_code(block) -> int:
+    """E8M0 code of the shared scale of one block of binary32 values:
+    floor(log2(max |v|)) - 8 + 127, clamped to [0, 254]; 127 for an all-zero block."""
+    v = np.ascontiguousarray(block, np.float32)
+    return int(lib().oracle_mx_scale_code(_ptr(v), len(v)))
+
+
+def quantize_mx_e4m3(v):
+    """MXFP8 quantisation of a [rows][cols] bf16/fp32 tensor (cols % 32 == 0): blocks of 32
+    along each row share an E8M0 scale X; codes = E4M3(v / X).  Returns (q uint8
+    [rows, cols], sf uint8 [rows, cols // 32]) with the scale codes in plain row order."""
     a, dt = _raw(v)
     a = a.reshape(-1, a.shape[-1])
     rows, cols = a.shape
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
     q = np.zeros((rows, cols), np.uint8)
-    sc = np.zeros(rows, np.float32)
-    lib().oracle_quantize_rows_e4m3(rows, cols, dt, _ptr(a), _ptr(q), _ptr(sc))
-    return q, sc
+    sf = np.zeros((rows, cols // 32), np.uint8)
+    lib().oracle_quantize_mx_e4m3(rows, cols, dt, _ptr(a), _ptr(q), _ptr(sf))
+    return q, sf
 
 
-def moe_forward_fp8(x, Wg, W1q, W3q, W2q, s1, s3, s2, n: int, K: int, tokens=None):
-    """Block output (unrounded, f64) with E4M3 expert weights and binary32 row scales for the
-    given token rows: W1q/W3q [n,F,d] and W2q [n,d,F] uint8 codes, s1/s3 [n,F], s2 [n,d].
-    Returns (y [len, d] f64, idx [len, K] i32, gate [len, K] f64)."""
+def moe_forward_fp8(x, Wg, W1q, W3q, W2q, sf1, sf3, sf2, n: int, K: int, tokens=None):
+    """Block output (unrounded, f64) with MXFP8 expert weights for the given token rows:
+    W1q/W3q [n,F,d] and W2q [n,d,F] uint8 E4M3 codes, sf1/sf3 [n,F,d//32] and sf2
+    [n,d,F//32] uint8 E8M0 block-scale codes.  Returns (y [len, d] f64, idx [len, K] i32,
+    gate [len, K] f64)."""
     xa, dt = _raw(x)
     if dt != BF16:
         raise TypeError("the FP8-weight block takes bf16 activations")
@@ -280,9 +300,11 @@ def moe_forward_fp8(x, Wg, W1q, W3q, W2q, s1, s3, s2, n: int, K: int, tokens=Non
     w3 = np.ascontiguousarray(W3q, np.uint8)
     w2 = np.ascontiguousarray(W2q, np.uint8)
     F = w1.shape[1]
-    a1 = np.ascontiguousarray(s1, np.float32)
-    a3 = np.ascontiguousarray(s3, np.float32)
-    a2 = np.ascontiguousarray(s2, np.float32)
+    a1 = np.ascontiguousarray(sf1, np.uint8)
+    a3 = np.ascontiguousarray(sf3, np.uint8)
+    a2 = np.ascontiguousarray(sf2, np.uint8)
+    if a1.size != n * F * d // 32 or a3.size != a1.size or a2.size != n * d * F // 32:
+        raise ValueError("block-scale arrays do not match the weights")
     tok = np.arange(T, dtype=np.int64) if tokens is None else np.asarray(tokens, np.int64)
     y = np.zeros((len(tok), d), np.float64)
     idx = np.zeros((len(tok), K), np.int32)

@@ -35,8 +35,9 @@
  *
  * Parity status: every function here is pinned by tests against closed forms, brute force
  * or library routines (see tests/test_oracle.py); none is "parity unpinned".  The FP8
- * functions at the end (E4M3 codes, row quantisation, the FP8-weight block) are pinned
- * against the format's defining values and torch's float8_e4m3fn conversion.
+ * functions at the end (E4M3 codes, E8M0 block scales, block quantisation, the FP8-weight
+ * block) are pinned against the formats' defining values, an independent numpy/torch
+ * restatement of the block-scale rule and torch's float8_e4m3fn conversion.
  */
 #include <math.h>
 #include <stdint.h>
@@ -335,20 +336,27 @@ int oracle_block_forward(int64_t rows, int64_t d, int64_t F, int n, int K, int d
 /* ---------------------------------------------------------------- FP8 expert weights
  *
  * The low-precision-weights variant (the pages mention only quantised community builds of
- * the model, so the format below is this library's own reading, the plainest one):
+ * the model, so the format below is this library's own reading: the OCP Microscaling (MX)
+ * format MXFP8 with E4M3 elements, which the sm_100a tensor cores scale in hardware):
  *   - OCP FP8 E4M3 ("fn" flavour): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
- *     no infinities, S.1111.111 is NaN, largest finite value 448, smallest subnormal 2^-9;
- *   - one binary32 scale per row of every weight matrix (W1, W3 rows f of [F][d], W2 rows i
- *     of [d][F]), per activation row (token) and per row of h:
- *       s = max_j |v_j| / 448  (s = 1 for an all-zero row),   q_j = E4M3(v_j / s)
- *     with E4M3 the nearest code, ties to the even mantissa, |v| > 448 clamped to 448;
- *     s and v_j / s are computed in binary32, as the kernels do, so that both sides decide
- *     the integer codes in the same precision;
- *   - a_f = s_x s1_f sum_j q_x,j q1_f,j and b_f likewise with W3 (the code products summed
- *     exactly, in double); h_f = silu(a_f) b_f rounded to binary32 and quantised per row
- *     (s_h, q_h); y_i = s_h s2_i sum_f q_h,f q2_i,f; out = sum_k G_k y_{e_k}, rounded once.
+ *     no infinities, S.1111.111 is NaN, largest finite value 448 = 1.75 * 2^8, smallest
+ *     subnormal 2^-9;
+ *   - every row of every matrix (W1, W3 rows f of [F][d]; W2 rows i of [d][F]; each token's
+ *     row of x; each row of h) is cut along its length into blocks of 32 consecutive
+ *     elements, and each block shares one scale X = 2^E, stored as an E8M0 code E + 127:
+ *       E = floor(log2(max_j |v_j|)) - 8   (8: the exponent of E4M3's largest normal),
+ *     clamped to [-127, 127]; an all-zero block takes E = 0;
+ *     element codes P_j = E4M3(v_j / X): the nearest code, ties to the even mantissa, values
+ *     above 448 (v_j / X can reach 512) clamped to 448 -- v_j / X is exact (X a power of two);
+ *   - a_f = sum over blocks b of X_x,b X_1,f,b sum_{j in b} P_x,j P_1,f,j (exact in double),
+ *     b_f likewise with W3; h_f = silu(a_f) b_f rounded to binary32 and block-quantised the
+ *     same way; y_i = sum_b X_h,b X_2,i,b sum_{f in b} P_h,f P_2,i,f;
+ *     out = sum_k G_k y_{e_k}, rounded once.
  *   Routing is the bf16 block's (the router reads the bf16 activations and fp32 W_g).
+ *   Scale codes are stored plainly here, [rows][cols / 32].
  */
+
+#define MX_BLOCK 32
 
 /* Value of an E4M3 code. */
 double oracle_e4m3_value(uint8_t c) {
@@ -374,28 +382,40 @@ uint8_t oracle_e4m3_code(float v) {
   return sign | (uint8_t)best;
 }
 
-/* Row scale in binary32: max |v| / 448, or 1 for an all-zero row. */
-static float e4m3_row_scale(const float* v, int64_t cols) {
+/* Value of an E8M0 scale code: 2^(c - 127); 255 is NaN. */
+double oracle_e8m0_value(uint8_t c) { return c == 255 ? NAN : ldexp(1.0, (int)c - 127); }
+
+/* E8M0 code of the shared scale of the block v[0..len). */
+uint8_t oracle_mx_scale_code(const float* v, int len) {
   float amax = 0.0f;
-  for (int64_t j = 0; j < cols; ++j) {
+  for (int j = 0; j < len; ++j) {
     const float a = fabsf(v[j]);
     if (a > amax) amax = a;
   }
-  return amax > 0.0f ? amax / 448.0f : 1.0f;
+  if (amax == 0.0f) return 127;
+  int ex;
+  frexp((double)amax, &ex);  /* amax = m * 2^ex with m in [0.5, 1): floor(log2 amax) = ex - 1 */
+  int E = ex - 1 - 8;
+  if (E < -127) E = -127;
+  if (E > 127) E = 127;
+  return (uint8_t)(E + 127);
 }
 
-static void e4m3_quantize_row(const float* v, int64_t cols, uint8_t* q, float* s) {
-  const volatile float sc = e4m3_row_scale(v, cols);
-  *s = sc;
-  for (int64_t j = 0; j < cols; ++j) {
-    const volatile float r = v[j] / sc;
-    q[j] = oracle_e4m3_code(r);
+/* One row of cols values (cols a multiple of 32): codes q[cols], scale codes sf[cols / 32]. */
+static void mx_quantize_row(const float* v, int64_t cols, uint8_t* q, uint8_t* sf) {
+  for (int64_t b = 0; b < cols / MX_BLOCK; ++b) {
+    const float* vb = v + b * MX_BLOCK;
+    const uint8_t c = oracle_mx_scale_code(vb, MX_BLOCK);
+    const double X = oracle_e8m0_value(c);
+    sf[b] = c;
+    for (int j = 0; j < MX_BLOCK; ++j) q[b * MX_BLOCK + j] = oracle_e4m3_code((float)(vb[j] / X));
   }
 }
 
-/* Per-row quantisation of a [rows][cols] matrix of dtype (bf16 or fp32) values. */
-void oracle_quantize_rows_e4m3(int64_t rows, int64_t cols, int dtype, const void* v,
-                               uint8_t* q, float* scales) {
+/* Block quantisation of a [rows][cols] matrix of dtype (bf16 or fp32) values; cols % 32 == 0.
+ * q [rows][cols] E4M3 codes, sf [rows][cols / 32] E8M0 codes. */
+void oracle_quantize_mx_e4m3(int64_t rows, int64_t cols, int dtype, const void* v, uint8_t* q,
+                             uint8_t* sf) {
 #pragma omp parallel
   {
     float* row = (float*)malloc(sizeof(float) * cols);
@@ -403,69 +423,75 @@ void oracle_quantize_rows_e4m3(int64_t rows, int64_t cols, int dtype, const void
     for (int64_t r = 0; r < rows; ++r) {
       if (!row) continue;
       for (int64_t j = 0; j < cols; ++j) row[j] = (float)elem(v, dtype, r * cols + j);
-      e4m3_quantize_row(row, cols, q + r * cols, scales + r);
+      mx_quantize_row(row, cols, q + r * cols, sf + r * (cols / MX_BLOCK));
     }
     free(row);
   }
 }
 
+/* sum over the blocks of (X_a,b X_w,b sum_{j in b} P_a,j P_w,j) for rows of len elements. */
+static double mx_dot(const uint8_t* qa, const uint8_t* sa, const uint8_t* qw, const uint8_t* sw,
+                     int64_t len, const double* lut) {
+  double total = 0.0;
+  for (int64_t b = 0; b < len / MX_BLOCK; ++b) {
+    double s = 0.0;
+    for (int j = 0; j < MX_BLOCK; ++j) s += lut[qa[b * MX_BLOCK + j]] * lut[qw[b * MX_BLOCK + j]];
+    total += oracle_e8m0_value(sa[b]) * oracle_e8m0_value(sw[b]) * s;
+  }
+  return total;
+}
+
 /* The block with FP8 expert weights for the tokens tok[0..n_tok): y[r][0..d) in double
- * (unrounded).  x bf16 [T][d]; W1q, W3q [n][F][d] and W2q [n][d][F] E4M3 codes; s1, s3
- * [n][F] and s2 [n][d] binary32 row scales. */
+ * (unrounded).  x bf16 [T][d]; W1q, W3q [n][F][d] and W2q [n][d][F] E4M3 codes; sf1, sf3
+ * [n][F][d / 32] and sf2 [n][d][F / 32] E8M0 block-scale codes.  d and F multiples of 32. */
 int oracle_moe_forward_fp8(int64_t T, int64_t d, int64_t F, int n, int K, const void* x,
                            const float* Wg, const uint8_t* W1q, const uint8_t* W3q,
-                           const uint8_t* W2q, const float* s1, const float* s3,
-                           const float* s2, int64_t n_tok, const int64_t* tok, double* y,
+                           const uint8_t* W2q, const uint8_t* sf1, const uint8_t* sf3,
+                           const uint8_t* sf2, int64_t n_tok, const int64_t* tok, double* y,
                            int32_t* idx_out, double* gate_out) {
-  if (n < 1 || n > 256 || K < 1 || K > n) return 1;
+  if (n < 1 || n > 256 || K < 1 || K > n || d % MX_BLOCK || F % MX_BLOCK) return 1;
   for (int64_t r = 0; r < n_tok; ++r) if (tok[r] < 0 || tok[r] >= T) return 2;
   double lut[256];
   for (int c = 0; c < 256; ++c) lut[c] = oracle_e4m3_value((uint8_t)c);
+  const int64_t bd = d / MX_BLOCK, bf = F / MX_BLOCK;
   int fail = 0;
 #pragma omp parallel
   {
     float* xf = (float*)malloc(sizeof(float) * d);
     uint8_t* qx = (uint8_t*)malloc(d);
+    uint8_t* sx = (uint8_t*)malloc(bd);
     float* hf = (float*)malloc(sizeof(float) * F);
     uint8_t* qh = (uint8_t*)malloc(F);
-    if (!xf || !qx || !hf || !qh) {
+    uint8_t* sh = (uint8_t*)malloc(bf);
+    const int ok = xf && qx && sx && hf && qh && sh;
+    if (!ok) {
 #pragma omp atomic write
       fail = 1;
     }
 #pragma omp for schedule(dynamic, 1)
     for (int64_t r = 0; r < n_tok; ++r) {
-      if (!xf || !qx || !hf || !qh) continue;
+      if (!ok) continue;
       const int64_t t = tok[r];
       double l[256], gate[256];
       int32_t idx[256];
       router_logits(d, n, ORACLE_BF16, x, t, Wg, l);
       topk_softmax(n, K, l, idx, gate);
       for (int64_t j = 0; j < d; ++j) xf[j] = (float)elem(x, ORACLE_BF16, t * d + j);
-      float sx;
-      e4m3_quantize_row(xf, d, qx, &sx);
+      mx_quantize_row(xf, d, qx, sx);
       double* yr = y + r * d;
       for (int64_t i = 0; i < d; ++i) yr[i] = 0.0;
       for (int k = 0; k < K; ++k) {
         const int e = idx[k];
         for (int64_t f = 0; f < F; ++f) {
-          const uint8_t* w1 = W1q + ((int64_t)e * F + f) * d;
-          const uint8_t* w3 = W3q + ((int64_t)e * F + f) * d;
-          double sa = 0.0, sb = 0.0;
-          for (int64_t j = 0; j < d; ++j) {
-            sa += lut[qx[j]] * lut[w1[j]];
-            sb += lut[qx[j]] * lut[w3[j]];
-          }
-          const double a = (double)sx * (double)s1[(int64_t)e * F + f] * sa;
-          const double b = (double)sx * (double)s3[(int64_t)e * F + f] * sb;
+          const int64_t wr = (int64_t)e * F + f;
+          const double a = mx_dot(qx, sx, W1q + wr * d, sf1 + wr * bd, d, lut);
+          const double b = mx_dot(qx, sx, W3q + wr * d, sf3 + wr * bd, d, lut);
           hf[f] = (float)(oracle_silu(a) * b);
         }
-        float sh;
-        e4m3_quantize_row(hf, F, qh, &sh);
+        mx_quantize_row(hf, F, qh, sh);
         for (int64_t i = 0; i < d; ++i) {
-          const uint8_t* w2 = W2q + ((int64_t)e * d + i) * F;
-          double sy = 0.0;
-          for (int64_t f = 0; f < F; ++f) sy += lut[qh[f]] * lut[w2[f]];
-          yr[i] += gate[k] * ((double)sh * (double)s2[(int64_t)e * d + i] * sy);
+          const int64_t wr = (int64_t)e * d + i;
+          yr[i] += gate[k] * mx_dot(qh, sh, W2q + wr * F, sf2 + wr * bf, F, lut);
         }
       }
       for (int k = 0; k < K; ++k) {
@@ -475,8 +501,10 @@ int oracle_moe_forward_fp8(int64_t T, int64_t d, int64_t F, int n, int K, const 
     }
     free(xf);
     free(qx);
+    free(sx);
     free(hf);
     free(qh);
+    free(sh);
   }
   return fail ? 3 : 0;
 }

@@ -331,31 +331,84 @@ def test_e4m3_rounding_matches_torch(oracle_lib):
     assert np.array_equal(ours, _e4m3_codes_torch(pts).numpy())
 
 
-def test_quantize_rows_e4m3(oracle_lib):
-    # s = max|v| / 448 in binary32, codes = E4M3(v / s): the largest element maps to +-448,
-    # an all-zero row gets s = 1 and zero codes, and codes match torch's conversion of v / s
+def _mx_exponent_by_search(amax: float) -> int:
+    """The block exponent from its defining inequality 2^(E + 8) <= amax < 2^(E + 9) (the
+    largest element lands in [256, 512) once divided by 2^E), found by stepping E; clamped
+    to [-127, 127]; 0 for an all-zero block."""
+    if amax == 0.0:
+        return 0
+    E = int(math.floor(math.log2(amax))) - 8
+    while 2.0 ** (E + 8) > amax:
+        E -= 1
+    while 2.0 ** (E + 9) <= amax:
+        E += 1
+    return max(-127, min(127, E))
+
+
+def _mx_quantize_ref(v: torch.Tensor):
+    """MXFP8 block quantisation by library steps: the exponent by search, the element codes by
+    torch's float8_e4m3fn conversion of v / 2^E clamped to +-448.  v float32 [rows, cols]."""
+    rows, cols = v.shape
+    blocks = v.reshape(rows, cols // 32, 32)
+    amax = blocks.abs().amax(dim=2).double().numpy()
+    E = np.vectorize(_mx_exponent_by_search, otypes=[np.int64])(amax)
+    X = torch.from_numpy(np.ldexp(1.0, E))
+    scaled = (blocks.double() / X[..., None]).clamp(-448.0, 448.0).float()
+    q = _e4m3_codes_torch(scaled).reshape(rows, cols)
+    return q.numpy(), (E + 127).astype(np.uint8)
+
+
+def test_e8m0_and_block_scale_closed_forms(oracle_lib):
+    assert oracle_lib.e8m0_value(127) == 1.0 and oracle_lib.e8m0_value(0) == 2.0 ** -127
+    assert oracle_lib.e8m0_value(254) == 2.0 ** 127 and math.isnan(oracle_lib.e8m0_value(255))
+    code = lambda v: oracle_lib.mx_scale_code(np.array(v, np.float32))
+    assert code([1.0] + [0.0] * 31) == 127 - 8          # max 1 -> X = 2^-8, 1 / X = 256
+    assert code([0.5, -1.999]) == 127 - 8               # floor(log2 1.999) = 0
+    assert code([-2.0, 1.0]) == 127 - 7                 # exactly 2: exponent 1
+    assert code([448.0, 3.0]) == 127                    # 448 = 1.75 * 2^8 -> X = 1
+    assert code([0.0] * 32) == 127                      # all-zero block: X = 1
+    assert code([2.0 ** -140, 0.0]) == 0                # clamped at 2^-127 (subnormal max)
+    assert code([3.0e38]) == 127 + 127 - 8              # floor(log2 3e38) = 127
+
+
+def test_quantize_mx_e4m3(oracle_lib):
+    # every block: the largest element divided by X lies in [256, 512), so its code is >= 256
+    # in value (448 when it saturates); codes match torch's conversion of v / X; the
+    # exponents match the search on the defining inequality; all-zero blocks read X = 1
     g = torch.Generator().manual_seed(11)
-    v = (torch.randn(6, 300, generator=g) * torch.tensor([1e-3, 1, 3, 50, 1e3, 0])[:, None]
-         ).to(torch.bfloat16)
-    q, s = oracle_lib.quantize_rows_e4m3(v)
-    vf = v.float()
-    amax = vf.abs().amax(dim=1)
-    assert s[5] == 1.0 and np.all((q[5] & 0x7F) == 0)  # signed zeros keep their sign
-    np.testing.assert_array_equal(s[:5], (amax[:5] / 448.0).numpy())
-    for r in range(5):
-        ref = _e4m3_codes_torch(vf[r] / torch.tensor(s[r])).numpy()
-        assert np.array_equal(q[r], ref)
-        j = int(vf[r].abs().argmax())
-        assert abs(oracle_lib.e4m3_value(int(q[r, j]))) == 448.0
+    scale = torch.tensor([1e-3, 1, 3, 50, 1e3, 0, 2.0 ** -130, 1e30])[:, None]
+    v = (torch.randn(8, 256, generator=g) * scale).to(torch.bfloat16).float()
+    v[1, :32] = torch.linspace(-1, 1, 32)             # exact power-of-two maximum
+    v[2, 32:64] = 0.0                                 # one zero block inside a row
+    q, sf = oracle_lib.quantize_mx_e4m3(v)
+    qr, sfr = _mx_quantize_ref(v)
+    np.testing.assert_array_equal(sf, sfr)
+    np.testing.assert_array_equal(q, qr)
+    X = np.ldexp(1.0, sf.astype(np.int64) - 127)
+    blocks = v.double().numpy().reshape(8, 8, 32)
+    amax = np.abs(blocks).max(axis=2)
+    nz = amax > 0
+    free = nz & (sf > 0)                 # exponent not clamped at -127 (row 6: below 2^-119)
+    assert np.all((amax / X)[free] >= 256) and np.all((amax / X)[free] < 512)
+    assert np.all(sf[nz & ~free] == 0) and np.all((amax / X)[nz & ~free] < 256)
+    assert np.all(sf[~nz] == 127)
+    deq = np.array([[oracle_lib.e4m3_value(int(c)) for c in row] for row in q]).reshape(8, 8, 32)
+    deq = deq * X[..., None]
+    # dequantised error: half a unit in the last place of E4M3 (relative 2^-4 in the normal
+    # range, 2^-10 X below it), or saturation at 448 X
+    tol = np.maximum(np.abs(blocks) * 2.0 ** -4, X[..., None] * 2.0 ** -10)
+    sat = np.abs(blocks) / X[..., None] > 448
+    assert np.all(np.abs(deq - blocks)[~sat] <= tol[~sat])
+    assert np.all(np.abs(deq[sat]) == 448 * np.broadcast_to(X[..., None], deq.shape)[sat])
 
 
 def _fp8_layer(T, d, F, n, seed):
     x, Wg, W1, W3, W2 = _layer(T, d, F, n, seed=seed, dtype=torch.bfloat16)
-    W1q, s1 = oracle_lib_module().quantize_rows_e4m3(W1.reshape(n * F, d))
-    W3q, s3 = oracle_lib_module().quantize_rows_e4m3(W3.reshape(n * F, d))
-    W2q, s2 = oracle_lib_module().quantize_rows_e4m3(W2.reshape(n * d, F))
+    W1q, s1 = oracle_lib_module().quantize_mx_e4m3(W1.reshape(n * F, d))
+    W3q, s3 = oracle_lib_module().quantize_mx_e4m3(W3.reshape(n * F, d))
+    W2q, s2 = oracle_lib_module().quantize_mx_e4m3(W2.reshape(n * d, F))
     return (x, Wg, W1q.reshape(n, F, d), W3q.reshape(n, F, d), W2q.reshape(n, d, F),
-            s1.reshape(n, F), s3.reshape(n, F), s2.reshape(n, d))
+            s1.reshape(n, F, d // 32), s3.reshape(n, F, d // 32), s2.reshape(n, d, F // 32))
 
 
 def oracle_lib_module():
@@ -363,28 +416,32 @@ def oracle_lib_module():
     return oracle
 
 
+def _dequant(q, sf):
+    """float64 values of E4M3 codes q [..., cols] with E8M0 block scales sf [..., cols / 32]."""
+    v = torch.from_numpy(np.ascontiguousarray(q)).view(E4M3).to(torch.float64)
+    X = torch.from_numpy(np.ldexp(1.0, sf.astype(np.int64) - 127))
+    return (v.reshape(*sf.shape, 32) * X[..., None]).reshape(v.shape)
+
+
 def _fp8_reference_torch(x, Wg, W1q, W3q, W2q, s1, s3, s2, K):
-    """The FP8-weight block from torch library steps: float8_e4m3fn conversions for every
-    quantisation, float64 matmuls for the code products."""
+    """The MXFP8 block from torch library steps: float64 matmuls on dequantised codes, x and h
+    block-quantised by the search-based reference quantiser."""
     T, d = x.shape
-    xf = x.float()
-    sx = xf.abs().amax(dim=1) / 448.0
-    xq = (xf / sx[:, None]).to(E4M3).to(torch.float64)
+    xq, xs = _mx_quantize_ref(x.float())
+    xd = _dequant(xq, xs)
     l = x.double() @ Wg.double()
     top = torch.topk(l, K, dim=1)
     G = torch.softmax(top.values, dim=1)
-    val = lambda q: torch.from_numpy(q).view(E4M3).to(torch.float64)
+    W1d, W3d, W2d = _dequant(W1q, s1), _dequant(W3q, s3), _dequant(W2q, s2)
     y = torch.zeros(T, d, dtype=torch.float64)
     for t in range(T):
         for k in range(K):
             e = int(top.indices[t, k])
-            a = sx[t].double() * torch.from_numpy(s1[e]).double() * (val(W1q[e]) @ xq[t])
-            b = sx[t].double() * torch.from_numpy(s3[e]).double() * (val(W3q[e]) @ xq[t])
+            a = W1d[e] @ xd[t]
+            b = W3d[e] @ xd[t]
             h = (torch.nn.functional.silu(a) * b).float()
-            sh = h.abs().amax() / 448.0
-            hq = (h / sh).to(E4M3).to(torch.float64)
-            y[t] += G[t, k] * (sh.double() * torch.from_numpy(s2[e]).double() *
-                               (val(W2q[e]) @ hq))
+            hq, hs = _mx_quantize_ref(h[None, :])
+            y[t] += G[t, k] * (W2d[e] @ _dequant(hq, hs)[0])
     return y.numpy(), top.indices.numpy()
 
 
@@ -398,12 +455,12 @@ def test_fp8_block_matches_library_reference(oracle_lib):
 
 
 def test_fp8_block_routing_and_scale_linearity(oracle_lib):
-    # routing is the bf16 block's, and y is linear in the W2 row scales: doubling s2 (a power
-    # of two) doubles y bit for bit
+    # routing is the bf16 block's, and y is linear in the W2 block scales: one more in every
+    # W2 scale code (X doubled) doubles y bit for bit
     T, d, F, n, K = 5, 64, 64, 8, 2
     x, Wg, W1q, W3q, W2q, s1, s3, s2 = _fp8_layer(T, d, F, n, seed=81)
     y, idx, gate = oracle_lib.moe_forward_fp8(x, Wg, W1q, W3q, W2q, s1, s3, s2, n, K)
     _, ridx, rgate = oracle_lib.route(x, Wg, n, K)
     assert np.array_equal(idx, ridx) and np.array_equal(gate, rgate)
-    y2, _, _ = oracle_lib.moe_forward_fp8(x, Wg, W1q, W3q, W2q, s1, s3, 2 * s2, n, K)
+    y2, _, _ = oracle_lib.moe_forward_fp8(x, Wg, W1q, W3q, W2q, s1, s3, s2 + 1, n, K)
     assert np.array_equal(y2, 2 * y)

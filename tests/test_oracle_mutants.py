@@ -33,15 +33,20 @@ MUTANTS = [
     ("rmsnorm_eps_dropped", "1.0 / sqrt(ss / (double)d + eps);", "1.0 / sqrt(ss / (double)d);"),
     ("residual_dropped", "round_to(x[r * d + i] + yr[i], dtype);", "round_to(yr[i], dtype);"),
     ("e4m3_ties_to_odd", "(dist == bd && (c & 1) == 0)", "(dist == bd && (c & 1) == 1)"),
-    ("e4m3_wrong_max", "return amax > 0.0f ? amax / 448.0f : 1.0f;",
-     "return amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    ("mx_emax_off_by_one", "int E = ex - 1 - 8;", "int E = ex - 1 - 7;"),
+    ("mx_ceil_not_floor", "int E = ex - 1 - 8;", "int E = ex - 8;"),
+    ("mx_low_clamp_dropped", "if (E < -127) E = -127;", "if (E < -200) E = -127;"),
+    ("mx_zero_block_scale", "if (amax == 0.0f) return 127;", "if (amax == 0.0f) return 0;"),
+    ("mx_overflow_to_nan", "if (a >= 448.0) return sign | 126;", "if (a > 464.0) return sign | 127;"),
     ("e4m3_subnormal_step", "ldexp((double)m, -9)", "ldexp((double)m, -10)"),
-    ("fp8_x_scale_dropped", "const double a = (double)sx * (double)s1[(int64_t)e * F + f] * sa;",
-     "const double a = (double)s1[(int64_t)e * F + f] * sa;"),
-    ("fp8_h_scale_dropped",
-     "yr[i] += gate[k] * ((double)sh * (double)s2[(int64_t)e * d + i] * sy);",
-     "yr[i] += gate[k] * ((double)s2[(int64_t)e * d + i] * sy);"),
-    ("fp8_w3_uses_w1", "sb += lut[qx[j]] * lut[w3[j]];", "sb += lut[qx[j]] * lut[w1[j]];"),
+    ("fp8_activation_scale_dropped",
+     "total += oracle_e8m0_value(sa[b]) * oracle_e8m0_value(sw[b]) * s;",
+     "total += oracle_e8m0_value(sw[b]) * s;"),
+    ("fp8_w3_uses_w1",
+     "const double b = mx_dot(qx, sx, W3q + wr * d, sf3 + wr * bd, d, lut);",
+     "const double b = mx_dot(qx, sx, W1q + wr * d, sf1 + wr * bd, d, lut);"),
+    ("fp8_h_block_scales_shifted", "mx_quantize_row(hf, F, qh, sh);",
+     "mx_quantize_row(hf, F, qh, sh); sh[0] = sh[bf - 1];"),
 ]
 
 
