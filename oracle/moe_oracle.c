@@ -344,10 +344,14 @@ int oracle_block_forward(int64_t rows, int64_t d, int64_t F, int n, int K, int d
  *   - every row of every matrix (W1, W3 rows f of [F][d]; W2 rows i of [d][F]; each token's
  *     row of x; each row of h) is cut along its length into blocks of 32 consecutive
  *     elements, and each block shares one scale X = 2^E, stored as an E8M0 code E + 127:
- *       E = floor(log2(max_j |v_j|)) - 8   (8: the exponent of E4M3's largest normal),
- *     clamped to [-127, 127]; an all-zero block takes E = 0;
- *     element codes P_j = E4M3(v_j / X): the nearest code, ties to the even mantissa, values
- *     above 448 (v_j / X can reach 512) clamped to 448 -- v_j / X is exact (X a power of two);
+ *     E is the smallest integer with max_j |v_j| <= 448 * 2^E, so that no element of the
+ *     block overflows E4M3's largest finite value (with max |v| = m 2^e, 1 <= m < 2:
+ *     E = e - 8 if m <= 1.75, else e - 7), clamped to [-127, 127]; an all-zero block takes
+ *     E = 0.  (The OCP text's E = floor(log2 max |v|) - 8 would clip block maxima in
+ *     [448, 512) X to 448.)
+ *     element codes P_j = E4M3(v_j / X): the nearest code, ties to the even mantissa (values
+ *     past 448, only possible when E was clamped, saturate) -- v_j / X is exact (X a power
+ *     of two);
  *   - a_f = sum over blocks b of X_x,b X_1,f,b sum_{j in b} P_x,j P_1,f,j (exact in double),
  *     b_f likewise with W3; h_f = silu(a_f) b_f rounded to binary32 and block-quantised the
  *     same way; y_i = sum_b X_h,b X_2,i,b sum_{f in b} P_h,f P_2,i,f;
@@ -394,8 +398,9 @@ uint8_t oracle_mx_scale_code(const float* v, int len) {
   }
   if (amax == 0.0f) return 127;
   int ex;
-  frexp((double)amax, &ex);  /* amax = m * 2^ex with m in [0.5, 1): floor(log2 amax) = ex - 1 */
-  int E = ex - 1 - 8;
+  const double f = frexp((double)amax, &ex);  /* amax = f 2^ex, f in [0.5, 1) */
+  /* amax <= 448 2^E = 0.875 2^(E + 9): the smallest such E */
+  int E = f <= 0.875 ? ex - 9 : ex - 8;
   if (E < -127) E = -127;
   if (E > 127) E = 127;
   return (uint8_t)(E + 127);

@@ -332,16 +332,16 @@ def test_e4m3_rounding_matches_torch(oracle_lib):
 
 
 def _mx_exponent_by_search(amax: float) -> int:
-    """The block exponent from its defining inequality 2^(E + 8) <= amax < 2^(E + 9) (the
-    largest element lands in [256, 512) once divided by 2^E), found by stepping E; clamped
-    to [-127, 127]; 0 for an all-zero block."""
+    """The block exponent from its definition, the smallest E with amax <= 448 2^E (no element
+    overflows E4M3 once divided by 2^E), found by stepping E; clamped to [-127, 127]; 0 for an
+    all-zero block."""
     if amax == 0.0:
         return 0
     E = int(math.floor(math.log2(amax))) - 8
-    while 2.0 ** (E + 8) > amax:
-        E -= 1
-    while 2.0 ** (E + 9) <= amax:
+    while 448.0 * 2.0 ** E < amax:
         E += 1
+    while 448.0 * 2.0 ** (E - 1) >= amax:
+        E -= 1
     return max(-127, min(127, E))
 
 
@@ -363,18 +363,20 @@ def test_e8m0_and_block_scale_closed_forms(oracle_lib):
     assert oracle_lib.e8m0_value(254) == 2.0 ** 127 and math.isnan(oracle_lib.e8m0_value(255))
     code = lambda v: oracle_lib.mx_scale_code(np.array(v, np.float32))
     assert code([1.0] + [0.0] * 31) == 127 - 8          # max 1 -> X = 2^-8, 1 / X = 256
-    assert code([0.5, -1.999]) == 127 - 8               # floor(log2 1.999) = 0
-    assert code([-2.0, 1.0]) == 127 - 7                 # exactly 2: exponent 1
+    assert code([0.5, -1.75]) == 127 - 8                # 1.75 / 2^-8 = 448 still fits
+    assert code([0.5, -1.7500001]) == 127 - 7           # just above: one binade up
+    assert code([-2.0, 1.0]) == 127 - 7                 # 2 / 2^-7 = 256
     assert code([448.0, 3.0]) == 127                    # 448 = 1.75 * 2^8 -> X = 1
+    assert code([449.0]) == 128                         # 449 > 448: X = 2
     assert code([0.0] * 32) == 127                      # all-zero block: X = 1
     assert code([2.0 ** -140, 0.0]) == 0                # clamped at 2^-127 (subnormal max)
-    assert code([3.0e38]) == 127 + 127 - 8              # floor(log2 3e38) = 127
+    assert code([3.0e38]) == 127 + 127 - 8 + 1          # 3e38 = 1.76 * 2^127 > 1.75 * 2^127
 
 
 def test_quantize_mx_e4m3(oracle_lib):
-    # every block: the largest element divided by X lies in [256, 512), so its code is >= 256
-    # in value (448 when it saturates); codes match torch's conversion of v / X; the
-    # exponents match the search on the defining inequality; all-zero blocks read X = 1
+    # every block: the largest element divided by X lies in (224, 448], so no code saturates;
+    # codes match torch's conversion of v / X; the exponents match the search on the defining
+    # inequality; all-zero blocks read X = 1
     g = torch.Generator().manual_seed(11)
     scale = torch.tensor([1e-3, 1, 3, 50, 1e3, 0, 2.0 ** -130, 1e30])[:, None]
     v = (torch.randn(8, 256, generator=g) * scale).to(torch.bfloat16).float()
@@ -389,17 +391,16 @@ def test_quantize_mx_e4m3(oracle_lib):
     amax = np.abs(blocks).max(axis=2)
     nz = amax > 0
     free = nz & (sf > 0)                 # exponent not clamped at -127 (row 6: below 2^-119)
-    assert np.all((amax / X)[free] >= 256) and np.all((amax / X)[free] < 512)
-    assert np.all(sf[nz & ~free] == 0) and np.all((amax / X)[nz & ~free] < 256)
+    assert np.all((amax / X)[free] > 224) and np.all((amax / X)[free] <= 448)
+    assert np.all(sf[nz & ~free] == 0) and np.all((amax / X)[nz & ~free] <= 224)
     assert np.all(sf[~nz] == 127)
     deq = np.array([[oracle_lib.e4m3_value(int(c)) for c in row] for row in q]).reshape(8, 8, 32)
     deq = deq * X[..., None]
     # dequantised error: half a unit in the last place of E4M3 (relative 2^-4 in the normal
-    # range, 2^-10 X below it), or saturation at 448 X
+    # range, 2^-10 X below it); nothing saturates
     tol = np.maximum(np.abs(blocks) * 2.0 ** -4, X[..., None] * 2.0 ** -10)
-    sat = np.abs(blocks) / X[..., None] > 448
-    assert np.all(np.abs(deq - blocks)[~sat] <= tol[~sat])
-    assert np.all(np.abs(deq[sat]) == 448 * np.broadcast_to(X[..., None], deq.shape)[sat])
+    assert not np.any(np.abs(blocks) / X[..., None] > 448)
+    assert np.all(np.abs(deq - blocks) <= tol)
 
 
 def _fp8_layer(T, d, F, n, seed):

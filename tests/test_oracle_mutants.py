@@ -33,8 +33,11 @@ MUTANTS = [
     ("rmsnorm_eps_dropped", "1.0 / sqrt(ss / (double)d + eps);", "1.0 / sqrt(ss / (double)d);"),
     ("residual_dropped", "round_to(x[r * d + i] + yr[i], dtype);", "round_to(yr[i], dtype);"),
     ("e4m3_ties_to_odd", "(dist == bd && (c & 1) == 0)", "(dist == bd && (c & 1) == 1)"),
-    ("mx_emax_off_by_one", "int E = ex - 1 - 8;", "int E = ex - 1 - 7;"),
-    ("mx_ceil_not_floor", "int E = ex - 1 - 8;", "int E = ex - 8;"),
+    ("mx_exponent_off_by_one", "int E = f <= 0.875 ? ex - 9 : ex - 8;",
+     "int E = f <= 0.875 ? ex - 8 : ex - 7;"),
+    ("mx_clipping_rule", "int E = f <= 0.875 ? ex - 9 : ex - 8;", "int E = ex - 9;"),
+    ("mx_threshold_at_one_and_a_half", "int E = f <= 0.875 ? ex - 9 : ex - 8;",
+     "int E = f <= 0.75 ? ex - 9 : ex - 8;"),
     ("mx_low_clamp_dropped", "if (E < -127) E = -127;", "if (E < -200) E = -127;"),
     ("mx_zero_block_scale", "if (amax == 0.0f) return 127;", "if (amax == 0.0f) return 0;"),
     ("mx_overflow_to_nan", "if (a >= 448.0) return sign | 126;", "if (a > 464.0) return sign | 127;"),
