@@ -380,7 +380,8 @@ def workload_label(w) -> str:
 
 
 def run_gpu_fp8(args, w):
-    """The FP8-weight variant (E4M3 expert weights with row scales) on a small-batch workload:
+    """The FP8-weight variant (MXFP8 expert weights: E4M3 codes, an E8M0 scale per 32
+    elements) on a small-batch workload:
     same step, timing and JSON line as run_gpu, one GPU (replicas as run_gpu for N > 1)."""
     import torch.distributed as dist
 
@@ -398,7 +399,7 @@ def run_gpu_fp8(args, w):
     layer = moe_inputs.make_layer(wr, device=dev)
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
-        q = {k: moe.moe_quantize_rows_e4m3(layer[k], stream=stream) for k in ("W1", "W3", "W2")}
+        q = {k: moe.moe_quantize_mx_e4m3(layer[k], stream=stream) for k in ("W1", "W3", "W2")}
     Wg = layer["Wg"]
     del layer
     args_q = (q["W1"][0], q["W3"][0], q["W2"][0], q["W1"][1], q["W3"][1], q["W2"][1])
@@ -474,30 +475,31 @@ def run_gpu_fp8(args, w):
     tok_s = world * w.T * args.steps / (ms / 1e3)
     g13 = statistics.mean(st[1] for st in stage_ms)
     stage_avg = [statistics.mean(st[j] for st in stage_ms) for j in range(5)]
-    bytes13 = n_active * 2 * w.F * (w.d + 4) + w.T * w.K * (w.d + 4)
-    step_bytes = n_active * 3 * w.F * w.d + n_active * (2 * w.F + w.d) * 4 + w.d * w.n * 4 \
-        + 2 * w.T * w.d * 2
+    # E4M3 codes plus one E8M0 scale byte per 32 of them
+    bytes13 = n_active * 2 * w.F * w.d * 33 // 32 + w.T * w.K * w.d * 33 // 32
+    step_bytes = n_active * 3 * w.F * w.d * 33 // 32 + w.d * w.n * 4 + 2 * w.T * w.d * 2
     achieved = bytes13 / (g13 / 1e3) / 1e9
     line = {
-        "metric": METRIC + " -- FP8 (E4M3) expert-weight variant", "value": round(tok_s, 2),
+        "metric": METRIC + " -- FP8 (MXFP8) expert-weight variant", "value": round(tok_s, 2),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3 weights and activations, fp32 accumulate, bf16 out",
+        "vs_baseline": None,
+        "dtype": "mxfp8 (e4m3 + e8m0 per 32) weights and activations, fp32 accumulate, bf16 out",
         "data": "synthetic (seeded N(0,1) activations, RMS-normalised; N(0,1/fan_in) weights "
-                "quantised per row to E4M3 on the device)",
+                "quantised to MXFP8 on the device)",
         "config": {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} n={w.n} K={w.K}, "
-                               "E4M3 expert weights",
+                               "MXFP8 expert weights",
                    "tokens_per_rank": w.T,
                    "l2": f"inputs larger than L2 ({3 * w.n * w.F * w.d / 1e9:.2f} GB of E4M3 "
-                         "expert weights)",
+                         "expert-weight codes)",
                    "parallelism": f"replicas x{world}",
                    "tiling": f"small-batch swap-AB split-K {plan['split13']}/{plan['split2']}, "
-                             "tcgen05 kind::f8f6f4", "active_experts": n_active},
+                             "tcgen05 kind::mxf8f6f4 block_scale", "active_experts": n_active},
         "pct_roofline": {"bound": "hbm", "frac": round(step_bytes / (ms_step / 1e3) / 1e9 /
                                                        peaks["hbm_gbs"], 4),
-                         "basis": "E4M3 weight bytes (+ row scales) of selected experts per "
+                         "basis": "E4M3 weight bytes (+ block scales) of selected experts per "
                                   "step / measured HBM copy GB/s"},
-        "roofline": {"bound": "hbm", "kernel": "tc_grouped_gemm G13 (E4M3)",
+        "roofline": {"bound": "hbm", "kernel": "tc_grouped_gemm G13 (MXFP8)",
                      "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": None, "peak_source": peaks["source"],

@@ -126,37 +126,46 @@ MOE_API moe_status moe_forward_debug(const void* x, const float* W_g, const void
 
 /* ---- FP8 expert weights (a variant for decode bandwidth; the pages only mention quantised
  * community builds -- the reader comments on the hada.io page -- and fix no format, so the
- * format is this library's plain reading; it is not the hardware's block-scaled MX format):
- * OCP FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
- * largest finite 448) with one fp32 scale per row of each weight matrix:
- *   s = max_j |w_j| / 448 (1 for a zero row), code_j = E4M3(w_j / s), nearest, ties to even,
- *   saturating; w_j ~ s * value(code_j).
- * The block then quantises each token's x row and each h row the same way (their scales
- * are computed on the device), accumulates code products in fp32 on the tensor cores
- * (tcgen05 kind::f8f6f4) and applies the row scales:
- *   a_f = s_x s1_f sum_j x_q,j W1q_f,j,  b_f likewise,  h_f = silu(a_f) b_f,
- *   y_i = s_h s2_i sum_f h_q,f W2q_i,f,  out = sum_k G_k y_{e_k} rounded once to bf16.
- * Routing is the bf16 block's (bf16 x, fp32 W_g). */
+ * format is this library's plain reading): MXFP8, the OCP Microscaling format with FP8 E4M3
+ * elements (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest
+ * finite 448) in blocks of 32 consecutive elements of a row sharing one E8M0 scale X = 2^E
+ * (code E + 127):
+ *   E = the smallest integer with max_j |w_j| <= 448 2^E (no element overflows), clamped to
+ *   [-127, 127] (E = 0 for an all-zero block);
+ *   code_j = E4M3(w_j / X), nearest, ties to even, saturating;  w_j ~ X value(code_j).
+ * The block quantises each token's x row and each h row the same way on the device, and the
+ * tensor cores apply both operands' block scales in the MMA (tcgen05 kind::mxf8f6f4,
+ * block_scale), accumulating in fp32:
+ *   a_f = sum_blocks X_x X_1,f sum_j x_q,j W1q_f,j,  b_f likewise,  h_f = silu(a_f) b_f,
+ *   y_i = sum_blocks X_h X_2,i sum_f h_q,f W2q_i,f,  out = sum_k G_k y_{e_k} rounded once.
+ * Routing is the bf16 block's (bf16 x, fp32 W_g).
+ *
+ * Scale layout ("tile order", what the tensor cores' scale copies read): for a [rows][cols]
+ * matrix (both multiples of 128) the scale code of row r, elements [32c, 32c + 32) is the byte
+ *   ((r / 128) * (cols / 128) + c / 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) / 32) + c % 4,
+ * i.e. one 512-byte chunk per 128 rows x 128 columns. */
 
-/* Per-row E4M3 codes and fp32 scales of a [rows][cols] bf16 matrix v (device pointers;
- * cols a multiple of 4; v 8-byte and q 4-byte aligned): q [rows][cols] uint8, scales [rows].
- * Enqueued on `stream`.  Use it once on W1 and W3 ([n*F][d]) and W2 ([n*d][F]). */
-MOE_API moe_status moe_quantize_rows_e4m3(const void* v, int64_t rows, int64_t cols,
-                                          uint8_t* q, float* scales, void* stream);
+/* MXFP8 codes and block scales of a [rows][cols] bf16 matrix v (device pointers; rows and
+ * cols multiples of 128; v 8-byte, q 4-byte and sf 16-byte aligned): q [rows][cols] uint8,
+ * sf rows * cols / 32 bytes in tile order.  Enqueued on `stream`.  Use it once on W1 and W3
+ * (as [n*F][d]) and W2 (as [n*d][F]). */
+MOE_API moe_status moe_quantize_mx_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
+                                        uint8_t* sf, void* stream);
 
 /* Workspace bytes for moe_forward_fp8 (0 if unsupported).  Supported: the small-batch
  * decode shapes (T <= 64, T*K <= 1024 and T*K < 64 n), d and F multiples of 128. */
 MOE_API size_t moe_workspace_bytes_fp8(int64_t T, int64_t d, int64_t F, int n, int K);
 
-/* The block with E4M3 expert weights:
+/* The block with MXFP8 expert weights:
  *   x [T][d] bf16, W_g [d][n] fp32, W1q, W3q [n][F][d] and W2q [n][d][F] E4M3 codes,
- *   s1, s3 [n][F] and s2 [n][d] fp32 row scales (16-byte aligned), out [T][d] bf16.
+ *   sf1, sf3 (of [n*F][d]) and sf2 (of [n*d][F]) their block scales in tile order as
+ *   moe_quantize_mx_e4m3 writes them (16-byte aligned), out [T][d] bf16.
  * events: NULL / 0, or six cudaEvent_t recorded at the stage boundaries (routing, G13,
- * reduction, G2, combine), as moe_forward_profiled.  Other conventions as moe_forward;
- * shapes outside the supported set return MOE_ERR_UNSUPPORTED. */
+ * SwiGLU + h quantisation, G2, combine), as moe_forward_profiled.  Other conventions as
+ * moe_forward; shapes outside the supported set return MOE_ERR_UNSUPPORTED. */
 MOE_API moe_status moe_forward_fp8(const void* x, const float* W_g, const uint8_t* W1q,
-                                   const uint8_t* W3q, const uint8_t* W2q, const float* s1,
-                                   const float* s3, const float* s2, int64_t T, int64_t d,
+                                   const uint8_t* W3q, const uint8_t* W2q, const uint8_t* sf1,
+                                   const uint8_t* sf3, const uint8_t* sf2, int64_t T, int64_t d,
                                    int64_t F, int n, int K, void* out, void* workspace,
                                    size_t workspace_bytes, void* stream, void* const* events,
                                    int n_events);

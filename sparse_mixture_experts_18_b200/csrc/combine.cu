@@ -77,14 +77,11 @@ struct Out4<float> {
   }
 };
 
-// SCALED (FP8-weight block): the expert outputs are code sums, scaled here by the row's h
-// scale row_scale[row] and the W2 row scales col_scale[e][column] of the slot's expert.
-template <typename Tout, bool RESID, bool SCALED = false>
+template <typename Tout, bool RESID>
 __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ Y, int S, int64_t split_stride, int64_t T, int d,
                    int K, const int32_t* __restrict__ inv, const float* __restrict__ gate,
-                   Tout* out, const Tout* resid, const float* __restrict__ row_scale,
-                   const float* __restrict__ col_scale, const int32_t* __restrict__ expert) {
+                   Tout* out, const Tout* resid) {
   pdl_wait();
   pdl_trigger();
   const int vpr = d / 4;
@@ -109,12 +106,6 @@ __global__ void __launch_bounds__(256)
         if (s < S) {
           yk.x += part[s].x; yk.y += part[s].y; yk.z += part[s].z; yk.w += part[s].w;
         }
-      if (SCALED) {
-        const float rs = row_scale[row];
-        const float4 cs = __ldg(reinterpret_cast<const float4*>(
-            col_scale + (int64_t)expert[t * K + k] * d + c));
-        yk.x *= rs * cs.x; yk.y *= rs * cs.y; yk.z *= rs * cs.z; yk.w *= rs * cs.w;
-      }
       acc[0] = fmaf(g, yk.x, acc[0]);
       acc[1] = fmaf(g, yk.y, acc[1]);
       acc[2] = fmaf(g, yk.z, acc[2]);
@@ -330,10 +321,10 @@ static cudaError_t combine_rows_t(const float* Y, int S, int64_t split_stride, i
   if (blocks < 1) blocks = 1;
   if (resid)
     pdl(combine_kernel<Tout, true>, (unsigned)blocks, 256, 0, s)(
-        Y, S, split_stride, T, d, K, inv, gate, out, resid, nullptr, nullptr, nullptr);
+        Y, S, split_stride, T, d, K, inv, gate, out, resid);
   else
     pdl(combine_kernel<Tout, false>, (unsigned)blocks, 256, 0, s)(
-        Y, S, split_stride, T, d, K, inv, gate, out, nullptr, nullptr, nullptr, nullptr);
+        Y, S, split_stride, T, d, K, inv, gate, out, nullptr);
   return cudaGetLastError();
 }
 
@@ -349,8 +340,7 @@ cudaError_t launch_combine_rows(const float* Y, int S, int64_t split_stride, int
 }
 
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
-                           cudaStream_t s, const float* s2, void* norm_out, float eps,
-                           bool* normed) {
+                           cudaStream_t s, void* norm_out, float eps, bool* normed) {
   if (normed) *normed = false;
   const float* g2 = p.gather_x ? nullptr : w.gate;
   if (norm_out && resid && p.dt == 1 && !p.fp8 && !p.swap &&
@@ -366,15 +356,6 @@ cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const v
   const int S = p.swap ? p.s2 : 1;
   const int64_t split_stride = p.rows_max * p.d;
   const float* gates = p.gather_x ? nullptr : w.gate;  // gather_x: G2 applied the gates
-  if (p.fp8) {  // small batches only (T <= 64), bf16 out, no residual
-    const int64_t total = p.T * (p.d / 4);
-    int64_t blocks = (total + 255) / 256;
-    if (blocks < 1) blocks = 1;
-    pdl(combine_kernel<__nv_bfloat16, false, true>, (unsigned)blocks, 256, 0, s)(
-        w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, w.gate,
-        static_cast<__nv_bfloat16*>(out), nullptr, w.sh, s2, w.idx);
-    return cudaGetLastError();
-  }
   return launch_combine_rows(w.y, S, split_stride, p.T, (int)p.d, p.K, w.inv, gates, out, resid,
                              p.dt == 0, s);
 }

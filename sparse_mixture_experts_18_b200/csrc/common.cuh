@@ -221,6 +221,72 @@ __device__ __forceinline__ void umma_e4m3(uint32_t tmem_d, uint64_t adesc, uint6
       : "memory");
 }
 
+// ---------------------------------------------------------------- MXFP8 (block-scaled E4M3)
+// Instruction descriptor, kind::mxf8f6f4 with E4M3 A and B (formats 0), both K-major, E8M0
+// scale factors (bit 23), N >> 3 (17-22), M >> 4 (24-28); the byte of each 32-bit TMEM scale
+// column that this MMA reads: B's in bits 4-5, A's in bits 29-30.
+__host__ __device__ constexpr uint32_t umma_idesc_mx_e4m3(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
+         (sf_id << 29);
+}
+
+// D[tmem] (+)= (A * SFA) (B * SFB)^T over K = 32 with E4M3 operands in shared memory and one
+// E8M0 scale per row of A and per row of B in TMEM (scale_vec 1X: one per 32 elements).  The
+// scale addresses carry the byte index in bits 30-31, like the descriptor's scale IDs.
+__device__ __forceinline__ void umma_mx_e4m3(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte matrix stored row after row (no swizzle:
+// 8-row core matrices of 128 bytes, 128 bytes apart), the source of tcgen05.cp below.
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t smem_addr) {
+  return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
+         ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
+// Copy 32 rows x 128 bits from shared memory into TMEM lanes 0-31, columns taddr .. taddr + 3,
+// and the same data into lanes 32-63, 64-95 and 96-127 (the scale-factor layout the MMA reads:
+// lane i, column c holds the 4 scales of row 32c + i).  Ordered with this thread's later MMAs.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Contiguous global -> shared copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned), completion signalled on `bar` as transaction bytes.  No multicast.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// E8M0 code of a 32-element block's scale X = 2^E: the smallest E with amax <= 448 2^E, so
+// that no element overflows E4M3 (amax = m 2^e, 1 <= m < 2: E = e - 8 for m <= 1.75, else
+// e - 7), clamped to [-127, 127]; 127 (X = 1) for an all-zero block.  amax >= 0 and finite.
+__device__ __forceinline__ uint32_t mx_scale_code(float amax) {
+  if (amax == 0.f) return 127u;
+  const uint32_t bits = __float_as_uint(amax);
+  const int ex = (int)(bits >> 23);  // biased exponent (sign bit is 0)
+  if (ex == 0) return 0u;  // subnormal: E would be below -127, so it is clamped there
+  const int E = ex - 127 - 8 + ((bits & 0x7FFFFFu) > 0x600000u ? 1 : 0);  // 0x600000: m = 1.75
+  return (uint32_t)(E < -127 ? 0 : E + 127);
+}
+
+// 1 / X for an E8M0 code c <= 253: 2^(127 - c), a normal binary32 (codes from mx_scale_code
+// never exceed 247).
+__device__ __forceinline__ float mx_inv_scale(uint32_t c) {
+  return __uint_as_float((254u - c) << 23);
+}
+
 // Two binary32 values to OCP FP8 E4M3 codes (nearest, ties to even, saturating to +-448):
 // lo's code in the low byte.
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {

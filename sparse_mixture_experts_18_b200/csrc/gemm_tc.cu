@@ -66,6 +66,18 @@ struct TcArgs {
   // will complete and runs out after wait_limit cycles (0 on every forward call)
   long long wait_limit = WAIT_LIMIT_CYCLES;
   int withhold_loads = 0;
+  // MXFP8 (E4M3 kernels): E8M0 block scales of the A rows (W1 or W2; sfa1: W3) in the tensor
+  // cores' tile order, one 512-byte chunk per (128-row tile, 128-wide K block); of the B rows
+  // (the expert's token or h rows) one 512-byte chunk per (expert, K block), row slot j at
+  // byte 16 (j % 32) + 4 (j / 32); sf_kb K blocks per row; sf_off: their copies in a stage
+  // (A0, A1, B at +0, +512, +1024); sf_col: first TMEM column of the scales (A0, A1, B at
+  // +0, +4, +8)
+  const uint8_t* sfa0 = nullptr;
+  const uint8_t* sfa1 = nullptr;
+  const uint8_t* sfb = nullptr;
+  int sf_kb = 0;
+  uint32_t sf_off = 0;
+  uint32_t sf_col = 0;
 };
 
 struct Ctrl {
@@ -122,18 +134,10 @@ __device__ __forceinline__ Work decode_work(const TcArgs& a, const Ctrl* c, int 
   return w;
 }
 
-// One MMA of the kernel's operand kind: bf16 (kind::f16) or E4M3 (kind::f8f6f4).
-template <bool E4M3>
-__device__ __forceinline__ void umma_kind(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  if constexpr (E4M3)
-    umma_e4m3(tmem_d, adesc, bdesc, idesc, accumulate);
-  else
-    umma_bf16(tmem_d, adesc, bdesc, idesc, accumulate);
-}
-
-// E4M3: operands are FP8 codes (128 per 128-byte row, so a K block is 128 elements wide);
-// the accumulators hold the code products, scaled later by the row scales.
+// E4M3 (small batch only): operands are FP8 codes (128 per 128-byte row, so a K block is 128
+// elements wide) with one E8M0 scale per 32 elements of every row; each stage also brings the
+// scales of its K block, which the MMA thread copies into TMEM (tcgen05.cp) ahead of the
+// block-scaled MMAs (kind::mxf8f6f4), so the accumulators hold real sums.
 template <int KIND, bool SWAP, bool E4M3 = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tc_grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
@@ -195,6 +199,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t phase = 0;
       for (int id = blockIdx.x; id < total && !a.withhold_loads; id += gridDim.x) {
         const Work w = decode_work<SWAP>(a, c, id);
+        // gathering: only the 4-row groups that hold this expert's rows are loaded; the MMA
+        // columns of the other slots read whatever the stage holds and are never stored
+        const int ngath = gather ? (w.count + 3) / 4 : 0;
+        const uint32_t tx =
+            gather ? a.tx_bytes - (uint32_t)(a.tok_tile / 4 - ngath) * 512u : a.tx_bytes;
         bool ok = true;
         for (int kb = 0; kb < a.num_kb; ++kb) {
           if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort, a.wait_limit)) {
@@ -203,7 +212,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
           uint8_t* st = smem + (size_t)stage * a.stage_bytes;
           uint64_t* fb = &c->full[stage];
-          mbar_arrive_expect_tx(fb, a.tx_bytes);
+          mbar_arrive_expect_tx(fb, tx);
           const int k = (SWAP ? w.s * a.num_kb + kb : kb) * (E4M3 ? 128 : 64);
           if (!SWAP) {
             tma_load_2d(st, &tmX, fb, k, w.mt * TILE_M, pol_x);
@@ -218,8 +227,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const int wr = w.e * a.nw + w.wblk * 128;
             tma_load_2d(st, &tmW0, fb, k, wr, pol_w);
             if (KIND == KIND_G13) tma_load_2d(st + TILE_BYTES, &tmW1, fb, k, wr, pol_w);
+            if constexpr (E4M3) {  // the K block's scale chunks (A rows, B row slots)
+              const int kbg = w.s * a.num_kb + kb;
+              const int64_t rt = ((int64_t)w.e * a.nw + w.wblk * 128) / 128;
+              bulk_load(st + a.sf_off, a.sfa0 + (rt * a.sf_kb + kbg) * 512, 512, fb);
+              if (KIND == KIND_G13)
+                bulk_load(st + a.sf_off + 512, a.sfa1 + (rt * a.sf_kb + kbg) * 512, 512, fb);
+              bulk_load(st + a.sf_off + 1024, a.sfb + ((int64_t)w.e * a.sf_kb + kbg) * 512, 512,
+                        fb);
+            }
             if (gather) {  // the expert's token rows straight from x, four per gather
-              for (int g = 0; g < a.tok_tile / 4; ++g) {
+              for (int g = 0; g < ngath; ++g) {
                 int tk[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
@@ -245,8 +263,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = E4M3 ? umma_idesc_e4m3(128, SWAP ? a.tok_tile : 256)
-                                  : umma_idesc_bf16(128, SWAP ? a.tok_tile : 256);
+      const uint32_t idesc = umma_idesc_bf16(128, SWAP ? a.tok_tile : 256);
       int stage = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -263,19 +280,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t sb = smem_u32(smem + (size_t)stage * a.stage_bytes);
+          if constexpr (E4M3) {
+            // the K block's scales into TMEM; the MMAs below read them after the copies (the
+            // tensor core runs this thread's tcgen05 operations in order)
+            const uint32_t sf = tmem_base + a.sf_col;
+            tmem_cp_32x128b_x4(sf, sdesc_rows16(sb + a.sf_off));
+            if (KIND == KIND_G13) tmem_cp_32x128b_x4(sf + 4, sdesc_rows16(sb + a.sf_off + 512));
+            tmem_cp_32x128b_x4(sf + 8, sdesc_rows16(sb + a.sf_off + 1024));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t kofs = kk * 32;  // 16 bf16 / 32 E4M3 along K in the 128-byte row
-            const uint32_t accum = (kb | kk) != 0;
-            if (!SWAP) {
-              umma_kind<E4M3>(dtm, umma_desc_k128(sb + kofs),
-                              umma_desc_k128(sb + TILE_BYTES + kofs), idesc, accum);
-            } else {
+            for (int kk = 0; kk < 4; ++kk) {  // 32 codes along K per MMA, scale byte kk
+              const uint32_t kofs = kk * 32;
+              const uint32_t accum = (kb | kk) != 0;
+              const uint32_t id = umma_idesc_mx_e4m3(128, a.tok_tile, (uint32_t)kk);
+              const uint32_t sbyte = (uint32_t)kk << 30;
               const uint64_t bd = umma_desc_k128(sb + a.x_off + kofs);
-              umma_kind<E4M3>(dtm, umma_desc_k128(sb + kofs), bd, idesc, accum);
+              umma_mx_e4m3(dtm, umma_desc_k128(sb + kofs), bd, id, sf + sbyte, sf + 8 + sbyte,
+                           accum);
               if (KIND == KIND_G13)
-                umma_kind<E4M3>(dtm + a.tok_tile, umma_desc_k128(sb + TILE_BYTES + kofs), bd,
-                                idesc, accum);
+                umma_mx_e4m3(dtm + a.tok_tile, umma_desc_k128(sb + TILE_BYTES + kofs), bd, id,
+                             sf + 4 + sbyte, sf + 8 + sbyte, accum);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t kofs = kk * 32;  // 16 bf16 along K in the 128-byte row
+              const uint32_t accum = (kb | kk) != 0;
+              if (!SWAP) {
+                umma_bf16(dtm, umma_desc_k128(sb + kofs), umma_desc_k128(sb + TILE_BYTES + kofs),
+                          idesc, accum);
+              } else {
+                const uint64_t bd = umma_desc_k128(sb + a.x_off + kofs);
+                umma_bf16(dtm, umma_desc_k128(sb + kofs), bd, idesc, accum);
+                if (KIND == KIND_G13)
+                  umma_bf16(dtm + a.tok_tile, umma_desc_k128(sb + TILE_BYTES + kofs), bd, idesc,
+                            accum);
+              }
             }
           }
           umma_commit(&c->empty[stage]);  // frees the stage once these MMAs have read it
@@ -803,118 +842,99 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// ---------------------------------------------------------------- FP8 (E4M3) weights
-// Row scale in binary32 as the E4M3 format is used here: max |v| / 448 (1 for a zero row),
-// codes E4M3(v / s), nearest with ties to even, saturating.
-constexpr int Q_THREADS = 512;
+// ---------------------------------------------------------------- FP8 (MXFP8) weights
+// Codes E4M3(v / X) in blocks of 32 consecutive elements of a row sharing the scale X = 2^E
+// (mx_scale_code / mx_inv_scale: the smallest E with max |v| <= 448 2^E; v / X is exact).
+// One warp per (row, 128 columns): lane c holds columns 4c .. 4c + 3, so a 32-element block is
+// 8 lanes and the K block's four scale codes are those of lanes 0, 8, 16 and 24.
 
-__device__ __forceinline__ float block_max(float v, float* wmax) {
+// Four E4M3 codes of v * inv (inv a power of two), lowest address in the lowest byte.
+__device__ __forceinline__ uint32_t e4m3x4_mul(float v0, float v1, float v2, float v3,
+                                               float inv) {
+  return (uint32_t)cvt_e4m3x2(v0 * inv, v1 * inv) |
+         ((uint32_t)cvt_e4m3x2(v2 * inv, v3 * inv) << 16);
+}
+
+// The block scale of this lane's 8-lane group and the K block's scale word (codes of the four
+// groups, the lowest columns in the lowest byte; the same value on every lane).
+__device__ __forceinline__ uint32_t mx_group_scale(float amax, float* inv, uint32_t* word) {
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float m = 0.f;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, wmax[w]);
-  return m;
+  for (int off = 1; off < 8; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const uint32_t code = mx_scale_code(amax);
+  *inv = mx_inv_scale(code);
+  *word = __shfl_sync(0xffffffffu, code, 0) | (__shfl_sync(0xffffffffu, code, 8) << 8) |
+          (__shfl_sync(0xffffffffu, code, 16) << 16) | (__shfl_sync(0xffffffffu, code, 24) << 24);
+  return code;
 }
 
-// One CTA per row of a [rows][cols] bf16 matrix (cols % 4 == 0).
-__global__ void __launch_bounds__(Q_THREADS)
-    quantize_rows_e4m3_kernel(const __nv_bfloat16* __restrict__ v, int64_t cols,
-                              uint8_t* __restrict__ q, float* __restrict__ scales) {
-  __shared__ float wmax[Q_THREADS / 32];
-  const __nv_bfloat16* row = v + (int64_t)blockIdx.x * cols;
-  float amax = 0.f;
-  for (int64_t c = threadIdx.x * 4; c < cols; c += Q_THREADS * 4) {
-    const uint2 r = *reinterpret_cast<const uint2*>(row + c);
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(r.x)), fabsf(bf16_hi(r.x))),
-                             fmaxf(fabsf(bf16_lo(r.y)), fabsf(bf16_hi(r.y)))));
-  }
-  const float s = e4m3_scale(block_max(amax, wmax));
-  if (threadIdx.x == 0) scales[blockIdx.x] = s;
-  uint8_t* qr = q + (int64_t)blockIdx.x * cols;
-  for (int64_t c = threadIdx.x * 4; c < cols; c += Q_THREADS * 4) {
-    const uint2 r = *reinterpret_cast<const uint2*>(row + c);
-    *reinterpret_cast<uint32_t*>(qr + c) =
-        e4m3x4(bf16_lo(r.x), bf16_hi(r.x), bf16_lo(r.y), bf16_hi(r.y), s);
+// Weights: [rows][cols] bf16 -> codes q [rows][cols] and scales in the tile order the GEMMs
+// read: the word of row r, K block kb at byte ((r / 128) * (cols / 128) + kb) * 512
+// + 16 (r % 32) + 4 ((r % 128) / 32).  rows and cols multiples of 128.
+__global__ void __launch_bounds__(256)
+    quantize_mx_e4m3_kernel(const __nv_bfloat16* __restrict__ v, int64_t rows, int64_t cols,
+                            uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  const int lane = threadIdx.x & 31;
+  const int64_t kbs = cols / 128;
+  for (int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); gw < rows * kbs;
+       gw += (int64_t)gridDim.x * 8) {  // warp-uniform
+    const int64_t r = gw / kbs, kb = gw % kbs;
+    const int64_t c = kb * 128 + lane * 4;
+    const uint2 raw = *reinterpret_cast<const uint2*>(v + r * cols + c);
+    const float f0 = bf16_lo(raw.x), f1 = bf16_hi(raw.x), f2 = bf16_lo(raw.y), f3 = bf16_hi(raw.y);
+    float inv;
+    uint32_t word;
+    mx_group_scale(fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))), &inv, &word);
+    *reinterpret_cast<uint32_t*>(q + r * cols + c) = e4m3x4_mul(f0, f1, f2, f3, inv);
+    if (lane == 0)
+      *reinterpret_cast<uint32_t*>(sf + ((r / 128) * kbs + kb) * 512 + 16 * (r % 32) +
+                                   4 * ((r % 128) / 32)) = word;
   }
 }
 
-// FP8 small batch: permuted row r of expert e (rows grouped by offsets) is handled by a
-// cluster of RQ_CLUSTER CTAs, each taking F / RQ_CLUSTER columns:
-//   a_f = (s_x s1[e][f]) sum_s A_s,  b_f = (s_x s3[e][f]) sum_s B_s  (splits in order; s_x the
-//   scale of the row's token), h_f = silu(a_f) b_f in binary32; the row's max |h| is combined
-//   across the cluster through
-//   distributed shared memory, then each CTA quantises its columns: s_h[r], hq[r][f].
-// h stays in shared memory between the two passes.
-constexpr int RQ_CLUSTER = 4;
-
-__global__ void __launch_bounds__(Q_THREADS)
-    swiglu_reduce_e4m3_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
-                              int F, int n, const int32_t* __restrict__ offsets,
-                              const int32_t* __restrict__ row_tok,
-                              const float* __restrict__ sx, const float* __restrict__ s1,
-                              const float* __restrict__ s3, uint8_t* __restrict__ hq,
-                              float* __restrict__ sh) {
+// FP8 small batch: permuted row r of expert e (rows grouped by offsets, slot j = r -
+// offsets[e]): a = sum_s A_s, b = sum_s B_s (splits in order; the block-scaled MMAs already
+// applied every scale), h = silu(a) b in binary32, then block-quantised: codes hq[r][f] and
+// the K block's scale word at slot j of the G2 B-operand chunk sfh[e][f / 128].
+__global__ void __launch_bounds__(256)
+    swiglu_quantize_mx_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
+                              int64_t rows, int F, int n, const int32_t* __restrict__ offsets,
+                              uint8_t* __restrict__ hq, uint32_t* __restrict__ sfh) {
   pdl_wait();
   pdl_trigger();
-  extern __shared__ float hbuf[];  // F / RQ_CLUSTER floats
-  __shared__ float wmax[Q_THREADS / 32];
-  __shared__ float cta_max;
-  __shared__ int s_e;
-  const uint32_t rank = cluster_ctarank();
-  const int64_t r = blockIdx.x / RQ_CLUSTER;
-  const int fc = F / RQ_CLUSTER, f0 = (int)rank * fc;
-  if (threadIdx.x == 0) {
+  const int lane = threadIdx.x & 31;
+  const int kbs = F / 128;
+  const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (gw >= rows * kbs) return;  // warp-uniform
+  const int64_t r = gw / kbs;
+  const int kb = (int)(gw % kbs);
+  const int c = kb * 128 + lane * 4;
+  const float* pa = p13 + r * 2 * F + c;
+  float4 ta[REDUCE_MAX_S], tb[REDUCE_MAX_S];
+#pragma unroll
+  for (int k = 0; k < REDUCE_MAX_S; ++k)
+    if (k < S) {
+      ta[k] = __ldg(reinterpret_cast<const float4*>(pa + k * split_stride));
+      tb[k] = __ldg(reinterpret_cast<const float4*>(pa + k * split_stride + F));
+    }
+  float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
+#pragma unroll
+  for (int k = 0; k < REDUCE_MAX_S; ++k)
+    if (k < S) {
+      sa.x += ta[k].x; sa.y += ta[k].y; sa.z += ta[k].z; sa.w += ta[k].w;
+      sb.x += tb[k].x; sb.y += tb[k].y; sb.z += tb[k].z; sb.w += tb[k].w;
+    }
+  const float h0 = silu_epilogue(sa.x) * sb.x, h1 = silu_epilogue(sa.y) * sb.y;
+  const float h2 = silu_epilogue(sa.z) * sb.z, h3 = silu_epilogue(sa.w) * sb.w;
+  float inv;
+  uint32_t word;
+  mx_group_scale(fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))), &inv, &word);
+  *reinterpret_cast<uint32_t*>(hq + r * F + c) = e4m3x4_mul(h0, h1, h2, h3, inv);
+  if (lane == 0) {
     int e = 0;
     while (e + 1 < n && r >= offsets[e + 1]) ++e;
-    s_e = e;
+    const int j = (int)(r - offsets[e]);  // < 128: an expert gets at most T <= 64 rows
+    sfh[((int64_t)e * kbs + kb) * 128 + 4 * (j & 31) + (j >> 5)] = word;
   }
-  __syncthreads();
-  const int e = s_e;
-  const float xs = sx[row_tok[r]];  // the scale of the row's token
-  const float* pa = p13 + r * 2 * F;
-  float amax = 0.f;
-  for (int cl = threadIdx.x * 4; cl < fc; cl += Q_THREADS * 4) {
-    const int c = f0 + cl;
-    float4 ta[REDUCE_MAX_S], tb[REDUCE_MAX_S];
-#pragma unroll
-    for (int k = 0; k < REDUCE_MAX_S; ++k)
-      if (k < S) {
-        ta[k] = __ldg(reinterpret_cast<const float4*>(pa + k * split_stride + c));
-        tb[k] = __ldg(reinterpret_cast<const float4*>(pa + k * split_stride + F + c));
-      }
-    float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
-#pragma unroll
-    for (int k = 0; k < REDUCE_MAX_S; ++k)
-      if (k < S) {
-        sa.x += ta[k].x; sa.y += ta[k].y; sa.z += ta[k].z; sa.w += ta[k].w;
-        sb.x += tb[k].x; sb.y += tb[k].y; sb.z += tb[k].z; sb.w += tb[k].w;
-      }
-    const float4 w1 = __ldg(reinterpret_cast<const float4*>(s1 + (int64_t)e * F + c));
-    const float4 w3 = __ldg(reinterpret_cast<const float4*>(s3 + (int64_t)e * F + c));
-    float4 h;
-    h.x = silu_epilogue((xs * w1.x) * sa.x) * ((xs * w3.x) * sb.x);
-    h.y = silu_epilogue((xs * w1.y) * sa.y) * ((xs * w3.y) * sb.y);
-    h.z = silu_epilogue((xs * w1.z) * sa.z) * ((xs * w3.z) * sb.z);
-    h.w = silu_epilogue((xs * w1.w) * sa.w) * ((xs * w3.w) * sb.w);
-    *reinterpret_cast<float4*>(hbuf + cl) = h;
-    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h.x), fabsf(h.y)), fmaxf(fabsf(h.z), fabsf(h.w))));
-  }
-  const float m = block_max(amax, wmax);  // (its barrier also orders hbuf)
-  if (threadIdx.x == 0) cta_max = m;
-  cluster_sync_all();  // every CTA's maximum is in its shared memory
-  float rmax = 0.f;
-#pragma unroll
-  for (int q = 0; q < RQ_CLUSTER; ++q)
-    rmax = fmaxf(rmax, ld_cluster_f32(map_to_rank(&cta_max, (uint32_t)q)));
-  const float s = e4m3_scale(rmax);
-  if (threadIdx.x == 0 && rank == 0) sh[r] = s;
-  for (int cl = threadIdx.x * 4; cl < fc; cl += Q_THREADS * 4) {
-    const float4 h = *reinterpret_cast<const float4*>(hbuf + cl);
-    *reinterpret_cast<uint32_t*>(hq + r * F + f0 + cl) = e4m3x4(h.x, h.y, h.z, h.w, s);
-  }
-  cluster_sync_all();  // no CTA leaves while a peer may still read its maximum
 }
 
 // ---------------------------------------------------------------- host side
@@ -1227,26 +1247,31 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   return record(ev, 2, s);
 }
 
-cudaError_t launch_quantize_rows_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
-                                      float* scales, cudaStream_t s) {
+cudaError_t launch_quantize_mx_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
+                                    uint8_t* sf, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  quantize_rows_e4m3_kernel<<<(unsigned)rows, Q_THREADS, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(v), cols, q, scales);
+  const int64_t warps = rows * (cols / 128);
+  int64_t blocks = (warps + 7) / 8;
+  if (blocks > 64 * (int64_t)num_sms()) blocks = 64 * (int64_t)num_sms();
+  quantize_mx_e4m3_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(v), rows, cols, q, sf);
   return cudaGetLastError();
 }
 
-// The small-batch tiling of launch_expert_gemms_tc on E4M3 codes: G13 partial sums, the
-// scaled SwiGLU with h quantised per row, G2 partial sums (scaled in the combine).
+// The small-batch tiling of launch_expert_gemms_tc on MXFP8 codes: G13 partial sums (block
+// scales applied by the MMAs), SwiGLU with h block-quantised, G2 partial sums.  The token
+// rows' codes are gathered from the per-token rows in w.xperm; the block scales of the B rows
+// come from the routing kernel (w.sfx) and from the SwiGLU kernel (w.sfh).
 cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const uint8_t* W3q,
-                                     const uint8_t* W2q, const float* s1, const float* s3,
-                                     const Workspace& w, cudaStream_t s,
-                                     cudaEvent_t const* ev) {
+                                     const uint8_t* W2q, const uint8_t* sf1,
+                                     const uint8_t* sf3, const uint8_t* sf2, const Workspace& w,
+                                     cudaStream_t s, cudaEvent_t const* ev) {
   CUtensorMap mX, mW1, mW3, mH, mW2;
   const int d = (int)p.d, F = (int)p.F, n = p.n;
-  const int tok = p.tok_tile;
+  const int tok = p.tok_tile;  // a multiple of 32 (the B scales' TMEM layout), <= 64
   const uint32_t xbytes = (uint32_t)tok * 128;
   const uint32_t xslot = (xbytes + 1023u) & ~1023u;
-  // the expert's token rows are gathered from the per-token E4M3 rows (one-row boxes)
+  constexpr uint32_t SF_SLOT = 2048;  // three 512-byte scale chunks, stage size 1024-aligned
   if (!make_map_u8(&mX, w.xperm, d, (uint64_t)p.T, 1) ||
       !make_map_u8(&mW1, W1q, d, (uint64_t)n * F, 128) ||
       !make_map_u8(&mW3, W3q, d, (uint64_t)n * F, 128) ||
@@ -1264,12 +1289,18 @@ cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const ui
   a.nw = F;
   a.wb = (F + 127) / 128;
   a.x_off = 2 * TILE_BYTES;
-  a.stage_bytes = 2 * TILE_BYTES + xslot;
-  a.tx_bytes = 2 * TILE_BYTES + xbytes;
+  a.sf_off = 2 * TILE_BYTES + xslot;
+  a.stage_bytes = 2 * TILE_BYTES + xslot + SF_SLOT;
+  a.tx_bytes = 2 * TILE_BYTES + xbytes + 3 * 512;
   a.stages = stages_for(a.stage_bytes);
   a.acc_cols = 2 * tok;
-  a.nacc = 2 * a.acc_cols <= 512 ? 2 : 1;
-  a.tmem_cols = pow2_cols(a.nacc * a.acc_cols);
+  a.nacc = 2 * a.acc_cols + 12 <= 512 ? 2 : 1;
+  a.sf_col = a.nacc * a.acc_cols;
+  a.tmem_cols = pow2_cols(a.sf_col + 12);
+  a.sfa0 = sf1;
+  a.sfa1 = sf3;
+  a.sfb = reinterpret_cast<const uint8_t*>(w.sfx);
+  a.sf_kb = d / 128;
   a.out = w.p13;
   a.out_ld = 2 * (int64_t)F;
   a.split_stride = p.rows_max * 2 * (int64_t)F;
@@ -1281,36 +1312,13 @@ cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const ui
     return err;
   a.row_tok = nullptr;
   if ((err = record(ev, 0, s)) != cudaSuccess) return err;
-  const size_t hsmem = (size_t)(F / RQ_CLUSTER) * sizeof(float);
   {
-    static size_t configured = 0;
-    if (configured < hsmem) {
-      if ((err = cudaFuncSetAttribute(swiglu_reduce_e4m3_kernel,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)hsmem)) != cudaSuccess)
-        return err;
-      configured = hsmem;
-    }
-    const int rows = (int)(p.T * p.K);
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = RQ_CLUSTER;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3((unsigned)(RQ_CLUSTER * (rows > 0 ? rows : 1)), 1, 1);
-    cfg.blockDim = dim3(Q_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = hsmem;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    if ((err = cudaLaunchKernelEx(&cfg, swiglu_reduce_e4m3_kernel, w.p13, p.s13, a.split_stride,
-                                  F, n, static_cast<const int32_t*>(w.offsets),
-                                  static_cast<const int32_t*>(w.row_tok), w.sx, s1, s3,
-                                  static_cast<uint8_t*>(w.h), w.sh)) != cudaSuccess)
-      return err;
+    const int64_t rows = p.T * p.K;
+    const int64_t warps = rows * (F / 128);
+    const unsigned blocks = (unsigned)((warps + 7) / 8 > 0 ? (warps + 7) / 8 : 1);
+    pdl(swiglu_quantize_mx_kernel, blocks, 256, 0, s)(
+        w.p13, p.s13, a.split_stride, rows, F, n, static_cast<const int32_t*>(w.offsets),
+        static_cast<uint8_t*>(w.h), w.sfh);
   }
   if ((err = cudaGetLastError()) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
     return err;
@@ -1319,12 +1327,18 @@ cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const ui
   a.nw = d;
   a.wb = (d + 127) / 128;
   a.x_off = TILE_BYTES;
-  a.stage_bytes = TILE_BYTES + xslot;
-  a.tx_bytes = TILE_BYTES + xbytes;
+  a.sf_off = TILE_BYTES + xslot;
+  a.stage_bytes = TILE_BYTES + xslot + SF_SLOT;
+  a.tx_bytes = TILE_BYTES + xbytes + 2 * 512;
   a.stages = stages_for(a.stage_bytes);
   a.acc_cols = tok;
-  a.nacc = 2 * a.acc_cols <= 512 ? 2 : 1;
-  a.tmem_cols = pow2_cols(a.nacc * a.acc_cols);
+  a.nacc = 2 * a.acc_cols + 12 <= 512 ? 2 : 1;
+  a.sf_col = a.nacc * a.acc_cols;
+  a.tmem_cols = pow2_cols(a.sf_col + 12);
+  a.sfa0 = sf2;
+  a.sfa1 = nullptr;
+  a.sfb = reinterpret_cast<const uint8_t*>(w.sfh);
+  a.sf_kb = F / 128;
   a.out = w.y;
   a.out_ld = d;
   a.split_stride = p.rows_max * (int64_t)d;

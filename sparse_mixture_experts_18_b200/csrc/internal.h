@@ -45,7 +45,8 @@ struct Plan {
   size_t o_rpart;          // small batch: partial router logits [ceil(d/64)][T][n]
   size_t o_rowtok;         // token of each permuted row [rows_max] (small batch, gather_x)
   size_t o_rowgate;        // gather_x: gate of each permuted row [rows_max]
-  size_t o_sx, o_sh;       // fp8: token-row scales [T] and h-row scales [rows_max]
+  size_t o_sx, o_sfx, o_sh;  // fp8 block scales: per token [T][d/128] words; per expert
+                             // row slot for G13's B [n][d/128][512 B] and G2's B [n][F/128][512 B]
   size_t o_wparts;         // tensor-core router: W_g as three bf16 parts [3n padded][d]
   size_t o_status, o_idx, o_gate, o_blk_counts, o_blk_base, o_counts, o_offsets, o_inv,
       o_xperm, o_h, o_y, o_p13, o_xn, total;
@@ -59,8 +60,9 @@ struct Workspace {
   float* rpart;          // small-batch routing: partial logits
   int32_t* row_tok;      // token of each permuted row (small batch, gather_x)
   float* row_gate;       // gather_x: gate of each permuted row
-  float* sx;             // fp8: scale of each token's row (the E4M3 rows are per token)
-  float* sh;             // fp8: scale of each h row
+  uint32_t* sxw;         // fp8: each token's block-scale words [T][d / 128]
+  uint32_t* sfx;         // fp8: the token rows' scales by expert row slot (G13 B operand)
+  uint32_t* sfh;         // fp8: the h rows' scales by expert row slot (G2 B operand)
   __nv_bfloat16* wparts; // tensor-core router: the W_g parts
   int32_t *idx, *blk_counts, *blk_base, *counts, *offsets, *inv;
   float* gate;
@@ -123,15 +125,17 @@ cudaError_t launch_route(const Plan& p, const void* x, const float* Wg, const Wo
 cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
                                    const void* W3, const void* W2, const Workspace& w,
                                    cudaStream_t s, cudaEvent_t const* ev = nullptr);
-// fp8: the small-batch GEMMs on E4M3 codes; W1q/W3q [n][F][d], W2q [n][d][F]; s1/s3 [n][F]
-// and s2 [n][d] row scales.  ev as for launch_expert_gemms_tc.
+// fp8: the small-batch GEMMs on MXFP8 codes; W1q/W3q [n][F][d], W2q [n][d][F] E4M3 codes;
+// sf1/sf3/sf2 their E8M0 block scales in the tile order of launch_quantize_mx_e4m3.  ev as
+// for launch_expert_gemms_tc.
 cudaError_t launch_expert_gemms_e4m3(const Plan& p, const uint8_t* W1q, const uint8_t* W3q,
-                                     const uint8_t* W2q, const float* s1, const float* s3,
-                                     const Workspace& w, cudaStream_t s,
-                                     cudaEvent_t const* ev = nullptr);
-// Per-row E4M3 quantisation of a [rows][cols] bf16 matrix (cols % 4 == 0).
-cudaError_t launch_quantize_rows_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
-                                      float* scales, cudaStream_t s);
+                                     const uint8_t* W2q, const uint8_t* sf1,
+                                     const uint8_t* sf3, const uint8_t* sf2, const Workspace& w,
+                                     cudaStream_t s, cudaEvent_t const* ev);
+// MXFP8 quantisation of [rows][cols] bf16 (multiples of 128): codes and block scales in the
+// GEMMs' tile order.
+cudaError_t launch_quantize_mx_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
+                                    uint8_t* sf, cudaStream_t s);
 cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float* W3,
                                      const float* W2, const Workspace& w, cudaStream_t s,
                                      cudaEvent_t const* ev = nullptr);
@@ -140,8 +144,8 @@ cudaError_t launch_expert_gemms_simt(const Plan& p, const float* W1, const float
 // it also writes the RMSNorm (unit gain, eps) of every result row there -- the next stacked
 // block's input -- and sets *normed; otherwise the caller runs launch_rmsnorm.
 cudaError_t launch_combine(const Plan& p, const Workspace& w, void* out, const void* resid,
-                           cudaStream_t s, const float* s2 = nullptr, void* norm_out = nullptr,
-                           float eps = 0.f, bool* normed = nullptr);
+                           cudaStream_t s, void* norm_out = nullptr, float eps = 0.f,
+                           bool* normed = nullptr);
 // out[t] = (resid[t] +) sum_k gate[t][k] * sum_{s < S} Y[s * split_stride + inv[t][k] row]
 // (gate null: weight 1), fp32 sums in split then slot order, rounded once to bf16, or kept
 // fp32 (out_f32).

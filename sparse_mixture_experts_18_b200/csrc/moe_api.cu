@@ -77,7 +77,7 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   }
   const int64_t P = T * K;
   q.rows_max = (P + (int64_t)n * (q.row_align - 1) + q.row_align - 1) / q.row_align * q.row_align;
-  if (q.swap) q.rows_max = (P + 15) / 16 * 16;  // >= tok_tile rows for the token TMA box
+  if (q.swap) q.rows_max = (P + 31) / 32 * 32;  // >= tok_tile rows for the token TMA box
   if (q.rows_max >= ((int64_t)1 << 31) / 2) return false;
   const int tokb = route_tokens_per_block(K);
   q.nblk = (T + tokb - 1) / tokb;
@@ -89,7 +89,8 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   if (route_only) q.rows_max = P;
   const int kbw = fp8 ? 128 : 64;  // elements per 128-byte K block
   if (q.swap) {
-    q.tok_tile = (int)((T + 15) / 16 * 16);
+    // (fp8: a multiple of 32, the granularity of the B operand's block scales in TMEM)
+    q.tok_tile = fp8 ? (int)((T + 31) / 32 * 32) : (int)((T + 15) / 16 * 16);
     const int sms = num_sms();
     q.s13 = choose_split((int)(d / kbw), n * (int)((F + 127) / 128), sms);
     q.s2 = choose_split((int)(F / kbw), n * (int)((d + 127) / 128), sms);
@@ -114,8 +115,10 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   // (the layout does not depend on gather_x, so a workspace sized earlier stays valid)
   q.o_rowtok = take(q.fused_route || q.pair ? (size_t)q.rows_max * 4 : 0);
   q.o_rowgate = take(q.pair ? (size_t)q.rows_max * 4 : 0);
-  q.o_sx = take(fp8 ? (size_t)q.rows_max * 4 : 0);  // X_perm and h hold E4M3 codes then
-  q.o_sh = take(fp8 ? (size_t)q.rows_max * 4 : 0);
+  // fp8: X_perm holds each token's E4M3 row (by token) and h the E4M3 rows; block scales
+  q.o_sx = take(fp8 ? (size_t)T * (d / 128) * 4 : 0);
+  q.o_sfx = take(fp8 ? (size_t)n * (d / 128) * 512 : 0);
+  q.o_sh = take(fp8 ? (size_t)n * (F / 128) * 512 : 0);
   q.o_wparts = take(router_tc_applies(q) ? router_tc_parts_bytes(d, n) : 0);
   q.total = o;
   *p = q;
@@ -131,8 +134,9 @@ Workspace carve(const Plan& p, void* base) {
   w.rpart = reinterpret_cast<float*>(b + p.o_rpart);
   w.row_tok = reinterpret_cast<int32_t*>(b + p.o_rowtok);
   w.row_gate = reinterpret_cast<float*>(b + p.o_rowgate);
-  w.sx = reinterpret_cast<float*>(b + p.o_sx);
-  w.sh = reinterpret_cast<float*>(b + p.o_sh);
+  w.sxw = reinterpret_cast<uint32_t*>(b + p.o_sx);
+  w.sfx = reinterpret_cast<uint32_t*>(b + p.o_sfx);
+  w.sfh = reinterpret_cast<uint32_t*>(b + p.o_sh);
   w.wparts = reinterpret_cast<__nv_bfloat16*>(b + p.o_wparts);
   w.idx = reinterpret_cast<int32_t*>(b + p.o_idx);
   w.gate = reinterpret_cast<float*>(b + p.o_gate);
@@ -187,7 +191,7 @@ static moe_status forward_impl(const Plan& p, const void* x, const float* W_g, c
                                            static_cast<const float*>(W2), w, s,
                                            ev ? ev + 2 : nullptr);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_combine(p, w, out, resid, s, nullptr, norm_out, eps, normed) != cudaSuccess)
+  if (launch_combine(p, w, out, resid, s, norm_out, eps, normed) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (ev && cudaEventRecord(ev[5], s) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
@@ -199,7 +203,7 @@ using namespace moe;
 
 extern "C" {
 
-int moe_abi_version(void) { return 2; }
+int moe_abi_version(void) { return 3; }
 
 const char* moe_status_string(moe_status s) {
   switch (s) {
@@ -270,19 +274,22 @@ size_t moe_workspace_bytes_fp8(int64_t T, int64_t d, int64_t F, int n, int K) {
   return p.total;
 }
 
-moe_status moe_quantize_rows_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
-                                  float* scales, void* stream) {
-  if (rows < 0 || cols <= 0 || cols % 4) return MOE_ERR_INVALID_ARG;
+moe_status moe_quantize_mx_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
+                                uint8_t* sf, void* stream) {
+  if (rows < 0 || cols <= 0 || rows % 128 || cols % 128) return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
-  if (!v || !q || !scales || !aligned(v, 8) || !aligned(q, 4)) return MOE_ERR_INVALID_ARG;
-  if (rows > ((int64_t)1 << 31) - 1) return MOE_ERR_UNSUPPORTED;
-  return launch_quantize_rows_e4m3(v, rows, cols, q, scales, static_cast<cudaStream_t>(stream))
-                 == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  if (!v || !q || !sf || !aligned(v, 8) || !aligned(q, 4) || !aligned(sf, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (rows > ((int64_t)1 << 31) - 1 || cols > ((int64_t)1 << 20)) return MOE_ERR_UNSUPPORTED;
+  return launch_quantize_mx_e4m3(v, rows, cols, q, sf, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 moe_status moe_forward_fp8(const void* x, const float* W_g, const uint8_t* W1q,
-                           const uint8_t* W3q, const uint8_t* W2q, const float* s1,
-                           const float* s3, const float* s2, int64_t T, int64_t d, int64_t F,
+                           const uint8_t* W3q, const uint8_t* W2q, const uint8_t* sf1,
+                           const uint8_t* sf3, const uint8_t* sf2, int64_t T, int64_t d, int64_t F,
                            int n, int K, void* out, void* workspace, size_t workspace_bytes,
                            void* stream, void* const* events, int n_events) {
   Plan p;
@@ -296,7 +303,7 @@ moe_status moe_forward_fp8(const void* x, const float* W_g, const uint8_t* W1q,
   if (T == 0) return MOE_OK;
   moe_status st = check_common(x, W_g, W1q, W3q, W2q, out, workspace);
   if (st != MOE_OK) return st;
-  if (!s1 || !s3 || !s2 || !aligned(s1, 16) || !aligned(s3, 16) || !aligned(s2, 16))
+  if (!sf1 || !sf3 || !sf2 || !aligned(sf1, 16) || !aligned(sf3, 16) || !aligned(sf2, 16))
     return MOE_ERR_INVALID_ARG;
   if (out == x) return MOE_ERR_INVALID_ARG;
   if (workspace_bytes < p.total) return MOE_ERR_WORKSPACE;
@@ -308,10 +315,10 @@ moe_status moe_forward_fp8(const void* x, const float* W_g, const uint8_t* W1q,
   if (evp && cudaEventRecord(ev[0], s) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_route(p, x, W_g, w, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (evp && cudaEventRecord(ev[1], s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_expert_gemms_e4m3(p, W1q, W3q, W2q, s1, s3, w, s, evp ? ev + 2 : nullptr) !=
-      cudaSuccess)
+  if (launch_expert_gemms_e4m3(p, W1q, W3q, W2q, sf1, sf3, sf2, w, s,
+                               evp ? ev + 2 : nullptr) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (launch_combine(p, w, out, nullptr, s, s2) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_combine(p, w, out, nullptr, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (evp && cudaEventRecord(ev[5], s) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

@@ -187,50 +187,45 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
   if (threadIdx.x < n) blk_counts[(int64_t)blockIdx.x * n + threadIdx.x] = hist[threadIdx.x];
 }
 
-// FP8-weight block: every token's bf16 x row as E4M3 codes with its own scale (max |x| /
-// 448) into xq[t] and sx[t]; one warp per token, two passes over the row.  The G13 kernel
-// gathers the rows of each expert from xq by token.
-__device__ __forceinline__ void quantize_tokens_e4m3(const __nv_bfloat16* __restrict__ x,
-                                                     int d, int T, uint8_t* __restrict__ xq,
-                                                     float* __restrict__ sx, int tid,
-                                                     int nthreads) {
-  constexpr int U = 4;  // 16-byte loads in flight per lane
+// FP8-weight block: every token's bf16 x row as MXFP8 -- E4M3 codes in blocks of 32 that
+// share an E8M0 scale (mx_scale_code) -- into xq[t], and per 128 columns the four scale codes
+// as one word (lowest columns in the lowest byte) into sxw[t][kb].  One warp per token; lane L
+// of a pass holds 8 columns, so a 32-element block is 4 lanes and a 128-column block 16.
+__device__ __forceinline__ void quantize_tokens_mx(const __nv_bfloat16* __restrict__ x, int d,
+                                                   int T, uint8_t* __restrict__ xq,
+                                                   uint32_t* __restrict__ sxw, int tid,
+                                                   int nthreads) {
   const int lane = tid & 31, nwarps = nthreads >> 5;
-  for (int r = tid >> 5; r < T; r += nwarps) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * d);
-    const int nv = d / 8;  // 8 bf16 per 16-byte vector
-    float amax = 0.f;
-    for (int v0 = lane; v0 < nv; v0 += 32 * U) {
-      uint4 t[U];
+  const int nv = d / 8;  // 16-byte vectors per row, a multiple of 16 (d % 128 == 0)
+  for (int t = tid >> 5; t < T; t += nwarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)t * d);
+    uint2* dst = reinterpret_cast<uint2*>(xq + (int64_t)t * d);
+    for (int v0 = 0; v0 < nv; v0 += 32) {  // warp-uniform
+      const int v = v0 + lane;
+      const bool in = v < nv;  // a whole 16-lane half of the warp is in or out
+      const uint4 r = in ? __ldg(src + v) : make_uint4(0u, 0u, 0u, 0u);
+      const float f[8] = {bf16_lo(r.x), bf16_hi(r.x), bf16_lo(r.y), bf16_hi(r.y),
+                          bf16_lo(r.z), bf16_hi(r.z), bf16_lo(r.w), bf16_hi(r.w)};
+      float amax = 0.f;
 #pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (v0 + 32 * u < nv) t[u] = __ldg(src + v0 + 32 * u);
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (v0 + 32 * u < nv) {
-          const uint32_t w[4] = {t[u].x, t[u].y, t[u].z, t[u].w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[k])), fabsf(bf16_hi(w[k]))));
-        }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1)
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    const float s = e4m3_scale(amax);
-    if (lane == 0) sx[r] = s;
-    uint2* dst = reinterpret_cast<uint2*>(xq + (int64_t)r * d);
-    for (int v0 = lane; v0 < nv; v0 += 32 * U) {
-      uint4 t[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (v0 + 32 * u < nv) t[u] = __ldg(src + v0 + 32 * u);
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (v0 + 32 * u < nv)
-          dst[v0 + 32 * u] = make_uint2(
-              e4m3x4(bf16_lo(t[u].x), bf16_hi(t[u].x), bf16_lo(t[u].y), bf16_hi(t[u].y), s),
-              e4m3x4(bf16_lo(t[u].z), bf16_hi(t[u].z), bf16_lo(t[u].w), bf16_hi(t[u].w), s));
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const uint32_t code = mx_scale_code(amax);
+      const float inv = mx_inv_scale(code);
+      const int h = lane & 16;  // first lane of this 128-column block
+      const uint32_t word = __shfl_sync(0xffffffffu, code, h) |
+                            (__shfl_sync(0xffffffffu, code, h + 4) << 8) |
+                            (__shfl_sync(0xffffffffu, code, h + 8) << 16) |
+                            (__shfl_sync(0xffffffffu, code, h + 12) << 24);
+      if (in) {
+        dst[v] = make_uint2(
+            (uint32_t)cvt_e4m3x2(f[0] * inv, f[1] * inv) |
+                ((uint32_t)cvt_e4m3x2(f[2] * inv, f[3] * inv) << 16),
+            (uint32_t)cvt_e4m3x2(f[4] * inv, f[5] * inv) |
+                ((uint32_t)cvt_e4m3x2(f[6] * inv, f[7] * inv) << 16));
+        if ((lane & 15) == 0) sxw[(int64_t)t * (d / 128) + v / 16] = word;
+      }
     }
   }
 }
@@ -270,8 +265,10 @@ __device__ __forceinline__ void gather_rows(const Tact* __restrict__ x, int64_t 
 // TopK and softmax, the expert counts, group offsets (padded to row_align), the stable rank
 // of every (token, slot) (per-warp match + per-expert prefix over 32-entry chunks), the
 // inverse map token -> row and the map row -> token.  Then, if xq is given (FP8 weights), the
-// token rows as E4M3 codes with their scales; else, if xperm is given, the bf16 rows in
-// permuted order.  The G13 kernel gathers token rows from x (bf16) or xq (FP8) otherwise.
+// token rows as MXFP8 codes and, by expert row slot, their block scales for G13 (sfx: slot j
+// of expert e, K block kb at word (e * d/128 + kb) * 128 + 4 (j % 32) + j / 32); else, if
+// xperm is given, the bf16 rows in permuted order.  The G13 kernel gathers token rows from x
+// (bf16) or xq (FP8) otherwise.
 constexpr int RS_THREADS = 1024;
 constexpr int RS_MAX_T = 64;
 constexpr int RS_MAX_ENTRIES = SMALL_ROUTE_MAX_ROWS;
@@ -285,7 +282,8 @@ __global__ void __launch_bounds__(RS_THREADS)
                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                        int32_t* __restrict__ inv, int32_t* __restrict__ row_tok,
                        Tact* __restrict__ xperm, uint32_t* status,
-                       uint8_t* __restrict__ xq, float* __restrict__ sx) {
+                       uint8_t* __restrict__ xq, uint32_t* __restrict__ sxw,
+                       uint32_t* __restrict__ sfx) {
   pdl_wait();
   pdl_trigger();
   constexpr int PER = RS_MAX_ENTRIES / RS_THREADS;  // entries per thread in the rank phase
@@ -464,9 +462,21 @@ __global__ void __launch_bounds__(RS_THREADS)
     inv[i] = row;
     if (row >= 0) row_tok[row] = i / K;
   }
-  if (xq != nullptr) {  // FP8-weight block: quantised token rows and their scales
-    if constexpr (std::is_same<Tact, __nv_bfloat16>::value)
-      quantize_tokens_e4m3(x, d, T, xq, sx, tid, RS_THREADS);
+  if (xq != nullptr) {  // FP8-weight block: quantised token rows and their block scales
+    if constexpr (std::is_same<Tact, __nv_bfloat16>::value) {
+      quantize_tokens_mx(x, d, T, xq, sxw, tid, RS_THREADS);
+      __syncthreads();  // sxw (global) and s_row are complete
+      const int kbs = d / 128;
+      for (int q = tid; q < E * kbs; q += RS_THREADS) {
+        const int i = q / kbs, kb = q % kbs;
+        const int row = s_row[i];
+        if (row < 0) continue;
+        const int e = s_idx[i];
+        const int j = row - s_off[e];  // < 64: an expert gets at most T rows
+        sfx[((int64_t)e * kbs + kb) * 128 + 4 * (j & 31) + (j >> 5)] =
+            sxw[(int64_t)(i / K) * kbs + kb];
+      }
+    }
     return;
   }
   if (xperm == nullptr) return;  // the G13 kernel gathers the token rows from x
@@ -723,7 +733,8 @@ static cudaError_t launch_route_small_t(const Plan& p, const Tact* x, const floa
       x, Wg, (int)p.T, (int)p.d, p.n, p.K, p.row_align, p.rows_max, w.rpart, w.ticket, w.idx,
       w.gate, w.counts, w.offsets, w.inv, w.row_tok,
       p.gather_small ? nullptr : static_cast<Tact*>(w.xperm), w.status,
-      p.fp8 ? static_cast<uint8_t*>(w.xperm) : nullptr, p.fp8 ? w.sx : nullptr);
+      p.fp8 ? static_cast<uint8_t*>(w.xperm) : nullptr, p.fp8 ? w.sxw : nullptr,
+      p.fp8 ? w.sfx : nullptr);
   return cudaGetLastError();
 }
 

@@ -91,8 +91,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.argtypes = [I32]
         L.moe_abi_version.restype = I32
         L.moe_abi_version.argtypes = []
-        L.moe_quantize_rows_e4m3.restype = I32
-        L.moe_quantize_rows_e4m3.argtypes = [P, I64, I64, P, P, P]
+        L.moe_quantize_mx_e4m3.restype = I32
+        L.moe_quantize_mx_e4m3.argtypes = [P, I64, I64, P, P, P]
         L.moe_workspace_bytes_fp8.restype = SZ
         L.moe_workspace_bytes_fp8.argtypes = [I64, I64, I64, I32, I32]
         L.moe_forward_fp8.restype = I32
@@ -368,32 +368,34 @@ def moe_combine(y_rows, token_rows, topk_gate, out, stream=None):
     return out
 
 
-# ------------------------------------------------------------------ FP8 (E4M3) expert weights
+# ------------------------------------------------------------------ FP8 (MXFP8) expert weights
 
-def moe_quantize_rows_e4m3(v: torch.Tensor, stream=None):
-    """Per-row E4M3 codes (uint8, same shape) and fp32 scales (one per row) of a bf16 CUDA
-    tensor whose last dimension is the row: s = max|v| / 448, code = E4M3(v / s)."""
+def moe_quantize_mx_e4m3(v: torch.Tensor, stream=None):
+    """MXFP8 codes (uint8, same shape) and E8M0 block scales (uint8, numel / 32, in the tile
+    order documented in moe.h) of a bf16 CUDA tensor whose last dimension is the row; rows
+    and columns multiples of 128."""
     if v.dtype != torch.bfloat16 or not v.is_cuda:
-        raise TypeError("moe_quantize_rows_e4m3 takes a bf16 CUDA tensor")
+        raise TypeError("moe_quantize_mx_e4m3 takes a bf16 CUDA tensor")
     v = v.contiguous()
     cols = v.shape[-1]
     rows = v.numel() // cols
     q = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
-    s = torch.empty(v.shape[:-1], dtype=torch.float32, device=v.device)
-    _check("moe_quantize_rows_e4m3", lib().moe_quantize_rows_e4m3(
-        _ptr(v), rows, cols, _ptr(q), _ptr(s), _stream(stream)))
-    return q, s
+    sf = torch.empty(v.numel() // 32, dtype=torch.uint8, device=v.device)
+    _check("moe_quantize_mx_e4m3", lib().moe_quantize_mx_e4m3(
+        _ptr(v), rows, cols, _ptr(q), _ptr(sf), _stream(stream)))
+    return q, sf
 
 
 def moe_workspace_bytes_fp8(T, d, F, n, K) -> int:
     return int(lib().moe_workspace_bytes_fp8(T, d, F, n, K))
 
 
-def moe_forward_fp8(x, W_g, W1q, W3q, W2q, s1, s3, s2, K: int, out=None, workspace=None,
+def moe_forward_fp8(x, W_g, W1q, W3q, W2q, sf1, sf3, sf2, K: int, out=None, workspace=None,
                     stream=None, events=None):
-    """The block with E4M3 expert weights (codes W1q/W3q [n,F,d], W2q [n,d,F]; fp32 row scales
-    s1/s3 [n,F], s2 [n,d]); x and out bf16.  events: None or six torch.cuda.Event recorded at
-    the stage boundaries by the library.  Returns out."""
+    """The block with MXFP8 expert weights (E4M3 codes W1q/W3q [n,F,d], W2q [n,d,F]; their
+    block scales sf1/sf3/sf2 as moe_quantize_mx_e4m3 returns them); x and out bf16.  events:
+    None or six torch.cuda.Event recorded at the stage boundaries by the library.  Returns
+    out."""
     T, d = x.shape
     n, F, _ = W1q.shape
     if out is None:
@@ -405,6 +407,6 @@ def moe_forward_fp8(x, W_g, W1q, W3q, W2q, s1, s3, s2, K: int, out=None, workspa
         ev = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
         nev = 6
     _check("moe_forward_fp8", lib().moe_forward_fp8(
-        _ptr(x), _ptr(W_g), _ptr(W1q), _ptr(W3q), _ptr(W2q), _ptr(s1), _ptr(s3), _ptr(s2),
+        _ptr(x), _ptr(W_g), _ptr(W1q), _ptr(W3q), _ptr(W2q), _ptr(sf1), _ptr(sf3), _ptr(sf2),
         T, d, F, n, K, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream), ev, nev))
     return out

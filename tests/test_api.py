@@ -264,9 +264,11 @@ def test_fp8_forward_rejects_bad_arguments_before_launch(L):
     assert _fwd8(L, T=0, x=0, out=0) == OK
 
 
-def test_quantize_rows_validation(L):
-    q = L.moe_quantize_rows_e4m3
-    assert q(P(0x1000), 4, 6, P(0x2000), P(0x3000), None) == INVALID      # cols % 4
-    assert q(None, 4, 8, P(0x2000), P(0x3000), None) == INVALID
-    assert q(P(0x1004), 4, 8, P(0x2000), P(0x3000), None) == INVALID      # v not 8-byte aligned
-    assert q(P(0x1000), 0, 8, None, None, None) == OK                     # no rows: no-op
+def test_quantize_mx_validation(L):
+    q = L.moe_quantize_mx_e4m3
+    assert q(P(0x1000), 128, 192, P(0x2000), P(0x3000), None) == INVALID    # cols % 128
+    assert q(P(0x1000), 96, 128, P(0x2000), P(0x3000), None) == INVALID     # rows % 128
+    assert q(None, 128, 128, P(0x2000), P(0x3000), None) == INVALID
+    assert q(P(0x1004), 128, 128, P(0x2000), P(0x3000), None) == INVALID    # v not 8-byte aligned
+    assert q(P(0x1000), 128, 128, P(0x2000), P(0x3008), None) == INVALID    # sf not 16-byte
+    assert q(P(0x1000), 0, 128, None, None, None) == OK                     # no rows: no-op

@@ -1,6 +1,6 @@
-"""GPU parity of the FP8-weight variant (E4M3 expert weights with per-row scales, on the
-small-batch decode path) against the oracle's FP8 block: quantisation codes and scales bit
-for bit, block outputs within the bf16 bars."""
+"""GPU parity of the FP8-weight variant (MXFP8: E4M3 expert weights with an E8M0 scale per
+32 elements, on the small-batch decode path) against the oracle's FP8 block: quantisation
+codes and block scales bit for bit, block outputs within the bf16 bars."""
 import numpy as np
 import pytest
 import torch
@@ -18,10 +18,20 @@ import sparse_mixture_experts_18_b200 as moe  # noqa: E402
 
 
 def _quantize_layer(L, n, F, d):
-    W1q, s1 = moe.moe_quantize_rows_e4m3(L["W1"])
-    W3q, s3 = moe.moe_quantize_rows_e4m3(L["W3"])
-    W2q, s2 = moe.moe_quantize_rows_e4m3(L["W2"])
+    W1q, s1 = moe.moe_quantize_mx_e4m3(L["W1"])
+    W3q, s3 = moe.moe_quantize_mx_e4m3(L["W3"])
+    W2q, s2 = moe.moe_quantize_mx_e4m3(L["W2"])
     return W1q, W3q, W2q, s1, s3, s2
+
+
+def _plain_scales(sf_tile, rows, cols):
+    """Block scales from the library's tile order (moe.h: the code of row r, elements
+    [32c, 32c + 32) at byte ((r / 128) (cols / 128) + c / 4) 512 + 16 (r % 32)
+    + 4 ((r % 128) / 32) + c % 4) to plain [rows][cols / 32]."""
+    r = np.arange(rows)[:, None]
+    c = np.arange(cols // 32)[None, :]
+    at = ((r // 128) * (cols // 128) + c // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + c % 4
+    return np.asarray(sf_tile).reshape(-1)[at]
 
 
 def _run_fp8(w, gen_device="cpu", budget=None):
@@ -34,7 +44,11 @@ def _run_fp8(w, gen_device="cpu", budget=None):
     torch.cuda.synchronize()
     xc = x.cpu()
     wg = layer["Wg"].cpu()
-    q = [t.cpu().numpy() for t in (W1q, W3q, W2q, s1, s3, s2)]
+    n, F, d = w.n, w.F, w.d
+    q = [t.cpu().numpy() for t in (W1q, W3q, W2q)]
+    q += [_plain_scales(s1.cpu().numpy(), n * F, d).reshape(n, F, d // 32),
+          _plain_scales(s3.cpu().numpy(), n * F, d).reshape(n, F, d // 32),
+          _plain_scales(s2.cpu().numpy(), n * d, F).reshape(n, d, F // 32)]
     del L
     logits, _, _ = parity.oracle.route(xc, wg, w.n, w.K)
     exempt = {t for t in range(w.T) if parity.oracle.tie_band(logits[t], w.K,
@@ -51,16 +65,20 @@ def _run_fp8(w, gen_device="cpu", budget=None):
     return rep
 
 
-def test_quantize_rows_bit_exact():
+def test_quantize_mx_bit_exact():
+    # codes and block scales against the oracle's quantiser, bit for bit: rows of very
+    # different magnitudes (tiny, subnormal-range, huge, all-zero), a block whose maximum is a
+    # power of two, and a dominant element that saturates its block's other codes' range
     g = torch.Generator().manual_seed(5)
-    scales = torch.tensor([1e-4, 0.01, 1.0, 7.0, 300.0, 0.0, 1e3, 2.5])[:, None]
-    v = (torch.randn(8, 1024, generator=g) * scales).to(torch.bfloat16)
-    v[3, 17] = -v[3, 17].abs().max() * 4          # a dominant negative element
-    q, s = moe.moe_quantize_rows_e4m3(v.cuda())
+    scales = torch.tensor([1e-4, 0.01, 1.0, 7.0, 300.0, 0.0, 1e3, 2.5, 2.0 ** -125, 1e30])
+    v = (torch.randn(256, 1024, generator=g) * scales.repeat(26)[:256, None]).to(torch.bfloat16)
+    v[3, 17] = -v[3, 17].abs().max() * 4
+    v[7, 64:96] = torch.linspace(-2, 2, 32).to(torch.bfloat16)
+    q, sf = moe.moe_quantize_mx_e4m3(v.cuda())
     torch.cuda.synchronize()
-    qo, so = parity.oracle.quantize_rows_e4m3(v)
+    qo, so = parity.oracle.quantize_mx_e4m3(v)
     np.testing.assert_array_equal(q.cpu().numpy(), qo)
-    np.testing.assert_array_equal(s.cpu().numpy(), so)
+    np.testing.assert_array_equal(_plain_scales(sf.cpu().numpy(), 256, 1024), so)
 
 
 @pytest.mark.parametrize("T", [1, 5, 16, 37, 64])
@@ -119,5 +137,5 @@ def test_fp8_decode_error_against_the_bf16_block():
     rep = {"tokens": w.T, "exempt": 0, "max_abs": float(np.max(np.abs(err))),
            "rel_l2": float(np.linalg.norm(err) / np.linalg.norm(ref)), "ok": True}
     rep["ok"] = rep["rel_l2"] <= 0.1
-    parity.record("decode_t16 FP8 (E4M3) weights vs the bf16 block (error of the format)", rep)
+    parity.record("decode_t16 MXFP8 weights vs the bf16 block (error of the format)", rep)
     assert rep["ok"], rep
