@@ -50,8 +50,9 @@ DEFAULT_WORKLOAD = "stack32_t8192"
 # of that kernel on the workload's shapes (for the stack: one T=8192 block), valid only for
 # the kernel source it was taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "stack32_t8192": {"bytes": 2700281856, "src": "482b80168b2c"},
-    "decode_t16": {"bytes": 1885220608, "src": "482b80168b2c"},
+    "stack32_t8192": {"bytes": 2661293824, "src": "90ac4cdb608c"},
+    "decode_t16": {"bytes": 1885336320, "src": "90ac4cdb608c"},
+    "decode_t16 mxfp8": {"bytes": 974726400, "src": "90ac4cdb608c"},
 }
 
 
@@ -479,6 +480,8 @@ def run_gpu_fp8(args, w):
     bytes13 = n_active * 2 * w.F * w.d * 33 // 32 + w.T * w.K * w.d * 33 // 32
     step_bytes = n_active * 3 * w.F * w.d * 33 // 32 + w.d * w.n * 4 + 2 * w.T * w.d * 2
     achieved = bytes13 / (g13 / 1e3) / 1e9
+    cap = TRAFFIC.get(w.name + " mxfp8")
+    traffic = cap["bytes"] if cap and cap["src"] == kernel_source_hash() else None
     line = {
         "metric": METRIC + " -- FP8 (MXFP8) expert-weight variant", "value": round(tok_s, 2),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -502,7 +505,7 @@ def run_gpu_fp8(args, w):
         "roofline": {"bound": "hbm", "kernel": "tc_grouped_gemm G13 (MXFP8)",
                      "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": None, "peak_source": peaks["source"],
+                     "traffic": traffic, "peak_source": peaks["source"],
                      "launch_ms": round(g13, 5)},
         "stage_ms": {"route": round(stage_avg[0], 5), "gemm13": round(stage_avg[1], 5),
                      "swiglu_quantize": round(stage_avg[2], 5),
