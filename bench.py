@@ -520,6 +520,128 @@ def run_gpu_fp8(args, w):
     return line
 
 
+NVLINK_GBS = 770.0  # measured peer copy per direction per GPU on this kind of node (GB/s)
+
+
+def run_ep_emulation(args, w):
+    """Expert parallelism over R ranks, emulated on one GPU.  Every virtual rank r holds the
+    experts [r n / R, (r + 1) n / R) and routes its own batch (the workload with its own seed).
+    The ranks' GPU stages run one after another on this GPU and are timed with CUDA events:
+    moe_route per rank, moe_experts_forward per rank on the rows it receives from every
+    source, moe_combine per rank.  The two all-to-alls are not run (one GPU): their time is
+    modelled from the bytes each rank sends and receives at the peer-copy rate NVLINK_GBS.
+    The modelled step is the slowest rank's route + dispatch + slowest experts stage + return
+    + slowest combine, with nothing overlapped."""
+    import sparse_mixture_experts_18_b200 as moe
+    from sparse_mixture_experts_18_b200 import ep
+
+    R = args.ep_emulate
+    if w.n % R:
+        raise SystemExit(f"{w.name}: n = {w.n} experts do not split over {R} ranks")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    layer = moe_inputs.make_layer(w, device=dev)
+    xs = [moe_inputs.make_x(replica_workload(w, r), device=dev) for r in range(R)]
+    part = ep.ExpertPartition(w.n, R, 0)
+    nl = part.n_local
+    local = [{k: layer[k][q * nl:(q + 1) * nl].contiguous() for k in ("W1", "W3", "W2")}
+             for q in range(R)]
+    Wg = layer["Wg"]
+    es = xs[0].element_size()
+    dt = 1 if xs[0].dtype == torch.bfloat16 else 0
+    lib = moe.lib()
+    ws_route = [moe.alloc_workspace(int(lib.moe_route_workspace_bytes(w.T, w.d, w.n, w.K, dt)),
+                                    dev) for _ in range(R)]
+    routed = [moe.moe_route(xs[r], Wg, w.K, workspace=ws_route[r]) for r in range(R)]
+    counts = [r[3].cpu() for r in routed]
+    send = [ep.ExpertPartition(w.n, R, s).send_splits(counts[s]) for s in range(R)]
+    seg = [torch.stack([counts[s][q * nl:(q + 1) * nl] for s in range(R)]).to(torch.int32)
+           .to(dev) for q in range(R)]
+    rows_q = [sum(send[s][q] for s in range(R)) for q in range(R)]
+    ws_exp = [moe.alloc_workspace(int(lib.moe_experts_workspace_bytes(max(rows_q[q], 1), w.d,
+                                                                       w.F, nl, dt)), dev)
+              for q in range(R)]
+    # the exchange, by slicing (untimed): rows grouped by expert go to their expert's rank
+    x_recv = [torch.cat([routed[s][0][sum(send[s][:q]):sum(send[s][:q + 1])] for s in range(R)])
+              for q in range(R)]
+    outs = [torch.empty_like(x) for x in xs]
+    t_route = [[] for _ in range(R)]
+    t_exp = [[] for _ in range(R)]
+    t_comb = [[] for _ in range(R)]
+    for it in range(args.warmup + args.steps):
+        timed = it >= args.warmup
+        ev = []
+        for r in range(R):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            routed[r] = moe.moe_route(xs[r], Wg, w.K, workspace=ws_route[r])
+            e1.record()
+            ev.append(("route", r, e0, e1))
+        y_recv = []
+        for q in range(R):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            y_recv.append(moe.moe_experts_forward(x_recv[q], seg[q], local[q]["W1"],
+                                                  local[q]["W3"], local[q]["W2"],
+                                                  workspace=ws_exp[q]))
+            e1.record()
+            ev.append(("experts", q, e0, e1))
+        for s in range(R):  # the return, by slicing (untimed)
+            parts_s = []
+            for q in range(R):
+                recv = ep.ExpertPartition.recv_splits(seg[q].cpu())
+                parts_s.append(y_recv[q][sum(recv[:s]):sum(recv[:s + 1])])
+            y_back = torch.cat(parts_s)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            moe.moe_combine(y_back, routed[s][4], routed[s][2], outs[s])
+            e1.record()
+            ev.append(("combine", s, e0, e1))
+        torch.cuda.synchronize()
+        if timed:
+            for kind, r, e0, e1 in ev:
+                {"route": t_route, "experts": t_exp, "combine": t_comb}[kind][r].append(
+                    e0.elapsed_time(e1))
+    for ws in ws_route + ws_exp:
+        code, raw = moe.moe_workspace_status(ws)
+        if code != 0:
+            raise RuntimeError(f"device status {code} ({raw:#x})")
+    med = lambda v: statistics.median(v)
+    route_ms = [med(t) for t in t_route]
+    exp_ms = [med(t) for t in t_exp]
+    comb_ms = [med(t) for t in t_comb]
+    # bytes that cross NVLink (rows for other ranks only): dispatch bf16 rows, return fp32
+    out_rows = [sum(send[s][q] for q in range(R) if q != s) for s in range(R)]
+    in_rows = [sum(send[s][q] for s in range(R) if s != q) for q in range(R)]
+    disp = max(max(o, i) for o, i in zip(out_rows, in_rows)) * w.d * es
+    ret = max(max(o, i) for o, i in zip(out_rows, in_rows)) * w.d * 4
+    t_disp = disp / (NVLINK_GBS * 1e9) * 1e3
+    t_ret = ret / (NVLINK_GBS * 1e9) * 1e3
+    step = max(route_ms) + t_disp + max(exp_ms) + t_ret + max(comb_ms)
+    flops = 2.0 * 3 * w.d * w.F * w.K * w.T * R
+    line = {
+        "metric": "expert-parallel MoE block, emulated on one GPU (modelled step)",
+        "value": round(R * w.T / (step / 1e3), 2), "unit": "tokens/s", "n_gpus": 1,
+        "ranks_emulated": R, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step_modelled": round(step, 5), "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic (seeded per rank)",
+        "config": {"workload": f"{workload_label(w)}, {R} ranks x {w.T} tokens, "
+                               f"{nl} experts per rank", "global_batch": R * w.T},
+        "stage_ms_per_rank": {"route": [round(v, 5) for v in route_ms],
+                              "experts": [round(v, 5) for v in exp_ms],
+                              "combine": [round(v, 5) for v in comb_ms]},
+        "rows_per_rank": rows_q,
+        "exchange": {"dispatch_bytes_max": disp, "return_bytes_max": ret,
+                     "dispatch_ms_modelled": round(t_disp, 5),
+                     "return_ms_modelled": round(t_ret, 5), "link_GBps": NVLINK_GBS},
+        "tflops_modelled": round(flops / (step / 1e3) / 1e12, 1),
+        "note": "GPU stages measured one rank after another on one GPU; all-to-alls modelled "
+                "at the peer-copy rate, not run",
+    }
+    print(json.dumps(line), flush=True)
+    return line
+
+
 def _oracle_block(oracle, w, x, layer, toks):
     """The oracle's result for token rows `toks` of the workload's (first) block, rounded to
     bf16 as the GPU's output is: the MoE block, or for stacked workloads one whole block
@@ -660,6 +782,9 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=None,
                     help="run only the first N blocks of a stacked workload (N=1: one MoE "
                          "block of its shape), e.g. for an ncu capture of a few GB")
+    ap.add_argument("--ep-emulate", type=int, default=0, metavar="R",
+                    help="expert parallelism over R ranks emulated on one GPU: measured GPU "
+                         "stages per rank, all-to-alls modelled from their bytes")
     ap.add_argument("--gather-x", action="store_true",
                     help="CTA-pair path: gather G13's A rows from x (TMA gather4) instead of "
                          "X_perm, gates applied in G2 (sets MOE_GATHER_X=1)")
@@ -677,6 +802,8 @@ def main(argv=None):
         ap.error("the bench measures the bf16 path")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.ep_emulate:
+        return run_ep_emulation(args, w)
     if args.weights == "e4m3":
         return run_gpu_fp8(args, w)
     return run_gpu(args, w)
