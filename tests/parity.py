@@ -160,3 +160,13 @@ REPORTS: list[tuple[str, dict]] = []
 def record(name: str, rep: dict):
     REPORTS.append((name, {k: rep[k] for k in ("tokens", "exempt", "max_abs", "rel_l2", "ok")
                            if k in rep}))
+
+
+def plain_scales(sf_tile, rows, cols):
+    """MXFP8 block scales from the library's tile order (include/moe.h: the code of row r,
+    elements [32c, 32c + 32) at byte ((r / 128) (cols / 128) + c / 4) 512 + 16 (r % 32)
+    + 4 ((r % 128) / 32) + c % 4) to the oracle's plain [rows][cols / 32]."""
+    r = np.arange(rows)[:, None]
+    c = np.arange(cols // 32)[None, :]
+    at = ((r // 128) * (cols // 128) + c // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + c % 4
+    return np.asarray(sf_tile).reshape(-1)[at]

@@ -24,14 +24,7 @@ def _quantize_layer(L, n, F, d):
     return W1q, W3q, W2q, s1, s3, s2
 
 
-def _plain_scales(sf_tile, rows, cols):
-    """Block scales from the library's tile order (moe.h: the code of row r, elements
-    [32c, 32c + 32) at byte ((r / 128) (cols / 128) + c / 4) 512 + 16 (r % 32)
-    + 4 ((r % 128) / 32) + c % 4) to plain [rows][cols / 32]."""
-    r = np.arange(rows)[:, None]
-    c = np.arange(cols // 32)[None, :]
-    at = ((r // 128) * (cols // 128) + c // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + c % 4
-    return np.asarray(sf_tile).reshape(-1)[at]
+_plain_scales = parity.plain_scales
 
 
 def _run_fp8(w, gen_device="cpu", budget=None):
