@@ -50,9 +50,9 @@ DEFAULT_WORKLOAD = "stack32_t8192"
 # of that kernel on the workload's shapes (for the stack: one T=8192 block), valid only for
 # the kernel source it was taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "stack32_t8192": {"bytes": 2661293824, "src": "90ac4cdb608c"},
-    "decode_t16": {"bytes": 1885336320, "src": "90ac4cdb608c"},
-    "decode_t16 mxfp8": {"bytes": 974726400, "src": "90ac4cdb608c"},
+    "stack32_t8192": {"bytes": 2871586816, "src": "2f50786d4371"},
+    "decode_t16": {"bytes": 1886672896, "src": "2f50786d4371"},
+    "decode_t16 mxfp8": {"bytes": 973194496, "src": "2f50786d4371"},
 }
 
 

@@ -203,24 +203,6 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint6
       : "memory");
 }
 
-// Instruction descriptor, kind::f8f6f4 with E4M3 A and B (format code 0 in bits 7-9 and
-// 10-12), fp32 accumulator, both K-major; other fields as umma_idesc_bf16.
-__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N) {
-  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T with 8-bit (E4M3) operands: K = 32 per instruction, so one
-// 128-byte swizzled row again spans four instructions.
-__device__ __forceinline__ void umma_e4m3(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // ---------------------------------------------------------------- MXFP8 (block-scaled E4M3)
 // Instruction descriptor, kind::mxf8f6f4 with E4M3 A and B (formats 0), both K-major, E8M0
 // scale factors (bit 23), N >> 3 (17-22), M >> 4 (24-28); the byte of each 32-bit TMEM scale
@@ -295,16 +277,6 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// Row scale of the E4M3 format as used here: max |v| / 448 in binary32 (1 for a zero row).
-__device__ __forceinline__ float e4m3_scale(float amax) {
-  return amax > 0.f ? amax / 448.0f : 1.0f;
-}
-
-// Codes of four consecutive values v / s (lowest address in the lowest byte).
-__device__ __forceinline__ uint32_t e4m3x4(float v0, float v1, float v2, float v3, float s) {
-  return (uint32_t)cvt_e4m3x2(v0 / s, v1 / s) | ((uint32_t)cvt_e4m3x2(v2 / s, v3 / s) << 16);
-}
-
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -361,13 +333,6 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
-}
-
-// Load a float from shared memory of a CTA of this cluster (address from map_to_rank).
-__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-  return v;
 }
 
 // Four floats from shared memory of a CTA of this cluster (16-byte aligned address).  Issue
