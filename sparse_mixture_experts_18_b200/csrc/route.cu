@@ -187,49 +187,6 @@ __global__ void __launch_bounds__(ROUTE_THREADS)
   if (threadIdx.x < n) blk_counts[(int64_t)blockIdx.x * n + threadIdx.x] = hist[threadIdx.x];
 }
 
-// FP8-weight block: every token's bf16 x row as MXFP8 -- E4M3 codes in blocks of 32 that
-// share an E8M0 scale (mx_scale_code) -- into xq[t], and per 128 columns the four scale codes
-// as one word (lowest columns in the lowest byte) into sxw[t][kb].  One warp per token; lane L
-// of a pass holds 8 columns, so a 32-element block is 4 lanes and a 128-column block 16.
-__device__ __forceinline__ void quantize_tokens_mx(const __nv_bfloat16* __restrict__ x, int d,
-                                                   int T, uint8_t* __restrict__ xq,
-                                                   uint32_t* __restrict__ sxw, int tid,
-                                                   int nthreads) {
-  const int lane = tid & 31, nwarps = nthreads >> 5;
-  const int nv = d / 8;  // 16-byte vectors per row, a multiple of 16 (d % 128 == 0)
-  for (int t = tid >> 5; t < T; t += nwarps) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)t * d);
-    uint2* dst = reinterpret_cast<uint2*>(xq + (int64_t)t * d);
-    for (int v0 = 0; v0 < nv; v0 += 32) {  // warp-uniform
-      const int v = v0 + lane;
-      const bool in = v < nv;  // a whole 16-lane half of the warp is in or out
-      const uint4 r = in ? __ldg(src + v) : make_uint4(0u, 0u, 0u, 0u);
-      const float f[8] = {bf16_lo(r.x), bf16_hi(r.x), bf16_lo(r.y), bf16_hi(r.y),
-                          bf16_lo(r.z), bf16_hi(r.z), bf16_lo(r.w), bf16_hi(r.w)};
-      float amax = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      const uint32_t code = mx_scale_code(amax);
-      const float inv = mx_inv_scale(code);
-      const int h = lane & 16;  // first lane of this 128-column block
-      const uint32_t word = __shfl_sync(0xffffffffu, code, h) |
-                            (__shfl_sync(0xffffffffu, code, h + 4) << 8) |
-                            (__shfl_sync(0xffffffffu, code, h + 8) << 16) |
-                            (__shfl_sync(0xffffffffu, code, h + 12) << 24);
-      if (in) {
-        dst[v] = make_uint2(
-            (uint32_t)cvt_e4m3x2(f[0] * inv, f[1] * inv) |
-                ((uint32_t)cvt_e4m3x2(f[2] * inv, f[3] * inv) << 16),
-            (uint32_t)cvt_e4m3x2(f[4] * inv, f[5] * inv) |
-                ((uint32_t)cvt_e4m3x2(f[6] * inv, f[7] * inv) << 16));
-        if ((lane & 15) == 0) sxw[(int64_t)t * (d / 128) + v / 16] = word;
-      }
-    }
-  }
-}
-
 // Copy the x rows of `E` entries (entry i = (token t0 + i / K, slot i % K)) to their
 // permuted rows (row[i] < 0: skip).  One warp per row, 16-byte vectors, U loads in flight per
 // lane before the stores; no per-vector index arithmetic beyond the lane stride.
@@ -265,10 +222,11 @@ __device__ __forceinline__ void gather_rows(const Tact* __restrict__ x, int64_t 
 // TopK and softmax, the expert counts, group offsets (padded to row_align), the stable rank
 // of every (token, slot) (per-warp match + per-expert prefix over 32-entry chunks), the
 // inverse map token -> row and the map row -> token.  Then, if xq is given (FP8 weights), the
-// token rows as MXFP8 codes and, by expert row slot, their block scales for G13 (sfx: slot j
-// of expert e, K block kb at word (e * d/128 + kb) * 128 + 4 (j % 32) + j / 32); else, if
-// xperm is given, the bf16 rows in permuted order.  The G13 kernel gathers token rows from x
-// (bf16) or xq (FP8) otherwise.
+// token rows' block scales by expert row slot for G13 (sfx: slot j of expert e, K block kb at
+// word (e * d/128 + kb) * 128 + 4 (j % 32) + j / 32) -- every CTA has already written its 64
+// columns of each token row as MXFP8 codes (xq) and their block scale codes (sxw: per token,
+// one byte per 32 columns); else, if xperm is given, the bf16 rows in permuted order.  The
+// G13 kernel gathers token rows from x (bf16) or xq (FP8) otherwise.
 constexpr int RS_THREADS = 1024;
 constexpr int RS_MAX_T = 64;
 constexpr int RS_MAX_ENTRIES = SMALL_ROUTE_MAX_ROWS;
@@ -308,6 +266,32 @@ __global__ void __launch_bounds__(RS_THREADS)
     for (int q = 0; q < CPL; ++q) {
       j0[q] = (c * 8 * CPL + q * 8 + sub) * 8;
       if (t < T && j0[q] < d) xv[q].load(x + (int64_t)t * d + j0[q]);
+    }
+    if constexpr (std::is_same<Tact, __nv_bfloat16>::value) {
+      if (xq != nullptr) {  // FP8-weight block: this CTA's 64 columns of the token as MXFP8
+        // lanes sub 0-3 and 4-7 of the token hold one 32-element block each
+        const bool have = t < T && j0[0] < d;
+        float f[8], amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          f[i] = have ? xv[0].get(i) : 0.f;
+          amax = fmaxf(amax, fabsf(f[i]));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const uint32_t code = mx_scale_code(amax);
+        const float inv = mx_inv_scale(code);
+        if (have) {
+          *reinterpret_cast<uint2*>(xq + (int64_t)t * d + j0[0]) = make_uint2(
+              (uint32_t)cvt_e4m3x2(f[0] * inv, f[1] * inv) |
+                  ((uint32_t)cvt_e4m3x2(f[2] * inv, f[3] * inv) << 16),
+              (uint32_t)cvt_e4m3x2(f[4] * inv, f[5] * inv) |
+                  ((uint32_t)cvt_e4m3x2(f[6] * inv, f[7] * inv) << 16));
+          // the block's code is byte j0 / 32 of the token's scale words (kb = j0 / 128)
+          if ((sub & 3) == 0)
+            reinterpret_cast<uint8_t*>(sxw)[(int64_t)t * (d / 32) + j0[0] / 32] = (uint8_t)code;
+        }
+      }
     }
     for (int eg = 0; eg < n; eg += 8) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -464,8 +448,7 @@ __global__ void __launch_bounds__(RS_THREADS)
   }
   if (xq != nullptr) {  // FP8-weight block: quantised token rows and their block scales
     if constexpr (std::is_same<Tact, __nv_bfloat16>::value) {
-      quantize_tokens_mx(x, d, T, xq, sxw, tid, RS_THREADS);
-      __syncthreads();  // sxw (global) and s_row are complete
+      __syncthreads();  // s_row is complete (sxw: written by every CTA before its ticket)
       const int kbs = d / 128;
       for (int q = tid; q < E * kbs; q += RS_THREADS) {
         const int i = q / kbs, kb = q % kbs;
