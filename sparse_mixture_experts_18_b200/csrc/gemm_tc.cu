@@ -20,7 +20,8 @@
 //   small batch (tc_grouped_gemm_kernel, SWAP): the weights are the 128-row MMA operand and
 //     the expert's tokens the N dimension (16..256), K split into `splits` ranges so that
 //     every SM streams weights; fp32 partial sums go to per-split slabs reduced in a fixed
-//     order afterwards.  With E4M3 the operands are FP8 codes (kind::f8f6f4).
+//     order afterwards.  With MXFP8 weights the operands are E4M3 codes with E8M0 block
+//     scales, applied by the MMA (kind::mxf8f6f4 block_scale).
 //   CTA pairs (tc_pair_gemm_kernel): cta_group::2 tiles of 256 rows x two 256-column blocks,
 //     M = 128 tiles for an expert's last 128 rows (see the section below).
 #include <stdio.h>

@@ -36,7 +36,7 @@ struct Plan {
   int tok_tile = 0;        // swap: MMA N (tokens per expert tile), multiple of 16
   int s13 = 1, s2 = 1;     // swap: split-K factors of the two expert GEMMs
   bool stack = false;      // workspace also holds the normalised activations
-  bool fp8 = false;        // E4M3 expert weights with row scales (small batch only)
+  bool fp8 = false;        // MXFP8 expert weights (small batch only)
   // failure-path test hook (moe_debug_forward_withheld only): the one-CTA G13 kernel issues
   // no loads and its pipeline waits give up after g13_wait_limit cycles
   bool g13_withhold = false;
