@@ -74,7 +74,7 @@ def test_quantize_mx_bit_exact():
     np.testing.assert_array_equal(_plain_scales(sf.cpu().numpy(), 256, 1024), so)
 
 
-@pytest.mark.parametrize("T", [1, 5, 16, 37, 64])
+@pytest.mark.parametrize("T", [1, 5, 16, 32, 33, 37, 64])   # 32 / 33: the 32-slot boundary
 def test_fp8_small_batch(T):
     _run_fp8(moe_inputs.small(T=T, d=512, F=768))
 
@@ -82,6 +82,11 @@ def test_fp8_small_batch(T):
 @pytest.mark.parametrize("n,K", [(16, 4), (64, 2), (1, 1), (8, 1)])
 def test_fp8_expert_counts(n, K):
     _run_fp8(moe_inputs.small(T=12, d=256, F=384, n=n, K=K))
+
+
+def test_fp8_minimal_widths():
+    # d = F = 128: one K block per row, one scale chunk per tile
+    _run_fp8(moe_inputs.small(T=9, d=128, F=128, n=4, K=2))
 
 
 def test_fp8_one_launch_routing_at_its_limit():
