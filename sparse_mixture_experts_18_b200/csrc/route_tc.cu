@@ -27,7 +27,6 @@ constexpr int RTC_THREADS = 192;
 constexpr int RTC_TILE = 128;         // tokens per tile (MMA M)
 constexpr int RTC_MAX_STAGES = 12;
 constexpr int RTC_MAX_N = 64;         // experts
-constexpr int RTC_MAX_NPAD = 192;     // 3 * 64 accumulator columns
 // one CTA per SM with as many stages in flight as shared memory holds (two CTAs per SM with
 // half the stages each measured slower)
 constexpr uint32_t RTC_SMEM_BUDGET = 200 * 1024;
