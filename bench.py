@@ -524,28 +524,28 @@ NVLINK_GBS = 770.0  # measured peer copy per direction per GPU on this kind of n
 
 
 def run_ep_emulation(args, w):
-    """Expert parallelism over R ranks, emulated on one GPU.  Every virtual rank r holds the
-    experts [r n / R, (r + 1) n / R) and routes its own batch (the workload with its own seed).
-    The ranks' GPU stages run one after another on this GPU and are timed with CUDA events:
-    moe_route per rank, moe_experts_forward per rank on the rows it receives from every
-    source, moe_combine per rank.  The two all-to-alls are not run (one GPU): their time is
-    modelled from the bytes each rank sends and receives at the peer-copy rate NVLINK_GBS.
-    The modelled step is the slowest rank's route + dispatch + slowest experts stage + return
-    + slowest combine, with nothing overlapped."""
+    """Expert parallelism over R ranks, emulated on one GPU.  Every virtual rank routes its own
+    batch (the workload with its own seed).  Experts are placed contiguously (n / R per rank),
+    or with --ep-slots C > n / R hot experts are replicated (ep.ExpertPlacement.balanced over
+    the global loads) and each source splits a replicated expert's rows evenly over its
+    replicas.  The ranks' GPU stages run one after another on this GPU and are timed with CUDA
+    events: moe_route (and the row gather into destination order when experts are
+    replicated) per rank; moe_experts_forward per rank on the rows it receives from every
+    source; the row gather back into grouped order and moe_combine per rank.  The two
+    all-to-alls are not run (one GPU): their time is modelled from the bytes each rank sends
+    and receives at the peer-copy rate NVLINK_GBS.  The modelled step is the slowest rank's
+    route + dispatch + slowest experts stage + return + slowest combine, nothing overlapped."""
     import sparse_mixture_experts_18_b200 as moe
     from sparse_mixture_experts_18_b200 import ep
 
     R = args.ep_emulate
     if w.n % R:
         raise SystemExit(f"{w.name}: n = {w.n} experts do not split over {R} ranks")
+    slots = args.ep_slots or w.n // R
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     layer = moe_inputs.make_layer(w, device=dev)
     xs = [moe_inputs.make_x(replica_workload(w, r), device=dev) for r in range(R)]
-    part = ep.ExpertPartition(w.n, R, 0)
-    nl = part.n_local
-    local = [{k: layer[k][q * nl:(q + 1) * nl].contiguous() for k in ("W1", "W3", "W2")}
-             for q in range(R)]
     Wg = layer["Wg"]
     es = xs[0].element_size()
     dt = 1 if xs[0].dtype == torch.bfloat16 else 0
@@ -553,68 +553,92 @@ def run_ep_emulation(args, w):
     ws_route = [moe.alloc_workspace(int(lib.moe_route_workspace_bytes(w.T, w.d, w.n, w.K, dt)),
                                     dev) for _ in range(R)]
     routed = [moe.moe_route(xs[r], Wg, w.K, workspace=ws_route[r]) for r in range(R)]
-    counts = [r[3].cpu() for r in routed]
-    send = [ep.ExpertPartition(w.n, R, s).send_splits(counts[s]) for s in range(R)]
-    seg = [torch.stack([counts[s][q * nl:(q + 1) * nl] for s in range(R)]).to(torch.int32)
-           .to(dev) for q in range(R)]
-    rows_q = [sum(send[s][q] for s in range(R)) for q in range(R)]
-    ws_exp = [moe.alloc_workspace(int(lib.moe_experts_workspace_bytes(max(rows_q[q], 1), w.d,
-                                                                       w.F, nl, dt)), dev)
-              for q in range(R)]
-    # the exchange, by slicing (untimed): rows grouped by expert go to their expert's rank
-    x_recv = [torch.cat([routed[s][0][sum(send[s][:q]):sum(send[s][:q + 1])] for s in range(R)])
-              for q in range(R)]
+    all_counts = torch.stack([r[3] for r in routed]).cpu()
+    loads = all_counts.sum(dim=0)
+    if slots == w.n // R:
+        pl = ep.ExpertPlacement.contiguous(w.n, R)
+    else:
+        pl = ep.ExpertPlacement.balanced(loads, R, slots)
+    plans = [pl.send_order(all_counts[s]) for s in range(R)]
+    ident = [order == list(range(len(order))) for order, _ in plans]
+    perms = [torch.tensor(o, dtype=torch.int32, device=dev) for o, _ in plans]
+    invs = []
+    for pm in perms:
+        inv = torch.empty_like(pm)
+        inv[pm.long()] = torch.arange(len(pm), dtype=torch.int32, device=dev)
+        invs.append(inv)
+    starts = [[sum(plans[s][1][:q]) for q in range(R + 1)] for s in range(R)]
+    segs = [torch.tensor(pl.recv_counts(all_counts, q), dtype=torch.int32, device=dev)
+            for q in range(R)]
+    rows_q = [int(sg.sum()) for sg in segs]
+    local = []
+    for q in range(R):
+        idx = torch.tensor(pl.local_experts(q), device=dev)
+        local.append({k: layer[k][idx].contiguous() for k in ("W1", "W3", "W2")})
+    del layer
+    ws_exp = [moe.alloc_workspace(int(lib.moe_experts_workspace_bytes(
+        max(rows_q[q], 1), w.d, w.F, len(pl.local_experts(q)), dt)), dev) for q in range(R)]
     outs = [torch.empty_like(x) for x in xs]
     t_route = [[] for _ in range(R)]
     t_exp = [[] for _ in range(R)]
     t_comb = [[] for _ in range(R)]
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        res = fn()
+        e1.record()
+        return res, (e0, e1)
+
     for it in range(args.warmup + args.steps):
-        timed = it >= args.warmup
         ev = []
+        x_send = [None] * R
         for r in range(R):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            routed[r] = moe.moe_route(xs[r], Wg, w.K, workspace=ws_route[r])
-            e1.record()
-            ev.append(("route", r, e0, e1))
+            def route_stage(r=r):
+                routed[r] = moe.moe_route(xs[r], Wg, w.K, workspace=ws_route[r])
+                return routed[r][0] if ident[r] else moe.moe_gather_rows(routed[r][0], perms[r])
+            x_send[r], e = timed(route_stage)
+            ev.append(("route", r, e))
+        # the dispatch, by slicing (untimed): rank q receives its slice of every source
+        x_recv = [torch.cat([x_send[s][starts[s][q]:starts[s][q + 1]] for s in range(R)])
+                  for q in range(R)]
         y_recv = []
         for q in range(R):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            y_recv.append(moe.moe_experts_forward(x_recv[q], seg[q], local[q]["W1"],
-                                                  local[q]["W3"], local[q]["W2"],
-                                                  workspace=ws_exp[q]))
-            e1.record()
-            ev.append(("experts", q, e0, e1))
+            y, e = timed(lambda q=q: moe.moe_experts_forward(
+                x_recv[q], segs[q], local[q]["W1"], local[q]["W3"], local[q]["W2"],
+                workspace=ws_exp[q]))
+            y_recv.append(y)
+            ev.append(("experts", q, e))
         for s in range(R):  # the return, by slicing (untimed)
             parts_s = []
             for q in range(R):
-                recv = ep.ExpertPartition.recv_splits(seg[q].cpu())
-                parts_s.append(y_recv[q][sum(recv[:s]):sum(recv[:s + 1])])
-            y_back = torch.cat(parts_s)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            moe.moe_combine(y_back, routed[s][4], routed[s][2], outs[s])
-            e1.record()
-            ev.append(("combine", s, e0, e1))
+                off = int(segs[q][:s].sum())
+                parts_s.append(y_recv[q][off:off + int(segs[q][s].sum())])
+            y_send_back = torch.cat(parts_s)
+
+            def combine_stage(s=s, y_send_back=y_send_back):
+                y_back = y_send_back if ident[s] else moe.moe_gather_rows(y_send_back, invs[s])
+                moe.moe_combine(y_back, routed[s][4], routed[s][2], outs[s])
+            _, e = timed(combine_stage)
+            ev.append(("combine", s, e))
         torch.cuda.synchronize()
-        if timed:
-            for kind, r, e0, e1 in ev:
+        if it >= args.warmup:
+            for kind, r, (e0, e1) in ev:
                 {"route": t_route, "experts": t_exp, "combine": t_comb}[kind][r].append(
                     e0.elapsed_time(e1))
-    for ws in ws_route + ws_exp:
-        code, raw = moe.moe_workspace_status(ws)
+    for wsp in ws_route + ws_exp:
+        code, raw = moe.moe_workspace_status(wsp)
         if code != 0:
             raise RuntimeError(f"device status {code} ({raw:#x})")
-    med = lambda v: statistics.median(v)
+    med = statistics.median
     route_ms = [med(t) for t in t_route]
     exp_ms = [med(t) for t in t_exp]
     comb_ms = [med(t) for t in t_comb]
-    # bytes that cross NVLink (rows for other ranks only): dispatch bf16 rows, return fp32
-    out_rows = [sum(send[s][q] for q in range(R) if q != s) for s in range(R)]
-    in_rows = [sum(send[s][q] for s in range(R) if s != q) for q in range(R)]
-    disp = max(max(o, i) for o, i in zip(out_rows, in_rows)) * w.d * es
-    ret = max(max(o, i) for o, i in zip(out_rows, in_rows)) * w.d * 4
+    # rows that cross NVLink (parts for other ranks only): dispatch bf16 rows, return fp32
+    out_rows = [sum(plans[s][1][q] for q in range(R) if q != s) for s in range(R)]
+    in_rows = [sum(int(segs[q][s].sum()) for s in range(R) if s != q) for q in range(R)]
+    worst = max(max(o, i) for o, i in zip(out_rows, in_rows))
+    disp, ret = worst * w.d * es, worst * w.d * 4
     t_disp = disp / (NVLINK_GBS * 1e9) * 1e3
     t_ret = ret / (NVLINK_GBS * 1e9) * 1e3
     step = max(route_ms) + t_disp + max(exp_ms) + t_ret + max(comb_ms)
@@ -622,11 +646,12 @@ def run_ep_emulation(args, w):
     line = {
         "metric": "expert-parallel MoE block, emulated on one GPU (modelled step)",
         "value": round(R * w.T / (step / 1e3), 2), "unit": "tokens/s", "n_gpus": 1,
-        "ranks_emulated": R, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step_modelled": round(step, 5), "higher_is_better": True, "dtype": "bf16",
-        "data": "synthetic (seeded per rank)",
+        "ranks_emulated": R, "expert_slots_per_rank": slots, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step_modelled": round(step, 5),
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded per rank)",
         "config": {"workload": f"{workload_label(w)}, {R} ranks x {w.T} tokens, "
-                               f"{nl} experts per rank", "global_batch": R * w.T},
+                               f"{slots} expert slots per rank", "global_batch": R * w.T},
+        "placement": [list(r) for r in pl.replicas],
         "stage_ms_per_rank": {"route": [round(v, 5) for v in route_ms],
                               "experts": [round(v, 5) for v in exp_ms],
                               "combine": [round(v, 5) for v in comb_ms]},
@@ -785,6 +810,9 @@ def main(argv=None):
     ap.add_argument("--ep-emulate", type=int, default=0, metavar="R",
                     help="expert parallelism over R ranks emulated on one GPU: measured GPU "
                          "stages per rank, all-to-alls modelled from their bytes")
+    ap.add_argument("--ep-slots", type=int, default=0, metavar="C",
+                    help="with --ep-emulate: expert slots per rank; more than n / R replicates "
+                         "the hot experts (balanced placement over the measured loads)")
     ap.add_argument("--gather-x", action="store_true",
                     help="CTA-pair path: gather G13's A rows from x (TMA gather4) instead of "
                          "X_perm, gates applied in G2 (sets MOE_GATHER_X=1)")

@@ -300,6 +300,16 @@ MOE_API moe_status moe_combine(const float* y_rows, const int32_t* token_rows,
                                const float* topk_gate, int64_t T, int64_t d, int K, moe_dtype dt,
                                void* out, void* stream);
 
+/* Row gather for the expert-parallel exchange when experts are replicated over ranks (the
+ * hada.io page, "Implementasi dan Efisiensi Inferensi": the load across GPUs must be
+ * balanced; moving rows is plumbing): out[i] = in[index[i]] for 0 <= i < rows, each row
+ * row_bytes bytes (a multiple of 16); in has in_rows rows; an index outside [0, in_rows)
+ * leaves out row i unwritten.  Device pointers: in and out 16-byte aligned and distinct,
+ * index int32 4-byte aligned.  Enqueued on `stream`; MOE_ERR_INVALID_ARG on bad arguments
+ * before any launch. */
+MOE_API moe_status moe_gather_rows(const void* in, int64_t in_rows, const int32_t* index,
+                                   int64_t rows, int64_t row_bytes, void* out, void* stream);
+
 /* Test hook for the failure path (no counterpart in the pages): moe_forward, except that the
  * one-CTA tensor-core kernel of the gate/up projection issues none of its loads, so its
  * tensor-core thread waits on a barrier that nothing will complete; that wait, and the other

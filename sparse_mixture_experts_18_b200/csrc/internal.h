@@ -157,6 +157,10 @@ cudaError_t launch_combine_rows(const float* Y, int S, int64_t split_stride, int
 // per-expert layout of the plan (X_perm, counts, offsets, inv = padded row of each row).
 cudaError_t launch_ep_regroup(const Plan& p, const void* x_rows, const int32_t* seg_counts,
                               int S, const Workspace& w, cudaStream_t s);
+// out[i] = in[index[i]], rows of row_bytes (a multiple of 16) bytes; indices outside
+// [0, in_rows) leave their row unwritten.
+cudaError_t launch_gather_rows(const void* in, int64_t in_rows, const int32_t* index,
+                               int64_t rows, int64_t row_bytes, void* out, cudaStream_t s);
 cudaError_t launch_rmsnorm(const void* x, void* xn, int64_t T, int64_t d, float eps,
                            cudaStream_t s);
 int num_sms();

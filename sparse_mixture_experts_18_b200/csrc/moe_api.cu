@@ -587,6 +587,20 @@ moe_status moe_combine(const float* y_rows, const int32_t* token_rows, const flo
              : MOE_ERR_CUDA;
 }
 
+moe_status moe_gather_rows(const void* in, int64_t in_rows, const int32_t* index, int64_t rows,
+                           int64_t row_bytes, void* out, void* stream) {
+  if (in_rows < 0 || rows < 0 || row_bytes <= 0 || row_bytes % 16) return MOE_ERR_INVALID_ARG;
+  if (row_bytes > ((int64_t)1 << 24) || rows > ((int64_t)1 << 40)) return MOE_ERR_UNSUPPORTED;
+  if (rows == 0) return MOE_OK;
+  if (!in || !index || !out || !aligned(in, 16) || !aligned(out, 16) || !aligned(index, 4) ||
+      in == out)
+    return MOE_ERR_INVALID_ARG;
+  return launch_gather_rows(in, in_rows, index, rows, row_bytes, out,
+                            static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
 moe_status moe_debug_forward_withheld(const void* x, const float* W_g, const void* W1,
                                       const void* W3, const void* W2, int64_t T, int64_t d,
                                       int64_t F, int n, int K, moe_dtype dt, void* out,

@@ -689,6 +689,49 @@ cudaError_t launch_ep_regroup(const Plan& p, const void* x_rows, const int32_t* 
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- row gather
+// out[i] = in[index[i]] for rows of vpr 16-byte vectors (the expert-parallel exchange with
+// replicated experts puts a rank's grouped rows in destination order and its returned rows
+// back in grouped order with it).  One warp per output row, U loads in flight per lane; an
+// index outside [0, in_rows) leaves its output row unwritten.
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint4* __restrict__ in, int64_t in_rows,
+                       const int32_t* __restrict__ index, int64_t rows, int vpr,
+                       uint4* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int U = 8;
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); r < rows;
+       r += (int64_t)gridDim.x * 8) {  // warp-uniform
+    const int64_t src = index[r];
+    if (src < 0 || src >= in_rows) continue;
+    const uint4* sp = in + src * vpr;
+    uint4* dp = out + r * vpr;
+    for (int c0 = lane; c0 < vpr; c0 += 32 * U) {
+      uint4 buf[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + 32 * u < vpr) buf[u] = __ldg(sp + c0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + 32 * u < vpr) dp[c0 + 32 * u] = buf[u];
+    }
+  }
+}
+
+cudaError_t launch_gather_rows(const void* in, int64_t in_rows, const int32_t* index,
+                               int64_t rows, int64_t row_bytes, void* out, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  int64_t blocks = (rows + 7) / 8;
+  const int64_t cap = 8 * (int64_t)num_sms();
+  if (blocks > cap) blocks = cap;
+  pdl(gather_rows_kernel, (unsigned)blocks, 256, 0, s)(
+      static_cast<const uint4*>(in), in_rows, index, rows, (int)(row_bytes / 16),
+      static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- host launchers
 
 // Tokens per router / permute block: eight, or fewer when K > 8 so that a block's

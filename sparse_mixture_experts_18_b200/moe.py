@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
                                           P]
         L.moe_combine.restype = I32
         L.moe_combine.argtypes = [P, P, P, I64, I64, I32, I32, P, P]
+        L.moe_gather_rows.restype = I32
+        L.moe_gather_rows.argtypes = [P, I64, P, I64, I64, P, P]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [I32]
         L.moe_abi_version.restype = I32
@@ -356,6 +358,21 @@ def moe_experts_forward(x_rows, seg_counts, W1, W3, W2, workspace=None, stream=N
         _ptr(x_rows), rows, _ptr(seg_counts.contiguous()), S, _ptr(W1), _ptr(W3), _ptr(W2), d,
         F, nl, dt, _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)))
     return y
+
+
+def moe_gather_rows(rows_in, index, out=None, stream=None):
+    """out[i] = rows_in[index[i]] (index: int32 on the device); rows of any dtype whose byte
+    width is a multiple of 16."""
+    n_out = index.shape[0]
+    if out is None:
+        out = torch.empty((n_out,) + tuple(rows_in.shape[1:]), dtype=rows_in.dtype,
+                          device=rows_in.device)
+    row_bytes = rows_in[0].numel() * rows_in.element_size() if rows_in.shape[0] else \
+        out[0].numel() * out.element_size() if n_out else 16
+    _check("moe_gather_rows", lib().moe_gather_rows(
+        _ptr(rows_in), rows_in.shape[0], _ptr(index.contiguous()), n_out, row_bytes, _ptr(out),
+        _stream(stream)))
+    return out
 
 
 def moe_combine(y_rows, token_rows, topk_gate, out, stream=None):

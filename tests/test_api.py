@@ -272,3 +272,14 @@ def test_quantize_mx_validation(L):
     assert q(P(0x1004), 128, 128, P(0x2000), P(0x3000), None) == INVALID    # v not 8-byte aligned
     assert q(P(0x1000), 128, 128, P(0x2000), P(0x3008), None) == INVALID    # sf not 16-byte
     assert q(P(0x1000), 0, 128, None, None, None) == OK                     # no rows: no-op
+
+
+def test_gather_rows_validation(L):
+    g = L.moe_gather_rows
+    assert g(P(0x1000), 10, P(0x2000), 5, 24, P(0x3000), None) == INVALID    # row bytes % 16
+    assert g(None, 10, P(0x2000), 5, 32, P(0x3000), None) == INVALID
+    assert g(P(0x1008), 10, P(0x2000), 5, 32, P(0x3000), None) == INVALID    # in not 16-byte
+    assert g(P(0x1000), 10, P(0x2002), 5, 32, P(0x3000), None) == INVALID    # index not 4-byte
+    assert g(P(0x1000), 10, P(0x2000), 5, 32, P(0x1000), None) == INVALID    # in == out
+    assert g(P(0x1000), -1, P(0x2000), 5, 32, P(0x3000), None) == INVALID
+    assert g(None, 0, None, 0, 32, None, None) == OK                          # no rows: no-op

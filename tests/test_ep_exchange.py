@@ -128,3 +128,111 @@ def test_partition_and_load_bookkeeping():
     loads = [28081, 12230, 7519, 5326, 4073, 3270, 2719, 2318]
     assert ep.load_per_rank(loads, 2) == [53156, 12380]
     assert max(ep.load_per_rank(loads, 8)) / sum(loads) == pytest.approx(0.4285, abs=1e-3)
+
+
+# ------------------------------------------------------------------ replicated experts
+
+SKEWED_LOADS = [28081, 12230, 7519, 5326, 4073, 3270, 2719, 2318]
+
+
+def test_balanced_placement_invariants():
+    from sparse_mixture_experts_18_b200 import ep
+    for world, slots in [(2, 4), (2, 6), (4, 2), (4, 3), (8, 1), (8, 2), (8, 4)]:
+        pl = ep.ExpertPlacement.balanced(SKEWED_LOADS, world, slots)
+        held = [pl.local_experts(q) for q in range(world)]
+        assert all(len(h) <= slots for h in held)
+        assert all(len(r) >= 1 for r in pl.replicas)
+        # the contiguous placement is kept: every expert stays on its home rank
+        assert all(e // (8 // world) in pl.replicas[e] for e in range(8))
+        load = pl.load_per_rank(SKEWED_LOADS)
+        assert sum(load) == pytest.approx(sum(SKEWED_LOADS))
+        if slots == 8 // world:
+            assert pl == ep.ExpertPlacement.contiguous(8, world)
+        else:  # more slots never make the busiest rank busier, and here they help
+            base = max(ep.load_per_rank(SKEWED_LOADS, world))
+            assert max(load) < base
+    # 8 ranks with two slots each: the busiest rank drops from 42.8% of the rows to <= 21.5%
+    pl = ep.ExpertPlacement.balanced(SKEWED_LOADS, 8, 2)
+    assert max(pl.load_per_rank(SKEWED_LOADS)) / sum(SKEWED_LOADS) <= 0.215
+    assert len(pl.replicas[0]) >= 4
+
+
+def test_send_order_and_receive_counts():
+    from sparse_mixture_experts_18_b200 import ep
+    pl = ep.ExpertPlacement(8, 4, ((0, 2, 3), (0, 1), (0, 1), (1,), (2,), (2,), (3,), (3,)))
+    counts = [5, 3, 2, 1, 0, 0, 1, 2]
+    order, send = pl.send_order(counts)
+    assert sorted(order) == list(range(sum(counts)))          # every grouped row once
+    assert order == [0, 1, 5, 6, 8, 7, 9, 10, 2, 3, 4, 11, 12, 13] and send == [5, 3, 2, 4]
+    assert ep.ExpertPlacement.split(5, 3) == [2, 2, 1] and ep.ExpertPlacement.split(0, 2) == [0, 0]
+    all_counts = [counts, [0, 4, 1, 0, 0, 0, 0, 0], [7, 0, 0, 0, 3, 0, 0, 0], [1] * 8]
+    for q in range(4):
+        seg = pl.recv_counts(all_counts, q)
+        # what q receives from s is what s sends to q
+        assert [sum(r) for r in seg] == [pl.send_order(all_counts[s])[1][q] for s in range(4)]
+    with pytest.raises(ValueError):
+        ep.ExpertPlacement(8, 4, ((0,),) * 7)
+    with pytest.raises(ValueError):
+        ep.ExpertPlacement(8, 4, ((1, 0),) * 8)
+
+
+def _placed_worker(rank, world, port, Ts, n, slots, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import moe_inputs
+    import oracle
+    from sparse_mixture_experts_18_b200 import ep
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        K, d = 2, 64
+        T = Ts[rank]
+        w = moe_inputs.small(T=max(T, 1), d=d, F=64, n=n, K=K, dtype="f32", rms_x=False,
+                             seed=300 + rank)
+        x = moe_inputs.make_x(w)[:T]
+        Wg = moe_inputs.make_layer(w.replace(seed=9))["Wg"]
+        idx = oracle.route(x, Wg, n, K)[1] if T else np.zeros((0, K), np.int32)
+        xg, rows, counts, row_expert = _group_rows(x, idx, n, K)
+        all_counts = ep.exchange_all_counts(torch.from_numpy(counts), world).numpy()
+        pl = ep.ExpertPlacement.balanced(all_counts.sum(axis=0), world, slots)
+        order, send = pl.send_order(all_counts[rank])
+        seg = pl.recv_counts(all_counts, rank)
+        recv = [sum(r) for r in seg]
+        x_send = xg[torch.tensor(order, dtype=torch.long)] if order else xg
+        x_recv = ep.dispatch(x_send, send, recv)
+        # the expert of every received row: source-major, the rank's experts in order
+        local = pl.local_experts(rank)
+        got_e = [e for s in range(world) for e, c in zip(local, seg[s]) for _ in range(c)]
+        y_recv = _stand_in_expert(x_recv, got_e)
+        y_send_back = ep.return_rows(y_recv, send, recv)
+        y_back = torch.empty_like(y_send_back)
+        if order:
+            y_back[torch.tensor(order, dtype=torch.long)] = y_send_back
+        back_ok = torch.equal(y_back, _stand_in_expert(xg, row_expert))
+        pos_ok = all(torch.equal(y_back[rows[t, k]], x[t] * (1.0 + float(idx[t, k])))
+                     for t in range(T) for k in range(K))
+        q.put((rank, back_ok, pos_ok, sum(recv), max(pl.load_per_rank(all_counts.sum(axis=0)))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,Ts,n,slots", [(2, (37, 21), 8, 6), (4, (11, 3, 20, 9), 8, 3)])
+def test_replicated_dispatch_and_return_over_gloo(world, Ts, n, slots):
+    """Rows of replicated experts reach every replica's rank in their parts and come back to
+    their sender's grouped order bit for bit."""
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_placed_worker, args=(r, world, port, Ts, n, slots, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, back_ok, pos_ok, _, _ in res:
+        assert back_ok, rank
+        assert pos_ok, rank
+    assert sum(r[3] for r in res) == sum(Ts) * 2

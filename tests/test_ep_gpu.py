@@ -121,6 +121,78 @@ def test_emulated_expert_parallel_mixtral_shapes():
                               outs[r], idxs[r], budget=48)
 
 
+def _emulated_ep_placed(ws, xs, layer, R, slots):
+    """As _emulated_ep with hot experts replicated (ExpertPlacement.balanced over the global
+    loads): each source's grouped rows go into destination order with moe_gather_rows, each
+    rank runs its experts (replicas included) on the parts it receives, and the returned rows
+    go back into grouped order with moe_gather_rows before the combine."""
+    n, K = ws[0].n, ws[0].K
+    routed = [moe.moe_route(x, layer["Wg"], K) for x in xs]     # (xg, idx, gate, counts, rows)
+    all_counts = torch.stack([r[3] for r in routed]).cpu()
+    pl = ep.ExpertPlacement.balanced(all_counts.sum(dim=0), R, slots)
+    plans = [pl.send_order(all_counts[s]) for s in range(R)]
+    perms = [torch.tensor(o, dtype=torch.int32, device="cuda") for o, _ in plans]
+    x_send = [moe.moe_gather_rows(routed[s][0], perms[s]) for s in range(R)]
+    starts = [[sum(plans[s][1][:q]) for q in range(R + 1)] for s in range(R)]
+    y_parts = [[None] * R for _ in range(R)]
+    for q in range(R):
+        local = pl.local_experts(q)
+        seg = torch.tensor(pl.recv_counts(all_counts, q), dtype=torch.int32)
+        x_recv = torch.cat([x_send[s][starts[s][q]:starts[s][q + 1]] for s in range(R)])
+        idx = torch.tensor(local, device="cuda")
+        y_recv = moe.moe_experts_forward(x_recv, seg.cuda(), layer["W1"][idx].contiguous(),
+                                         layer["W3"][idx].contiguous(),
+                                         layer["W2"][idx].contiguous())
+        off = 0
+        for s in range(R):
+            c = int(seg[s].sum())
+            y_parts[s][q] = y_recv[off:off + c]
+            off += c
+    outs = []
+    for s in range(R):
+        y_send_back = torch.cat(y_parts[s])
+        inv = torch.empty_like(perms[s])
+        inv[perms[s].long()] = torch.arange(len(perms[s]), dtype=torch.int32, device="cuda")
+        y_back = moe.moe_gather_rows(y_send_back, inv)
+        out = torch.empty_like(xs[s])
+        moe.moe_combine(y_back, routed[s][4], routed[s][2], out)
+        outs.append(out)
+    torch.cuda.synchronize()
+    return outs, [r[1] for r in routed], pl
+
+
+@pytest.mark.parametrize("R,T,n,slots", [(2, 700, 8, 6), (4, 333, 8, 3), (4, 1500, 8, 4)])
+def test_emulated_expert_parallel_with_replicas(R, T, n, slots):
+    ws = [moe_inputs.small(name=f"epr{R}_rank{r}", T=T + 13 * r, d=256, F=384, n=n, K=2,
+                           seed=40 + r) for r in range(R)]
+    layer = {k: v.cuda() for k, v in moe_inputs.make_layer(ws[0].replace(seed=5)).items()}
+    xs = [moe_inputs.make_x(w).cuda() for w in ws]
+    outs, idxs, pl = _emulated_ep_placed(ws, xs, layer, R, slots)
+    assert any(len(r) > 1 for r in pl.replicas)
+    for r in range(R):
+        _check_against_oracle(f"EP x{R} replicated ({slots} slots) rank {r}: T={ws[r].T}",
+                              ws[r], xs[r], layer, outs[r], idxs[r])
+
+
+def test_gather_rows():
+    g = torch.Generator().manual_seed(2)
+    src = torch.randn(300, 64, generator=g).cuda()
+    index = torch.randint(0, 300, (500,), generator=g, dtype=torch.int32).cuda()
+    index[7] = -1                                   # out of range: row left unwritten
+    index[9] = 300
+    out = torch.full((500, 64), 7.0, device="cuda")
+    moe.moe_gather_rows(src, index, out=out)
+    torch.cuda.synchronize()
+    ok = index.long().clamp(0, 299)
+    ref = src[ok]
+    ref[7] = 7.0
+    ref[9] = 7.0
+    assert torch.equal(out, ref)
+    xb = torch.randn(10, 4096, generator=g).to(torch.bfloat16).cuda()
+    assert torch.equal(moe.moe_gather_rows(xb, torch.tensor([9, 0, 3], dtype=torch.int32,
+                                                            device="cuda")), xb[[9, 0, 3]])
+
+
 @pytest.mark.parametrize("w", [moe_inputs.small(T=200, d=256, F=384),
                                moe_inputs.WORKLOADS["decode_t16"]], ids=["small", "decode_t16"])
 def test_forward_ep_single_rank(w):
