@@ -244,9 +244,11 @@ def _forward_placed(x, W_g, W1_local, W3_local, W2_local, K, placement, group, o
     order, send = placement.send_order(all_counts[rank])
     seg = placement.recv_counts(all_counts, rank)
     recv = [sum(r) for r in seg]
-    perm = torch.tensor(order, dtype=torch.int32, device=x.device)
-    inv = torch.empty_like(perm)
-    inv[perm.long()] = torch.arange(len(order), dtype=torch.int32, device=x.device)
+    inv_order = [0] * len(order)  # host bookkeeping: where each grouped row went
+    for i, r in enumerate(order):
+        inv_order[r] = i
+    perm = torch.tensor(order, dtype=torch.int32).to(x.device)
+    inv = torch.tensor(inv_order, dtype=torch.int32).to(x.device)
     x_send = moe.moe_gather_rows(xg, perm, stream=stream) if len(order) else xg
     x_recv = dispatch(x_send, send, recv, group)
     y_recv = moe.moe_experts_forward(
