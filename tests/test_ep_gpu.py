@@ -205,3 +205,20 @@ def test_forward_ep_single_rank(w):
     assert rep["ok"], rep
     _, idx, _, _, _ = moe.moe_route(x, L["Wg"], w.K)
     _check_against_oracle(f"EP x1: {w.name} T={w.T}", w, x, L, out, idx)
+
+
+def test_forward_ep_placed_single_rank():
+    """The placement path of moe_forward_ep on one rank (counts all-gather, row gathers, the
+    local experts, combine) against moe_forward and the oracle."""
+    w = moe_inputs.small(T=300, d=256, F=384)
+    x = moe_inputs.make_x(w, device="cuda")
+    L = moe_inputs.make_layer(w, device="cuda")
+    pl = ep.ExpertPlacement.contiguous(w.n, 1)
+    out = ep.moe_forward_ep(x, L["Wg"], L["W1"], L["W3"], L["W2"], w.K, placement=pl)
+    ref = moe.moe_forward(x, L["Wg"], L["W1"], L["W3"], L["W2"], w.K)
+    torch.cuda.synchronize()
+    rep = parity.compare_outputs(out.float().cpu().numpy(), ref.double().cpu().numpy(), x.dtype)
+    assert rep["ok"], rep
+    _, idx, _, _, _ = moe.moe_route(x, L["Wg"], w.K)
+    _check_against_oracle(f"EP x1 placed: T={w.T}", w, x, L, out, idx)
+
