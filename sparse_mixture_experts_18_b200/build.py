@@ -19,7 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = ["route.cu", "route_tc.cu", "gemm_tc.cu", "gemm_simt.cu", "combine.cu", "moe_api.cu", "moe_noalloc.cu"]
+SOURCES = ["route.cu", "route_tc.cu", "gemm_tc.cu", "gemm_simt.cu", "combine.cu", "quantize.cu",
+           "moe_api.cu", "moe_noalloc.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",

@@ -277,6 +277,13 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Four E4M3 codes of v * inv (inv a power of two), lowest address in the lowest byte.
+__device__ __forceinline__ uint32_t e4m3x4_mul(float v0, float v1, float v2, float v3,
+                                               float inv) {
+  return (uint32_t)cvt_e4m3x2(v0 * inv, v1 * inv) |
+         ((uint32_t)cvt_e4m3x2(v2 * inv, v3 * inv) << 16);
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(

@@ -849,13 +849,6 @@ __global__ void __launch_bounds__(256)
 // One warp per (row, 128 columns): lane c holds columns 4c .. 4c + 3, so a 32-element block is
 // 8 lanes and the K block's four scale codes are those of lanes 0, 8, 16 and 24.
 
-// Four E4M3 codes of v * inv (inv a power of two), lowest address in the lowest byte.
-__device__ __forceinline__ uint32_t e4m3x4_mul(float v0, float v1, float v2, float v3,
-                                               float inv) {
-  return (uint32_t)cvt_e4m3x2(v0 * inv, v1 * inv) |
-         ((uint32_t)cvt_e4m3x2(v2 * inv, v3 * inv) << 16);
-}
-
 // The block scale of this lane's 8-lane group and the K block's scale word (codes of the four
 // groups, the lowest columns in the lowest byte; the same value on every lane).
 __device__ __forceinline__ uint32_t mx_group_scale(float amax, float* inv, uint32_t* word) {
@@ -866,30 +859,6 @@ __device__ __forceinline__ uint32_t mx_group_scale(float amax, float* inv, uint3
   *word = __shfl_sync(0xffffffffu, code, 0) | (__shfl_sync(0xffffffffu, code, 8) << 8) |
           (__shfl_sync(0xffffffffu, code, 16) << 16) | (__shfl_sync(0xffffffffu, code, 24) << 24);
   return code;
-}
-
-// Weights: [rows][cols] bf16 -> codes q [rows][cols] and scales in the tile order the GEMMs
-// read: the word of row r, K block kb at byte ((r / 128) * (cols / 128) + kb) * 512
-// + 16 (r % 32) + 4 ((r % 128) / 32).  rows and cols multiples of 128.
-__global__ void __launch_bounds__(256)
-    quantize_mx_e4m3_kernel(const __nv_bfloat16* __restrict__ v, int64_t rows, int64_t cols,
-                            uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
-  const int lane = threadIdx.x & 31;
-  const int64_t kbs = cols / 128;
-  for (int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); gw < rows * kbs;
-       gw += (int64_t)gridDim.x * 8) {  // warp-uniform
-    const int64_t r = gw / kbs, kb = gw % kbs;
-    const int64_t c = kb * 128 + lane * 4;
-    const uint2 raw = *reinterpret_cast<const uint2*>(v + r * cols + c);
-    const float f0 = bf16_lo(raw.x), f1 = bf16_hi(raw.x), f2 = bf16_lo(raw.y), f3 = bf16_hi(raw.y);
-    float inv;
-    uint32_t word;
-    mx_group_scale(fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))), &inv, &word);
-    *reinterpret_cast<uint32_t*>(q + r * cols + c) = e4m3x4_mul(f0, f1, f2, f3, inv);
-    if (lane == 0)
-      *reinterpret_cast<uint32_t*>(sf + ((r / 128) * kbs + kb) * 512 + 16 * (r % 32) +
-                                   4 * ((r % 128) / 32)) = word;
-  }
 }
 
 // FP8 small batch: permuted row r of expert e (rows grouped by offsets, slot j = r -
@@ -1246,17 +1215,6 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
       cudaSuccess)
     return err;
   return record(ev, 2, s);
-}
-
-cudaError_t launch_quantize_mx_e4m3(const void* v, int64_t rows, int64_t cols, uint8_t* q,
-                                    uint8_t* sf, cudaStream_t s) {
-  if (rows <= 0) return cudaSuccess;
-  const int64_t warps = rows * (cols / 128);
-  int64_t blocks = (warps + 7) / 8;
-  if (blocks > 64 * (int64_t)num_sms()) blocks = 64 * (int64_t)num_sms();
-  quantize_mx_e4m3_kernel<<<(unsigned)blocks, 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(v), rows, cols, q, sf);
-  return cudaGetLastError();
 }
 
 // The small-batch tiling of launch_expert_gemms_tc on MXFP8 codes: G13 partial sums (block
