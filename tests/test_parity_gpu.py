@@ -109,6 +109,20 @@ def test_small_batch_tiling(T):
     _run(moe_inputs.small(T=T, d=512, F=768))
 
 
+@pytest.mark.parametrize("T,small,pair", [(64, True, False), (65, True, False),
+                                           (255, True, False), (256, False, False),
+                                           (1023, False, False), (1024, False, False),
+                                           (2559, False, False), (2560, False, True)])
+def test_path_selection_boundaries(T, small, pair):
+    """Both sides of every tiling switch (n = 8, K = 2): the one-launch routing (T <= 64), the
+    small-batch tiling (T*K < 64 n), the tensor-core router (T >= 1024) and the CTA pairs
+    (T*K >= 640 n)."""
+    w = moe_inputs.small(T=T, d=256, F=384)
+    plan = moe.moe_plan_info(w.T, w.d, w.F, w.n, w.K)
+    assert plan["small_batch"] == small and plan["pair"] == pair, plan
+    _run(w, budget=200)
+
+
 @pytest.mark.parametrize("n,K", [(8, 1), (4, 4), (16, 2), (64, 2), (1, 1), (32, 3)])
 def test_expert_counts(n, K):
     _run(moe_inputs.small(T=333, d=256, F=256, n=n, K=K))
