@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(RS_THREADS)
       if (t < T && j0[q] < d) xv[q].load(x + (int64_t)t * d + j0[q]);
     }
     if constexpr (std::is_same<Tact, __nv_bfloat16>::value) {
+      static_assert(CPL == 1, "the MXFP8 blocks below assume 8 columns per lane");
       if (xq != nullptr) {  // FP8-weight block: this CTA's 64 columns of the token as MXFP8
         // lanes sub 0-3 and 4-7 of the token hold one 32-element block each
         const bool have = t < T && j0[0] < d;
