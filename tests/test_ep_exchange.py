@@ -217,7 +217,8 @@ def _placed_worker(rank, world, port, Ts, n, slots, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,Ts,n,slots", [(2, (37, 21), 8, 6), (4, (11, 3, 20, 9), 8, 3)])
+@pytest.mark.parametrize("world,Ts,n,slots", [(2, (37, 21), 8, 6), (4, (11, 3, 20, 9), 8, 3),
+                                              (2, (0, 9), 8, 5)])
 def test_replicated_dispatch_and_return_over_gloo(world, Ts, n, slots):
     """Rows of replicated experts reach every replica's rank in their parts and come back to
     their sender's grouped order bit for bit."""
