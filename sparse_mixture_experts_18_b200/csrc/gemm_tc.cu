@@ -971,13 +971,9 @@ static cudaError_t launch_one(const CUtensorMap& mx, const CUtensorMap& mw0,
                               const CUtensorMap& mw1, TcArgs a, int max_work, cudaStream_t s) {
   const size_t smem = (size_t)a.stages * a.stage_bytes + sizeof(Ctrl) + 1024;
   auto kern = tc_grouped_gemm_kernel<KIND, SWAP, E4M3>;
-  static int configured = 0;
-  if (configured < (int)smem) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = (int)smem;
-  }
+  static int configured[MAX_DEVICES] = {0};
+  const cudaError_t e = ensure_dynamic_smem(kern, smem, configured);
+  if (e != cudaSuccess) return e;
   const int grid = max_work < num_sms() ? (max_work > 0 ? max_work : 1) : num_sms();
   pdl(kern, grid, GEMM_THREADS, smem, s)(mx, mw0, mw1, a);
   return cudaGetLastError();
@@ -989,8 +985,8 @@ static cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw0,
                                const CUtensorMap& mw1h, TcArgs a, int max_work, cudaStream_t s) {
   const size_t smem = (size_t)a.stages * a.stage_bytes + sizeof(PairCtrl) + 1024;
   auto kern = tc_pair_gemm_kernel<KIND>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static int configured[MAX_DEVICES] = {0};
+  cudaError_t e = ensure_dynamic_smem(kern, smem, configured);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];

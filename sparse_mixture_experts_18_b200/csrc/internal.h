@@ -165,4 +165,20 @@ cudaError_t launch_rmsnorm(const void* x, void* xn, int64_t T, int64_t d, float 
                            cudaStream_t s);
 int num_sms();
 
+// Raise kernel `kern`'s dynamic shared-memory limit to at least `smem` bytes on the current
+// device; `configured` is the caller's per-device record for that kernel instance (a repeated
+// or concurrent first call only sets the attribute again).
+constexpr int MAX_DEVICES = 64;
+template <typename Kern>
+cudaError_t ensure_dynamic_smem(Kern kern, size_t smem, int (&configured)[MAX_DEVICES]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool tracked = dev >= 0 && dev < MAX_DEVICES;
+  if (tracked && configured[dev] >= (int)smem) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && tracked) configured[dev] = (int)smem;
+  return e;
+}
+
 }  // namespace moe

@@ -319,13 +319,9 @@ static cudaError_t launch_rtc(const CUtensorMap& mx, const CUtensorMap& mw, cons
   int stages = 0;
   const size_t smem = rtc_smem(npad, &stages);
   auto kern = router_tc_kernel<CS, MAXN>;
-  static int configured = 0;
-  if (configured < (int)smem) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = (int)smem;
-  }
+  static int configured[MAX_DEVICES] = {0};
+  const cudaError_t e = ensure_dynamic_smem(kern, smem, configured);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
