@@ -50,9 +50,9 @@ DEFAULT_WORKLOAD = "stack32_t8192"
 # of that kernel on the workload's shapes (for the stack: one T=8192 block), valid only for
 # the kernel source it was taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "stack32_t8192": {"bytes": 2811173376, "src": "21044c931415"},
-    "decode_t16": {"bytes": 1886850816, "src": "21044c931415"},
-    "decode_t16 mxfp8": {"bytes": 970451968, "src": "21044c931415"},
+    "stack32_t8192": {"bytes": 2668023552, "src": "c7be512be9be"},
+    "decode_t16": {"bytes": 1886525440, "src": "c7be512be9be"},
+    "decode_t16 mxfp8": {"bytes": 973218816, "src": "c7be512be9be"},
 }
 
 
