@@ -94,12 +94,13 @@ def test_all_tokens_to_two_experts_gather_x(monkeypatch, T):
 
 @pytest.mark.parametrize("T,d,n,K", [(1024, 4096, 8, 2), (1100, 4096, 8, 2), (2501, 4096, 8, 2),
                                      (1500, 256, 5, 2), (1300, 320, 12, 3), (1030, 512, 16, 8),
-                                     (1100, 256, 32, 3), (1500, 512, 48, 2), (1024, 256, 64, 4)])
+                                     (1100, 256, 32, 3), (1500, 512, 48, 2), (1024, 256, 64, 4),
+                                     (1030, 64, 8, 2), (1100, 192, 8, 2), (4100, 8192, 8, 2)])
 def test_router_tc_tiles(T, d, n, K):
     # the tensor-core router (T >= 1024, n <= 64, K <= 8): an exact multiple of its 128-token
-    # tile, ragged last tiles, clusters splitting d (4 where d / 64 allows, 1 at d = 320), and
-    # accumulators of 16 (n = 5) to 192 (n = 64) columns; a narrow expert width keeps the
-    # oracle quick
+    # tile, ragged last tiles, clusters splitting d (4 where d / 64 allows, 1 at d = 320), a
+    # single and three K blocks (d = 64, 192), a wide d (8192), and accumulators of 16
+    # (n = 5) to 192 (n = 64) columns; a narrow expert width keeps the oracle quick
     _run(moe_inputs.small(T=T, d=d, F=128, n=n, K=K), budget=300)
 
 
