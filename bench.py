@@ -50,9 +50,11 @@ DEFAULT_WORKLOAD = "stack32_t8192"
 # of that kernel on the workload's shapes (for the stack: one T=8192 block), valid only for
 # the kernel source it was taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "stack32_t8192": {"bytes": 2668023552, "src": "c7be512be9be"},
-    "decode_t16": {"bytes": 1886525440, "src": "c7be512be9be"},
-    "decode_t16 mxfp8": {"bytes": 973218816, "src": "c7be512be9be"},
+    "stack32_t8192": {"bytes": 2651231232, "src": "0b8972a94db6"},
+    "decode_t16": {"bytes": 1885249024, "src": "0b8972a94db6"},
+    "decode_t16 mxfp8": {"bytes": 970611456, "src": "0b8972a94db6"},
+    # captured at n = 8, T = 512 (the same 128 rows per expert), scaled by 8 to n = 64
+    "experts64_top2_t4096": {"bytes": 15262502912, "src": "0b8972a94db6"},
 }
 
 
@@ -313,7 +315,9 @@ def run_gpu(args, w):
     step_frac = (step_bytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"] if step_hbm
                  else tflops / bf16_peak)
     tiling = (f"small-batch swap-AB split-K {s13}/{s2}" if small_batch else
-              "CTA-pair 256-row tiles" if plan["pair"] else "128-row tiles")
+              "CTA-pair 256-row tiles" if plan["pair"] else
+              "weight-stationary tiles (128 weight rows x up to 256 token rows)" if plan["mid"]
+              else "128-row tiles")
     cap = TRAFFIC.get(w.name)
     traffic = cap["bytes"] if cap and cap["src"] == kernel_source_hash() else None
     workload = workload_label(w)

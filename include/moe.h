@@ -200,11 +200,14 @@ MOE_API moe_status moe_forward_profiled(const void* x, const float* W_g, const v
  *   *split13 / *split2 = K-splits of the two expert GEMMs on that path (1 otherwise);
  *   *launches = kernels one forward launches (a stack of them launches one more, the first
  *              block's RMSNorm, on the large-batch tilings);
- *   *pair = 1 if the expert GEMMs run on CTA pairs (256-row tiles).
+ *   *tiling = the expert GEMMs' tiling: 0 = 128-row token tiles (or the small-batch tiles
+ *             when *small_batch = 1), 1 = CTA pairs (256-row token tiles), 2 = mid-size
+ *             weight-stationary tiles (128 weight rows as the MMA's M, up to 256 of an
+ *             expert's token rows as its N).
  * Any output may be NULL. */
 MOE_API moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt,
                                  int* small_batch, int* split13, int* split2, int* launches,
-                                 int* pair);
+                                 int* tiling);
 
 /* Stack of L blocks on a residual stream (attention omitted), in place on x [T][d]:
  *   for l in 0..L-1:  x <- round(x + MoE_l(RMSNorm(x)))

@@ -67,6 +67,10 @@ struct TcArgs {
   // will complete and runs out after wait_limit cycles (0 on every forward call)
   long long wait_limit = WAIT_LIMIT_CYCLES;
   int withhold_loads = 0;
+  // weight-stationary tiles for mid-size groups (SWAP kernels): an expert's rows are taken
+  // in passes of up to tok_tile, each MMA's N is its pass's rows rounded up to 16, B rows come
+  // in 64-row boxes, and G13 writes h = bf16(silu(a) b) itself (no split-K)
+  int mid = 0;
   // MXFP8 (E4M3 kernels): E8M0 block scales of the A rows (W1 or W2; sfa1: W3) in the tensor
   // cores' tile order, one 512-byte chunk per (128-row tile, 128-wide K block); of the B rows
   // (the expert's token or h rows) one 512-byte chunk per (expert, K block), row slot j at
@@ -93,6 +97,7 @@ struct Ctrl {
   int nact;
   int off[MAX_EXPERTS + 1];
   int act[MAX_EXPERTS];
+  int pbase[MAX_EXPERTS + 1];      // mid: passes of the active experts before each
   int gtok[SMALL_ROUTE_MAX_ROWS];  // small batch gathering from x: token of each row
 };
 
@@ -104,7 +109,7 @@ struct Work {
 
 template <bool SWAP>
 __device__ __forceinline__ int total_work(const TcArgs& a, const Ctrl* c) {
-  if (SWAP) return c->nact * a.wb * a.splits;
+  if (SWAP) return a.mid ? c->pbase[c->nact] * a.wb : c->nact * a.wb * a.splits;
   return (c->off[a.n] / TILE_M) * a.n_tiles;
 }
 
@@ -113,7 +118,21 @@ __device__ __forceinline__ int total_work(const TcArgs& a, const Ctrl* c) {
 template <bool SWAP>
 __device__ __forceinline__ Work decode_work(const TcArgs& a, const Ctrl* c, int id) {
   Work w{};
-  if (SWAP) {
+  if (SWAP && a.mid) {
+    // active expert, then weight block, then pass (the passes over one weight block run side
+    // by side and share its stream through L2)
+    int ai = 0;
+    while (ai + 1 < c->nact && id >= c->pbase[ai + 1] * a.wb) ++ai;
+    const int np = c->pbase[ai + 1] - c->pbase[ai];
+    const int local = id - c->pbase[ai] * a.wb;
+    const int pass = local % np;
+    w.e = c->act[ai];
+    w.wblk = local / np;
+    w.s = 0;
+    w.row0 = c->off[w.e] + pass * a.tok_tile;
+    const int left = c->off[w.e + 1] - w.row0;
+    w.count = left < a.tok_tile ? left : a.tok_tile;
+  } else if (SWAP) {
     const int per = a.wb * a.splits;
     const int ai = id / per, rem = id % per;
     w.e = c->act[ai];
@@ -181,8 +200,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     int na = 0;
+    c->pbase[0] = 0;
     for (int e = 0; e < a.n; ++e)
-      if (c->off[e + 1] > c->off[e]) c->act[na++] = e;
+      if (c->off[e + 1] > c->off[e]) {
+        c->act[na] = e;
+        c->pbase[na + 1] = c->pbase[na] + (c->off[e + 1] - c->off[e] + a.tok_tile - 1) /
+                                              (a.tok_tile > 0 ? a.tok_tile : 1);
+        ++na;
+      }
     c->nact = na;
   }
   tc_fence_before();
@@ -203,8 +228,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // gathering: only the 4-row groups that hold this expert's rows are loaded; the MMA
         // columns of the other slots read whatever the stage holds and are never stored
         const int ngath = gather ? (w.count + 3) / 4 : 0;
+        const int nbox = a.mid ? (w.count + 63) / 64 : 0;  // mid: 64-row boxes of B rows
         const uint32_t tx =
-            gather ? a.tx_bytes - (uint32_t)(a.tok_tile / 4 - ngath) * 512u : a.tx_bytes;
+            gather ? a.tx_bytes - (uint32_t)(a.tok_tile / 4 - ngath) * 512u
+            : a.mid ? a.tx_bytes - (uint32_t)(a.tok_tile / 64 - nbox) * 8192u
+                    : a.tx_bytes;
         bool ok = true;
         for (int kb = 0; kb < a.num_kb; ++kb) {
           if (!mbar_wait(&c->empty[stage], phase ^ 1u, a.status, &c->abort, a.wait_limit)) {
@@ -246,6 +274,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 tma_gather4(st + a.x_off + g * 512, &tmX, fb, k, tk[0], tk[1], tk[2], tk[3],
                             pol_x);
               }
+            } else if (a.mid) {
+              for (int b = 0; b < nbox; ++b)
+                tma_load_2d(st + a.x_off + b * 8192, &tmX, fb, k, w.row0 + 64 * b, pol_x);
             } else {
               tma_load_2d(st + a.x_off, &tmX, fb, k, w.row0, pol_x);
             }
@@ -274,6 +305,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (!mbar_wait(&c->tempty[acc], aph ^ 1u, a.status, &c->abort, a.wait_limit)) break;
         tc_fence_after();
         const uint32_t dtm = tmem_base + acc * a.acc_cols;
+        uint32_t idesc_u = idesc;  // mid: N = this pass's rows rounded up to 16
+        if (SWAP && !E4M3 && a.mid) {
+          const Work wq = decode_work<SWAP>(a, c, id);
+          idesc_u = umma_idesc_bf16(128, (wq.count + 15) & ~15);
+        }
         for (int kb = 0; kb < a.num_kb; ++kb) {
           if (!mbar_wait(&c->full[stage], phase, a.status, &c->abort, a.wait_limit)) {
             ok = false;
@@ -311,10 +347,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                           idesc, accum);
               } else {
                 const uint64_t bd = umma_desc_k128(sb + a.x_off + kofs);
-                umma_bf16(dtm, umma_desc_k128(sb + kofs), bd, idesc, accum);
+                umma_bf16(dtm, umma_desc_k128(sb + kofs), bd, idesc_u, accum);
                 if (KIND == KIND_G13)
-                  umma_bf16(dtm + a.tok_tile, umma_desc_k128(sb + TILE_BYTES + kofs), bd, idesc,
-                            accum);
+                  umma_bf16(dtm + a.tok_tile, umma_desc_k128(sb + TILE_BYTES + kofs), bd,
+                            idesc_u, accum);
               }
             }
           }
@@ -389,8 +425,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         float* p = static_cast<float*>(a.out) + (int64_t)w.s * a.split_stride;
         const int f = w.wblk * 128 + r;
         const bool frow = f < a.nw;
+        // mid: only the pass's rows; G13 writes h = bf16(silu(a) b) straight away
+        const int ncc = a.mid ? (w.count + 15) / 16 : a.tok_tile / 16;
+        __nv_bfloat16* hm = static_cast<__nv_bfloat16*>(a.out);
 #pragma unroll 1
-        for (int cc = 0; cc < a.tok_tile / 16; ++cc) {
+        for (int cc = 0; cc < ncc; ++cc) {
           uint32_t v1[16], v3[16];
           tmem_ld16(tb + cc * 16, v1);
           if (KIND == KIND_G13) tmem_ld16(tb + a.tok_tile + cc * 16, v3);
@@ -399,9 +438,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int jj = 0; jj < 16; ++jj) {
             const int j = cc * 16 + jj;
             if (frow && j < w.count) {
-              float* rowp = p + (int64_t)(w.row0 + j) * a.out_ld;
-              rowp[f] = __uint_as_float(v1[jj]);
-              if (KIND == KIND_G13) rowp[a.nw + f] = __uint_as_float(v3[jj]);
+              if (KIND == KIND_G13 && a.mid) {
+                hm[(int64_t)(w.row0 + j) * a.out_ld + f] = __float2bfloat16_rn(
+                    silu_epilogue(__uint_as_float(v1[jj])) * __uint_as_float(v3[jj]));
+              } else {
+                float* rowp = p + (int64_t)(w.row0 + j) * a.out_ld;
+                rowp[f] = __uint_as_float(v1[jj]);
+                if (KIND == KIND_G13) rowp[a.nw + f] = __uint_as_float(v3[jj]);
+              }
             }
           }
         }
@@ -1088,6 +1132,65 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
     a.counts = nullptr;
     if (p.gather_x) a.row_gate = w.row_gate;
     if ((err = launch_pair<KIND_G2>(mH, mW2, mW2, mW2, mW2, a, pair_tiles_max * a.n_tiles, s)) !=
+        cudaSuccess)
+      return err;
+    return record(ev, 2, s);
+  }
+  if (p.mid) {  // mid-size groups: weight-stationary tiles, the expert's rows as the MMA's N
+    const int tok = p.tok_tile;
+    if (!make_map(&mX, w.xperm, d, p.rows_max, 64) ||
+        !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||
+        !make_map(&mW3, W3, d, (uint64_t)n * F, 128) || !make_map(&mH, w.h, F, p.rows_max, 64) ||
+        !make_map(&mW2, W2, F, (uint64_t)n * d, 128))
+      return cudaErrorInvalidValue;
+    // passes over all experts: one per tok rows, plus at most one partial pass per expert
+    const int64_t max_passes = n + (p.T * p.K + tok - 1) / tok;
+    TcArgs a{};
+    a.offsets = w.offsets;
+    a.n = n;
+    a.tok_tile = tok;
+    a.status = w.status;
+    a.mid = 1;
+    a.splits = 1;
+    // G13 with SwiGLU: h = bf16(silu(x.W1) * (x.W3)), W1 and W3 accumulators fill TMEM
+    a.num_kb = d / 64;
+    a.nw = F;
+    a.wb = (F + 127) / 128;
+    a.x_off = 2 * TILE_BYTES;
+    a.stage_bytes = 2 * TILE_BYTES + (uint32_t)tok * 128;
+    a.tx_bytes = a.stage_bytes;
+    a.stages = stages_for(a.stage_bytes);
+    a.acc_cols = 2 * tok;
+    a.nacc = 1;
+    a.tmem_cols = 512;
+    a.out = w.h;
+    a.out_ld = F;
+    if (p.g13_withhold) {
+      a.withhold_loads = 1;
+      a.wait_limit = p.g13_wait_limit;
+    }
+    if ((err = launch_one<KIND_G13, true>(mX, mW1, mW3, a, (int)(max_passes * a.wb), s)) !=
+        cudaSuccess)
+      return err;
+    a.withhold_loads = 0;
+    a.wait_limit = WAIT_LIMIT_CYCLES;
+    if ((err = record(ev, 0, s)) != cudaSuccess || (err = record(ev, 1, s)) != cudaSuccess)
+      return err;
+    // G2: Y = h.W2 in fp32
+    a.num_kb = F / 64;
+    a.nw = d;
+    a.wb = (d + 127) / 128;
+    a.x_off = TILE_BYTES;
+    a.stage_bytes = TILE_BYTES + (uint32_t)tok * 128;
+    a.tx_bytes = a.stage_bytes;
+    a.stages = stages_for(a.stage_bytes);
+    a.acc_cols = tok;
+    a.nacc = 2;
+    a.tmem_cols = pow2_cols(2 * tok);
+    a.out = w.y;
+    a.out_ld = d;
+    a.split_stride = 0;
+    if ((err = launch_one<KIND_G2, true>(mH, mW2, mW2, a, (int)(max_passes * a.wb), s)) !=
         cudaSuccess)
       return err;
     return record(ev, 2, s);

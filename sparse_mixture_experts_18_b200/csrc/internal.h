@@ -15,6 +15,7 @@ namespace moe {
 
 constexpr int TILE_M = 128;       // rows of one tensor-core accumulator tile
 constexpr int SIMT_TILE = 64;     // rows of one fp32 SIMT tile
+constexpr int MID_TOK = 256;      // mid-size tiling: an expert's rows per pass (the MMA's N)
 constexpr int MAX_EXPERTS = 64;
 constexpr int SMALL_ROUTE_MAX_ROWS = 1024;  // T*K limit of the one-launch routing
 
@@ -25,6 +26,8 @@ struct Plan {
   int dt = 1;              // 0 = fp32 (SIMT path), 1 = bf16 (tensor-core path)
   bool swap = false;       // small-batch path: weights are the MMA's 128-row operand
   bool pair = false;       // large batches: 256-row tiles on 2-CTA clusters (cta_group::2)
+  bool mid = false;        // mid-size groups: weight-stationary tiles, an expert's rows (up to
+                           // 256 per pass) as the MMA's N, SwiGLU fused into G13
   bool gather_x = false;   // pair path: G13 gathers its A rows from x by token (no X_perm),
                            // G2 applies the gates in its epilogue
   int row_align = 1;       // each expert's group is padded to a multiple of this

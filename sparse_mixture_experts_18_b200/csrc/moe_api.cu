@@ -69,15 +69,25 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   q.swap = dt == 1 && T <= 256 && T * K < 64 * (int64_t)n;
   // CTA pairs (256-row tiles, 128-row tails) from about 80 rows per expert on.
   q.pair = dt == 1 && !q.swap && T * K >= 640 * (int64_t)n;
-  q.row_align = dt == 0 ? SIMT_TILE : (q.swap ? 1 : TILE_M);
+  // Mid-size groups (at most 192 rows per expert on average): each CTA keeps a 128-row block
+  // of the expert's weights as the MMA's M and takes all the expert's rows (256 per pass) as
+  // N, so the weights stream once per pass instead of once per 128-row tile.  From ~256 rows
+  // on the 128-row tiles are faster (the W1 and W3 accumulators of a 256-row pass fill TMEM,
+  // so its epilogue cannot overlap the next pass; measured at n = 16, K = 1).
+  q.mid = dt == 1 && !q.swap && !q.pair && T * K <= 192 * (int64_t)n;
+  q.row_align = dt == 0 ? SIMT_TILE : (q.swap || q.mid ? 1 : TILE_M);
   q.gather_x = q.pair && gather_x_requested();
   if (route_only) {  // experts' rows contiguous and unpadded, in the caller's buffer
-    q.swap = q.pair = q.gather_x = false;
+    q.swap = q.pair = q.mid = q.gather_x = false;
     q.row_align = 1;
   }
   const int64_t P = T * K;
   q.rows_max = (P + (int64_t)n * (q.row_align - 1) + q.row_align - 1) / q.row_align * q.row_align;
   if (q.swap) q.rows_max = (P + 31) / 32 * 32;  // >= tok_tile rows for the token TMA box
+  if (q.mid) {
+    q.tok_tile = MID_TOK;
+    q.rows_max = (P + 63) / 64 * 64;  // whole 64-row boxes of B rows
+  }
   if (q.rows_max >= ((int64_t)1 << 31) / 2) return false;
   const int tokb = route_tokens_per_block(K);
   q.nblk = (T + tokb - 1) / tokb;
@@ -346,7 +356,8 @@ moe_status moe_forward_profiled(const void* x, const float* W_g, const void* W1,
 }
 
 moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtype dt,
-                         int* small_batch, int* split13, int* split2, int* launches, int* pair) {
+                         int* small_batch, int* split13, int* split2, int* launches,
+                         int* tiling) {
   Plan p;
   if (!make_plan(T, d, F, n, K, (int)dt, false, &p)) return shape_status(T, d, F, n, K, dt);
   if (small_batch) *small_batch = p.swap ? 1 : 0;
@@ -356,7 +367,7 @@ moe_status moe_plan_info(int64_t T, int64_t d, int64_t F, int n, int K, moe_dtyp
     *launches = T == 0 ? 0
                        : (p.fused_route ? 1 : 3) + (router_tc_applies(p) ? 1 : 0) +
                              (p.swap ? 3 : 2) + 1;
-  if (pair) *pair = p.pair ? 1 : 0;
+  if (tiling) *tiling = p.pair ? 1 : p.mid ? 2 : 0;
   return MOE_OK;
 }
 

@@ -209,7 +209,7 @@ def moe_plan_info(T, d, F, n, K, dtype=torch.bfloat16) -> dict:
     v = [ctypes.c_int(0) for _ in range(5)]
     _check("moe_plan_info", lib().moe_plan_info(T, d, F, n, K, dt, *[ctypes.byref(i) for i in v]))
     return {"small_batch": bool(v[0].value), "split13": v[1].value, "split2": v[2].value,
-            "launches": v[3].value, "pair": bool(v[4].value)}
+            "launches": v[3].value, "pair": v[4].value == 1, "mid": v[4].value == 2}
 
 
 def moe_forward_debug(x, W_g, W1, W3, W2, K: int, out=None, workspace=None, stream=None):

@@ -93,7 +93,7 @@ def _emulated_ep(ws, xs, layer, R):
 
 @pytest.mark.parametrize("R,T,d,F,n,K,dtype", [
     (2, 40, 256, 384, 8, 2, "bf16"),       # small batches on every rank's local stage
-    (2, 700, 256, 384, 8, 2, "bf16"),      # 128-row tiles locally
+    (2, 700, 256, 384, 8, 2, "bf16"),      # mid-size tiles locally
     (4, 1500, 256, 384, 8, 2, "bf16"),     # CTA-pair tiles locally (2 experts per rank)
     (2, 64, 64, 96, 8, 2, "f32"),          # fp32 SIMT path
     (4, 333, 320, 448, 16, 3, "bf16"),     # n = 16 over 4 ranks, K = 3, ragged d and F

@@ -42,11 +42,11 @@ def test_status_word_is_reported_and_cleared(bits, code):
     assert moe.moe_workspace_status(ws) == (MOE_OK, 0)
 
 
-@pytest.mark.parametrize("T", [16, 400], ids=["small_batch", "128_row_tiles"])
+@pytest.mark.parametrize("T", [16, 400, 2000], ids=["small_batch", "mid_size", "128_row_tiles"])
 def test_withheld_loads_time_out_and_the_workspace_recovers(T):
     w = moe_inputs.small(T=T, d=256, F=384)
     plan = moe.moe_plan_info(w.T, w.d, w.F, w.n, w.K)
-    assert not plan["pair"] and plan["small_batch"] == (T == 16)
+    assert not plan["pair"] and plan["small_batch"] == (T == 16) and plan["mid"] == (T == 400)
     x = moe_inputs.make_x(w).cuda()
     L = {k: v.cuda() for k, v in moe_inputs.make_layer(w).items()}
     nbytes = moe.moe_workspace_bytes(w.T, w.d, w.F, w.n, w.K, torch.bfloat16)

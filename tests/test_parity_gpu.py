@@ -64,10 +64,24 @@ def test_tiny_f32_full():
     assert rep["tokens"] == 64
 
 
-@pytest.mark.parametrize("T,d,F", [(700, 320, 448), (1000, 256, 384), (600, 512, 1024)])
+@pytest.mark.parametrize("T,d,F", [(1400, 320, 448), (2000, 256, 384), (1000, 512, 1024)])
 def test_prefill_tiling_small(T, d, F):
-    # T*K >= 64*n: the 128-row tile path; d % 256 and F % 128 ragged in the first case
-    _run(moe_inputs.small(T=T, d=d, F=F))
+    # 192 n < T*K < 640 n: the 128-row tile path; d % 256 and F % 128 ragged in the first case
+    plan = moe.moe_plan_info(T, d, F, 8, 2)
+    assert not (plan["small_batch"] or plan["pair"] or plan["mid"]), plan
+    _run(moe_inputs.small(T=T, d=d, F=F), budget=400)
+
+
+@pytest.mark.parametrize("T,d,F,n,K", [(300, 320, 448, 8, 2), (700, 256, 384, 8, 2),
+                                       (768, 512, 1024, 8, 2), (600, 256, 384, 16, 1),
+                                       (1024, 256, 384, 16, 2), (1000, 256, 256, 64, 2),
+                                       (300, 192, 320, 5, 3)])
+def test_mid_tiling(T, d, F, n, K):
+    # 64 n <= T*K <= 192 n: weight-stationary tiles, each expert's rows (256 per pass) as the
+    # MMA's N, SwiGLU fused into the up-projection; ragged d, F and pass tails
+    plan = moe.moe_plan_info(T, d, F, n, K)
+    assert plan["mid"] and not plan["small_batch"], plan
+    _run(moe_inputs.small(T=T, d=d, F=F, n=n, K=K), budget=400)
 
 
 @pytest.mark.parametrize("T,d,F,n,K", [(3000, 256, 384, 8, 2), (2700, 320, 448, 8, 2),
@@ -152,7 +166,7 @@ def _biased_layer(w, bias):
 @pytest.mark.parametrize("T", [16, 900, 2600])
 def test_all_tokens_to_two_experts(T):
     # T = 2600 takes the CTA-pair tiling: 2600 rows per expert are ten 256-row tiles and one
-    # 128-row tile (M = 128), and six experts have no rows
+    # 128-row tile (M = 128), and six experts have no rows; T = 900 the 128-row tiling
     w = moe_inputs.small(T=T, d=256, F=384, zipf=0.0)
     x = moe_inputs.make_x(w)
     x[:, 0] = 1.0
