@@ -97,8 +97,8 @@ struct Ctrl {
   int nact;
   int off[MAX_EXPERTS + 1];
   int act[MAX_EXPERTS];
-  int pbase[MAX_EXPERTS + 1];      // mid: passes of the active experts before each
-  int gtok[SMALL_ROUTE_MAX_ROWS];  // small batch gathering from x: token of each row
+  int pbase[MAX_EXPERTS + 1];  // mid: passes of the active experts before each
+  // small batch gathering from x: the token of each row follows the block (gather_rows ints)
 };
 
 struct Work {
@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Ctrl* c = reinterpret_cast<Ctrl*>(smem + (size_t)a.stages * a.stage_bytes);
+  int* gtok = reinterpret_cast<int*>(c + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (threadIdx.x <= a.n) c->off[threadIdx.x] = a.offsets[threadIdx.x];
   const bool gather = SWAP && KIND == KIND_G13 && a.row_tok != nullptr;
   if (gather)
-    for (int i = threadIdx.x; i < a.gather_rows; i += blockDim.x) c->gtok[i] = a.row_tok[i];
+    for (int i = threadIdx.x; i < a.gather_rows; i += blockDim.x) gtok[i] = a.row_tok[i];
   __syncthreads();
   if (threadIdx.x == 0) {
     int na = 0;
@@ -228,10 +229,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // gathering: only the 4-row groups that hold this expert's rows are loaded; the MMA
         // columns of the other slots read whatever the stage holds and are never stored
         const int ngath = gather ? (w.count + 3) / 4 : 0;
-        const int nbox = a.mid ? (w.count + 63) / 64 : 0;  // mid: 64-row boxes of B rows
+        const int nbox = a.mid ? (w.count + MID_BOX - 1) / MID_BOX : 0;  // mid: boxes of B rows
         const uint32_t tx =
             gather ? a.tx_bytes - (uint32_t)(a.tok_tile / 4 - ngath) * 512u
-            : a.mid ? a.tx_bytes - (uint32_t)(a.tok_tile / 64 - nbox) * 8192u
+            : a.mid ? a.tx_bytes - (uint32_t)(a.tok_tile / MID_BOX - nbox) * (MID_BOX * 128u)
                     : a.tx_bytes;
         bool ok = true;
         for (int kb = 0; kb < a.num_kb; ++kb) {
@@ -270,13 +271,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 int tk[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                  tk[j] = 4 * g + j < w.count ? c->gtok[w.row0 + 4 * g + j] : a.gather_T;
+                  tk[j] = 4 * g + j < w.count ? gtok[w.row0 + 4 * g + j] : a.gather_T;
                 tma_gather4(st + a.x_off + g * 512, &tmX, fb, k, tk[0], tk[1], tk[2], tk[3],
                             pol_x);
               }
             } else if (a.mid) {
               for (int b = 0; b < nbox; ++b)
-                tma_load_2d(st + a.x_off + b * 8192, &tmX, fb, k, w.row0 + 64 * b, pol_x);
+                tma_load_2d(st + a.x_off + b * (MID_BOX * 128), &tmX, fb, k,
+                            w.row0 + MID_BOX * b, pol_x);
             } else {
               tma_load_2d(st + a.x_off, &tmX, fb, k, w.row0, pol_x);
             }
@@ -1009,11 +1011,17 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ou
 }
 
 constexpr uint32_t SMEM_STAGE_BUDGET = 200 * 1024;
+// mid-size tiling: the stages may take all the shared memory a CTA can have (227 KB) beside
+// the control block (four 56 KB stages of 192-row passes); the weight tiles in flight set the
+// rate at which a CTA streams weights
+constexpr uint32_t MID_STAGE_BUDGET = 232448 - (uint32_t)sizeof(Ctrl) - 1024;
+static_assert(MID_STAGE_BUDGET >= 4 * (2 * TILE_BYTES + 192 * 128), "four 192-row stages");
 
 template <int KIND, bool SWAP, bool E4M3 = false>
 static cudaError_t launch_one(const CUtensorMap& mx, const CUtensorMap& mw0,
                               const CUtensorMap& mw1, TcArgs a, int max_work, cudaStream_t s) {
-  const size_t smem = (size_t)a.stages * a.stage_bytes + sizeof(Ctrl) + 1024;
+  const size_t gath = SWAP && KIND == KIND_G13 && a.row_tok ? (size_t)a.gather_rows * 4 : 0;
+  const size_t smem = (size_t)a.stages * a.stage_bytes + sizeof(Ctrl) + gath + 1024;
   auto kern = tc_grouped_gemm_kernel<KIND, SWAP, E4M3>;
   static int configured[MAX_DEVICES] = {0};
   const cudaError_t e = ensure_dynamic_smem(kern, smem, configured);
@@ -1065,8 +1073,8 @@ static cudaError_t launch_pair(const CUtensorMap& mx, const CUtensorMap& mw0,
   return cudaGetLastError();
 }
 
-static int stages_for(uint32_t stage_bytes) {
-  int st = (int)(SMEM_STAGE_BUDGET / stage_bytes);
+static int stages_for(uint32_t stage_bytes, uint32_t budget = SMEM_STAGE_BUDGET) {
+  int st = (int)(budget / stage_bytes);
   return st > MAX_STAGES ? MAX_STAGES : st;
 }
 
@@ -1138,9 +1146,10 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
   }
   if (p.mid) {  // mid-size groups: weight-stationary tiles, the expert's rows as the MMA's N
     const int tok = p.tok_tile;
-    if (!make_map(&mX, w.xperm, d, p.rows_max, 64) ||
+    if (!make_map(&mX, w.xperm, d, p.rows_max, MID_BOX) ||
         !make_map(&mW1, W1, d, (uint64_t)n * F, 128) ||
-        !make_map(&mW3, W3, d, (uint64_t)n * F, 128) || !make_map(&mH, w.h, F, p.rows_max, 64) ||
+        !make_map(&mW3, W3, d, (uint64_t)n * F, 128) ||
+        !make_map(&mH, w.h, F, p.rows_max, MID_BOX) ||
         !make_map(&mW2, W2, F, (uint64_t)n * d, 128))
       return cudaErrorInvalidValue;
     // passes over all experts: one per tok rows, plus at most one partial pass per expert
@@ -1159,10 +1168,12 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
     a.x_off = 2 * TILE_BYTES;
     a.stage_bytes = 2 * TILE_BYTES + (uint32_t)tok * 128;
     a.tx_bytes = a.stage_bytes;
-    a.stages = stages_for(a.stage_bytes);
+    a.stages = stages_for(a.stage_bytes, MID_STAGE_BUDGET);
+    // W1's and W3's accumulators side by side; two such slots (the epilogue of one pass
+    // overlapping the next pass's MMAs) while they fit in TMEM's 512 columns
     a.acc_cols = 2 * tok;
-    a.nacc = 1;
-    a.tmem_cols = 512;
+    a.nacc = 2 * a.acc_cols <= 512 ? 2 : 1;
+    a.tmem_cols = pow2_cols(a.nacc * a.acc_cols);
     a.out = w.h;
     a.out_ld = F;
     if (p.g13_withhold) {
@@ -1183,7 +1194,7 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
     a.x_off = TILE_BYTES;
     a.stage_bytes = TILE_BYTES + (uint32_t)tok * 128;
     a.tx_bytes = a.stage_bytes;
-    a.stages = stages_for(a.stage_bytes);
+    a.stages = stages_for(a.stage_bytes, MID_STAGE_BUDGET);
     a.acc_cols = tok;
     a.nacc = 2;
     a.tmem_cols = pow2_cols(2 * tok);

@@ -15,7 +15,8 @@ namespace moe {
 
 constexpr int TILE_M = 128;       // rows of one tensor-core accumulator tile
 constexpr int SIMT_TILE = 64;     // rows of one fp32 SIMT tile
-constexpr int MID_TOK = 256;      // mid-size tiling: an expert's rows per pass (the MMA's N)
+constexpr int MID_TOK_MAX = 256;  // mid-size tiling: most rows of an expert per pass (MMA N)
+constexpr int MID_BOX = 64;       // mid-size tiling: rows of one TMA box of B rows
 constexpr int MAX_EXPERTS = 64;
 constexpr int SMALL_ROUTE_MAX_ROWS = 1024;  // T*K limit of the one-launch routing
 
@@ -36,7 +37,8 @@ struct Plan {
   bool fused_route = false;  // small batch: routing in one launch (route_split_kernel)
   bool gather_small = false; // small batch (bf16, fused routing): G13 gathers its token rows
                              // from x (TMA gather4); routing writes no X_perm
-  int tok_tile = 0;        // swap: MMA N (tokens per expert tile), multiple of 16
+  int tok_tile = 0;        // swap: MMA N (tokens per expert tile), multiple of 16; mid: rows
+                           // of an expert per pass, multiple of MID_BOX
   int s13 = 1, s2 = 1;     // swap: split-K factors of the two expert GEMMs
   bool stack = false;      // workspace also holds the normalised activations
   bool fp8 = false;        // MXFP8 expert weights (small batch only)

@@ -77,11 +77,21 @@ def test_prefill_tiling_small(T, d, F):
                                        (1024, 256, 384, 16, 2), (1000, 256, 256, 64, 2),
                                        (300, 192, 320, 5, 3)])
 def test_mid_tiling(T, d, F, n, K):
-    # 64 n <= T*K <= 192 n: weight-stationary tiles, each expert's rows (256 per pass) as the
-    # MMA's N, SwiGLU fused into the up-projection; ragged d, F and pass tails
+    # 64 n <= T*K <= 192 n: weight-stationary tiles, each expert's rows (64 to 256 per pass,
+    # from the mean group size) as the MMA's N, SwiGLU fused into the up-projection; ragged
+    # d, F and pass tails
     plan = moe.moe_plan_info(T, d, F, n, K)
     assert plan["mid"] and not plan["small_batch"], plan
     _run(moe_inputs.small(T=T, d=d, F=F, n=n, K=K), budget=400)
+
+
+@pytest.mark.parametrize("T", [500, 700])
+def test_mid_tiling_skewed(T):
+    # Zipf(1.2) routing over 8 experts: the largest group (~43% of the rows) takes three
+    # passes over each weight block, the smallest (~4%) part of one
+    w = moe_inputs.small(T=T, d=256, F=384, zipf=1.2)
+    assert moe.moe_plan_info(w.T, w.d, w.F, w.n, w.K)["mid"]
+    _run(w, budget=T)
 
 
 @pytest.mark.parametrize("T,d,F,n,K", [(3000, 256, 384, 8, 2), (2700, 320, 448, 8, 2),
