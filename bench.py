@@ -50,11 +50,11 @@ DEFAULT_WORKLOAD = "stack32_t8192"
 # of that kernel on the workload's shapes (for the stack: one T=8192 block), valid only for
 # the kernel source it was taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "stack32_t8192": {"bytes": 2651231232, "src": "0b8972a94db6"},
-    "decode_t16": {"bytes": 1885249024, "src": "0b8972a94db6"},
-    "decode_t16 mxfp8": {"bytes": 970611456, "src": "0b8972a94db6"},
+    "stack32_t8192": {"bytes": 3661249024, "src": "a845ecde58d3"},
+    "decode_t16": {"bytes": 1885158144, "src": "a845ecde58d3"},
+    "decode_t16 mxfp8": {"bytes": 971447552, "src": "a845ecde58d3"},
     # captured at n = 8, T = 512 (the same 128 rows per expert), scaled by 8 to n = 64
-    "experts64_top2_t4096": {"bytes": 15262502912, "src": "0b8972a94db6"},
+    "experts64_top2_t4096": {"bytes": 15148277760, "src": "a845ecde58d3"},
 }
 
 
