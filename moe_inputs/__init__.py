@@ -72,6 +72,9 @@ WORKLOADS = {
     "experts64_top2_t4096": Workload("experts64_top2_t4096", T=4096, d=4096, F=14336, n=64,
                                      K=2),
     "experts64_top4_t16": Workload("experts64_top4_t16", T=16, d=4096, F=14336, n=64, K=4),
+    # the rows per expert of experts64_top2_t4096 (M_e = 128) on 8 experts: the mid-size
+    # tiling at an eighth of the weights (a case small enough for full profiler captures)
+    "experts8_top2_t512": Workload("experts8_top2_t512", T=512, d=4096, F=14336),
 }
 
 
