@@ -75,11 +75,14 @@ def test_prefill_tiling_small(T, d, F):
 @pytest.mark.parametrize("T,d,F,n,K", [(300, 320, 448, 8, 2), (700, 256, 384, 8, 2),
                                        (768, 512, 1024, 8, 2), (600, 256, 384, 16, 1),
                                        (1024, 256, 384, 16, 2), (1000, 256, 256, 64, 2),
-                                       (300, 192, 320, 5, 3)])
+                                       (300, 192, 320, 5, 3), (150, 256, 384, 1, 1),
+                                       (150, 256, 384, 4, 4), (300, 256, 384, 64, 1),
+                                       (257, 192, 256, 2, 1)])
 def test_mid_tiling(T, d, F, n, K):
     # 64 n <= T*K <= 192 n: weight-stationary tiles, each expert's rows (64 to 256 per pass,
     # from the mean group size) as the MMA's N, SwiGLU fused into the up-projection; ragged
-    # d, F and pass tails
+    # d, F and pass tails; one expert (n = 1), every expert chosen (K = n), 64 experts with
+    # about five rows each (many empty), T just above the small-batch bound
     plan = moe.moe_plan_info(T, d, F, n, K)
     assert plan["mid"] and not plan["small_batch"], plan
     _run(moe_inputs.small(T=T, d=d, F=F, n=n, K=K), budget=400)
