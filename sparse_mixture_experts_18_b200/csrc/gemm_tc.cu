@@ -22,6 +22,9 @@
 //     every SM streams weights; fp32 partial sums go to per-split slabs reduced in a fixed
 //     order afterwards.  With MXFP8 weights the operands are E4M3 codes with E8M0 block
 //     scales, applied by the MMA (kind::mxf8f6f4 block_scale).
+//   mid-size groups (tc_grouped_gemm_kernel, SWAP with `mid`): the same orientation without
+//     the K split: a unit is (expert, 128 weight rows, pass of up to tok_tile of the expert's
+//     rows), each weight byte streamed once per pass; G13 writes h itself.
 //   CTA pairs (tc_pair_gemm_kernel): cta_group::2 tiles of 256 rows x two 256-column blocks,
 //     M = 128 tiles for an expert's last 128 rows (see the section below).
 #include <stdio.h>
