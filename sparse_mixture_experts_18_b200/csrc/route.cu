@@ -256,9 +256,12 @@ __global__ void __launch_bounds__(RS_THREADS)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, c = blockIdx.x;
 
-  // ---- partial logits of this CTA's 64 hidden elements
+  // ---- partial logits of this CTA's 64 hidden elements: a warp takes four tokens and eight
+  // experts at a time (work items (token quad, expert octet) spread over the warps)
   const int sub = lane & 7;
-  for (int tb = warp * 4; tb < T; tb += (RS_THREADS / 32) * 4) {
+  const int neg = (n + 7) / 8;
+  for (int wi = warp; wi < ((T + 3) / 4) * neg; wi += RS_THREADS / 32) {
+    const int tb = (wi / neg) * 4, eg = (wi % neg) * 8;
     const int t = tb + (lane >> 3);
     Vec8<Tact> xv[CPL];
     int j0[CPL];
@@ -269,7 +272,7 @@ __global__ void __launch_bounds__(RS_THREADS)
     }
     if constexpr (std::is_same<Tact, __nv_bfloat16>::value) {
       static_assert(CPL == 1, "the MXFP8 blocks below assume 8 columns per lane");
-      if (xq != nullptr) {  // FP8-weight block: this CTA's 64 columns of the token as MXFP8
+      if (xq != nullptr && eg == 0) {  // FP8-weight block: this CTA's 64 columns as MXFP8
         // lanes sub 0-3 and 4-7 of the token hold one 32-element block each
         const bool have = t < T && j0[0] < d;
         float f[8], amax = 0.f;
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(RS_THREADS)
         }
       }
     }
-    for (int eg = 0; eg < n; eg += 8) {
+    {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < CPL; ++q) {
@@ -303,7 +306,7 @@ __global__ void __launch_bounds__(RS_THREADS)
         for (int i = 0; i < 8; ++i) {
           const float xi = xv[q].get(i);
           const float* wr = Wg + (int64_t)(j0[q] + i) * n + eg;
-          if (n == 8) {
+          if (n % 4 == 0 && eg + 8 <= n) {  // 16-byte aligned: two float4 loads
             const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr));
             const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr) + 1);
             acc[0] = fmaf(xi, w0.x, acc[0]); acc[1] = fmaf(xi, w0.y, acc[1]);
