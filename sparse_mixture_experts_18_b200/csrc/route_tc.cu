@@ -14,11 +14,12 @@
 //     (S_hi + S_mid) + S_lo of its three accumulator columns.
 //
 // One CTA per 128-token tile and K range: a cluster of CS CTAs (CS = 1, 2 or 4) splits the
-// hidden dimension, and the leader adds the others' partial sums in rank order through
-// distributed shared memory.  Warp 0 streams x and the W_g parts with TMA (no multicast), one
-// thread of warp 1 issues the MMAs, warps 2-5 read the accumulators (one token per thread) and
-// run TopK (ties to the lower index) and the softmax over the kept logits, and write the
-// token block histograms the scan kernel takes (8-token blocks, as router_topk_kernel).
+// hidden dimension; each CTA then takes a share of the tile's tokens and adds all ranks'
+// partial sums of them in rank order through distributed shared memory.  Warp 0 streams x
+// and the W_g parts with TMA (no multicast), one thread of warp 1 issues the MMAs, warps 2-5
+// read the accumulators (one token per thread) and run TopK (ties to the lower index) and the
+// softmax over the kept logits, and write the token block histograms the scan kernel takes
+// (8-token blocks, as router_topk_kernel).
 #include "internal.h"
 
 namespace moe {
@@ -204,18 +205,24 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
   }
 
   if (CS > 1) cluster_sync_all();  // every CTA's partial sums are in its shared memory
-  if (warp >= 2 && rank == 0) {
+  // the tile's 32-token quarters are shared out over the cluster (quarter q to rank q % CS):
+  // the CTA adds every rank's partial sums of its quarters' tokens in rank order, then runs
+  // TopK, the softmax and the histograms for them
+  if (warp >= 2 && (uint32_t)((warp & 3) % CS) == rank) {
     const int q = warp & 3, r = q * 32 + lane;
     const int64_t t = t0 + r;
     float* mine = part + r * pstride;
-    if (CS > 1) {  // add the other CTAs' K ranges in rank order, 48 columns per batch of loads
+    if (CS > 1) {  // the K ranges in rank order, 48 columns per batch of loads
       float4* m4 = reinterpret_cast<float4*>(mine);
       constexpr int CH = 12;  // float4 per batch
       for (int c4 = 0; c4 < npad / 4; c4 += CH) {
         float4 sum[CH];
+        {
+          const uint32_t base0 = map_to_rank(mine, 0) + 16u * (uint32_t)c4;
 #pragma unroll
-        for (int i = 0; i < CH; ++i)
-          if (c4 + i < npad / 4) sum[i] = m4[c4 + i];
+          for (int i = 0; i < CH; ++i)
+            if (c4 + i < npad / 4) sum[i] = ld_cluster_v4(base0 + 16u * (uint32_t)i);
+        }
         for (uint32_t p = 1; p < (uint32_t)CS; ++p) {
           const uint32_t base = map_to_rank(mine, p) + 16u * (uint32_t)c4;
           float4 t4[CH];
@@ -284,7 +291,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
       if ((lane & 7) == (e & 7) && b < nblk) blk_counts[b * n + e] = cnt;
     }
   }
-  if (CS > 1) cluster_sync_all();  // the leader has read every peer's partial sums
+  if (CS > 1) cluster_sync_all();  // every rank has read the partial sums it needs
 
   tc_fence_before();
   __syncthreads();
