@@ -75,6 +75,8 @@ WORKLOADS = {
     # the rows per expert of experts64_top2_t4096 (M_e = 128) on 8 experts: the mid-size
     # tiling at an eighth of the weights (a case small enough for full profiler captures)
     "experts8_top2_t512": Workload("experts8_top2_t512", T=512, d=4096, F=14336),
+    # the rows per expert of experts16_top1_t4096 (M_e = 256) on 4 experts (profiler captures)
+    "experts4_top1_t1024": Workload("experts4_top1_t1024", T=1024, d=4096, F=14336, n=4, K=1),
 }
 
 

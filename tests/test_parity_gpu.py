@@ -368,7 +368,7 @@ def test_skewed_t32768_sampled():
 
 @pytest.mark.parametrize("name", ["experts16_top1_t4096", "experts16_top4_t4096",
                                   "experts64_top2_t4096", "experts64_top4_t16",
-                                  "experts8_top2_t512"])
+                                  "experts8_top2_t512", "experts4_top1_t1024"])
 def test_expert_count_variants_full_size(name):
     """n = 16 / 64 experts with K = 1 / 2 / 4 at Mixtral's hidden and expert widths: every
     token's routing, the grouping, and sampled tokens' outputs."""
