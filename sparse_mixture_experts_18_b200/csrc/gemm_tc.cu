@@ -1164,7 +1164,7 @@ cudaError_t launch_expert_gemms_tc(const Plan& p, const void* x, const void* W1,
     a.status = w.status;
     a.mid = 1;
     a.splits = 1;
-    // G13 with SwiGLU: h = bf16(silu(x.W1) * (x.W3)), W1 and W3 accumulators fill TMEM
+    // G13 with SwiGLU: h = bf16(silu(x.W1) * (x.W3))
     a.num_kb = d / 64;
     a.nw = F;
     a.wb = (F + 127) / 128;
