@@ -50,12 +50,12 @@ DEFAULT_WORKLOAD = "stack32_t8192"
 # of that kernel on the workload's shapes (for the stack: one T=8192 block), valid only for
 # the kernel source it was taken on (hash of csrc/gemm_tc.cu + csrc/common.cuh).
 TRAFFIC = {
-    "stack32_t8192": {"bytes": 3000929024, "src": "a845ecde58d3"},
-    "decode_t16": {"bytes": 1885158144, "src": "a845ecde58d3"},
-    "decode_t16 mxfp8": {"bytes": 971447552, "src": "a845ecde58d3"},
-    "experts8_top2_t512": {"bytes": 1893885184, "src": "a845ecde58d3"},
+    "stack32_t8192": {"bytes": 2961393408, "src": "f189b48f7381"},
+    "decode_t16": {"bytes": 1885246976, "src": "f189b48f7381"},
+    "decode_t16 mxfp8": {"bytes": 971478528, "src": "f189b48f7381"},
+    "experts8_top2_t512": {"bytes": 1894018304, "src": "f189b48f7381"},
     # experts8_top2_t512's capture (the same 128 rows per expert) scaled by 8 to n = 64
-    "experts64_top2_t4096": {"bytes": 15151081472, "src": "a845ecde58d3"},
+    "experts64_top2_t4096": {"bytes": 15152146432, "src": "f189b48f7381"},
 }
 
 

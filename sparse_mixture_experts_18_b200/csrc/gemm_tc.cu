@@ -855,9 +855,34 @@ __global__ void __launch_bounds__(PAIR_THREADS, 1)
   }
 }
 
-// Small batch: h = bf16(silu(sum_s A_s) * sum_s B_s), splits summed in order 0..S-1.  All
-// 2*S loads of a thread are issued before the sums (splits unrolled up to 8).
-constexpr int REDUCE_MAX_S = 8;
+// Small batch: h = bf16(silu(sum_s A_s) * sum_s B_s), splits summed in order 0..S-1.  A
+// thread's loads go out four splits (eight float4) at a time before their sums: holding all
+// eight splits' loads took 102 registers, two CTAs per SM, and a second wave for the last
+// CTAs of a decode step's 448.
+
+// The four-wide column slice at p of the split sums of A (p[s * split_stride]) and of B (F
+// further on), in split order.
+__device__ __forceinline__ void sum_splits(const float* __restrict__ p, int S,
+                                           int64_t split_stride, int F, float4* a, float4* b) {
+  float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
+  for (int s0 = 0; s0 < S; s0 += 4) {
+    float4 ta[4], tb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (s0 + u < S) {
+        ta[u] = __ldg(reinterpret_cast<const float4*>(p + (s0 + u) * split_stride));
+        tb[u] = __ldg(reinterpret_cast<const float4*>(p + (s0 + u) * split_stride + F));
+      }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (s0 + u < S) {
+        sa.x += ta[u].x; sa.y += ta[u].y; sa.z += ta[u].z; sa.w += ta[u].w;
+        sb.x += tb[u].x; sb.y += tb[u].y; sb.z += tb[u].z; sb.w += tb[u].w;
+      }
+  }
+  *a = sa;
+  *b = sb;
+}
 
 __global__ void __launch_bounds__(256)
     swiglu_reduce_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
@@ -870,21 +895,8 @@ __global__ void __launch_bounds__(256)
        v += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = v / vpr;
     const int c = (int)(v % vpr) * 4;
-    const float* pa = p13 + r * 2 * F + c;
-    float4 ta[REDUCE_MAX_S], tb[REDUCE_MAX_S];
-#pragma unroll
-    for (int s = 0; s < REDUCE_MAX_S; ++s)
-      if (s < S) {
-        ta[s] = __ldg(reinterpret_cast<const float4*>(pa + s * split_stride));
-        tb[s] = __ldg(reinterpret_cast<const float4*>(pa + s * split_stride + F));
-      }
-    float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
-#pragma unroll
-    for (int s = 0; s < REDUCE_MAX_S; ++s)
-      if (s < S) {
-        sa.x += ta[s].x; sa.y += ta[s].y; sa.z += ta[s].z; sa.w += ta[s].w;
-        sb.x += tb[s].x; sb.y += tb[s].y; sb.z += tb[s].z; sb.w += tb[s].w;
-      }
+    float4 sa, sb;
+    sum_splits(p13 + r * 2 * F + c, S, split_stride, F, &sa, &sb);
     uint2 o;
     o.x = pack_bf16x2(silu_epilogue(sa.x) * sb.x, silu_epilogue(sa.y) * sb.y);
     o.y = pack_bf16x2(silu_epilogue(sa.z) * sb.z, silu_epilogue(sa.w) * sb.w);
@@ -914,7 +926,8 @@ __device__ __forceinline__ uint32_t mx_group_scale(float amax, float* inv, uint3
 // offsets[e]): a = sum_s A_s, b = sum_s B_s (splits in order; the block-scaled MMAs already
 // applied every scale), h = silu(a) b in binary32, then block-quantised: codes hq[r][f] and
 // the K block's scale word at slot j of the G2 B-operand chunk sfh[e][f / 128].
-__global__ void __launch_bounds__(256)
+// four CTAs per SM (at most 64 registers), so that a decode step's 448 CTAs take one wave
+__global__ void __launch_bounds__(256, 4)
     swiglu_quantize_mx_kernel(const float* __restrict__ p13, int S, int64_t split_stride,
                               int64_t rows, int F, int n, const int32_t* __restrict__ offsets,
                               uint8_t* __restrict__ hq, uint32_t* __restrict__ sfh) {
@@ -927,21 +940,8 @@ __global__ void __launch_bounds__(256)
   const int64_t r = gw / kbs;
   const int kb = (int)(gw % kbs);
   const int c = kb * 128 + lane * 4;
-  const float* pa = p13 + r * 2 * F + c;
-  float4 ta[REDUCE_MAX_S], tb[REDUCE_MAX_S];
-#pragma unroll
-  for (int k = 0; k < REDUCE_MAX_S; ++k)
-    if (k < S) {
-      ta[k] = __ldg(reinterpret_cast<const float4*>(pa + k * split_stride));
-      tb[k] = __ldg(reinterpret_cast<const float4*>(pa + k * split_stride + F));
-    }
-  float4 sa = make_float4(0.f, 0.f, 0.f, 0.f), sb = sa;
-#pragma unroll
-  for (int k = 0; k < REDUCE_MAX_S; ++k)
-    if (k < S) {
-      sa.x += ta[k].x; sa.y += ta[k].y; sa.z += ta[k].z; sa.w += ta[k].w;
-      sb.x += tb[k].x; sb.y += tb[k].y; sb.z += tb[k].z; sb.w += tb[k].w;
-    }
+  float4 sa, sb;
+  sum_splits(p13 + r * 2 * F + c, S, split_stride, F, &sa, &sb);
   const float h0 = silu_epilogue(sa.x) * sb.x, h1 = silu_epilogue(sa.y) * sb.y;
   const float h2 = silu_epilogue(sa.z) * sb.z, h3 = silu_epilogue(sa.w) * sb.w;
   float inv;
