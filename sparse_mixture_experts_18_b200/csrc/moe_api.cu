@@ -84,12 +84,14 @@ bool make_plan(int64_t T, int64_t d, int64_t F, int n, int K, int dt, bool stack
   q.swap = dt == 1 && T <= 256 && T * K < 64 * (int64_t)n;
   // CTA pairs (256-row tiles, 128-row tails) from about 80 rows per expert on.
   q.pair = dt == 1 && !q.swap && T * K >= 640 * (int64_t)n;
-  // Mid-size groups (at most 192 rows per expert on average): each CTA keeps a 128-row block
-  // of the expert's weights as the MMA's M and takes all the expert's rows (256 per pass) as
-  // N, so the weights stream once per pass instead of once per 128-row tile.  From ~256 rows
-  // on the 128-row tiles are faster (the W1 and W3 accumulators of a 256-row pass fill TMEM,
-  // so its epilogue cannot overlap the next pass; measured at n = 16, K = 1).
-  q.mid = dt == 1 && !q.swap && !q.pair && T * K <= 192 * (int64_t)n;
+  // Mid-size groups (at most 160 rows per expert on average): each CTA keeps a 128-row block
+  // of the expert's weights as the MMA's M and takes the expert's rows (up to 192 per pass at
+  // this mean) as N, so the weights stream once per pass instead of once per 128-row tile.
+  // Above it passes grow to 256 rows, whose W1 and W3 accumulators fill TMEM (no overlap of
+  // a pass's epilogue with the next) in three stages: the 128-row tiles were faster from a
+  // mean of 192 rows on (n = 16, K = 1: 1489 against 1559 us per block), the mid-size tiles
+  // at 160 (1271 against 1385 us).
+  q.mid = dt == 1 && !q.swap && !q.pair && T * K <= 160 * (int64_t)n;
   q.row_align = dt == 0 ? SIMT_TILE : (q.swap || q.mid ? 1 : TILE_M);
   q.gather_x = q.pair && gather_x_requested();
   if (route_only) {  // experts' rows contiguous and unpadded, in the caller's buffer

@@ -64,8 +64,8 @@ def test_workspace_bytes(L):
     assert ws(16, 4096, 14336, 8, 9, BF16) == 0                 # K > n
     assert ws(16, 4096, 14336, 8, 0, BF16) == 0                 # K < 1
     # the prefill layouts hold at least the routed rows of X, h and Y (mid-size tiles at
-    # T = 700, 128-row tiles at T = 2000, CTA pairs at T = 4096)
-    for T, d, F in ((700, 4096, 14336), (2000, 4096, 14336), (4096, 4096, 14336)):
+    # T = 600, 128-row tiles at T = 2000, CTA pairs at T = 4096)
+    for T, d, F in ((600, 4096, 14336), (2000, 4096, 14336), (4096, 4096, 14336)):
         assert ws(T, d, F, 8, 2, BF16) >= T * 2 * (d * 2 + F * 2 + d * 4)
     assert moe.moe_stack_workspace_bytes(8192, 4096, 14336, 8, 2) > ws(8192, 4096, 14336, 8, 2,
                                                                        BF16)
@@ -87,13 +87,13 @@ def test_plan_selection(L):
     assert rc == OK and small == 0 and s13 == 1 and s2 == 1 and launches == 7 and pair == 1
     rc, (_, _, _, launches, _) = _plan(L, 512, 4096, 14336, 8, 2)   # CUDA-core router
     assert rc == OK and launches == 6
-    rc, (small, _, _, _, tiling) = _plan(L, 700, 4096, 14336, 8, 2)   # mid-size tiles
+    rc, (small, _, _, _, tiling) = _plan(L, 600, 4096, 14336, 8, 2)   # mid-size tiles
     assert rc == OK and small == 0 and tiling == 2
     rc, (small, _, _, _, tiling) = _plan(L, 4096, 4096, 14336, 64, 2)
     assert rc == OK and small == 0 and tiling == 2
     rc, (small, _, _, _, tiling) = _plan(L, 4096, 4096, 14336, 16, 1)   # 256 rows per expert
     assert rc == OK and small == 0 and tiling == 0
-    rc, (small, _, _, _, tiling) = _plan(L, 700, 4096, 14336, 8, 2, F32)  # bf16 only
+    rc, (small, _, _, _, tiling) = _plan(L, 600, 4096, 14336, 8, 2, F32)  # bf16 only
     assert rc == OK and small == 0 and tiling == 0
     rc, (small, _, _, launches, pair) = _plan(L, 2000, 4096, 14336, 8, 2)  # 128-row tiles
     assert rc == OK and small == 0 and pair == 0 and launches == 7

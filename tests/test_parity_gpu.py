@@ -66,20 +66,20 @@ def test_tiny_f32_full():
 
 @pytest.mark.parametrize("T,d,F", [(1400, 320, 448), (2000, 256, 384), (1000, 512, 1024)])
 def test_prefill_tiling_small(T, d, F):
-    # 192 n < T*K < 640 n: the 128-row tile path; d % 256 and F % 128 ragged in the first case
+    # 160 n < T*K < 640 n: the 128-row tile path; d % 256 and F % 128 ragged in the first case
     plan = moe.moe_plan_info(T, d, F, 8, 2)
     assert not (plan["small_batch"] or plan["pair"] or plan["mid"]), plan
     _run(moe_inputs.small(T=T, d=d, F=F), budget=400)
 
 
-@pytest.mark.parametrize("T,d,F,n,K", [(300, 320, 448, 8, 2), (700, 256, 384, 8, 2),
-                                       (768, 512, 1024, 8, 2), (600, 256, 384, 16, 1),
+@pytest.mark.parametrize("T,d,F,n,K", [(300, 320, 448, 8, 2), (640, 256, 384, 8, 2),
+                                       (600, 512, 1024, 8, 2), (600, 256, 384, 16, 1),
                                        (1024, 256, 384, 16, 2), (1000, 256, 256, 64, 2),
-                                       (300, 192, 320, 5, 3), (150, 256, 384, 1, 1),
+                                       (260, 192, 320, 5, 3), (150, 256, 384, 1, 1),
                                        (150, 256, 384, 4, 4), (300, 256, 384, 64, 1),
                                        (257, 192, 256, 2, 1)])
 def test_mid_tiling(T, d, F, n, K):
-    # 64 n <= T*K <= 192 n: weight-stationary tiles, each expert's rows (64 to 256 per pass,
+    # 64 n <= T*K <= 160 n: weight-stationary tiles, each expert's rows (64 to 192 per pass,
     # from the mean group size) as the MMA's N, SwiGLU fused into the up-projection; ragged
     # d, F and pass tails; one expert (n = 1), every expert chosen (K = n), 64 experts with
     # about five rows each (many empty), T just above the small-batch bound
@@ -88,7 +88,7 @@ def test_mid_tiling(T, d, F, n, K):
     _run(moe_inputs.small(T=T, d=d, F=F, n=n, K=K), budget=400)
 
 
-@pytest.mark.parametrize("T", [500, 700])
+@pytest.mark.parametrize("T", [500, 640])
 def test_mid_tiling_skewed(T):
     # Zipf(1.2) routing over 8 experts: the largest group (~43% of the rows) takes three
     # passes over each weight block, the smallest (~4%) part of one
